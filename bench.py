@@ -1,0 +1,424 @@
+"""Benchmark: CSA2 decode over an NVFP4 main-KV cache at 1M context, batch 8.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--config 2|4]
+
+One step = one FP4 quant-append of the new token of every sequence + the 20
+decoder layers (Full + 3 Reuse, then 4 x (Reindex + 3 Reuse)), each layer
+launched on its own through the C ABI, captured once in a CUDA graph.  The
+cache (8 x 1,048,576 entries, random page permutation, 64-entry pages) is filled
+before timing; L2 is flushed (a 256 MiB write, not timed) before every timed
+step.  Prints one JSON line (rank 0).
+
+Multi-GPU: one process per GPU (torchrun), each rank runs its own batch of 8
+sequences (weak scaling, no collective on the data path); the step time is the
+max over ranks.
+
+--impl reference times the CPU oracle (the plain C restatement of the method)
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode attn tokens/s @1M ctx & achieved HBM GB/s (fraction of roofline)"
+UNIT = "tokens/s"
+PAGE = 64
+CH = 256
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    p.add_argument("--config", type=int, default=4, choices=[2, 4])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--kernel-reps", type=int, default=300)
+    p.add_argument("--contiguous-pages", action="store_true")
+    return p.parse_args()
+
+
+def workload(cfg_id: int) -> dict:
+    import synth
+    c = synth.CONFIGS[cfg_id]
+    return dict(workload=c["name"], L=c["L"], B=c["B"], layers=c["layers"], seed=c["seed"])
+
+
+def unique_bytes_per_seq(L: int, layers: int = 20) -> dict:
+    """Algorithmic bytes one decode step must move for one sequence (each byte
+    counted once per step)."""
+    nblk = (L + 7) // 8
+    blk = nblk * 128 if nblk > 2048 else 0
+    tok = min(L, 16384) * 128
+    n_sets = 5  # Full + 4 Reindex layers
+    kv = n_sets * min(512, L) * 144
+    swa = layers * min(128, L) * 512
+    append = 256 * 4 + 64 * 2 + 144 + 128
+    q = layers * 16 * 128 * 2 + n_sets * (4 * 64 * 2 + 16)
+    out = layers * (16 * 128 * 4 + 16 * 4)
+    return dict(block=blk, token=tok, kv=kv, swa=swa, append=append, q=q, out=out,
+                total=blk + tok + kv + swa + append + q + out)
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+
+def run_cuda(args, rank: int, world: int, local_rank: int):
+    import torch
+    import synth
+    import fp4_kv_cache_nvfp4_b200 as csa2
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    csa2.lib()
+    W = workload(args.config)
+    B, L, layers, seed = W["B"], W["L"], W["layers"], W["seed"] + 100 * rank
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+
+    # ---- cache: B sequences of L entries, pages permuted ----------------------
+    lens = np.full(B, L, np.int64)
+    table, n_phys = synth.page_table(seed, lens, PAGE, shuffle=not args.contiguous_pages)
+    cache = csa2.KVCache(n_phys, PAGE, torch.from_numpy(table), device=dev)
+    gain = torch.from_numpy(synth.gain(seed)).to(dev)
+    tab_d = torch.from_numpy(table).to(dev).long()
+    chunk = 1 << 16
+    for b in range(B):
+        for s0 in range(0, L, chunk):
+            m = min(chunk, L - s0)
+            pos = torch.arange(s0, s0 + m, device=dev)
+            slots = (tab_d[b, pos // PAGE] * PAGE + pos % PAGE).contiguous()
+            kv = torch.randn((m, CH), generator=gen, device=dev) * gain
+            ik = torch.randn((m, 64), generator=gen, device=dev).to(torch.bfloat16).view(torch.int16)
+            csa2.kv_quant_append(cache, kv, ik, slots)
+    torch.cuda.synchronize()
+
+    # ---- per-layer inputs -------------------------------------------------------
+    modes = csa2.schedule(True)[:layers]
+    descs = [csa2.default_desc(m, 1) for m in modes]
+    n_idx = sum(1 for m in modes if m != csa2.REUSE)
+    # one packed device buffer holds every per-step input, so one H2D copy refreshes it
+    sizes = dict(q=layers * B * 16 * 128 * 2, qi=layers * B * 4 * 64 * 2, w=layers * B * 4 * 4, kv=B * CH * 4,
+                 ik=B * 64 * 2)
+    offs, o = {}, 0
+    for k, v in sizes.items():
+        offs[k] = o
+        o += (v + 255) // 256 * 256
+    step_in = torch.empty(o, dtype=torch.uint8, device=dev)
+
+    def view(k, shape, dtype):
+        return step_in[offs[k]:offs[k] + sizes[k]].view(dtype).view(shape)
+
+    q_all = view("q", (layers, B, 16, 128), torch.int16)
+    qi_all = view("qi", (layers, B, 4, 64), torch.int16)
+    w_all = view("w", (layers, B, 4), torch.float32)
+    kv_new = view("kv", (B, CH), torch.float32)
+    ik_new = view("ik", (B, 64), torch.int16)
+    q_all.copy_(torch.randn(q_all.shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16))
+    qi_all.copy_(torch.randn(qi_all.shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16))
+    w_all.copy_(torch.rand(w_all.shape, generator=gen, device=dev))
+    kv_new.copy_(torch.randn(kv_new.shape, generator=gen, device=dev) * gain)
+    ik_new.copy_(torch.randn(ik_new.shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16))
+    swa = torch.randn((layers, B, 128, CH), generator=gen, device=dev).mul_(gain).to(torch.bfloat16).view(
+        torch.int16).contiguous()
+    seq_lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    pos_new = torch.full((B,), L - 1, dtype=torch.int64, device=dev)  # the step (re)writes the newest entry
+    slot_new = (tab_d[torch.arange(B, device=dev), pos_new // PAGE] * PAGE + pos_new % PAGE).contiguous()
+    outs = [torch.empty((B, 16, 128), dtype=torch.float32, device=dev) for _ in range(layers)]
+    lses = [torch.empty((B, 16), dtype=torch.float32, device=dev) for _ in range(layers)]
+    cand = torch.empty((B, 2048), dtype=torch.int32, device=dev)
+    sets = torch.empty((layers, B, 512), dtype=torch.int32, device=dev)
+    ws = torch.zeros(csa2.workspace_bytes(descs[0], csa2.BLOCK, B, L), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, err=err, stream=stream)
+        csa2.decode_layers(descs, cache, [qi_all[l] for l in range(layers)], [w_all[l] for l in range(layers)],
+                           [q_all[l] for l in range(layers)], [swa[l] for l in range(layers)], seq_lens, cand, sets,
+                           outs, lses, B, L, ws, err=err, stream=stream)
+
+    # eager run, then capture
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = 1 + sum({csa2.FULL: 4, csa2.REINDEX: 2, csa2.REUSE: 1}[m] for m in modes)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                graph.replay()
+        torch.cuda.synchronize()
+        # ---- timed: K steps, L2 flushed before each (flush not timed) ---------
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for k in range(args.steps):
+                flush.fill_(k & 0xFF)
+                ev[k][0].record(stream)
+                graph.replay()
+                ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        total_ms = sum(step_ms)
+        if world > 1:
+            t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            total_ms = float(t.item())
+        ms_per_step = total_ms / args.steps
+
+        # ---- dominant kernel: block-level indexer (block scoring + select) ----
+        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.kernel_reps)]
+        with torch.cuda.stream(stream):
+            for k in range(args.kernel_reps):
+                flush.fill_(k & 0xFF)
+                kev[k][0].record(stream)
+                csa2.indexer_topk(descs[0], cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens, cand, B, L, ws,
+                                  err=err, stream=stream)
+                kev[k][1].record(stream)
+        torch.cuda.synchronize()
+        k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+        # ---- end to end: pinned host inputs -> device, step, result -> host ----
+        host_in = torch.empty(step_in.numel(), dtype=torch.uint8, pin_memory=True)
+        host_in.copy_(step_in.cpu())
+        host_swa = torch.empty((layers, B, CH), dtype=torch.int16, pin_memory=True)
+        host_swa.copy_(swa[:, :, (L - 1) % 128, :].cpu())
+        host_out = torch.empty((B, 16, 128), dtype=torch.float32, pin_memory=True)
+        host_lse = torch.empty((B, 16), dtype=torch.float32, pin_memory=True)
+        cudart = _cudart()
+        ring = (L - 1) % 128
+        e2e_steps = max(10, min(args.steps, 100))
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+        with torch.cuda.stream(stream):
+            for k in range(e2e_steps):
+                flush.fill_(k & 0xFF)
+                eev[k][0].record(stream)
+                step_in.copy_(host_in, non_blocking=True)
+                for l in range(layers):  # the new token's SWA row of every layer into its ring slot
+                    dst = swa[l, :, ring, :]
+                    rc = cudart.cudaMemcpy2DAsync(ctypes.c_void_p(dst.data_ptr()), ctypes.c_size_t(128 * CH * 2),
+                                                  ctypes.c_void_p(host_swa[l].data_ptr()), ctypes.c_size_t(CH * 2),
+                                                  ctypes.c_size_t(CH * 2), ctypes.c_size_t(B), 1,
+                                                  ctypes.c_void_p(stream.cuda_stream))
+                    assert rc == 0
+                graph.replay()
+                host_out.copy_(outs[-1], non_blocking=True)
+                host_lse.copy_(lses[-1], non_blocking=True)
+                eev[k][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in eev)
+    clocks = sampler.summary()
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    h2d = step_in.numel() + layers * B * CH * 2
+    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+    ub = unique_bytes_per_seq(L, layers)
+    peaks = _peaks()
+    hbm = peaks.get("hbm_gbs")
+    k_bytes = B * ((L + 7) // 8) * 128
+    k_gbs = k_bytes / (k_ms * 1e-3) / 1e9
+    res = dict(metric=METRIC, value=world * B / (ms_per_step * 1e-3), unit=UNIT, n_gpus=world, steps=args.steps,
+               warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
+               vs_baseline=None, dtype="fp4(e2m1)+e4m3 cache; bf16 q/idx; fp32 accumulate", data="synthetic",
+               config=dict(workload=W["workload"], seq_len=L, batch_per_gpu=B, global_batch=world * B,
+                           layers=layers, schedule="decoder: F+3R, 4x(RI+3R)", page_size=PAGE,
+                           pages="contiguous" if args.contiguous_pages else "random permutation",
+                           l2="flushed before every timed step (256 MiB write, not timed)", parallelism=f"dp{world}",
+                           graph="one CUDA graph per step, programmatic dependent launch between kernels"),
+               step_bytes_unique=B * ub["total"], step_gbs=B * ub["total"] / (ms_per_step * 1e-3) / 1e9,
+               step_frac_of_hbm=(B * ub["total"] / (ms_per_step * 1e-3) / 1e9) / hbm if hbm else None,
+               roofline=dict(kernel="block-level indexer (block_score_kernel + block_select_kernel)", bound="hbm",
+                             achieved=k_gbs, peak=hbm, unit="GB/s", frac=k_gbs / hbm if hbm else None,
+                             traffic=None, bytes_per_launch=k_bytes, ms_per_launch=k_ms,
+                             peak_source="MEASURED_PEAKS.json hbm_gbs (measured)" if hbm else "fallback 6650"),
+               e2e=dict(value=world * B / (e2e_ms * 1e-3), unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                        ms_per_step=e2e_ms),
+               gpu_launches=launches_per_step * args.steps, launches_per_step=launches_per_step,
+               clocks=clocks)
+    return res
+
+
+def _cudart():
+    import torch  # noqa: F401  (loads the runtime torch ships)
+    for name in ("libcudart.so.12", "libcudart.so"):
+        try:
+            lib = ctypes.CDLL(name)
+            lib.cudaMemcpy2DAsync.restype = ctypes.c_int
+            return lib
+        except OSError:
+            continue
+    raise RuntimeError("libcudart not found")
+
+
+def _peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f)
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg_id: int, budget_s: float = 15.0, max_steps: int = 1000):
+    """Time the oracle's decode step on the host cores: the same 20-layer step
+    on sequences of the workload's length, one OpenMP thread per sequence."""
+    import oracle
+    import synth
+    W = workload(cfg_id)
+    L, layers, seed = W["L"], W["layers"], W["seed"]
+    n_seq = min(W["B"], os.cpu_count() or 1)
+    # one sequence's cache, built by the oracle itself (not timed), shared by the sampled sequences
+    kv = synth.kv_rows(seed, 0, 0, L)
+    codes, scales = oracle.quant_rows(kv)
+    del kv
+    idx = synth.idx_k_rows(seed, 0, 0, L)
+    pooled = oracle.pool_blocks(idx)
+    modes = oracle.schedule(True)[:layers]
+    q_idx = np.stack([np.concatenate([synth.q_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
+    w = np.stack([np.concatenate([synth.w_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
+    q = np.stack([np.concatenate([synth.q_heads(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
+    swa = np.stack([np.stack([synth.swa_rows(seed, l, b, 128) for l in range(layers)]) for b in range(n_seq)])
+    steps, t0 = 0, time.perf_counter()
+    while steps < max_steps:
+        oracle.decode_batch(modes, [L] * n_seq, [codes] * n_seq, [scales] * n_seq, [idx] * n_seq,
+                            [pooled] * n_seq, q_idx, w, q, swa)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return dict(value=steps * n_seq / dt, unit=UNIT, cores=n_seq, kind="oracle",
+                sample=f"{steps} decode step(s) x {n_seq} sequences of the {W['workload']} workload "
+                       f"({layers} layers, L={L}); the quant-append of the step is not in the sample; "
+                       f"{dt:.1f} s on {n_seq} of {os.cpu_count()} host threads (one per sequence)")
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    W = workload(args.config)
+    cb = oracle_sample(args.config, budget_s=max(10.0, min(60.0, 2.0 * args.steps)), max_steps=max(args.steps, 1))
+    return dict(metric=METRIC, value=cb["value"], unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=W["B"] / cb["value"] * 1e3 if cb["value"] else None, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f32 decisions / f64 attention (oracle)", data="synthetic",
+                config=dict(workload=W["workload"], seq_len=W["L"], batch_per_gpu=W["B"], layers=W["layers"],
+                            parallelism="host cores"),
+                impl="reference", cpu_baseline=cb,
+                e2e=dict(value=cb["value"], unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_cuda(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = oracle_sample(args.config, budget_s=15.0)
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

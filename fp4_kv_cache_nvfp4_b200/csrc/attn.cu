@@ -1,0 +1,354 @@
+// K6/K7: sparse attention over gathered FP4 main-KV entries plus the layer's
+// bf16 SWA window, merged by log-sum-exp.
+//
+// Pages: "Como funciona" (e-cogni.com.br): a Reuse layer runs sparse attention
+// directly on the re-used Top-K indices; every layer keeps its own global Q and
+// its own SWA KV.  The 128-token SWA window runs in every layer
+// (conexaotc.com.br, Causal Encoder-Decoder paragraph).  Merge of the two
+// branches by log-sum-exp: workload statement.
+//
+// Design (one "row" = one decode sequence or one prefill query, 16 heads that
+// share one K and one V):
+//   * a cluster of 8 CTAs per row; CTA s takes selected keys [64s, 64s+64)
+//     (four warps of 16) and window keys [16s, 16s+16) (a fifth warp);
+//   * each warp gathers its 16 rows (144 B per FP4 entry: codes + scales, or
+//     512 B per bf16 window token) with cp.async, dequantises E2M1 x E4M3 to
+//     fp16 in registers (exact: <= 6 significant bits, magnitudes 2^-10..2688)
+//     straight into the mma.sync B fragments of S = Q K^T (m16n8k16, the 16
+//     heads are the M dimension), takes an exp2-domain softmax over its keys,
+//     and multiplies P (fp16) by V (fp16 tile in shared memory, ldmatrix.trans);
+//   * warps merge their (max, sum, O) in shared memory, CTAs of the cluster
+//     through distributed shared memory: CTA s writes heads 2s and 2s+1.
+// The work per row is ~5 MFLOP against 136 KiB of gathered bytes, so the kernel
+// is bound by gather latency and HBM/L2 bandwidth; mma.sync keeps the math off
+// the critical path.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace csa2 {
+
+constexpr int ATT_SPLIT = 8;   // CTAs (cluster) per row
+constexpr int ATT_WARPS = 5;   // 4 selected-key warps + 1 window warp
+constexpr int ATT_THREADS = ATT_WARPS * 32;
+constexpr int KPW = 16;        // keys per warp
+constexpr int FP4_ROW = 144;   // staged FP4 entry: 128 code bytes + 16 scale bytes
+constexpr int SWA_ROW = 528;   // staged bf16 token: 512 B + 16 B pad (bank spread)
+constexpr int VT_ROW = 272;    // fp16 V tile row: 256 B + 16 B pad
+constexpr int OACC_ROW = 132;  // fp32 merged O row (floats)
+
+constexpr size_t ATT_OFF_FP4 = 0;
+constexpr size_t ATT_OFF_SWA = ATT_OFF_FP4 + 4 * KPW * FP4_ROW;
+constexpr size_t ATT_OFF_VT = ATT_OFF_SWA + KPW * SWA_ROW;
+constexpr size_t ATT_OFF_OACC = ATT_OFF_VT + ATT_WARPS * KPW * VT_ROW;
+constexpr size_t ATT_OFF_MS = ATT_OFF_OACC + kH * OACC_ROW * 4;
+constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;
+constexpr size_t ATT_OFF_MC = ATT_OFF_L + kH * 4;
+constexpr size_t ATT_OFF_VALID = ATT_OFF_MC + kH * 4;
+constexpr size_t ATT_SMEM = ATT_OFF_VALID + ATT_WARPS * KPW * 4;
+
+__device__ __forceinline__ uint32_t e2m1_low_byte_to_h2(uint32_t x) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+        : "=r"(out)
+        : "r"(x));
+    return out;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int split = (int)cluster.block_rank();
+    const int row = blockIdx.x / ATT_SPLIT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const bool prefill = a.q_pos != nullptr;
+    float* oacc = reinterpret_cast<float*>(smem + ATT_OFF_OACC);
+    float* ms = reinterpret_cast<float*>(smem + ATT_OFF_MS);
+    float* lacc = reinterpret_cast<float*>(smem + ATT_OFF_L);
+    float* mc = reinterpret_cast<float*>(smem + ATT_OFF_MC);
+    int* valid = reinterpret_cast<int*>(smem + ATT_OFF_VALID) + warp * KPW;
+    uint8_t* vt = smem + ATT_OFF_VT + warp * KPW * VT_ROW;
+
+    pdl_wait();
+    pdl_trigger();
+
+    // ---- sequence, window --------------------------------------------------
+    const int seq = prefill ? 0 : row;
+    int64_t L = prefill ? a.seq_len_prefill : a.seq_lens[row];
+    const uint16_t* swa_base;
+    int n_swa;
+    if (prefill) {
+        const int p = a.q_pos[row];
+        const int lo = max(0, p - a.window + 1);
+        swa_base = a.swa + (int64_t)(lo - a.swa_start) * kCh;
+        n_swa = (lo >= a.swa_start) ? p - lo + 1 : 0;
+        if (lo < a.swa_start && tid == 0 && split == 0) dev_error(a.err, CSA2_DEV_INDEX);
+    } else {
+        swa_base = a.swa + (int64_t)row * a.window * kCh;
+        n_swa = a.swa_lens ? a.swa_lens[row] : (int)(L < a.window ? L : a.window);
+        n_swa = max(0, min(n_swa, a.window));
+    }
+
+    // ---- gather this warp's 16 keys into shared memory ---------------------
+    if (warp < 4) {
+        uint8_t* st = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW;
+        const int k0 = split * 64 + warp * KPW;
+        int64_t slot = -1;
+        if (lane < KPW) {
+            const int kidx = k0 + lane;
+            if (kidx < a.topk) {
+                const int32_t pos = a.idx[(int64_t)row * a.topk + kidx];
+                if (pos >= 0) {
+                    if (pos < L) slot = entry_slot(a.cache, seq, pos, a.err);
+                    else dev_error(a.err, CSA2_DEV_INDEX);
+                }
+            }
+            valid[lane] = slot >= 0;
+        }
+        // 16 rows x 9 chunks of 16 B; every lane runs all 5 trips (the shuffle
+        // needs the full warp), trips past the 144 chunks copy nothing
+#pragma unroll
+        for (int it = 0; it < (KPW * 9 + 31) / 32; ++it) {
+            const int c = lane + 32 * it;
+            const int r = min(c / 9, KPW - 1), ch = c % 9;
+            const int64_t s = __shfl_sync(0xffffffffu, slot, r);
+            if (c < KPW * 9) {
+                uint8_t* dst = st + r * FP4_ROW + ch * 16;
+                if (s >= 0) {
+                    if (ch < 8) cp_async16(dst, a.cache.codes + s * kCodeBytes + ch * 16);
+                    else cp_async16(dst, a.cache.scales + s * kScales);
+                } else {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+    } else {
+        uint8_t* st = smem + ATT_OFF_SWA;
+        const int k0 = split * KPW;
+        if (lane < KPW) valid[lane] = (k0 + lane) < n_swa;
+        for (int c = lane; c < KPW * 32; c += 32) {
+            const int r = c >> 5, ch = c & 31;
+            uint8_t* dst = st + r * SWA_ROW + ch * 16;
+            if (k0 + r < n_swa) cp_async16(dst, swa_base + (int64_t)(k0 + r) * kCh + ch * 8);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    cp_async_commit();
+
+    // ---- Q fragments (A operand, 16 heads x 128 dims, fp16) ----------------
+    uint32_t qa[8][4];
+    {
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
+        const uint32_t* qg8 = qg + 8 * kD / 2;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            qa[c][0] = bf2_to_h2(__ldg(qg + 8 * c + t));
+            qa[c][1] = bf2_to_h2(__ldg(qg8 + 8 * c + t));
+            qa[c][2] = bf2_to_h2(__ldg(qg + 8 * c + 4 + t));
+            qa[c][3] = bf2_to_h2(__ldg(qg8 + 8 * c + 4 + t));
+        }
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+
+    // ---- S = Q K^T for the warp's two n8 tiles of keys ---------------------
+    float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    if (warp < 4) {
+        const uint8_t* st = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint8_t* r = st + (8 * j + g) * FP4_ROW;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t sc = e4m3_to_h2(r[128 + c]);
+                const uint32_t wl = *reinterpret_cast<const uint32_t*>(r + 8 * c);
+                const uint32_t wh = *reinterpret_cast<const uint32_t*>(r + 8 * c + 4);
+                const uint32_t b0 = hmul2(e2m1_low_byte_to_h2(wl >> (8 * t)), sc);
+                const uint32_t b1 = hmul2(e2m1_low_byte_to_h2(wh >> (8 * t)), sc);
+                mma16816(S[j], qa[c], b0, b1);
+            }
+        }
+    } else {
+        const uint8_t* st = smem + ATT_OFF_SWA;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t* r = reinterpret_cast<const uint32_t*>(st + (8 * j + g) * SWA_ROW);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mma16816(S[j], qa[c], bf2_to_h2(r[8 * c + t]), bf2_to_h2(r[8 * c + 4 + t]));
+        }
+    }
+
+    // ---- V tile (fp16, [key][dim]) ------------------------------------------
+    {
+        const int key = lane >> 1, half = lane & 1;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
+        if (warp < 4) {
+            const uint8_t* r = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW + key * FP4_ROW;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(r + 64 + 32 * half + 4 * i);
+                const uint32_t sc = e4m3_to_h2(r[128 + 8 + 4 * half + (i >> 1)]);
+                uint32_t h0, h1, h2, h3;
+                e2m1x8_to_h2x4(w, h0, h1, h2, h3);
+                *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc),
+                                                                    hmul2(h3, sc));
+            }
+        } else {
+            const uint32_t* r = reinterpret_cast<const uint32_t*>(smem + ATT_OFF_SWA + key * SWA_ROW) + 64 + 32 * half;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]),
+                                                                    bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+        }
+    }
+
+    // ---- softmax over the warp's keys (log2 domain) ------------------------
+    const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    float mg = -INFINITY, mg8 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const bool ok = valid[8 * j + 2 * t + e] != 0;
+            S[j][e] = ok ? S[j][e] * kScaleLog2 : -INFINITY;
+            S[j][2 + e] = ok ? S[j][2 + e] * kScaleLog2 : -INFINITY;
+            mg = fmaxf(mg, S[j][e]);
+            mg8 = fmaxf(mg8, S[j][2 + e]);
+        }
+    }
+    mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 1));
+    mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 2));
+    mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 1));
+    mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 2));
+    float lg = 0.f, lg8 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            S[j][e] = mg == -INFINITY ? 0.f : exp2f(S[j][e] - mg);
+            S[j][2 + e] = mg8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - mg8);
+            lg += S[j][e];
+            lg8 += S[j][2 + e];
+        }
+    }
+    lg += __shfl_xor_sync(0xffffffffu, lg, 1);
+    lg += __shfl_xor_sync(0xffffffffu, lg, 2);
+    lg8 += __shfl_xor_sync(0xffffffffu, lg8, 1);
+    lg8 += __shfl_xor_sync(0xffffffffu, lg8, 2);
+
+    // ---- O = P V --------------------------------------------------------------
+    const uint32_t pa[4] = {f2_to_h2(S[0][0], S[0][1]), f2_to_h2(S[0][2], S[0][3]), f2_to_h2(S[1][0], S[1][1]),
+                            f2_to_h2(S[1][2], S[1][3])};
+    __syncwarp();
+    float O[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+    {
+        const int m = lane >> 3, r = lane & 7;
+        const uint32_t base = (uint32_t)__cvta_generic_to_shared(vt) + ((m & 1) * 8 + r) * VT_ROW + (m >> 1) * 16;
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_trans(base + j * 16, b0, b1, b2, b3);
+            mma16816(O[j], pa, b0, b1);
+            mma16816(O[j + 1], pa, b2, b3);
+        }
+    }
+
+    // ---- merge the 5 warps of this CTA -------------------------------------
+    if (t == 0) {
+        ms[warp * kH + g] = mg;
+        ms[warp * kH + g + 8] = mg8;
+    }
+    __syncthreads();
+    float Mg = -INFINITY, Mg8 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < ATT_WARPS; ++w) {
+        Mg = fmaxf(Mg, ms[w * kH + g]);
+        Mg8 = fmaxf(Mg8, ms[w * kH + g + 8]);
+    }
+    const float fg = mg == -INFINITY ? 0.f : exp2f(mg - Mg);
+    const float fg8 = mg8 == -INFINITY ? 0.f : exp2f(mg8 - Mg8);
+    for (int w = 0; w < ATT_WARPS; ++w) {
+        if (warp == w) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float* p0 = oacc + g * OACC_ROW + 8 * j + 2 * t;
+                float* p1 = oacc + (g + 8) * OACC_ROW + 8 * j + 2 * t;
+                if (w == 0) {
+                    p0[0] = O[j][0] * fg;
+                    p0[1] = O[j][1] * fg;
+                    p1[0] = O[j][2] * fg8;
+                    p1[1] = O[j][3] * fg8;
+                } else {
+                    p0[0] += O[j][0] * fg;
+                    p0[1] += O[j][1] * fg;
+                    p1[0] += O[j][2] * fg8;
+                    p1[1] += O[j][3] * fg8;
+                }
+            }
+            if (t == 0) {
+                lacc[g] = (w == 0 ? 0.f : lacc[g]) + lg * fg;
+                lacc[g + 8] = (w == 0 ? 0.f : lacc[g + 8]) + lg8 * fg8;
+                if (w == 0) {
+                    mc[g] = Mg;
+                    mc[g + 8] = Mg8;
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- merge the 8 CTAs of the cluster: CTA s writes heads 2s, 2s+1 ------
+    cluster.sync();
+    for (int i = tid; i < 2 * kD; i += ATT_THREADS) {
+        const int h = 2 * split + (i >> 7), d = i & (kD - 1);
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < ATT_SPLIT; ++c) M = fmaxf(M, *cluster.map_shared_rank(mc + h, c));
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int c = 0; c < ATT_SPLIT; ++c) {
+            const float mcv = *cluster.map_shared_rank(mc + h, c);
+            const float f = mcv == -INFINITY ? 0.f : exp2f(mcv - M);
+            num += *cluster.map_shared_rank(oacc + h * OACC_ROW + d, c) * f;
+            den += *cluster.map_shared_rank(lacc + h, c) * f;
+        }
+        a.out[((int64_t)row * kH + h) * kD + d] = den > 0.f ? num / den : 0.f;
+        if (d == 0) a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+    }
+    cluster.sync();
+}
+
+cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
+    static bool init = false;
+    if (!init) {
+        cudaError_t e = cudaFuncSetAttribute((const void*)sparse_attn_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM);
+        if (e != cudaSuccess) return e;
+        init = true;
+    }
+    if (a.rows <= 0) return cudaSuccess;
+    LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), ATT_SMEM, stream, ATT_SPLIT);
+    return cudaLaunchKernelEx(&c.cfg, sparse_attn_kernel, a);
+}
+
+}  // namespace csa2

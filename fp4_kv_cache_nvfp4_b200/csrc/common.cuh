@@ -1,0 +1,193 @@
+// Shared device helpers of the CSA2 library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+constexpr int kCh = 256;        // channels per main-KV entry (K 0..127, V 128..255)
+constexpr int kCodeBytes = 128; // packed E2M1 codes per entry
+constexpr int kScales = 16;     // E4M3 scales per entry (one per 16 channels)
+constexpr int kIH = 4;          // indexer heads
+constexpr int kID = 64;         // indexer dim
+constexpr int kH = 16;          // query heads
+constexpr int kD = 128;         // head dim
+constexpr int kBlk = 8;         // positions per indexer block
+constexpr int kMaxTopk = 512;
+constexpr int kMaxKeep = 2048;
+constexpr int kMaxWindow = 128;
+constexpr int kMaxCand = kMaxKeep * kBlk;         // 16,384 token candidates
+constexpr int64_t kMaxBlockLevelLen = 1ll << 21;  // entries, block-level indexer
+constexpr int kHistBits = 12;                     // first radix digit of a score key
+constexpr int kHistBins = 1 << kHistBits;
+
+// --- bf16 / fp16 bit helpers -------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// --- programmatic dependent launch ---------------------------------------------
+// Every kernel waits on its predecessor before touching global memory, so the
+// chain of completions stays transitive.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void dev_error(int32_t* err, int32_t bit) {
+    if (err) atomicOr(err, bit);
+}
+
+// Order-preserving 32-bit key of an fp32 score: larger score -> larger key,
+// -0 and +0 share one key.  Key 0 is reserved for "not a candidate".
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    if ((u << 1) == 0u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Physical slot of entry `pos` of sequence `seq`, or -1 (and an error bit)
+// when the page table has no page there.
+__device__ __forceinline__ int64_t entry_slot(const csa2_kv_cache& c, int seq, int64_t pos, int32_t* err) {
+    int64_t pg = pos / c.page_size;
+    if (pos < 0 || pg >= c.max_pages_per_seq) {
+        dev_error(err, CSA2_DEV_PAGE);
+        return -1;
+    }
+    int32_t phys = __ldg(c.page_table + (int64_t)seq * c.max_pages_per_seq + pg);
+    if (phys < 0 || phys >= c.n_phys_pages) {
+        dev_error(err, CSA2_DEV_PAGE);
+        return -1;
+    }
+    return (int64_t)phys * c.page_size + (pos - pg * c.page_size);
+}
+
+// --- cp.async (16 B, L2-only) -------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// --- E2M1 / E4M3 ----------------------------------------------------------------
+// Nearest E2M1 code of y, ties to the even code, saturating at 6, sign copied.
+// The magnitude code is the number of rounding boundaries below |y|; at a tie
+// the boundary counts only when the upper neighbour has the even code.
+__device__ __forceinline__ uint32_t e2m1_encode(float y) {
+    float a = fabsf(y);
+    uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+    return c | ((__float_as_uint(y) >> 28) & 8u);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+__device__ __forceinline__ uint32_t e4m3_to_h2(uint8_t b) {  // (s, s) as f16x2
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+    return uint32_t(h.x) | (uint32_t(h.x) << 16);
+}
+
+// Four packed bytes = eight E2M1 codes -> four f16x2 (byte i -> h[i]; the low
+// nibble of a byte lands in the low half), hardware conversion.
+__device__ __forceinline__ void e2m1x8_to_h2x4(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2, uint32_t& h3) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(w));
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// bf16x2 -> f16x2 (exact for normal-range values)
+__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t w) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(bf16_hi(w)), "f"(bf16_lo(w)));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// --- warp / block scans ------------------------------------------------------------
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+    int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Exclusive scan of one value per thread over the whole block (blockDim a
+// multiple of 32, <= 1024).  `tmp` holds >= 33 words of shared memory.
+// Returns the exclusive prefix; *total receives the block sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+    int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t inc = warp_incl_scan(v);
+    if (lane == 31) tmp[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        uint32_t s = lane < nw ? tmp[lane] : 0u;
+        uint32_t si = warp_incl_scan(s);
+        if (lane < nw) tmp[lane] = si - s;
+        if (lane == 31) tmp[32] = si;
+    }
+    __syncthreads();
+    uint32_t r = tmp[wid] + inc - v;
+    *total = tmp[32];
+    __syncthreads();
+    return r;
+}
+
+// Given a histogram `hist[nbins]` in shared memory (descending rank = from the
+// top bin down) find the bin holding the k-th largest item (1-based k <= total):
+// *bin_out = that bin, *above_out = items in higher bins.  Whole block calls.
+__device__ __forceinline__ void find_kth_bin(const uint32_t* hist, int nbins, uint32_t k, uint32_t* tmp,
+                                             int* bin_out, uint32_t* above_out) {
+    // each thread owns a contiguous run of bins counted from the top
+    int per = (nbins + blockDim.x - 1) / blockDim.x;
+    int hi = nbins - 1 - threadIdx.x * per;  // first (highest) bin of this thread
+    uint32_t mine = 0;
+    for (int i = 0; i < per; ++i) {
+        int b = hi - i;
+        if (b >= 0) mine += hist[b];
+    }
+    uint32_t total;
+    uint32_t before = block_excl_scan(mine, tmp, &total);
+    if (before < k && before + mine >= k) {
+        uint32_t acc = before;
+        for (int i = 0; i < per; ++i) {
+            int b = hi - i;
+            if (b < 0) break;
+            if (acc + hist[b] >= k) {
+                tmp[40] = (uint32_t)b;
+                tmp[41] = acc;
+                break;
+            }
+            acc += hist[b];
+        }
+    }
+    __syncthreads();
+    *bin_out = (int)tmp[40];
+    *above_out = tmp[41];
+    __syncthreads();
+}
+
+}  // namespace csa2

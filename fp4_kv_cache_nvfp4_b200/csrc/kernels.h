@@ -1,0 +1,85 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+// Launch configuration with programmatic dependent launch enabled, and an
+// optional thread-block cluster.
+struct LaunchCfg {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[2];
+    LaunchCfg(dim3 grid, dim3 block, size_t smem, cudaStream_t stream, unsigned cluster_x = 0) {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        int n = 0;
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+        if (cluster_x > 1) {
+            attr[n].id = cudaLaunchAttributeClusterDimension;
+            attr[n].val.clusterDim.x = cluster_x;
+            attr[n].val.clusterDim.y = 1;
+            attr[n].val.clusterDim.z = 1;
+            ++n;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = n;
+    }
+};
+
+// Workspace layout of the decode indexer (byte offsets; all 256-aligned).
+struct DecodeWs {
+    size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt;
+    size_t tok_keys, tok_ctr;
+    size_t total;
+    int64_t nblk_pad;  // per-sequence stride of block arrays
+};
+DecodeWs decode_ws_layout(int n, int64_t max_len);
+
+struct PrefillWs {
+    size_t keys, total;
+    int64_t stride;
+};
+PrefillWs prefill_ws_layout(int T, int64_t n_entries);
+
+cudaError_t launch_quant_append(const csa2_kv_cache& cache, const void* src, bool bf16, const uint16_t* idx_src,
+                                int64_t n, int ratio, const int64_t* slot_mapping, int32_t* err,
+                                cudaStream_t stream);
+
+cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
+                              const int32_t* seq_lens, int keep, int32_t* out, int n, int64_t max_len,
+                              char* ws, int32_t* err, cudaStream_t stream);
+
+cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
+                              const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,
+                              int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream);
+
+cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
+                                const int32_t* seq_lens, const int32_t* q_pos, int ratio, int topk, int32_t* out,
+                                int T, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream);
+
+// Attention rows: decode (row = sequence) or prefill (row = query of sequence 0).
+struct AttnArgs {
+    csa2_kv_cache cache;
+    const uint16_t* q;        // [rows][16][128] bf16
+    const int32_t* idx;       // [rows][topk]
+    const uint16_t* swa;      // decode: [rows][window][256]; prefill: token rows from swa_start
+    const int32_t* seq_lens;  // decode: [rows]; prefill: nullptr
+    const int32_t* swa_lens;  // decode: nullable
+    const int32_t* q_pos;     // prefill: [rows]; decode: nullptr
+    float* out;
+    float* lse;
+    int32_t* err;
+    int rows, topk, window, swa_start, seq_len_prefill;
+};
+cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace csa2

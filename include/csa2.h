@@ -1,0 +1,226 @@
+/*
+ * csa2.h -- C ABI of the CSA2 sparse global-attention step over an NVFP4
+ * main-KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * What the method is (pages: "DeepSeek lanca V4.1-Flash com contexto de um
+ * milhao de tokens", conexaotc.com.br, paragraphs on CSA2 and on the FP4 KV;
+ * "Como funciona", e-cogni.com.br; "Atencion escasa comprimida 2 (CSA2)" and
+ * "FP4 KV, repeticion limitada", 7minutos.es):
+ *   - every CSA2 layer is statically Full, Reindex or Reuse.  Full computes its
+ *     own main KV, projects the indexer K from it and selects new Top-512
+ *     indices; Reindex re-scores the last Full layer's indexer K with its own
+ *     indexer Q; Reuse re-uses the main KV and the most recent Top-K and skips
+ *     the indexer.  Every layer keeps its own query and its own 128-token SWA
+ *     KV;
+ *   - in the decoder a hierarchical indexer lets the Full layer keep up to
+ *     2048 blocks of 8 positions (16,384 candidates) that later indexers score;
+ *   - the main KV is E2M1 with one E4M3 scale per 16 channels, i.e. NVFP4
+ *     without its global scale.
+ * Dimensions (fixed by the workload statement, compiled in): 16 query heads of
+ * dim 128 sharing one 128-d K and one 128-d V; indexer 4 heads x 64 with score
+ * = sum_h w_h * ReLU(q_h . k); main-KV entry = 256 channels (K = 0..127,
+ * V = 128..255) stored as 128 code bytes + 16 scale bytes.
+ *
+ * Conventions for every call:
+ *   - all array arguments are DEVICE pointers owned by the caller, except the
+ *     descriptor/cache structs and the per-layer pointer tables of
+ *     csa2_decode_layers, which are HOST memory read during the call;
+ *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and may be captured in a CUDA graph;
+ *   - kernels are launched with programmatic dependent launch: each waits for
+ *     the preceding kernel in the stream before touching memory;
+ *   - host-side checks return a status and launch nothing; errors found on the
+ *     device (a slot, page or index out of range) never fault: the access is
+ *     skipped and a CSA2_DEV_* bit is OR-ed into *err_word (if non-NULL),
+ *     which the caller reads after synchronising;
+ *   - no exception crosses the ABI; the library allocates no device memory.
+ *   - bf16 values are passed as their uint16_t bit patterns.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA2_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad mode/level, misalignment */
+    CSA2_ERR_UNSUPPORTED = 2, /* a dimension other than the compiled ones */
+    CSA2_ERR_CUDA = 3,        /* a CUDA API call or launch failed */
+    CSA2_ERR_WORKSPACE = 4    /* workspace missing or smaller than required */
+} csa2_status;
+
+/* bits OR-ed into *err_word by kernels */
+#define CSA2_DEV_SLOT 0x1   /* slot_mapping entry outside the cache */
+#define CSA2_DEV_PAGE 0x2   /* page-table entry missing or outside the cache */
+#define CSA2_DEV_INDEX 0x4  /* a Top-K index >= the sequence length */
+#define CSA2_DEV_LEN 0x8    /* a sequence length outside [1, capacity] */
+
+typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
+typedef enum { CSA2_LEVEL_BLOCK = 0, CSA2_LEVEL_TOKEN = 1 } csa2_level;
+typedef enum { CSA2_SRC_F32 = 0, CSA2_SRC_BF16 = 1 } csa2_src_dtype;
+
+/* Per-layer descriptor.  Supported values: ratio 1 or 2; 1 <= topk <= 512;
+ * block 8; 1 <= keep_blocks <= 2048; 1 <= window <= 128; n_heads 16;
+ * head_dim 128; idx_heads 4; idx_dim 64. */
+typedef struct {
+    int32_t mode;        /* csa2_mode */
+    int32_t ratio;       /* tokens per main-KV entry: 1 decoder, 2 encoder */
+    int32_t topk;        /* indices kept per Full/Reindex layer (512) */
+    int32_t block;       /* positions per indexer block (8) */
+    int32_t keep_blocks; /* blocks kept by the Full layer (2048) */
+    int32_t window;      /* SWA window in tokens (128) */
+    int32_t n_heads;     /* 16 */
+    int32_t head_dim;    /* 128 */
+    int32_t idx_heads;   /* 4 */
+    int32_t idx_dim;     /* 64 */
+} csa2_layer_desc;
+
+/* Paged global-KV cache (caller-owned device memory).  Entry e of sequence b
+ * lives in slot page_table[b][e / page_size] * page_size + e % page_size.
+ *   codes        [n_slots][128] u8  : channel 2j in the low nibble of byte j
+ *   scales       [n_slots][16]  u8  : E4M3 bits, scale i covers channels 16i..16i+15
+ *   idx_k        [n_slots][64]  bf16: indexer K of each entry
+ *   idx_k_pooled [n_slots/8][64] bf16: mean of the rows present in each
+ *                block of 8 (slot / 8); NULL if no hierarchical indexer is used
+ * n_slots = n_phys_pages * page_size; page_size is a multiple of 8; every
+ * array base is 16-byte aligned; page_table is [n_seqs][max_pages_per_seq]
+ * int32 with -1 for unused pages. */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    uint16_t* idx_k;
+    uint16_t* idx_k_pooled;
+    const int32_t* page_table;
+    int32_t page_size;
+    int32_t max_pages_per_seq;
+    int64_t n_phys_pages;
+} csa2_kv_cache;
+
+/* Fill a descriptor with the pages' defaults (topk 512, block 8, keep 2048,
+ * window 128, 16x128 heads, 4x64 indexer) for the given mode and ratio. */
+CSA2_API void csa2_layer_desc_default(csa2_layer_desc* desc, int32_t mode, int32_t ratio);
+
+/* Layer modes of the decoder (20 layers: Full + 3 Reuse, then 4 x (Reindex +
+ * 3 Reuse)) or the encoder (18 CSA2 layers: 3 x (Full + 5 Reuse)), as stated
+ * by the CSA2 paragraph of the conexaotc.com.br page and the "CSA2" section of
+ * 7minutos.es.  modes must hold 20 entries; returns the layer count. */
+CSA2_API int32_t csa2_schedule(int32_t decoder, int32_t* modes);
+
+/* ---------------------------------------------------------------------- */
+/* (1) FP4 quant-append.  Pages: FP4 KV paragraph of conexaotc.com.br, bullet
+ * "Cache KV principal em FP4" of plugged.ninja: E2M1 codes with one E4M3
+ * scale per 16 channels, no global scale.  Per 16-channel block:
+ * s = E4M3_RNE_satfinite(amax / 6) (fp32 division); code = E2M1 nearest
+ * (ties to even, saturating, sign copied) of x / s; all codes 0 when s == 0.
+ * At ratio 2 entry e is the fp32 mean (x_2e + x_2e+1) * 0.5 of two source
+ * rows.  Also copies the entry's indexer-K row and, if the cache has a pooled
+ * array, recomputes the pooled row of every block this call touches as
+ * bf16(fp32 sequential sum of the rows present / count).
+ *   kv_src       [n_entries * ratio][256] fp32 or bf16 (src_dtype)
+ *   idx_k_src    [n_entries][64] bf16, or NULL to leave idx_k and pooled alone
+ *   slot_mapping [n_entries] int64 physical slots
+ * Entries of one sequence must be contiguous and in ascending position order,
+ * and the earlier positions of a touched block must already be in the cache.
+ * n_entries == 0 is a no-op. */
+CSA2_API csa2_status csa2_kv_quant_append(const csa2_kv_cache* cache, const void* kv_src, int32_t src_dtype,
+                                 const uint16_t* idx_k_src, int64_t n_entries, int32_t ratio,
+                                 const int64_t* slot_mapping, int32_t* err_word, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* (2) Indexer Top-K.  Pages: CSA2 paragraph of conexaotc.com.br (Top-512;
+ * hierarchical indexer of up to 2048 blocks of 8 = 16,384 positions) and
+ * "Como funciona" of e-cogni.com.br (Reindex re-scores the shared indexer K
+ * with its own indexer Q).  score = sum_h w_h * max(q_h . k, 0), each dot a
+ * sequential fp32 FMA chain over the 64 dims, the head sum a sequential fp32
+ * FMA chain over h; Top-K by (score desc, index asc); outputs ascending and
+ * padded with -1.  The mode must be Full or Reindex (Reuse: INVALID_ARG).
+ *
+ * Decode (q_pos == NULL): n sequences, q_idx [n][4][64] bf16, w [n][4] fp32,
+ * seq_lens [n] entries.
+ *   level BLOCK: idx_out [n][keep_blocks] = the Top-keep blocks by the pooled
+ *     indexer K score, or every block when ceil(L/8) <= keep_blocks.
+ *   level TOKEN: idx_out [n][topk] = Top-min(topk, C) positions among the
+ *     C candidates: the positions < L of the blocks in cand_blocks
+ *     [n][keep_blocks] (ascending, -1 padded; normally the BLOCK output of
+ *     the Full layer of this step), or all L positions if cand_blocks is NULL
+ *     (then L <= 8 * keep_blocks).
+ * Prefill (q_pos != NULL, level TOKEN): n queries of sequence 0 of the page
+ *   table, q_idx [n][4][64], w [n][4], q_pos [n] absolute token positions,
+ *   seq_lens [1] = entries in the cache (<= 16384); entry j is visible to the
+ *   query at p iff (j+1)*ratio - 1 <= p; idx_out [n][topk].
+ * score_out is reserved (pass NULL).
+ * workspace: device memory of csa2_indexer_workspace_bytes() bytes, 256-byte
+ * aligned, zero-filled before its first use; every call leaves it zero-filled
+ * again.  Calls sharing one workspace must not overlap on the GPU. */
+CSA2_API size_t csa2_indexer_workspace_bytes(const csa2_layer_desc* desc, int32_t level, int32_t n, int64_t max_len,
+                                    int32_t prefill);
+CSA2_API csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
+                              const uint16_t* q_idx, const float* w, const int32_t* seq_lens, const int32_t* q_pos,
+                              const int32_t* cand_blocks, int32_t* idx_out, float* score_out, int32_t n,
+                              int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* (3) Sparse attention, decode.  Pages: "Como funciona" of e-cogni.com.br
+ * (Reuse runs sparse attention directly on the re-used indices; every layer
+ * keeps its own Q and SWA KV), SWA window of 128 tokens in every layer
+ * (conexaotc.com.br, Causal Encoder-Decoder paragraph).  Per head h:
+ * branch 1 = softmax((q_h . k_j) / sqrt(128)) weighted V over the selected
+ * entries (index -1 skipped), k_j|v_j = e2m1(code) * e4m3(scale); branch 2 =
+ * the same over the layer's SWA tokens; out = LSE merge of the two, lse =
+ * log(sum of exp over both).  No de-duplication between the two branches.
+ *   q        [B][16][128] bf16        topk_idx [B][topk] int32
+ *   swa_kv   [B][window][256] bf16 (K|V), rows 0..swa_len-1 valid (any order)
+ *   seq_lens [B] entries               swa_lens [B] or NULL (= min(window, L))
+ *   out      [B][16][128] fp32         lse      [B][16] fp32 (natural log) */
+CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
+                                    const int32_t* topk_idx, const uint16_t* swa_kv, const int32_t* seq_lens,
+                                    const int32_t* swa_lens, float* out, float* lse, int32_t B, int32_t* err_word,
+                                    void* stream);
+
+/* Sparse attention, prefill: T queries of sequence 0 of the page table at
+ * absolute token positions q_pos [T]; topk_idx [T][topk]; swa_kv holds the
+ * bf16 K|V rows of tokens swa_start, swa_start+1, ... and the window of the
+ * query at p is tokens [max(0, p - window + 1), p] (requires swa_start <= that
+ * start); seq_len = entries in the cache; out [T][16][128], lse [T][16]. */
+CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
+                                     const int32_t* topk_idx, const int32_t* q_pos, const uint16_t* swa_kv,
+                                     int32_t swa_start, int32_t seq_len, float* out, float* lse, int32_t T,
+                                     int32_t* err_word, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Schedule driver: one decode step of n_layers layers in order, each layer
+ * launched on its own (Full: BLOCK then TOKEN indexer then attention;
+ * Reindex: TOKEN indexer on the Full layer's cand_blocks with its own q_idx/w,
+ * then attention; Reuse: attention on the latest index set).  Host arrays of
+ * device pointers, one per layer: q_idx[l], w[l] (read for Full/Reindex
+ * layers only), q[l], swa_kv[l], out[l], lse[l].  cand_blocks
+ * [B][keep_blocks] and idx_sets [n_layers][B][topk] are device outputs; a
+ * Reuse layer writes no set and reads the latest one.  Layer 0 must be Full. */
+CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, const csa2_kv_cache* cache,
+                               const uint16_t* const* q_idx, const float* const* w, const uint16_t* const* q,
+                               const uint16_t* const* swa_kv, const int32_t* seq_lens, const int32_t* swa_lens,
+                               int32_t* cand_blocks, int32_t* idx_sets, float* const* out, float* const* lse,
+                               int32_t B, int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word,
+                               void* stream);
+
+/* ---------------------------------------------------------------------- */
+CSA2_API const char* csa2_status_string(csa2_status s);
+CSA2_API int32_t csa2_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

@@ -1,0 +1,347 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs spanning
+several tiles and ragged tails.  Bit-exact for codes, scales, indexer K,
+pooled K and Top-K sets; attention within max-abs 2e-3 and rel-L2 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from _gpu_util import PagedSeqs, bits16, check_attn, check_sets, dev
+
+pytestmark = pytest.mark.gpu
+SEED = 1001
+
+
+@pytest.fixture(scope="module")
+def csa2():
+    import fp4_kv_cache_nvfp4_b200 as m
+    assert torch.cuda.is_available()
+    m.lib()
+    return m
+
+
+def _fill(ps, seq, L, ratio=1, chunk=None, bf16=False, seed=SEED):
+    kv = synth.kv_rows(seed, seq, 0, L * ratio)
+    idx = synth.idx_k_rows(seed, seq, 0, L)
+    src = synth.to_bf16_bits(kv) if bf16 else kv
+    ps.append(seq, 0, src, idx, ratio=ratio, chunk=chunk)
+    return kv, idx
+
+
+# ---------------------------------------------------------------------------
+# quant-append
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("ratio,bf16,chunk", [(1, False, None), (1, False, 37), (1, True, 1000), (2, False, 513),
+                                              (2, True, None)])
+def test_quant_append_bitexact(csa2, orc, ratio, bf16, chunk):
+    lens = [4096 + 37, 1000, 9]
+    ps = PagedSeqs(csa2, lens)
+    for b, L in enumerate(lens):
+        kv, idx = _fill(ps, b, L, ratio=ratio, chunk=chunk, bf16=bf16)
+        if bf16:
+            kv = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+        codes, scales = orc.quant_rows(kv, ratio=ratio)
+        gc, gs, gk, gp = ps.unpage(b, L)
+        np.testing.assert_array_equal(gc, codes)
+        np.testing.assert_array_equal(gs, scales)
+        np.testing.assert_array_equal(gk, idx)
+        np.testing.assert_array_equal(gp, orc.pool_blocks(idx))
+    assert ps.errors() == 0
+
+
+def test_quant_append_decode_steps(csa2, orc):
+    """One entry per sequence per call, the way a decode step appends."""
+    lens = [70, 9]
+    ps = PagedSeqs(csa2, lens)
+    kvs = [synth.kv_rows(SEED, b, 0, L) for b, L in enumerate(lens)]
+    idxs = [synth.idx_k_rows(SEED, b, 0, L) for b, L in enumerate(lens)]
+    for p in range(max(lens)):
+        seqs = [b for b, L in enumerate(lens) if p < L]
+        sl = np.concatenate([ps.slots(b, [p]) for b in seqs]).astype(np.int64)
+        kv = np.concatenate([kvs[b][p:p + 1] for b in seqs])
+        ik = np.concatenate([idxs[b][p:p + 1] for b in seqs])
+        csa2.kv_quant_append(ps.cache, dev(kv), bits16(ik), dev(sl), err=ps.err)
+    for b, L in enumerate(lens):
+        gc, gs, gk, gp = ps.unpage(b, L)
+        codes, scales = orc.quant_rows(kvs[b])
+        np.testing.assert_array_equal(gc, codes)
+        np.testing.assert_array_equal(gs, scales)
+        np.testing.assert_array_equal(gp, orc.pool_blocks(idxs[b]))
+    assert ps.errors() == 0
+
+
+def test_quant_append_special_values(csa2, orc):
+    x = np.zeros((4, 256), np.float32)
+    x[0, :16] = [6, -6, 0.5, -0.5, 1, 1.5, 2, 3, 4, -4, 0, -0.0, 1.25, -2.5, 5, -0.01]
+    x[1, :16] = 5.0 * 2.0 ** -10        # amax / 6 below 2^-10: zero scale
+    x[2] = np.linspace(-1e4, 1e4, 256)  # saturating scales
+    x[3, 16:32] = -0.0
+    ps = PagedSeqs(csa2, [4])
+    ps.append(0, 0, x, np.zeros((4, 64), np.uint16))
+    gc, gs, _, _ = ps.unpage(0, 4)
+    codes, scales = orc.quant_rows(x)
+    np.testing.assert_array_equal(gc, codes)
+    np.testing.assert_array_equal(gs, scales)
+
+
+# ---------------------------------------------------------------------------
+# indexer
+# ---------------------------------------------------------------------------
+
+def _ws(csa2, n, max_len, prefill=False):
+    d = csa2.default_desc(csa2.FULL, 1)
+    nb = csa2.workspace_bytes(d, csa2.BLOCK, n, max_len, prefill)
+    return torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+
+def _indexer_inputs(B, layer=0, seed=SEED):
+    q = np.concatenate([synth.q_idx(seed, layer, b) for b in range(B)])
+    w = np.concatenate([synth.w_idx(seed, layer, b) for b in range(B)])
+    return q, w
+
+
+def test_block_topk_bitexact(csa2, orc):
+    lens = [16392, 20001, 70000, 1000, 16384]
+    B, max_len = len(lens), max(lens)
+    ps = PagedSeqs(csa2, lens)
+    idxs = [_fill(ps, b, L)[1] for b, L in enumerate(lens)]
+    q, w = _indexer_inputs(B)
+    ws = _ws(csa2, B, max_len)
+    out = torch.full((B, 2048), -7, dtype=torch.int32, device="cuda")
+    sl = dev(np.array(lens, np.int32))
+    d = csa2.default_desc(csa2.FULL, 1)
+    for rep in range(2):  # the workspace is left clean for the next call
+        csa2.indexer_topk(d, ps.cache, csa2.BLOCK, bits16(q), dev(w), sl, out, B, max_len, ws, err=ps.err)
+        got = out.cpu().numpy()
+        for b, L in enumerate(lens):
+            want = orc.select_blocks(orc.pool_blocks(idxs[b]), L, q[b], w[b])
+            check_sets(got[b], want, f"seq {b} rep {rep}")
+    assert ps.errors() == 0
+
+
+def test_block_topk_all_ties(csa2, orc):
+    L = 8 * 5000 + 3
+    ps = PagedSeqs(csa2, [L])
+    _fill(ps, 0, L)
+    ws = _ws(csa2, 1, L)
+    out = torch.empty((1, 2048), dtype=torch.int32, device="cuda")
+    q = np.zeros((1, 4, 64), np.uint16)  # every score is 0: the lowest 2048 blocks win
+    w = np.ones((1, 4), np.float32)
+    csa2.indexer_topk(csa2.default_desc(), ps.cache, csa2.BLOCK, bits16(q), dev(w), dev(np.array([L], np.int32)),
+                      out, 1, L, ws)
+    assert out.cpu().numpy()[0].tolist() == list(range(2048))
+
+
+@pytest.mark.parametrize("lens", [[16392, 20001, 70000], [1, 7, 8, 9, 511, 512, 513, 4096, 16384]])
+def test_token_topk_bitexact(csa2, orc, lens):
+    B, max_len = len(lens), max(lens)
+    ps = PagedSeqs(csa2, lens)
+    idxs = [_fill(ps, b, L)[1] for b, L in enumerate(lens)]
+    ws = _ws(csa2, B, max_len)
+    sl = dev(np.array(lens, np.int32))
+    d = csa2.default_desc(csa2.FULL, 1)
+    blocks = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
+    q0, w0 = _indexer_inputs(B, 0)
+    csa2.indexer_topk(d, ps.cache, csa2.BLOCK, bits16(q0), dev(w0), sl, blocks, B, max_len, ws, err=ps.err)
+    for layer in (0, 4):  # the Full layer's own q, then a Reindex layer's q on the same blocks
+        q, w = _indexer_inputs(B, layer)
+        out = torch.empty((B, 512), dtype=torch.int32, device="cuda")
+        csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q), dev(w), sl, out, B, max_len, ws, cand_blocks=blocks,
+                          err=ps.err)
+        got = out.cpu().numpy()
+        for b, L in enumerate(lens):
+            ob = orc.select_blocks(orc.pool_blocks(idxs[b]), L, q0[b], w0[b])
+            want = orc.select_tokens(idxs[b], L, ob, q[b], w[b])
+            check_sets(got[b], want, f"layer {layer} seq {b}")
+    if max_len <= 16384:  # flat path (no candidate blocks)
+        out = torch.empty((B, 512), dtype=torch.int32, device="cuda")
+        csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q0), dev(w0), sl, out, B, max_len, ws, err=ps.err)
+        for b, L in enumerate(lens):
+            check_sets(out.cpu().numpy()[b], orc.select_tokens(idxs[b], L, None, q0[b], w0[b]), f"flat {b}")
+    assert ps.errors() == 0
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def _swa(B, L_list, layer=0, window=128, seed=SEED):
+    s = np.zeros((B, window, 256), np.uint16)
+    for b, L in enumerate(L_list):
+        n = min(window, L)
+        s[b, :n] = synth.swa_rows(seed, layer, b, n)
+    return s
+
+
+def test_attn_decode_parity(csa2, orc):
+    lens = [5000, 300, 100, 1]
+    B = len(lens)
+    ps = PagedSeqs(csa2, lens)
+    data = [_fill(ps, b, L) for b, L in enumerate(lens)]
+    rng = np.random.default_rng(0)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, L in enumerate(lens):
+        k = min(512, L)
+        idx[b, :k] = np.sort(rng.choice(L, k, replace=False))
+    idx[0, 100] = -1  # a hole in the middle of a set is skipped
+    q = np.concatenate([synth.q_heads(SEED, 0, b) for b in range(B)])
+    swa = _swa(B, lens)
+    out = torch.empty((B, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_decode(csa2.default_desc(), ps.cache, bits16(q), dev(idx), bits16(swa),
+                            dev(np.array(lens, np.int32)), out, lse, B, err=ps.err)
+    o, l = out.cpu().numpy(), lse.cpu().numpy()
+    for b, L in enumerate(lens):
+        codes, scales = orc.quant_rows(data[b][0])
+        ro, rl = orc.attend(q[b], idx[b], codes, scales, swa[b, :min(128, L)])
+        check_attn(o[b], l[b], ro, rl, f"seq {b}")
+    assert ps.errors() == 0
+
+
+def test_attn_decode_swa_lens(csa2, orc):
+    L = 3000
+    ps = PagedSeqs(csa2, [L, L])
+    kv, _ = _fill(ps, 0, L)
+    _fill(ps, 1, L)
+    idx = np.tile(np.arange(0, 1024, 2, dtype=np.int32), (2, 1))
+    q = np.concatenate([synth.q_heads(SEED, 3, b) for b in range(2)])
+    swa = _swa(2, [L, L], layer=3)
+    swl = np.array([128, 5], np.int32)
+    out = torch.empty((2, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((2, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_decode(csa2.default_desc(), ps.cache, bits16(q), dev(idx), bits16(swa),
+                            dev(np.array([L, L], np.int32)), out, lse, 2, swa_lens=dev(swl))
+    codes, scales = orc.quant_rows(kv)
+    ro, rl = orc.attend(q[1], idx[1], codes, scales, swa[1, :5])
+    kv1 = synth.kv_rows(SEED, 1, 0, L)
+    c1, s1 = orc.quant_rows(kv1)
+    ro, rl = orc.attend(q[1], idx[1], c1, s1, swa[1, :5])
+    check_attn(out.cpu().numpy()[1], lse.cpu().numpy()[1], ro, rl, "swa_lens 5")
+
+
+# ---------------------------------------------------------------------------
+# schedule
+# ---------------------------------------------------------------------------
+
+def _decode_layer_inputs(B, lens, n_layers=20, seed=SEED):
+    q_idx = np.stack([np.concatenate([synth.q_idx(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    w = np.stack([np.concatenate([synth.w_idx(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    q = np.stack([np.concatenate([synth.q_heads(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    swa = np.zeros((B, n_layers, 128, 256), np.uint16)
+    for b, L in enumerate(lens):
+        for l in range(n_layers):
+            n = min(128, L)
+            swa[b, l, :n] = synth.swa_rows(seed, l, b, n)
+    return q_idx, w, q, swa  # [B, layers, ...]
+
+
+def run_decode_layers(csa2, ps, lens, q_idx, w, q, swa, max_len, ws=None):
+    B = len(lens)
+    modes = csa2.schedule(True)
+    n = len(modes)
+    descs = [csa2.default_desc(m, 1) for m in modes]
+    qi_t = [bits16(np.ascontiguousarray(q_idx[:, l])) for l in range(n)]
+    w_t = [dev(np.ascontiguousarray(w[:, l])) for l in range(n)]
+    q_t = [bits16(np.ascontiguousarray(q[:, l])) for l in range(n)]
+    s_t = [bits16(np.ascontiguousarray(swa[:, l])) for l in range(n)]
+    out = [torch.empty((B, 16, 128), dtype=torch.float32, device="cuda") for _ in range(n)]
+    lse = [torch.empty((B, 16), dtype=torch.float32, device="cuda") for _ in range(n)]
+    cand = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
+    sets = torch.full((n, B, 512), -9, dtype=torch.int32, device="cuda")
+    ws = _ws(csa2, B, max_len) if ws is None else ws
+    csa2.decode_layers(descs, ps.cache, qi_t, w_t, q_t, s_t, dev(np.array(lens, np.int32)), cand, sets, out, lse, B,
+                       max_len, ws, err=ps.err)
+    torch.cuda.synchronize()
+    return dict(blocks=cand.cpu().numpy(), sets=sets.cpu().numpy(), out=[o.cpu().numpy() for o in out],
+                lse=[x.cpu().numpy() for x in lse], modes=modes)
+
+
+def test_decode_layers_vs_oracle(csa2, orc):
+    lens = [20000, 9000, 130]
+    B, max_len = len(lens), max(lens)
+    ps = PagedSeqs(csa2, lens)
+    data = [_fill(ps, b, L) for b, L in enumerate(lens)]
+    q_idx, w, q, swa = _decode_layer_inputs(B, lens)
+    snap = [t.clone() for t in (ps.cache.codes, ps.cache.scales, ps.cache.idx_k, ps.cache.pooled)]
+    r = run_decode_layers(csa2, ps, lens, q_idx, w, q, swa, max_len)
+    for a, b_ in zip(snap, (ps.cache.codes, ps.cache.scales, ps.cache.idx_k, ps.cache.pooled)):
+        assert torch.equal(a, b_)  # Reindex/Reuse layers never write the shared cache
+    modes = orc.schedule(True)
+    for b, L in enumerate(lens):
+        codes, scales = orc.quant_rows(data[b][0])
+        idx = data[b][1]
+        ref = orc.decode_step(modes, L, codes, scales, idx, orc.pool_blocks(idx), q_idx[b], w[b], q[b], swa[b])
+        check_sets(r["blocks"][b], ref["blocks"], f"blocks {b}")
+        last = None
+        for l, m in enumerate(modes):
+            if m != 2:
+                check_sets(r["sets"][l, b], ref["idx"][l], f"set layer {l} seq {b}")
+                last = l
+            else:
+                check_sets(r["sets"][last, b], ref["idx"][l], f"reuse layer {l} seq {b}")
+            check_attn(r["out"][l][b], r["lse"][l][b], ref["out"][l], ref["lse"][l], f"layer {l} seq {b}")
+    assert ps.errors() == 0
+
+
+# ---------------------------------------------------------------------------
+# prefill
+# ---------------------------------------------------------------------------
+
+def test_prefill_parity(csa2, orc):
+    seed = 1003
+    tokens, T = 4096 + 62, 700
+    ratio = 2
+    n_ent = tokens // 2
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 0, 0, tokens)
+    idx_k = synth.idx_k_rows(seed, 0, 0, n_ent)
+    ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=999)
+    kvb = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+    codes, scales = orc.quant_rows(kvb, ratio=2)
+    q_pos = np.arange(tokens - T, tokens, dtype=np.int32)
+    q_idx = synth.q_idx(seed, 0, 0, T)
+    w = synth.w_idx(seed, 0, 0, T)
+    d = csa2.default_desc(csa2.FULL, 2)
+    ws = _ws(csa2, T, n_ent, prefill=True)
+    out_idx = torch.empty((T, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q_idx), dev(w), dev(np.array([n_ent], np.int32)), out_idx, T,
+                      n_ent, ws, q_pos=dev(q_pos), err=ps.err)
+    got = out_idx.cpu().numpy()
+    want = orc.prefill_indexer(q_pos, ratio, n_ent, idx_k, q_idx, w)
+    check_sets(got, want, "prefill indexer")
+    swa_start = int(q_pos[0]) - 127
+    swa = synth.swa_rows(seed, 0, 0, tokens - swa_start)
+    q = synth.q_heads(seed, 0, 0, T)
+    out = torch.empty((T, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_prefill(d, ps.cache, bits16(q), out_idx, dev(q_pos), bits16(swa), swa_start, n_ent, out, lse,
+                             T, err=ps.err)
+    ro, rl = orc.prefill_attn(q_pos, q, want, codes, scales, swa, swa_start)
+    check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, "prefill attention")
+    assert ps.errors() == 0
+
+
+# ---------------------------------------------------------------------------
+# device-side error reporting (bounds checks turn bad input into flags)
+# ---------------------------------------------------------------------------
+
+def test_device_errors_are_flagged(csa2):
+    ps = PagedSeqs(csa2, [100])
+    kv = synth.kv_rows(SEED, 0, 0, 2)
+    n_slots = ps.cache.codes.shape[0]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa2.kv_quant_append(ps.cache, dev(kv), None, dev(np.array([0, n_slots + 5], np.int64)), err=err)
+    torch.cuda.synchronize()
+    assert err.item() & 0x1
+    err.zero_()
+    idx = np.full((1, 512), -1, np.int32)
+    idx[0, :3] = [0, 5, 100]  # 100 >= L
+    out = torch.empty((1, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((1, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_decode(csa2.default_desc(), ps.cache, bits16(synth.q_heads(SEED, 0, 0)), dev(idx),
+                            bits16(np.zeros((1, 128, 256), np.uint16)), dev(np.array([100], np.int32)), out, lse, 1,
+                            err=err)
+    torch.cuda.synchronize()
+    assert err.item() & 0x4
+    assert np.isfinite(out.cpu().numpy()).all()
