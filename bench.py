@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--kernel-reps", type=int, default=300)
     p.add_argument("--contiguous-pages", action="store_true")
+    p.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
+    p.add_argument("--seq-len", type=int, default=0, help="override the context (profiling runs)")
+    p.add_argument("--breakdown", action="store_true", help="also time every call of the step on its own")
     return p.parse_args()
 
 
@@ -141,6 +144,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(dev)
     csa2.lib()
     W = workload(args.config)
+    if args.batch:
+        W["B"] = args.batch
+    if args.seq_len:
+        W["L"] = args.seq_len
+    if args.batch or args.seq_len:
+        W["workload"] += f"-override-b{W['B']}-l{W['L']}"
     B, L, layers, seed = W["B"], W["L"], W["layers"], W["seed"] + 100 * rank
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
@@ -242,11 +251,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize()
         barrier()
         step_ms = [a.elapsed_time(b) for a, b in ev]
-        total_ms = sum(step_ms)
-        if world > 1:
-            t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            total_ms = float(t.item())
+        total_ms = max_over_ranks(sum(step_ms), world, dev)
         ms_per_step = total_ms / args.steps
 
         # ---- dominant kernel: block-level indexer (block scoring + select) ----
@@ -293,6 +298,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in eev)
     clocks = sampler.summary()
     assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+    breakdown = _breakdown(csa2, cache, descs, modes, qi_all, w_all, q_all, swa, seq_lens, cand, sets, outs, lses,
+                           kv_new, ik_new, slot_new, ws, err, flush, stream, B, L) if args.breakdown else None
 
     h2d = step_in.numel() + layers * B * CH * 2
     d2h = host_out.numel() * 4 + host_lse.numel() * 4
@@ -301,7 +308,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     hbm = peaks.get("hbm_gbs")
     k_bytes = B * ((L + 7) // 8) * 128
     k_gbs = k_bytes / (k_ms * 1e-3) / 1e9
-    res = dict(metric=METRIC, value=world * B / (ms_per_step * 1e-3), unit=UNIT, n_gpus=world, steps=args.steps,
+    res = dict(metric=METRIC, value=whole_job_tokens_per_s(B, world, ms_per_step), unit=UNIT, n_gpus=world,
+               steps=args.steps,
                warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
                vs_baseline=None, dtype="fp4(e2m1)+e4m3 cache; bf16 q/idx; fp32 accumulate", data="synthetic",
                config=dict(workload=W["workload"], seq_len=L, batch_per_gpu=B, global_batch=world * B,
@@ -315,11 +323,74 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                              achieved=k_gbs, peak=hbm, unit="GB/s", frac=k_gbs / hbm if hbm else None,
                              traffic=None, bytes_per_launch=k_bytes, ms_per_launch=k_ms,
                              peak_source="MEASURED_PEAKS.json hbm_gbs (measured)" if hbm else "fallback 6650"),
-               e2e=dict(value=world * B / (e2e_ms * 1e-3), unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+               e2e=dict(value=whole_job_tokens_per_s(B, world, max_over_ranks(e2e_ms, world, dev)), unit=UNIT,
+                        h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                         ms_per_step=e2e_ms),
                gpu_launches=launches_per_step * args.steps, launches_per_step=launches_per_step,
                clocks=clocks)
+    if breakdown is not None:
+        res["breakdown_us"] = breakdown
     return res
+
+
+def _breakdown(csa2, cache, descs, modes, qi_all, w_all, q_all, swa, seq_lens, cand, sets, outs, lses, kv_new,
+               ik_new, slot_new, ws, err, flush, stream, B, L, reps=50):
+    """Every call of the step timed on its own with CUDA events (mean over
+    reps), once after an L2 flush (cold) and once right after the same call
+    (warm)."""
+    import torch
+    full = descs[0]
+    rei = next(d for d, m in zip(descs, modes) if m == csa2.REINDEX)
+    reuse = next(d for d, m in zip(descs, modes) if m == csa2.REUSE)
+    calls = {
+        "quant_append (B entries)": lambda: csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, err=err,
+                                                                  stream=stream),
+        "indexer block level (block_score + block_select)": lambda: csa2.indexer_topk(
+            full, cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens, cand, B, L, ws, err=err, stream=stream),
+        "indexer token level (token_topk)": lambda: csa2.indexer_topk(
+            rei, cache, csa2.TOKEN, qi_all[4], w_all[4], seq_lens, sets[4], B, L, ws, cand_blocks=cand, err=err,
+            stream=stream),
+        "attention, Full/Reindex layer": lambda: csa2.sparse_attn_decode(
+            full, cache, q_all[0], sets[0], swa[0], seq_lens, outs[0], lses[0], B, err=err, stream=stream),
+        "attention, Reuse layer": lambda: csa2.sparse_attn_decode(
+            reuse, cache, q_all[1], sets[0], swa[1], seq_lens, outs[1], lses[1], B, err=err, stream=stream),
+    }
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, fn in calls.items():
+            fn()
+            out = {}
+            for mode in ("cold", "warm"):
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+                for k in range(reps):
+                    if mode == "cold":
+                        flush.fill_(k & 0xFF)
+                    else:
+                        fn()
+                    ev[k][0].record(stream)
+                    fn()
+                    ev[k][1].record(stream)
+                torch.cuda.synchronize()
+                out[mode] = round(statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3, 2)
+            res[name] = out
+    return res
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (the step time of a weak-scaling
+    job is its slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(batch_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens decoded per second by all ranks together: each rank decodes its
+    own batch of sequences per step."""
+    return world * batch_per_rank / (ms_per_step * 1e-3)
 
 
 def _cudart():

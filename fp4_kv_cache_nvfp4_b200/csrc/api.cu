@@ -27,8 +27,10 @@ csa2_status check_desc(const csa2_layer_desc* d) {
 csa2_status check_cache(const csa2_kv_cache* c, bool need_idx, bool need_pooled) {
     if (!c || !c->codes || !c->scales || !c->page_table) return CSA2_ERR_INVALID_ARG;
     if (!aligned(c->codes, 16) || !aligned(c->scales, 16) || !aligned(c->page_table, 4)) return CSA2_ERR_INVALID_ARG;
-    if (c->page_size < 8 || c->page_size % 8 != 0 || c->max_pages_per_seq < 1 || c->n_phys_pages < 1)
+    if (c->page_size < 8 || (c->page_size & (c->page_size - 1)) != 0 || c->page_size > (1 << 20) ||
+        c->max_pages_per_seq < 1 || c->n_phys_pages < 1)
         return CSA2_ERR_INVALID_ARG;
+    if ((int64_t)c->max_pages_per_seq * c->page_size > (int64_t(1) << 31)) return CSA2_ERR_INVALID_ARG;
     if (c->n_phys_pages > (int64_t(1) << 40) / c->page_size) return CSA2_ERR_INVALID_ARG;
     if (need_idx && (!c->idx_k || !aligned(c->idx_k, 16))) return CSA2_ERR_INVALID_ARG;
     if (need_pooled && (!c->idx_k_pooled || !aligned(c->idx_k_pooled, 16))) return CSA2_ERR_INVALID_ARG;
@@ -110,7 +112,8 @@ csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* 
     if (!aligned(q_idx, 4) || !aligned(w, 16) || !aligned(seq_lens, 4) || !aligned(idx_out, 4))
         return CSA2_ERR_INVALID_ARG;
     if (cand_blocks && (!aligned(cand_blocks, 4) || prefill || level != CSA2_LEVEL_TOKEN)) return CSA2_ERR_INVALID_ARG;
-    if (level == CSA2_LEVEL_BLOCK && max_len > kMaxBlockLevelLen) return CSA2_ERR_UNSUPPORTED;
+    if (level == CSA2_LEVEL_BLOCK && (max_len > kMaxBlockLevelLen || n > 1024)) return CSA2_ERR_UNSUPPORTED;
+    if (level == CSA2_LEVEL_BLOCK && cache->n_phys_pages * cache->page_size / 8 > 0x7fffffff) return CSA2_ERR_UNSUPPORTED;
     if (prefill && max_len > kMaxCand) return CSA2_ERR_UNSUPPORTED;
     if (max_len > (int64_t)cache->max_pages_per_seq * cache->page_size) return CSA2_ERR_INVALID_ARG;
     const size_t need = csa2_indexer_workspace_bytes(desc, level, n, max_len, prefill ? 1 : 0);
@@ -157,6 +160,8 @@ csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const csa2_kv_c
     a.rows = B;
     a.topk = desc->topk;
     a.window = desc->window;
+    a.page_shift = page_shift_of(*cache);
+    a.early = desc->mode == CSA2_MODE_REUSE;
     return from_cuda(launch_sparse_attn(a, (cudaStream_t)stream));
 }
 
@@ -191,6 +196,8 @@ csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_
     a.window = desc->window;
     a.swa_start = swa_start;
     a.seq_len_prefill = seq_len;
+    a.page_shift = page_shift_of(*cache);
+    a.early = 0;
     return from_cuda(launch_sparse_attn(a, (cudaStream_t)stream));
 }
 

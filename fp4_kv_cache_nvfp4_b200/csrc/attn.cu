@@ -43,12 +43,20 @@ constexpr int OACC_ROW = 132;  // fp32 merged O row (floats)
 constexpr size_t ATT_OFF_FP4 = 0;
 constexpr size_t ATT_OFF_SWA = ATT_OFF_FP4 + 4 * KPW * FP4_ROW;
 constexpr size_t ATT_OFF_VT = ATT_OFF_SWA + KPW * SWA_ROW;
-constexpr size_t ATT_OFF_OACC = ATT_OFF_VT + ATT_WARPS * KPW * VT_ROW;
+constexpr size_t ATT_END_STAGE = ATT_OFF_VT + ATT_WARPS * KPW * VT_ROW;
+// per-warp rescaled O partials reuse the staging area once every warp is past P.V
+constexpr size_t ATT_OFF_OPART = 0;
+constexpr size_t ATT_END_OPART = ATT_OFF_OPART + (size_t)ATT_WARPS * kH * OACC_ROW * 4;
+constexpr size_t ATT_OFF_OACC = ATT_END_STAGE > ATT_END_OPART ? ATT_END_STAGE : ATT_END_OPART;
 constexpr size_t ATT_OFF_MS = ATT_OFF_OACC + kH * OACC_ROW * 4;
 constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;
 constexpr size_t ATT_OFF_MC = ATT_OFF_L + kH * 4;
-constexpr size_t ATT_OFF_VALID = ATT_OFF_MC + kH * 4;
+constexpr size_t ATT_OFF_LPART = ATT_OFF_MC + kH * 4;
+constexpr size_t ATT_OFF_VALID = ATT_OFF_LPART + ATT_WARPS * kH * 4;
 constexpr size_t ATT_SMEM = ATT_OFF_VALID + ATT_WARPS * KPW * 4;
+static_assert(ATT_OFF_SWA % 16 == 0 && ATT_OFF_VT % 16 == 0 && ATT_OFF_OACC % 16 == 0 && ATT_OFF_MS % 16 == 0 &&
+                  ATT_OFF_VALID % 16 == 0,
+              "attention shared-memory layout");
 
 __device__ __forceinline__ uint32_t e2m1_low_byte_to_h2(uint32_t x) {
     uint32_t out;
@@ -84,17 +92,22 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     float* ms = reinterpret_cast<float*>(smem + ATT_OFF_MS);
     float* lacc = reinterpret_cast<float*>(smem + ATT_OFF_L);
     float* mc = reinterpret_cast<float*>(smem + ATT_OFF_MC);
+    float* opart = reinterpret_cast<float*>(smem + ATT_OFF_OPART);
+    float* lpart = reinterpret_cast<float*>(smem + ATT_OFF_LPART);
     int* valid = reinterpret_cast<int*>(smem + ATT_OFF_VALID) + warp * KPW;
     uint8_t* vt = smem + ATT_OFF_VT + warp * KPW * VT_ROW;
 
-    pdl_wait();
-    pdl_trigger();
+    // A Reuse layer's index set, the cache and the SWA history come from kernels
+    // at least two launches back, so they are gathered before waiting on the
+    // preceding kernel; the query and the newest SWA row are read after it.
+    const bool early = a.early != 0;
+    if (!early) pdl_wait();
 
     // ---- sequence, window --------------------------------------------------
     const int seq = prefill ? 0 : row;
-    int64_t L = prefill ? a.seq_len_prefill : a.seq_lens[row];
+    const int32_t L = prefill ? a.seq_len_prefill : a.seq_lens[row];
     const uint16_t* swa_base;
-    int n_swa;
+    int n_swa, newest = -1;
     if (prefill) {
         const int p = a.q_pos[row];
         const int lo = max(0, p - a.window + 1);
@@ -103,21 +116,23 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         if (lo < a.swa_start && tid == 0 && split == 0) dev_error(a.err, CSA2_DEV_INDEX);
     } else {
         swa_base = a.swa + (int64_t)row * a.window * kCh;
-        n_swa = a.swa_lens ? a.swa_lens[row] : (int)(L < a.window ? L : a.window);
+        n_swa = a.swa_lens ? a.swa_lens[row] : (L < a.window ? L : a.window);
         n_swa = max(0, min(n_swa, a.window));
+        if (early && L > 0) newest = (L - 1) % a.window;
     }
 
     // ---- gather this warp's 16 keys into shared memory ---------------------
+    uint8_t* st_fp4 = smem + ATT_OFF_FP4 + (warp < 4 ? warp : 0) * KPW * FP4_ROW;
+    uint8_t* st_swa = smem + ATT_OFF_SWA;
+    const int k0 = warp < 4 ? split * 64 + warp * KPW : split * KPW;
     if (warp < 4) {
-        uint8_t* st = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW;
-        const int k0 = split * 64 + warp * KPW;
         int64_t slot = -1;
         if (lane < KPW) {
             const int kidx = k0 + lane;
             if (kidx < a.topk) {
                 const int32_t pos = a.idx[(int64_t)row * a.topk + kidx];
                 if (pos >= 0) {
-                    if (pos < L) slot = entry_slot(a.cache, seq, pos, a.err);
+                    if (pos < L) slot = entry_slot(a.cache, a.page_shift, seq, pos, a.err);
                     else dev_error(a.err, CSA2_DEV_INDEX);
                 }
             }
@@ -131,7 +146,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             const int r = min(c / 9, KPW - 1), ch = c % 9;
             const int64_t s = __shfl_sync(0xffffffffu, slot, r);
             if (c < KPW * 9) {
-                uint8_t* dst = st + r * FP4_ROW + ch * 16;
+                uint8_t* dst = st_fp4 + r * FP4_ROW + ch * 16;
                 if (s >= 0) {
                     if (ch < 8) cp_async16(dst, a.cache.codes + s * kCodeBytes + ch * 16);
                     else cp_async16(dst, a.cache.scales + s * kScales);
@@ -141,67 +156,40 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             }
         }
     } else {
-        uint8_t* st = smem + ATT_OFF_SWA;
-        const int k0 = split * KPW;
         if (lane < KPW) valid[lane] = (k0 + lane) < n_swa;
         for (int c = lane; c < KPW * 32; c += 32) {
             const int r = c >> 5, ch = c & 31;
-            uint8_t* dst = st + r * SWA_ROW + ch * 16;
-            if (k0 + r < n_swa) cp_async16(dst, swa_base + (int64_t)(k0 + r) * kCh + ch * 8);
-            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            uint8_t* dst = st_swa + r * SWA_ROW + ch * 16;
+            if (k0 + r < n_swa) {
+                if (k0 + r != newest) cp_async16(dst, swa_base + (int64_t)(k0 + r) * kCh + ch * 8);
+            } else {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            }
         }
     }
     cp_async_commit();
 
-    // ---- Q fragments (A operand, 16 heads x 128 dims, fp16) ----------------
-    uint32_t qa[8][4];
-    {
-        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
-        const uint32_t* qg8 = qg + 8 * kD / 2;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            qa[c][0] = bf2_to_h2(__ldg(qg + 8 * c + t));
-            qa[c][1] = bf2_to_h2(__ldg(qg8 + 8 * c + t));
-            qa[c][2] = bf2_to_h2(__ldg(qg + 8 * c + 4 + t));
-            qa[c][3] = bf2_to_h2(__ldg(qg8 + 8 * c + 4 + t));
-        }
-    }
-    cp_async_wait<0>();
-    __syncwarp();
-
-    // ---- S = Q K^T for the warp's two n8 tiles of keys ---------------------
-    float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    if (warp < 4) {
-        const uint8_t* st = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const uint8_t* r = st + (8 * j + g) * FP4_ROW;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint32_t sc = e4m3_to_h2(r[128 + c]);
-                const uint32_t wl = *reinterpret_cast<const uint32_t*>(r + 8 * c);
-                const uint32_t wh = *reinterpret_cast<const uint32_t*>(r + 8 * c + 4);
-                const uint32_t b0 = hmul2(e2m1_low_byte_to_h2(wl >> (8 * t)), sc);
-                const uint32_t b1 = hmul2(e2m1_low_byte_to_h2(wh >> (8 * t)), sc);
-                mma16816(S[j], qa[c], b0, b1);
-            }
-        }
-    } else {
-        const uint8_t* st = smem + ATT_OFF_SWA;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const uint32_t* r = reinterpret_cast<const uint32_t*>(st + (8 * j + g) * SWA_ROW);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) mma16816(S[j], qa[c], bf2_to_h2(r[8 * c + t]), bf2_to_h2(r[8 * c + 4 + t]));
-        }
-    }
-
-    // ---- V tile (fp16, [key][dim]) ------------------------------------------
-    {
+    // B fragments of S = Q K^T (fp16) for the warp's two n8 tiles of keys, and
+    // the fp16 V tile [key][dim] in shared memory.  In a Reuse layer the four
+    // selected-key warps build both before waiting on the preceding kernel.
+    uint32_t bk[2][8][2];
+    auto build_kv = [&]() {
         const int key = lane >> 1, half = lane & 1;
         uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
         if (warp < 4) {
-            const uint8_t* r = smem + ATT_OFF_FP4 + warp * KPW * FP4_ROW + key * FP4_ROW;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint8_t* r = st_fp4 + (8 * j + g) * FP4_ROW;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t sc = e4m3_to_h2(r[128 + c]);
+                    const uint32_t wl = *reinterpret_cast<const uint32_t*>(r + 8 * c);
+                    const uint32_t wh = *reinterpret_cast<const uint32_t*>(r + 8 * c + 4);
+                    bk[j][c][0] = hmul2(e2m1_low_byte_to_h2(wl >> (8 * t)), sc);
+                    bk[j][c][1] = hmul2(e2m1_low_byte_to_h2(wh >> (8 * t)), sc);
+                }
+            }
+            const uint8_t* r = st_fp4 + key * FP4_ROW;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(r + 64 + 32 * half + 4 * i);
@@ -212,11 +200,63 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
                                                                     hmul2(h3, sc));
             }
         } else {
-            const uint32_t* r = reinterpret_cast<const uint32_t*>(smem + ATT_OFF_SWA + key * SWA_ROW) + 64 + 32 * half;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t* r = reinterpret_cast<const uint32_t*>(st_swa + (8 * j + g) * SWA_ROW);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    bk[j][c][0] = bf2_to_h2(r[8 * c + t]);
+                    bk[j][c][1] = bf2_to_h2(r[8 * c + 4 + t]);
+                }
+            }
+            const uint32_t* r = reinterpret_cast<const uint32_t*>(st_swa + key * SWA_ROW) + 64 + 32 * half;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]),
                                                                     bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+        }
+    };
+    if (early) {
+        if (warp < 4) {
+            cp_async_wait<0>();
+            __syncwarp();
+            build_kv();
+            pdl_wait();
+        } else {
+            pdl_wait();
+            if (newest >= k0 && newest < k0 + KPW && newest < n_swa)
+                cp_async16(st_swa + (newest - k0) * SWA_ROW + lane * 16, swa_base + (int64_t)newest * kCh + lane * 8);
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            build_kv();
+        }
+    } else {
+        cp_async_wait<0>();
+        __syncwarp();
+        build_kv();
+    }
+    pdl_trigger();
+
+    // ---- Q fragments (A operand, 16 heads x 128 dims, fp16) and S = Q K^T ---
+    float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
+        const uint32_t* qg8 = qg + 8 * kD / 2;
+        uint32_t qraw[8][4];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            qraw[c][0] = __ldg(qg + 8 * c + t);
+            qraw[c][1] = __ldg(qg8 + 8 * c + t);
+            qraw[c][2] = __ldg(qg + 8 * c + 4 + t);
+            qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t qa[4] = {bf2_to_h2(qraw[c][0]), bf2_to_h2(qraw[c][1]), bf2_to_h2(qraw[c][2]),
+                                    bf2_to_h2(qraw[c][3])};
+            mma16816(S[0], qa, bk[0][c][0], bk[0][c][1]);
+            mma16816(S[1], qa, bk[1][c][0], bk[1][c][1]);
         }
     }
 
@@ -238,6 +278,10 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 2));
     mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 1));
     mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 2));
+    if (t == 0) {
+        ms[warp * kH + g] = mg;
+        ms[warp * kH + g + 8] = mg8;
+    }
     float lg = 0.f, lg8 = 0.f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -273,12 +317,9 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         }
     }
 
-    // ---- merge the 5 warps of this CTA -------------------------------------
-    if (t == 0) {
-        ms[warp * kH + g] = mg;
-        ms[warp * kH + g + 8] = mg8;
-    }
-    __syncthreads();
+    // ---- merge the 5 warps of this CTA: each writes its rescaled partial,
+    // then every thread sums the five for its share of the 16 x 128 outputs --
+    __syncthreads();  // ms complete
     float Mg = -INFINITY, Mg8 = -INFINITY;
 #pragma unroll
     for (int w = 0; w < ATT_WARPS; ++w) {
@@ -287,64 +328,92 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     }
     const float fg = mg == -INFINITY ? 0.f : exp2f(mg - Mg);
     const float fg8 = mg8 == -INFINITY ? 0.f : exp2f(mg8 - Mg8);
-    for (int w = 0; w < ATT_WARPS; ++w) {
-        if (warp == w) {
+    {
+        float* part = opart + warp * kH * OACC_ROW;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float* p0 = oacc + g * OACC_ROW + 8 * j + 2 * t;
-                float* p1 = oacc + (g + 8) * OACC_ROW + 8 * j + 2 * t;
-                if (w == 0) {
-                    p0[0] = O[j][0] * fg;
-                    p0[1] = O[j][1] * fg;
-                    p1[0] = O[j][2] * fg8;
-                    p1[1] = O[j][3] * fg8;
-                } else {
-                    p0[0] += O[j][0] * fg;
-                    p0[1] += O[j][1] * fg;
-                    p1[0] += O[j][2] * fg8;
-                    p1[1] += O[j][3] * fg8;
-                }
-            }
-            if (t == 0) {
-                lacc[g] = (w == 0 ? 0.f : lacc[g]) + lg * fg;
-                lacc[g + 8] = (w == 0 ? 0.f : lacc[g + 8]) + lg8 * fg8;
-                if (w == 0) {
-                    mc[g] = Mg;
-                    mc[g + 8] = Mg8;
-                }
+        for (int j = 0; j < 16; ++j) {
+            *reinterpret_cast<float2*>(part + g * OACC_ROW + 8 * j + 2 * t) = make_float2(O[j][0] * fg, O[j][1] * fg);
+            *reinterpret_cast<float2*>(part + (g + 8) * OACC_ROW + 8 * j + 2 * t) =
+                make_float2(O[j][2] * fg8, O[j][3] * fg8);
+        }
+        if (t == 0) {
+            lpart[warp * kH + g] = lg * fg;
+            lpart[warp * kH + g + 8] = lg8 * fg8;
+            if (warp == 0) {
+                mc[g] = Mg;
+                mc[g + 8] = Mg8;
             }
         }
-        __syncthreads();
+    }
+    __syncthreads();
+    for (int i = tid; i < kH * kD / 4; i += ATT_THREADS) {
+        const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
+        float4 acc = *reinterpret_cast<const float4*>(opart + h * OACC_ROW + d4);
+#pragma unroll
+        for (int w = 1; w < ATT_WARPS; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(opart + w * kH * OACC_ROW + h * OACC_ROW + d4);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(oacc + h * OACC_ROW + d4) = acc;
+    }
+    if (tid < kH) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < ATT_WARPS; ++w) l += lpart[w * kH + tid];
+        lacc[tid] = l;
     }
 
     // ---- merge the 8 CTAs of the cluster: CTA s writes heads 2s, 2s+1 ------
+    __shared__ float fct[2][ATT_SPLIT], sden[2];
     cluster.sync();
-    for (int i = tid; i < 2 * kD; i += ATT_THREADS) {
-        const int h = 2 * split + (i >> 7), d = i & (kD - 1);
-        float M = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < ATT_SPLIT; ++c) M = fmaxf(M, *cluster.map_shared_rank(mc + h, c));
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int c = 0; c < ATT_SPLIT; ++c) {
-            const float mcv = *cluster.map_shared_rank(mc + h, c);
-            const float f = mcv == -INFINITY ? 0.f : exp2f(mcv - M);
-            num += *cluster.map_shared_rank(oacc + h * OACC_ROW + d, c) * f;
-            den += *cluster.map_shared_rank(lacc + h, c) * f;
+    if (warp == 0) {
+        const int hh = (lane >> 3) & 1, c = lane & 7, h = 2 * split + hh;
+        float mcv = -INFINITY, lv = 0.f;
+        if (lane < 2 * ATT_SPLIT) {
+            mcv = *cluster.map_shared_rank(mc + h, c);
+            lv = *cluster.map_shared_rank(lacc + h, c);
         }
+        float M = mcv;
+#pragma unroll
+        for (int o = 1; o < ATT_SPLIT; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float f = (lane < 2 * ATT_SPLIT && mcv != -INFINITY) ? exp2f(mcv - M) : 0.f;
+        float den = lv * f;
+#pragma unroll
+        for (int o = 1; o < ATT_SPLIT; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        if (lane < 2 * ATT_SPLIT) {
+            fct[hh][c] = f;
+            if (c == 0) {
+                sden[hh] = den;
+                a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 2 * kD; i += ATT_THREADS) {
+        const int hh = i >> 7, h = 2 * split + hh, d = i & (kD - 1);
+        float num = 0.f;
+#pragma unroll
+        for (int c = 0; c < ATT_SPLIT; ++c) num += *cluster.map_shared_rank(oacc + h * OACC_ROW + d, c) * fct[hh][c];
+        const float den = sden[hh];
         a.out[((int64_t)row * kH + h) * kD + d] = den > 0.f ? num / den : 0.f;
-        if (d == 0) a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
     }
     cluster.sync();
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
-    static bool init = false;
-    if (!init) {
-        cudaError_t e = cudaFuncSetAttribute((const void*)sparse_attn_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM);
+    static bool init[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!init[dev]) {
+        e = cudaFuncSetAttribute((const void*)sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ATT_SMEM);
         if (e != cudaSuccess) return e;
-        init = true;
+        init[dev] = true;
     }
     if (a.rows <= 0) return cudaSuccess;
     LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), ATT_SMEM, stream, ATT_SPLIT);

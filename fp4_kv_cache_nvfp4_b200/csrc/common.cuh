@@ -27,6 +27,10 @@ constexpr int64_t kMaxBlockLevelLen = 1ll << 21;  // entries, block-level indexe
 constexpr int kHistBits = 12;                     // first radix digit of a score key
 constexpr int kHistBins = 1 << kHistBits;
 
+// Round a shared-memory offset up to a multiple of 16 bytes (mbarriers need 8,
+// vector and bulk accesses 16).
+constexpr size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
 // --- bf16 / fp16 bit helpers -------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -50,20 +54,20 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Physical slot of entry `pos` of sequence `seq`, or -1 (and an error bit)
-// when the page table has no page there.
-__device__ __forceinline__ int64_t entry_slot(const csa2_kv_cache& c, int seq, int64_t pos, int32_t* err) {
-    int64_t pg = pos / c.page_size;
+// Physical slot of entry `pos` of sequence `seq` (page size 1 << shift), or -1
+// (and an error bit) when the page table has no page there.
+__device__ __forceinline__ int64_t entry_slot(const csa2_kv_cache& c, int shift, int seq, int32_t pos, int32_t* err) {
+    const int32_t pg = pos >> shift;
     if (pos < 0 || pg >= c.max_pages_per_seq) {
         dev_error(err, CSA2_DEV_PAGE);
         return -1;
     }
-    int32_t phys = __ldg(c.page_table + (int64_t)seq * c.max_pages_per_seq + pg);
+    const int32_t phys = __ldg(c.page_table + (int64_t)seq * c.max_pages_per_seq + pg);
     if (phys < 0 || phys >= c.n_phys_pages) {
         dev_error(err, CSA2_DEV_PAGE);
         return -1;
     }
-    return (int64_t)phys * c.page_size + (pos - pg * c.page_size);
+    return ((int64_t)phys << shift) | (int64_t)(pos & ((1 << shift) - 1));
 }
 
 // --- cp.async (16 B, L2-only) -------------------------------------------------
@@ -74,6 +78,41 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// --- mbarrier + TMA (bulk tensor copies, no multicast) ------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Wait for the phase with the given parity; gives up after `limit` polls and
+// returns false (the caller reports a timeout instead of hanging).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// 2-D tiled bulk copy global -> this CTA's shared memory, completion counted
+// in bytes on `bar`.  x (innermost) must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int32_t x, int32_t y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 
 // --- E2M1 / E4M3 ----------------------------------------------------------------
 // Nearest E2M1 code of y, ties to the even code, saturating at 6, sign copied.

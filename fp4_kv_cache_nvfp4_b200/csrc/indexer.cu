@@ -12,54 +12,42 @@
 // (score desc, index asc).  Every score is therefore bit-identical to the
 // oracle's and the selected sets are exact.
 //
+// Selection is a most-significant-digit radix select on order-preserving
+// 32-bit keys: a 12-bit first digit (bits 31..20), then two 10-bit digits
+// that only look at the slots left in the threshold bin, then an ordered
+// emission (ballots in slot order) that keeps ties at the lowest index.
+//
 // Kernels
-//   block_score_kernel  (K2)  stream the pooled indexer K of every block of a
-//                              sequence, write fp32 scores and a 4096-bin
-//                              histogram of the top 12 key bits; the last CTA
-//                              of a sequence finds the bin holding the
-//                              keep-th largest score.  HBM-bound: 128 B/block.
-//   block_select_kernel (K3)  mark blocks above that bin in a bitmap, collect
-//                              the bin's members; the last CTA refines the
-//                              boundary with two 10-bit passes and emits the
-//                              kept blocks in ascending order.
+//   block_score_kernel  (K2)  stream the pooled indexer K of every block,
+//                              write fp32 scores and a per-sequence histogram
+//                              of the first digit; the last CTA of a sequence
+//                              finds the bin holding the keep-th score.
+//                              HBM-bound: 128 B per block.
+//   block_select_kernel (K3)  mark blocks above that bin in a bitmap and
+//                              collect the bin's members; the last CTA refines
+//                              the boundary and emits the kept blocks in order.
 //   token_topk_kernel   (K4)  score the <= 16,384 candidates (1 KiB runs of 8
-//                              indexer-K rows), the last CTA of a sequence
-//                              selects the Top-K with a 12/10/10-bit radix
-//                              select in shared memory.
+//                              indexer-K rows) and histogram them; the last CTA
+//                              of a sequence refines and emits the Top-K.
 //   prefill_score_kernel / prefill_select_kernel: the same per query over the
 //                              entries visible to it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace csa2 {
 
 // ----------------------------------------------------------------------------
 // score of one indexer-K row held as 32 bf16x2 words; qd[d] = (q_0..q_3)[d]
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ float idx_score(const uint32_t (&k)[32], const float4* __restrict__ qd, float4 w) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float k0 = bf16_lo(k[i]), k1 = bf16_hi(k[i]);
-        const float4 q0 = qd[2 * i], q1 = qd[2 * i + 1];
-        a0 = __fmaf_rn(q0.x, k0, a0);
-        a1 = __fmaf_rn(q0.y, k0, a1);
-        a2 = __fmaf_rn(q0.z, k0, a2);
-        a3 = __fmaf_rn(q0.w, k0, a3);
-        a0 = __fmaf_rn(q1.x, k1, a0);
-        a1 = __fmaf_rn(q1.y, k1, a1);
-        a2 = __fmaf_rn(q1.z, k1, a2);
-        a3 = __fmaf_rn(q1.w, k1, a3);
-    }
-    float s = 0.f;
-    s = __fmaf_rn(w.x, a0 > 0.f ? a0 : 0.f, s);
-    s = __fmaf_rn(w.y, a1 > 0.f ? a1 : 0.f, s);
-    s = __fmaf_rn(w.z, a2 > 0.f ? a2 : 0.f, s);
-    s = __fmaf_rn(w.w, a3 > 0.f ? a3 : 0.f, s);
-    return s;
-}
-
-// Two rows at once (amortises the q reads from shared memory).
 __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32_t (&m)[32],
                                            const float4* __restrict__ qd, float4 w, float& s_k, float& s_m) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
@@ -99,6 +87,29 @@ __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32
     s_m = t;
 }
 
+__device__ __forceinline__ float idx_score1(const uint32_t (&k)[32], const float4* __restrict__ qd, float4 w) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float k0 = bf16_lo(k[i]), k1 = bf16_hi(k[i]);
+        const float4 q0 = qd[2 * i], q1 = qd[2 * i + 1];
+        a0 = __fmaf_rn(q0.x, k0, a0);
+        a1 = __fmaf_rn(q0.y, k0, a1);
+        a2 = __fmaf_rn(q0.z, k0, a2);
+        a3 = __fmaf_rn(q0.w, k0, a3);
+        a0 = __fmaf_rn(q1.x, k1, a0);
+        a1 = __fmaf_rn(q1.y, k1, a1);
+        a2 = __fmaf_rn(q1.z, k1, a2);
+        a3 = __fmaf_rn(q1.w, k1, a3);
+    }
+    float s = 0.f;
+    s = __fmaf_rn(w.x, a0 > 0.f ? a0 : 0.f, s);
+    s = __fmaf_rn(w.y, a1 > 0.f ? a1 : 0.f, s);
+    s = __fmaf_rn(w.z, a2 > 0.f ? a2 : 0.f, s);
+    s = __fmaf_rn(w.w, a3 > 0.f ? a3 : 0.f, s);
+    return s;
+}
+
 // Load q_idx [4][64] bf16 of one sequence/query into qd[64] (transposed, fp32).
 __device__ __forceinline__ void load_q_idx(const uint16_t* q, float4* qd) {
     for (int d = threadIdx.x; d < kID; d += blockDim.x) {
@@ -123,60 +134,104 @@ __device__ __forceinline__ void read_row(const uint8_t* tile, int r, uint32_t (&
 }
 
 // ----------------------------------------------------------------------------
-// Top-K of the keys[0..nslots) held in shared memory (key 0 = not a candidate):
-// emits pos_of(slot) of the Top-min(topk, valid) slots, ascending by slot, and
-// -1 after them.  Whole block; scratch: hist[4096], list[nslots] (u16), tmp[64].
+// Warp-aggregated shared-memory counters.  Every lane of the warp must call.
 // ----------------------------------------------------------------------------
-template <class PosFn>
-__device__ void select_sorted(const uint32_t* keys, int nslots, int topk, int32_t* __restrict__ out, uint32_t* hist,
-                              uint16_t* list, uint32_t* tmp, PosFn pos_of) {
-    const int tid = threadIdx.x, nt = blockDim.x;
-    for (int i = tid; i < kHistBins; i += nt) hist[i] = 0;
-    if (tid == 0) tmp[48] = 0;
-    __syncthreads();
-    uint32_t nv = 0;
-    for (int i = tid; i < nslots; i += nt) {
-        const uint32_t k = keys[i];
-        if (k) {
-            atomicAdd(&hist[k >> 20], 1u);
-            ++nv;
-        }
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+    const unsigned m = __ballot_sync(0xffffffffu, active);
+    if (active) {
+        const unsigned peers = __match_any_sync(m, bin);
+        if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
-    uint32_t n_valid;
-    block_excl_scan(nv, tmp, &n_valid);  // also orders the histogram writes
-    const uint32_t kk = min((uint32_t)topk, n_valid);
-    if (kk == 0) {
-        for (int i = tid; i < topk; i += nt) out[i] = -1;
+}
+
+__device__ __forceinline__ void list_append(uint16_t* list, uint32_t* cnt, uint32_t v, bool pred) {
+    const unsigned m = __ballot_sync(0xffffffffu, pred);
+    if (m == 0u) return;
+    const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+    uint32_t pos = 0;
+    if (lane == leader) pos = atomicAdd(cnt, (uint32_t)__popc(m));
+    pos = __shfl_sync(0xffffffffu, pos, leader);
+    if (pred) list[pos + __popc(m & ((1u << lane) - 1u))] = (uint16_t)v;
+}
+
+// Copy n32 words global -> shared, 16 B per load (when both pointers allow),
+// many loads in flight.
+__device__ __forceinline__ void load_words(uint32_t* dst, const uint32_t* src, int n32) {
+    const int nt = blockDim.x;
+    if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) {
+        for (int j = threadIdx.x; j < n32; j += nt) dst[j] = __ldcg(src + j);
         return;
     }
-    int b1, d2, d3;
-    uint32_t above;
-    find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
-    uint32_t need = kk - above;
-    for (int i = tid; i < nslots; i += nt) {
-        const uint32_t k = keys[i];
-        if (k && (int)(k >> 20) == b1) list[atomicAdd(&tmp[48], 1u)] = (uint16_t)i;
+    const int n4 = n32 >> 2;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    int i = threadIdx.x;
+    for (; i + 3 * nt < n4; i += 4 * nt) {
+        const uint4 a = __ldcg(s4 + i), b = __ldcg(s4 + i + nt), c = __ldcg(s4 + i + 2 * nt),
+                    d = __ldcg(s4 + i + 3 * nt);
+        d4[i] = a;
+        d4[i + nt] = b;
+        d4[i + 2 * nt] = c;
+        d4[i + 3 * nt] = d;
+    }
+    for (; i < n4; i += nt) d4[i] = __ldcg(s4 + i);
+    for (int j = 4 * n4 + threadIdx.x; j < n32; j += nt) dst[j] = __ldcg(src + j);
+}
+
+// ----------------------------------------------------------------------------
+// Threshold refinement: the first digit b1 (key bits 31..20) holds the kk-th
+// largest key and `need` of its members are still to be taken.  Two 10-bit
+// digits over the shrinking member list give the exact key T; *need_out is
+// then the number of ties at T to take (lowest slots first).  Whole block.
+// ----------------------------------------------------------------------------
+__device__ void refine_threshold(const uint32_t* keys, int nslots, uint32_t b1, uint32_t need, uint32_t* hist,
+                                 uint16_t* list0, uint16_t* list1, uint32_t* tmp, uint32_t* T_out,
+                                 uint32_t* need_out) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) {
+        tmp[48] = 0;
+        tmp[49] = 0;
     }
     for (int i = tid; i < 1024; i += nt) hist[i] = 0;
     __syncthreads();
-    const int nl = (int)tmp[48];
-    for (int i = tid; i < nl; i += nt) atomicAdd(&hist[(keys[list[i]] >> 10) & 1023u], 1u);
+    for (int base = wid * 32; base < nslots; base += nt) {
+        const int i = base + lane;
+        const uint32_t k = i < nslots ? keys[i] : 0u;
+        const bool in = k != 0u && (k >> 20) == b1;
+        list_append(list0, &tmp[48], (uint32_t)i, in);
+        hist_add(hist, (k >> 10) & 1023u, in);
+    }
     __syncthreads();
+    const int n0 = (int)tmp[48];
+    int d2, d3;
+    uint32_t above;
     find_kth_bin(hist, 1024, need, tmp, &d2, &above);
     need -= above;
     for (int i = tid; i < 1024; i += nt) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < nl; i += nt) {
-        const uint32_t k = keys[list[i]];
-        if ((int)((k >> 10) & 1023u) == d2) atomicAdd(&hist[k & 1023u], 1u);
+    for (int base = wid * 32; base < n0; base += nt) {
+        const int i = base + lane;
+        const int slot = i < n0 ? (int)list0[i] : 0;
+        const uint32_t k = i < n0 ? keys[slot] : 0u;
+        const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
+        list_append(list1, &tmp[49], (uint32_t)slot, in);
+        hist_add(hist, k & 1023u, in);
     }
     __syncthreads();
     find_kth_bin(hist, 1024, need, tmp, &d3, &above);
-    need -= above;  // ties at the threshold key still to take, lowest slots first
-    const uint32_t T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+    need -= above;
+    *T_out = (b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+    *need_out = need;
+}
 
-    // ordered emission: warp w owns slots [w*seg, (w+1)*seg), 32 at a time
-    const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+// Ordered emission: warp w owns slots [w*seg, (w+1)*seg), 32 at a time;
+// writes pos_of(slot) of every key > T and of the first `need` keys == T, in
+// slot order, then -1 from kk to topk.  Whole block.
+template <class PosFn>
+__device__ void emit_sorted(const uint32_t* keys, int nslots, uint32_t T, uint32_t need, uint32_t kk, int topk,
+                            int32_t* __restrict__ out, uint32_t* tmp, PosFn pos_of) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+    const unsigned lt = (1u << lane) - 1u;
     const int seg = ((nslots + nw - 1) / nw + 31) & ~31;
     const int lo = wid * seg, hi = min(nslots, lo + seg);
     uint32_t n_gt = 0, n_eq = 0;
@@ -186,24 +241,18 @@ __device__ void select_sorted(const uint32_t* keys, int nslots, int topk, int32_
         n_gt += __popc(__ballot_sync(0xffffffffu, k > T));
         n_eq += __popc(__ballot_sync(0xffffffffu, k == T));
     }
-    // per-warp totals -> exclusive prefixes of ties and of selections
-    uint32_t* wt = tmp;  // [0..nw) ties, [32..32+nw) selections
     __syncthreads();
     if (lane == 0) {
-        wt[wid] = n_eq;
-        wt[32 + wid] = n_gt;
+        tmp[wid] = n_eq;
+        tmp[32 + wid] = n_gt;
     }
     __syncthreads();
     uint32_t tie_base = 0, sel_base = 0;
-    for (int v = 0; v < wid; ++v) tie_base += wt[v];
     for (int v = 0; v < wid; ++v) {
-        const uint32_t ties_v = wt[v];
-        uint32_t tb = 0;
-        for (int u = 0; u < v; ++u) tb += wt[u];
-        const uint32_t take = tb >= need ? 0u : min(ties_v, need - tb);
-        sel_base += wt[32 + v] + take;
+        const uint32_t take = tie_base >= need ? 0u : min(tmp[v], need - tie_base);
+        sel_base += tmp[32 + v] + take;
+        tie_base += tmp[v];
     }
-    const unsigned lt = (1u << lane) - 1u;
     for (int base = lo; base < hi; base += 32) {
         const int i = base + lane;
         const uint32_t k = i < hi ? keys[i] : 0u;
@@ -215,18 +264,57 @@ __device__ void select_sorted(const uint32_t* keys, int nslots, int topk, int32_
         sel_base += __popc(msel);
         tie_base += __popc(meq);
     }
-    for (int i = kk + tid; i < topk; i += nt) out[i] = -1;
+    for (int i = (int)kk + tid; i < topk; i += nt) out[i] = -1;
+}
+
+__device__ __forceinline__ int32_t seq_len_checked(const int32_t* seq_lens, int b, int64_t max_len, int32_t* err) {
+    const int32_t L = seq_lens[b];
+    if (L < 1 || L > max_len) {
+        if (threadIdx.x == 0) dev_error(err, CSA2_DEV_LEN);
+        return 0;
+    }
+    return L;
+}
+
+// Physical page of every page of entries [e0, e1) of one sequence, staged in
+// shared memory once per CTA (-1 where the page table has none).
+__device__ __forceinline__ void stage_pages(const csa2_kv_cache& c, int shift, int seq, int32_t e0, int32_t e1,
+                                            int32_t* pg, int32_t* err) {
+    const int32_t p0 = e0 >> shift, p1 = (e1 - 1) >> shift;
+    for (int32_t p = p0 + threadIdx.x; p <= p1; p += blockDim.x) {
+        int32_t phys = -1;
+        if (p < c.max_pages_per_seq) phys = __ldg(c.page_table + (int64_t)seq * c.max_pages_per_seq + p);
+        if (phys < 0 || phys >= c.n_phys_pages) {
+            dev_error(err, CSA2_DEV_PAGE);
+            phys = -1;
+        }
+        pg[p - p0] = phys;
+    }
 }
 
 // ============================================================================
-// K2: block scores + histogram
+// K2: block scores + first-digit histogram
+//
+// Persistent: one CTA per SM walks a contiguous range of the flattened list of
+// 512-row tiles of every sequence that needs block selection, so a ragged batch
+// balances across the SMs.  A 3-stage ring of 64 KiB tiles is filled by 2-D
+// bulk tensor copies (one box = the pooled rows of one page run, 128B swizzle:
+// chunk c of row r lands at chunk c ^ (r & 7), the layout read_row expects);
+// warp 0 runs two tiles ahead.  Each of the 512 threads scores one row.
 // ============================================================================
-constexpr int K2_THREADS = 256;
-constexpr int K2_ROW = 2 * K2_THREADS;  // rows per round (two per thread)
-constexpr int K2_ROUNDS = 4;
-constexpr int K2_CHUNK = K2_ROW * K2_ROUNDS;  // 2048 blocks per CTA
-constexpr size_t K2_STAGE = (size_t)K2_ROW * 128;
-constexpr size_t K2_SMEM = 2 * K2_STAGE + kHistBins * 4 + kID * 16 + 64 * 4;
+constexpr int K2_THREADS = 512;
+constexpr int K2_TILE = 512;                    // pooled rows per tile (one per thread)
+constexpr int K2_STAGES = 3;
+constexpr size_t K2_STAGE_BYTES = (size_t)K2_TILE * 128;
+constexpr int K2_MAX_SEQS = 1024;
+constexpr size_t K2_OFF_HIST = K2_STAGES * K2_STAGE_BYTES;
+constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
+constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
+constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
+constexpr size_t K2_OFF_BAR = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
+constexpr size_t K2_SMEM = align16(K2_OFF_BAR + K2_STAGES * 8) + 1024;  // + alignment slack for the 1 KiB-aligned ring
+constexpr uint32_t kWaitLimit = 1u << 22;
+static_assert(K2_OFF_BAR % 8 == 0 && K2_OFF_QD % 16 == 0 && K2_OFF_HIST % 1024 == 0, "K2 shared-memory layout");
 
 struct BlockArgs {
     csa2_kv_cache cache;
@@ -237,123 +325,186 @@ struct BlockArgs {
     float* scores;     // [n][nblk_pad]
     uint32_t* hist;    // [n][4096]
     int32_t* thr;      // [n][4]
-    uint32_t* ctr;     // [n][2]
+    uint32_t* ctr;     // [n][2]: tiles scored (K2), chunks filtered (K3)
     uint32_t* bitmap;  // [n][nblk_pad/32]
     uint64_t* bnd;     // [n][nblk_pad]
     uint32_t* bnd_cnt; // [n]
     int32_t* err;
     int64_t nblk_pad;
     int64_t max_len;
-    int keep;
+    int n, keep, page_shift, box_rows;
 };
 
-__device__ __forceinline__ int64_t seq_len_checked(const int32_t* seq_lens, int b, int64_t max_len, int32_t* err) {
-    int64_t L = seq_lens[b];
-    if (L < 1 || L > max_len) {
-        if (threadIdx.x == 0) dev_error(err, CSA2_DEV_LEN);
-        return 0;
+// tile_start[b] = first tile of sequence b; returns the sequence of tile t
+__device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int n, int32_t t) {
+    int lo = 0, hi = n;  // tile_start[lo] <= t < tile_start[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_start[mid] <= t) lo = mid;
+        else hi = mid;
     }
-    return L;
+    return lo;
 }
 
-__device__ __forceinline__ void k2_issue(const BlockArgs& a, int b, int64_t j0, int64_t c1, uint8_t* stage) {
-    // 8 x 16 B per row; copy ci = tid + 256 i covers row ci/8, chunk ci%8
-#pragma unroll
-    for (int i = 0; i < 8 * K2_ROW / K2_THREADS; ++i) {
-        const int ci = threadIdx.x + K2_THREADS * i;
-        const int r = ci >> 3, c = ci & 7;
-        const int64_t j = j0 + r;
-        uint8_t* dst = stage + r * 128 + ((c ^ (r & 7)) << 4);
-        if (j < c1) {
-            const int64_t slot = entry_slot(a.cache, b, j * kBlk, a.err);
-            if (slot >= 0) {
-                cp_async16(dst, a.cache.idx_k_pooled + (slot >> 3) * kID + c * 8);
-                continue;
-            }
-        }
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-    }
-}
-
-__global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* stage = smem;
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + 2 * K2_STAGE);
-    float4* qd = reinterpret_cast<float4*>(hist + kHistBins);
-    uint32_t* tmp = reinterpret_cast<uint32_t*>(qd + kID);
-    __shared__ int s_last;
+__global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                 BlockArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K2_OFF_HIST);
+    float4* qd = reinterpret_cast<float4*>(smem + K2_OFF_QD);
+    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K2_OFF_TMP);
+    int32_t* tile_start = reinterpret_cast<int32_t*>(smem + K2_OFF_TS);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K2_OFF_BAR);
+    __shared__ float4 s_w;
+    __shared__ int s_last, s_timeout;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
     pdl_trigger();
-    const int b = blockIdx.y;
-    const int64_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
-    const int64_t nblk = (L + kBlk - 1) / kBlk;
-    if (nblk <= a.keep) return;
-    const int64_t c0 = (int64_t)blockIdx.x * K2_CHUNK;
-    if (c0 >= nblk) return;
-    const int64_t c1 = min(c0 + K2_CHUNK, nblk);
-    const int nrounds = (int)((c1 - c0 + K2_ROW - 1) / K2_ROW);
-
-    k2_issue(a, b, c0, c1, stage);
-    cp_async_commit();
-    load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
-    const float4 w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
-    for (int i = threadIdx.x; i < kHistBins; i += K2_THREADS) hist[i] = 0;
-    float* scores = a.scores + (int64_t)b * a.nblk_pad;
-
-    for (int r = 0; r < nrounds; ++r) {
-        if (r + 1 < nrounds) {
-            k2_issue(a, b, c0 + (int64_t)(r + 1) * K2_ROW, c1, stage + ((r + 1) & 1) * K2_STAGE);
-            cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    // ---- tiles of every sequence (0 for sequences that keep all blocks) ------
+    {
+        const int per = (a.n + K2_THREADS - 1) / K2_THREADS;
+        uint32_t mine = 0;
+        for (int i = 0; i < per; ++i) {
+            const int b = tid * per + i;
+            if (b < a.n) {
+                const int32_t L = a.seq_lens[b];
+                const int32_t nblk = (L >= 1 && L <= a.max_len) ? (L + kBlk - 1) / kBlk : 0;
+                if (L < 1 || L > a.max_len) dev_error(a.err, CSA2_DEV_LEN);
+                mine += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
+            }
         }
-        __syncthreads();
-        const uint8_t* tile = stage + (r & 1) * K2_STAGE;
-        const int r0 = threadIdx.x, r1 = threadIdx.x + K2_THREADS;
-        const int64_t j0 = c0 + (int64_t)r * K2_ROW + r0, j1 = c0 + (int64_t)r * K2_ROW + r1;
-        uint32_t k[32], m[32];
-        read_row(tile, r0, k);
-        read_row(tile, r1, m);
-        float s0, s1;
-        idx_score2(k, m, qd, w, s0, s1);
-        if (j0 < c1) {
-            scores[j0] = s0;
-            atomicAdd(&hist[score_key(s0) >> 20], 1u);
+        uint32_t total;
+        uint32_t base = block_excl_scan(mine, tmp, &total);
+        for (int i = 0; i < per; ++i) {
+            const int b = tid * per + i;
+            if (b < a.n) {
+                tile_start[b] = (int32_t)base;
+                const int32_t L = a.seq_lens[b];
+                const int32_t nblk = (L >= 1 && L <= a.max_len) ? (L + kBlk - 1) / kBlk : 0;
+                base += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
+            }
         }
-        if (j1 < c1) {
-            scores[j1] = s1;
-            atomicAdd(&hist[score_key(s1) >> 20], 1u);
+        if (tid == 0) tile_start[a.n] = (int32_t)total;
+        if (tid < K2_STAGES) mbar_init(&full[tid], 1);
+        if (tid == 0) {
+            s_timeout = 0;
+            mbar_init_fence();
         }
+        for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
         __syncthreads();
     }
+    const int32_t T = tile_start[a.n];
+    const int32_t t0 = (int32_t)((int64_t)T * blockIdx.x / gridDim.x);
+    const int32_t t1 = (int32_t)((int64_t)T * (blockIdx.x + 1) / gridDim.x);
+    const int ntiles = t1 - t0;
+    if (ntiles <= 0) return;
 
-    uint32_t* gh = a.hist + (int64_t)b * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += K2_THREADS)
-        if (hist[i]) atomicAdd(&gh[i], hist[i]);
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t nch = (uint32_t)((nblk + K2_CHUNK - 1) / K2_CHUNK);
-        s_last = atomicAdd(&a.ctr[2 * b], 1u) == nch - 1;
+    const int sh = a.page_shift, br = a.box_rows;
+    const int32_t emask = (1 << sh) - 1;
+    // warp 0: issue the boxes of tile t into stage s (lane-parallel)
+    auto issue = [&](int32_t t, int s) {
+        const int b = seq_of_tile(tile_start, a.n, t);
+        const int32_t L = a.seq_lens[b];
+        const int32_t nblk = (L + kBlk - 1) / kBlk;
+        const int32_t r0 = (t - tile_start[b]) * K2_TILE, r1 = min(r0 + K2_TILE, nblk);
+        const int nbox = (r1 - r0 + br - 1) / br;
+        uint8_t* stage = smem + (size_t)s * K2_STAGE_BYTES;
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * br * 128));
+        }
+        __syncwarp();
+        for (int x = lane; x < nbox; x += 32) {
+            const int32_t e = (r0 + x * br) * kBlk;  // first entry of the box
+            const int32_t pg = e >> sh;
+            int32_t phys = pg < a.cache.max_pages_per_seq
+                               ? __ldg(a.cache.page_table + (int64_t)b * a.cache.max_pages_per_seq + pg)
+                               : -1;
+            if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                dev_error(a.err, CSA2_DEV_PAGE);
+                phys = 0;  // keep the byte count; results of this call are undefined
+            }
+            const int32_t prow = (int32_t)((((int64_t)phys << sh) | (e & emask)) >> 3);
+            tma_load_2d(stage + (size_t)x * br * 128, &tmap, 0, prow, &full[s]);
+        }
+    };
+    if (wid == 0) {
+        for (int i = 0; i < min(2, ntiles); ++i) issue(t0 + i, i);
     }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int i = threadIdx.x; i < kHistBins; i += K2_THREADS) {
-        hist[i] = __ldcg(&gh[i]);
-        gh[i] = 0;
+
+    int cur_b = -1, nloc = 0;
+    auto flush = [&](int b, int nt) {
+        __syncthreads();
+        uint32_t* gh = a.hist + (int64_t)b * kHistBins;
+        for (int i = tid; i < kHistBins; i += K2_THREADS) {
+            const uint32_t v = hist[i];
+            if (v) atomicAdd(&gh[i], v);
+            hist[i] = 0;
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const int32_t L = a.seq_lens[b];
+            const int32_t nblk = (L + kBlk - 1) / kBlk;
+            const uint32_t need_t = (uint32_t)((nblk + K2_TILE - 1) / K2_TILE);
+            s_last = atomicAdd(&a.ctr[2 * b], (uint32_t)nt) + (uint32_t)nt == need_t;
+        }
+        __syncthreads();
+        if (s_last) {  // the sequence's last tile is done: find the bin of the keep-th score
+            __threadfence();
+            load_words(hist, gh, kHistBins);
+            __syncthreads();
+            for (int i = tid; i < kHistBins / 4; i += K2_THREADS)
+                reinterpret_cast<uint4*>(gh)[i] = make_uint4(0, 0, 0, 0);
+            int bin;
+            uint32_t above;
+            find_kth_bin(hist, kHistBins, (uint32_t)a.keep, tmp, &bin, &above);
+            if (tid == 0) {
+                a.thr[4 * b] = bin;
+                a.thr[4 * b + 1] = (int32_t)above;
+                a.ctr[2 * b] = 0;
+            }
+            for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
+            __syncthreads();
+        }
+    };
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int32_t t = t0 + i;
+        const int s = i % K2_STAGES;
+        if (wid == 0 && i + 2 < ntiles) issue(t + 2, (i + 2) % K2_STAGES);
+        const int b = seq_of_tile(tile_start, a.n, t);
+        if (b != cur_b) {
+            if (cur_b >= 0) flush(cur_b, nloc);
+            load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
+            if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
+            cur_b = b;
+            nloc = 0;
+            __syncthreads();
+        }
+        const int32_t L = a.seq_lens[b];
+        const int32_t nblk = (L + kBlk - 1) / kBlk;
+        const int32_t r0 = (t - tile_start[b]) * K2_TILE;
+        const int32_t j = r0 + tid;
+        if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, kWaitLimit)) s_timeout = 1;
+        uint32_t k[32];
+        read_row(smem + (size_t)s * K2_STAGE_BYTES, tid, k);
+        const float s0 = idx_score1(k, qd, s_w);
+        const bool act = j < nblk;
+        if (act) a.scores[(int64_t)b * a.nblk_pad + j] = s0;
+        hist_add(hist, score_key(s0) >> 20, act);
+        ++nloc;
+        __syncthreads();
+        if (s_timeout) break;
     }
-    __syncthreads();
-    int bin;
-    uint32_t above;
-    find_kth_bin(hist, kHistBins, (uint32_t)a.keep, tmp, &bin, &above);
-    if (threadIdx.x == 0) {
-        a.thr[4 * b] = bin;
-        a.thr[4 * b + 1] = (int32_t)above;
-        a.ctr[2 * b] = 0;
+    if (s_timeout) {
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        // let every copy this CTA issued land before the shared memory goes away
+        for (int i = 0; i < K2_STAGES; ++i) mbar_wait(&full[i], 0u, kWaitLimit);
+        return;
     }
+    if (cur_b >= 0) flush(cur_b, nloc);
 }
 
 // ============================================================================
@@ -361,7 +512,9 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
 // ============================================================================
 constexpr int K3_THREADS = 512;
 constexpr int K3_CHUNK = 8192;
-constexpr size_t K3_SMEM = (size_t)2 * (kMaxBlockLevelLen / kBlk / 32) * 4 + 1024 * 4 + 64 * 4;
+constexpr int K3_WORDS = (int)(kMaxBlockLevelLen / kBlk / 32);  // bitmap words for the largest context
+constexpr int K3_BND_CAP = 12288;                               // boundary entries held in shared memory
+constexpr size_t K3_SMEM = (size_t)2 * K3_WORDS * 4 + 1024 * 4 + 64 * 4 + (size_t)K3_BND_CAP * 8;
 
 __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -369,36 +522,48 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     pdl_wait();
     pdl_trigger();
     const int b = blockIdx.y;
-    const int64_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
-    const int64_t nblk = (L + kBlk - 1) / kBlk;
+    const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
+    const int32_t nblk = (L + kBlk - 1) / kBlk;
     int32_t* out = a.out + (int64_t)b * a.keep;
     if (nblk <= a.keep) {
         if (blockIdx.x == 0)
             for (int i = threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = i < nblk ? i : -1;
         return;
     }
-    const int64_t c0 = (int64_t)blockIdx.x * K3_CHUNK;
+    const int32_t c0 = blockIdx.x * K3_CHUNK;
     if (c0 >= nblk) return;
-    const int64_t c1 = min(c0 + K3_CHUNK, nblk);
+    const int32_t c1 = min(c0 + K3_CHUNK, nblk);
     const uint32_t bstar = (uint32_t)__ldcg(&a.thr[4 * b]);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const float* scores = a.scores + (int64_t)b * a.nblk_pad;
     uint32_t* bitmap = a.bitmap + (int64_t)b * (a.nblk_pad >> 5);
     uint64_t* bnd = a.bnd + (int64_t)b * a.nblk_pad;
-    for (int64_t base = c0 + wid * 32; base < c1; base += K3_THREADS) {
-        const int64_t j = base + lane;
-        const uint32_t key = j < c1 ? score_key(__ldcg(&scores[j])) : 0u;
-        const uint32_t bin = key >> 20;
-        const unsigned mgt = __ballot_sync(0xffffffffu, j < c1 && bin > bstar);
-        const unsigned meq = __ballot_sync(0xffffffffu, j < c1 && bin == bstar);
-        if (lane == 0) bitmap[base >> 5] = mgt;
-        if (meq) {
-            const int leader = __ffs(meq) - 1;
-            uint32_t pos = 0;
-            if (lane == leader) pos = atomicAdd(&a.bnd_cnt[b], (uint32_t)__popc(meq));
-            pos = __shfl_sync(0xffffffffu, pos, leader);
-            if ((meq >> lane) & 1u)
-                bnd[pos + __popc(meq & ((1u << lane) - 1u))] = ((uint64_t)key << 32) | (uint64_t)j;
+    constexpr int U = 4;  // loads in flight per thread
+    for (int32_t base = c0 + wid * 32; base < c1; base += U * K3_THREADS) {
+        float v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int32_t j = base + u * K3_THREADS + lane;
+            v[u] = j < c1 ? __ldcg(&scores[j]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int32_t wbase = base + u * K3_THREADS;
+            if (wbase >= c1) break;
+            const int32_t j = wbase + lane;
+            const uint32_t key = score_key(v[u]);
+            const uint32_t bin = key >> 20;
+            const unsigned mgt = __ballot_sync(0xffffffffu, j < c1 && bin > bstar);
+            const unsigned meq = __ballot_sync(0xffffffffu, j < c1 && bin == bstar);
+            if (lane == 0) bitmap[wbase >> 5] = mgt;
+            if (meq) {
+                const int leader = __ffs(meq) - 1;
+                uint32_t pos = 0;
+                if (lane == leader) pos = atomicAdd(&a.bnd_cnt[b], (uint32_t)__popc(meq));
+                pos = __shfl_sync(0xffffffffu, pos, leader);
+                if ((meq >> lane) & 1u)
+                    bnd[pos + __popc(meq & ((1u << lane) - 1u))] = ((uint64_t)key << 32) | (uint64_t)j;
+            }
         }
     }
     __threadfence();
@@ -412,40 +577,46 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     __threadfence();
 
     // ---- finalize: exact threshold inside the boundary bin -----------------
-    const int nwords = (int)((nblk + 31) >> 5);
+    const int nwords = (nblk + 31) >> 5;
     uint32_t* bm = reinterpret_cast<uint32_t*>(smem);
-    uint32_t* tie = bm + (kMaxBlockLevelLen / kBlk / 32);
-    uint32_t* hist = tie + (kMaxBlockLevelLen / kBlk / 32);
+    uint32_t* tie = bm + K3_WORDS;
+    uint32_t* hist = tie + K3_WORDS;
     uint32_t* tmp = hist + 1024;
+    uint64_t* sbnd = reinterpret_cast<uint64_t*>(tmp + 64);
     const uint32_t n_bnd = __ldcg(&a.bnd_cnt[b]);
+    const uint64_t* B = bnd;
+    if (n_bnd <= (uint32_t)K3_BND_CAP) {  // stage the boundary list (the common case)
+        load_words(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd), 2 * (int)n_bnd);
+        B = sbnd;
+    }
+    load_words(bm, bitmap, nwords);
+    for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
     uint32_t need = (uint32_t)a.keep - (uint32_t)__ldcg(&a.thr[4 * b + 1]);
     int d2, d3;
     uint32_t above;
     for (int i = threadIdx.x; i < 1024; i += K3_THREADS) hist[i] = 0;
     __syncthreads();
-    for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS)
-        atomicAdd(&hist[(uint32_t)(__ldcg(&bnd[i]) >> 42) & 1023u], 1u);
+    for (int base = wid * 32; base < (int)n_bnd; base += K3_THREADS) {
+        const int i = base + lane;
+        const uint32_t key = i < (int)n_bnd ? (uint32_t)(B[i] >> 32) : 0u;
+        hist_add(hist, (key >> 10) & 1023u, i < (int)n_bnd);
+    }
     __syncthreads();
     find_kth_bin(hist, 1024, need, tmp, &d2, &above);
     need -= above;
     for (int i = threadIdx.x; i < 1024; i += K3_THREADS) hist[i] = 0;
     __syncthreads();
-    for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) {
-        const uint32_t key = (uint32_t)(__ldcg(&bnd[i]) >> 32);
-        if ((int)((key >> 10) & 1023u) == d2) atomicAdd(&hist[key & 1023u], 1u);
+    for (int base = wid * 32; base < (int)n_bnd; base += K3_THREADS) {
+        const int i = base + lane;
+        const uint32_t key = i < (int)n_bnd ? (uint32_t)(B[i] >> 32) : 0u;
+        hist_add(hist, key & 1023u, i < (int)n_bnd && (int)((key >> 10) & 1023u) == d2);
     }
     __syncthreads();
     find_kth_bin(hist, 1024, need, tmp, &d3, &above);
     need -= above;
     const uint32_t T = (bstar << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
-
-    for (int i = threadIdx.x; i < nwords; i += K3_THREADS) {
-        bm[i] = __ldcg(&bitmap[i]);
-        tie[i] = 0;
-    }
-    __syncthreads();
     for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) {
-        const uint64_t v = __ldcg(&bnd[i]);
+        const uint64_t v = B[i];
         const uint32_t key = (uint32_t)(v >> 32), j = (uint32_t)v;
         if (key > T) atomicOr(&bm[j >> 5], 1u << (j & 31));
         else if (key == T) atomicOr(&tie[j >> 5], 1u << (j & 31));
@@ -489,14 +660,43 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
 }
 
 // ============================================================================
-// K4: token scores over the candidates + last-CTA Top-K
+// K4: token scores over the candidates + Top-K, one 8-CTA cluster per sequence
+//
+// CTA r of a sequence's cluster scores candidate slots [2048 r, 2048 r + 2048):
+// the indexer-K rows of its 256 candidate blocks (one 1 KiB box each) arrive by
+// 2-D bulk tensor copies into a 2-stage ring; every thread scores one row per
+// round.  The radix select then runs across the cluster: each CTA histograms
+// its own keys, CTA r sums slice r of the histogram over the 8 CTAs through
+// distributed shared memory, every CTA locates the slice and bin holding the
+// K-th key, and the next digit repeats this on the survivors only.  The
+// ordered emission exchanges per-CTA counts the same way, so every CTA writes
+// its selected positions at its own offset, ascending.
 // ============================================================================
-constexpr int K4_THREADS = 512;
-constexpr int K4_CHUNK = 1024;  // candidate slots per CTA (two rounds of 512)
-constexpr size_t K4_STAGE = (size_t)K4_THREADS * 128;
-constexpr size_t K4_SMEM_SCORE = 2 * K4_STAGE + kID * 16;
-constexpr size_t K4_SMEM_SELECT = (size_t)kMaxCand * 4 + kHistBins * 4 + kMaxCand * 2 + 64 * 4;
-constexpr size_t K4_SMEM = K4_SMEM_SCORE > K4_SMEM_SELECT ? K4_SMEM_SCORE : K4_SMEM_SELECT;
+constexpr int TK_CL = 8;
+constexpr int TK_THREADS = 512;
+constexpr int TK_SLOTS = kMaxCand / TK_CL;  // 2048 candidate slots per CTA
+constexpr int TK_ROUND = TK_THREADS;        // rows per round
+constexpr int TK_BLKS = TK_SLOTS / kBlk;    // 256 candidate blocks per CTA
+constexpr size_t TK_STAGE_BYTES = (size_t)TK_ROUND * 128;
+constexpr size_t TK_OFF_KEYS = 2 * TK_STAGE_BYTES;
+constexpr size_t TK_OFF_HIST = align16(TK_OFF_KEYS + TK_SLOTS * 4);
+constexpr size_t TK_OFF_SLICE = align16(TK_OFF_HIST + kHistBins * 4);        // this CTA's reduced slice
+constexpr size_t TK_OFF_L0 = align16(TK_OFF_SLICE + (kHistBins / TK_CL) * 4);
+constexpr size_t TK_OFF_L1 = align16(TK_OFF_L0 + TK_SLOTS * 2);
+constexpr size_t TK_OFF_BSLOT = align16(TK_OFF_L1 + TK_SLOTS * 2);
+constexpr size_t TK_OFF_BPOS = align16(TK_OFF_BSLOT + TK_BLKS * 8);
+constexpr size_t TK_OFF_QD = align16(TK_OFF_BPOS + TK_BLKS * 4);
+constexpr size_t TK_OFF_TMP = align16(TK_OFF_QD + kID * 16);
+constexpr size_t TK_OFF_X = align16(TK_OFF_TMP + (64 + kHistBins / TK_CL) * 4);  // exchanged words
+constexpr size_t TK_OFF_BAR = align16(TK_OFF_X + 16 * 4);
+constexpr size_t TK_SMEM = align16(TK_OFF_BAR + 2 * 8) + 1024;
+static_assert(TK_OFF_BAR % 8 == 0 && TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0, "K4 shared-memory layout");
+
+// The earlier (non-cluster) layout constants are still used by the prefill select.
+constexpr size_t K4_OFF_HIST = (size_t)kMaxCand * 4;
+constexpr size_t K4_OFF_L0 = K4_OFF_HIST + kHistBins * 4;
+constexpr size_t K4_OFF_L1 = K4_OFF_L0 + (size_t)kMaxCand * 2;
+constexpr size_t K4_OFF_CB = K4_OFF_L1 + (size_t)kMaxCand * 2;
 
 struct TokenArgs {
     csa2_kv_cache cache;
@@ -505,102 +705,250 @@ struct TokenArgs {
     const int32_t* seq_lens;
     const int32_t* cand;  // [n][keep] or null (flat)
     int32_t* out;         // [n][topk]
-    uint32_t* keys;       // [n][kMaxCand]
-    uint32_t* ctr;        // [n]
     int32_t* err;
     int64_t max_len;
-    int keep, topk;
+    int keep, topk, page_shift;
 };
 
-// position of candidate slot i, or -1 if the slot is empty
-__device__ __forceinline__ int64_t cand_pos(const TokenArgs& a, int b, int i, int64_t L) {
-    int64_t blk = i >> 3;
-    if (a.cand) {
-        blk = __ldg(a.cand + (int64_t)b * a.keep + (i >> 3));
-        if (blk < 0) return -1;
-    }
-    const int64_t p = blk * kBlk + (i & 7);
-    return p < L ? p : -1;
-}
-
-__device__ __forceinline__ void k4_issue(const TokenArgs& a, int b, int i0, int nslots, int64_t L, uint8_t* stage) {
+// Cluster-wide "which bin holds the need-th largest" over a histogram of
+// nbins bins split across the 8 CTAs (each CTA holds a full local histogram).
+// Returns the bin and the count of items in higher bins.  Whole CTA, all 8 CTAs.
+__device__ void cluster_kth_bin(cg::cluster_group& cl, const uint32_t* hist, int nbins, uint32_t need, uint32_t* slice,
+                                uint32_t* xw, uint32_t* tmp, int* bin_out, uint32_t* above_out) {
+    const int r = (int)cl.block_rank(), per = nbins / TK_CL;
+    cl.sync();  // local histograms complete
+    uint32_t tot = 0;
+    for (int i = threadIdx.x; i < per; i += blockDim.x) {
+        uint32_t v = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int ci = threadIdx.x + K4_THREADS * i;
-        const int r = ci >> 3, c = ci & 7;
-        uint8_t* dst = stage + r * 128 + ((c ^ (r & 7)) << 4);
-        const int slot_i = i0 + r;
-        if (slot_i < nslots) {
-            const int64_t p = cand_pos(a, b, slot_i, L);
-            if (p >= 0) {
-                const int64_t slot = entry_slot(a.cache, b, p, a.err);
-                if (slot >= 0) {
-                    cp_async16(dst, a.cache.idx_k + slot * kID + c * 8);
-                    continue;
-                }
-            }
-        }
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < TK_CL; ++c) v += *cl.map_shared_rank(hist + r * per + i, c);
+        slice[i] = v;
+        tot += v;
     }
+    uint32_t sum;
+    block_excl_scan(tot, tmp, &sum);
+    if (threadIdx.x == 0) xw[0] = sum;
+    cl.sync();  // slices and their totals complete
+    // slices from the top: slice TK_CL-1 holds the highest bins
+    uint32_t above = 0;
+    int sstar = 0;
+    for (int c = TK_CL - 1; c >= 0; --c) {
+        const uint32_t t = *cl.map_shared_rank(xw, c);
+        if (above + t >= need) {
+            sstar = c;
+            break;
+        }
+        above += t;
+    }
+    const uint32_t* src = cl.map_shared_rank(slice, sstar);
+    for (int i = threadIdx.x; i < per; i += blockDim.x) tmp[64 + i] = src[i];  // tmp has room for a 512-bin slice
+    __syncthreads();
+    int b;
+    uint32_t ab;
+    find_kth_bin(tmp + 64, per, need - above, tmp, &b, &ab);
+    *bin_out = sstar * per + b;
+    *above_out = above + ab;
 }
 
-__global__ void __launch_bounds__(K4_THREADS) token_topk_kernel(TokenArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_last;
+__global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
+    token_topk_kernel(const __grid_constant__ CUtensorMap tmap, TokenArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + TK_OFF_KEYS);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);
+    uint32_t* slice = reinterpret_cast<uint32_t*>(smem + TK_OFF_SLICE);
+    uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L0);
+    uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L1);
+    int64_t* bslot = reinterpret_cast<int64_t*>(smem + TK_OFF_BSLOT);
+    int32_t* bpos = reinterpret_cast<int32_t*>(smem + TK_OFF_BPOS);
+    float4* qd = reinterpret_cast<float4*>(smem + TK_OFF_QD);
+    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
+    uint32_t* xw = reinterpret_cast<uint32_t*>(smem + TK_OFF_X);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + TK_OFF_BAR);
+    __shared__ float4 s_w;
+    __shared__ int s_timeout;
+    cg::cluster_group cl = cg::this_cluster();
+    const int r = (int)cl.block_rank();
+    const int b = blockIdx.x / TK_CL;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+
     pdl_wait();
     pdl_trigger();
-    const int b = blockIdx.y;
-    int64_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
-    int nslots = a.cand ? a.keep * kBlk : (int)(L < (int64_t)a.keep * kBlk ? L : (int64_t)a.keep * kBlk);
-    if (!a.cand && L > (int64_t)a.keep * kBlk) {
-        if (threadIdx.x == 0) dev_error(a.err, CSA2_DEV_LEN);
-    }
-    const int nch = (nslots + K4_CHUNK - 1) / K4_CHUNK;
-    if (L == 0 || nch == 0) {
-        if (blockIdx.x == 0)
-            for (int i = threadIdx.x; i < a.topk; i += K4_THREADS) a.out[(int64_t)b * a.topk + i] = -1;
-        return;
-    }
-    const int i0 = blockIdx.x * K4_CHUNK;
-    if (i0 >= nslots) return;
+    const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
+    const int32_t cap = a.keep * kBlk;
+    const int nslots = a.cand ? cap : min(L, cap);
+    if (!a.cand && L > cap && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_LEN);
+    const int s0 = r * TK_SLOTS, s1 = max(s0, min(s0 + TK_SLOTS, nslots));
 
-    uint8_t* stage = smem;
-    float4* qd = reinterpret_cast<float4*>(smem + 2 * K4_STAGE);
-    k4_issue(a, b, i0, nslots, L, stage);
-    cp_async_commit();
-    k4_issue(a, b, i0 + K4_THREADS, nslots, L, stage + K4_STAGE);
-    cp_async_commit();
+    // candidate blocks of this CTA: first position and first slot
+    for (int k = tid; k < TK_BLKS; k += TK_THREADS) {
+        const int i = s0 + k * kBlk;
+        int32_t p = -1;
+        int64_t sl = -1;
+        if (i < s1) {
+            const int32_t blk = a.cand ? __ldg(a.cand + (int64_t)b * a.keep + (i >> 3)) : (i >> 3);
+            if (blk >= 0 && blk * kBlk < L) {
+                p = blk * kBlk;
+                sl = entry_slot(a.cache, a.page_shift, b, p, a.err);
+            }
+        }
+        bpos[k] = sl >= 0 ? p : -1;
+        bslot[k] = sl;
+    }
     load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
-    const float4 w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
-    uint32_t* keys = a.keys + (int64_t)b * kMaxCand;
-    cp_async_wait<0>();
-    __syncthreads();
-    {
-        uint32_t k[32], m[32];
-        read_row(stage, threadIdx.x, k);
-        read_row(stage + K4_STAGE, threadIdx.x, m);
-        float s0, s1;
-        idx_score2(k, m, qd, w, s0, s1);
-        const int sa = i0 + threadIdx.x, sb = i0 + K4_THREADS + threadIdx.x;
-        if (sa < nslots) keys[sa] = cand_pos(a, b, sa, L) >= 0 ? score_key(s0) : 0u;
-        if (sb < nslots) keys[sb] = cand_pos(a, b, sb, L) >= 0 ? score_key(s1) : 0u;
+    if (tid == 0) {
+        s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
+        s_timeout = 0;
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init_fence();
     }
-    __threadfence();
+    for (int i = tid; i < kHistBins; i += TK_THREADS) hist[i] = 0;
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&a.ctr[b], 1u) == (uint32_t)nch - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
 
-    uint32_t* skeys = reinterpret_cast<uint32_t*>(smem);
-    uint32_t* hist = skeys + kMaxCand;
-    uint16_t* list = reinterpret_cast<uint16_t*>(hist + kHistBins);
-    uint32_t* tmp = reinterpret_cast<uint32_t*>(list + kMaxCand);
-    for (int i = threadIdx.x; i < nslots; i += K4_THREADS) skeys[i] = __ldcg(&keys[i]);
+    const int nrounds = (s1 - s0 + TK_ROUND - 1) / TK_ROUND;
+    auto issue = [&](int k) {  // warp 0: round k into stage k & 1
+        const int st = k & 1;
+        uint8_t* stage = smem + (size_t)st * TK_STAGE_BYTES;
+        uint32_t nvalid = 0;
+        for (int x = lane; x < TK_ROUND / kBlk; x += 32) nvalid += bslot[k * (TK_ROUND / kBlk) + x] >= 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&full[st], nvalid * kBlk * 128);
+        }
+        __syncwarp();
+        for (int x = lane; x < TK_ROUND / kBlk; x += 32) {
+            const int64_t sl = bslot[k * (TK_ROUND / kBlk) + x];
+            if (sl >= 0) tma_load_2d(stage + (size_t)x * kBlk * 128, &tmap, 0, (int32_t)sl, &full[st]);
+        }
+    };
+    if (wid == 0) {
+        for (int k = 0; k < min(2, nrounds); ++k) issue(k);
+    }
+    for (int k = 0; k < nrounds; ++k) {
+        const int st = k & 1;
+        if (!mbar_wait(&full[st], (uint32_t)(k >> 1) & 1u, kWaitLimit)) s_timeout = 1;
+        const int blk = k * (TK_ROUND / kBlk) + (tid >> 3), e = tid & 7;
+        const bool valid = s0 + k * TK_ROUND + tid < s1 && bpos[blk] >= 0 && bpos[blk] + e < L;
+        uint32_t key = 0u;
+        if (valid) {
+            uint32_t kr[32];
+            read_row(smem + (size_t)st * TK_STAGE_BYTES, tid, kr);
+            key = score_key(idx_score1(kr, qd, s_w));
+        }
+        keys[k * TK_ROUND + tid] = key;
+        hist_add(hist, key >> 20, key != 0u);
+        __syncthreads();
+        if (wid == 0 && k + 2 < nrounds) issue(k + 2);
+    }
+    for (int i = nrounds * TK_ROUND + tid; i < TK_SLOTS; i += TK_THREADS) keys[i] = 0u;
+    if (s_timeout && tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+
+    // ---- cluster radix select ---------------------------------------------
+    uint32_t nv = 0;
+    for (int i = tid; i < kHistBins; i += TK_THREADS) nv += hist[i];
+    uint32_t mine_valid;
+    block_excl_scan(nv, tmp, &mine_valid);
+    if (tid == 0) xw[1] = mine_valid;
+    cl.sync();
+    uint32_t n_valid = 0;
+#pragma unroll
+    for (int c = 0; c < TK_CL; ++c) n_valid += *cl.map_shared_rank(xw + 1, c);
+    const uint32_t kk = min((uint32_t)a.topk, n_valid);
+    int32_t* out = a.out + (int64_t)b * a.topk;
+    uint32_t T = 0xffffffffu, need = 0;
+    if (kk > 0) {  // uniform across the cluster
+        int b1, d2, d3;
+        uint32_t above;
+        cluster_kth_bin(cl, hist, kHistBins, kk, slice, xw, tmp, &b1, &above);
+        need = kk - above;
+        // survivors of digit 1, histogram of digit 2 (bits 19..10)
+        if (tid == 0) {
+            xw[2] = 0;
+            xw[3] = 0;
+        }
+        for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int base = wid * 32; base < TK_SLOTS; base += TK_THREADS) {
+            const int i = base + lane;
+            const uint32_t k = keys[i];
+            const bool in = k != 0u && (int)(k >> 20) == b1;
+            list_append(l0, &xw[2], (uint32_t)i, in);
+            hist_add(hist, (k >> 10) & 1023u, in);
+        }
+        __syncthreads();
+        cluster_kth_bin(cl, hist, 1024, need, slice, xw + 4, tmp, &d2, &above);
+        need -= above;
+        const int n0 = (int)xw[2];
+        for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int base = wid * 32; base < n0; base += TK_THREADS) {
+            const int i = base + lane;
+            const int slot = i < n0 ? (int)l0[i] : 0;
+            const uint32_t k = i < n0 ? keys[slot] : 0u;
+            const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
+            list_append(l1, &xw[3], (uint32_t)slot, in);
+            hist_add(hist, k & 1023u, in);
+        }
+        __syncthreads();
+        cluster_kth_bin(cl, hist, 1024, need, slice, xw + 6, tmp, &d3, &above);
+        need -= above;
+        T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+    }
+
+    // ---- ordered emission: counts per CTA, then each CTA writes at its offset
+    const unsigned lt = (1u << lane) - 1u;
+    constexpr int SEG = TK_SLOTS / (TK_THREADS / 32);  // 128 slots per warp
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int base = wid * SEG; base < wid * SEG + SEG; base += 32) {
+        const uint32_t k = keys[base + lane];
+        n_gt += __popc(__ballot_sync(0xffffffffu, k > T && T != 0xffffffffu));
+        n_eq += __popc(__ballot_sync(0xffffffffu, k == T));
+    }
     __syncthreads();
-    select_sorted(skeys, nslots, a.topk, a.out + (int64_t)b * a.topk, hist, list, tmp,
-                  [&](int i) { return (int32_t)cand_pos(a, b, i, L); });
-    if (threadIdx.x == 0) a.ctr[b] = 0;
+    if (lane == 0) {
+        tmp[wid] = n_eq;
+        tmp[32 + wid] = n_gt;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t e = 0, g = 0;
+        for (int v = 0; v < TK_THREADS / 32; ++v) {
+            e += tmp[v];
+            g += tmp[32 + v];
+        }
+        xw[8] = e;
+        xw[9] = g;
+    }
+    cl.sync();
+    uint32_t tie_base = 0, sel_base = 0;
+    for (int c = 0; c < r; ++c) {
+        const uint32_t e = *cl.map_shared_rank(xw + 8, c), g = *cl.map_shared_rank(xw + 9, c);
+        const uint32_t take = tie_base >= need ? 0u : min(e, need - tie_base);
+        sel_base += g + take;
+        tie_base += e;
+    }
+    for (int v = 0; v < wid; ++v) {
+        const uint32_t take = tie_base >= need ? 0u : min(tmp[v], need - tie_base);
+        sel_base += tmp[32 + v] + take;
+        tie_base += tmp[v];
+    }
+    for (int base = wid * SEG; base < wid * SEG + SEG; base += 32) {
+        const int i = base + lane;
+        const uint32_t k = keys[i];
+        const unsigned meq = __ballot_sync(0xffffffffu, k == T);
+        const uint32_t rank = tie_base + __popc(meq & lt);
+        const bool sel = (k > T && T != 0xffffffffu) || (k == T && rank < need);
+        const unsigned msel = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[sel_base + __popc(msel & lt)] = bpos[i >> 3] + (i & 7);
+        sel_base += __popc(msel);
+        tie_base += __popc(meq);
+    }
+    if (r == 0)
+        for (int i = (int)kk + tid; i < a.topk; i += TK_THREADS) out[i] = -1;
+    cl.sync();  // peers may still read this CTA's shared memory
 }
 
 // ============================================================================
@@ -618,18 +966,18 @@ struct PrefillArgs {
     uint32_t* keys;  // [T][stride]
     int32_t* err;
     int64_t stride;
-    int T, ratio, topk, n_entries;
+    int T, ratio, topk, n_entries, page_shift;
 };
 
 __device__ __forceinline__ int visible(int p, int ratio, int n) { return min((p + 1) / ratio, n); }
 
-// Thread (qi, ei) of a 16 x 16 grid computes queries 2qi, 2qi+1 against entries
-// 4ei .. 4ei+3 of the tile: 32 sequential fp32 FMA chains.
 constexpr size_t PS_SMEM = (size_t)kID * PS_E * 4 + (size_t)kID * PS_Q * kIH * 4;
 
+// Thread (qi, ei) of a 16 x 16 grid computes queries 2qi, 2qi+1 against entries
+// 4ei .. 4ei+3 of the tile: 32 sequential fp32 FMA chains.
 __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    float (*kt)[PS_E] = reinterpret_cast<float (*)[PS_E]>(smem);                               // [d][entry]
+    float (*kt)[PS_E] = reinterpret_cast<float (*)[PS_E]>(smem);                                      // [d][entry]
     float (*qs)[PS_Q][kIH] = reinterpret_cast<float (*)[PS_Q][kIH]>(smem + (size_t)kID * PS_E * 4);  // [d][q][h]
     __shared__ float ws_[PS_Q][kIH];
     __shared__ int vis[PS_Q];
@@ -661,7 +1009,7 @@ __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a
                 const int e = e0 + r;
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (e < max_vis) {
-                    const int64_t slot = entry_slot(a.cache, 0, e, a.err);
+                    const int64_t slot = entry_slot(a.cache, a.page_shift, 0, e, a.err);
                     if (slot >= 0) v = __ldg(reinterpret_cast<const uint4*>(a.cache.idx_k + slot * kID) + c);
                 }
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -725,7 +1073,7 @@ __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a
 }
 
 constexpr int PSEL_THREADS = 512;
-constexpr size_t PSEL_SMEM = K4_SMEM_SELECT;
+constexpr size_t PSEL_SMEM = K4_OFF_CB + 64 * 4;  // keys | hist | list0 | list1 | tmp
 
 __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -734,13 +1082,34 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
     const int t = blockIdx.x;
     const int n = (int)a.stride;
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem);
-    uint32_t* hist = skeys + kMaxCand;
-    uint16_t* list = reinterpret_cast<uint16_t*>(hist + kHistBins);
-    uint32_t* tmp = reinterpret_cast<uint32_t*>(list + kMaxCand);
-    const uint4* src = reinterpret_cast<const uint4*>(a.keys + (int64_t)t * a.stride);
-    for (int i = threadIdx.x; i < n / 4; i += PSEL_THREADS) reinterpret_cast<uint4*>(skeys)[i] = __ldcs(src + i);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K4_OFF_HIST);
+    uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + K4_OFF_L0);
+    uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + K4_OFF_L1);
+    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K4_OFF_CB);
+    for (int i = threadIdx.x; i < kHistBins; i += PSEL_THREADS) hist[i] = 0;
+    load_words(skeys, a.keys + (int64_t)t * a.stride, n);
     __syncthreads();
-    select_sorted(skeys, n, a.topk, a.out + (int64_t)t * a.topk, hist, list, tmp, [](int i) { return (int32_t)i; });
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint32_t nv = 0;
+    for (int base = wid * 32; base < n; base += PSEL_THREADS) {
+        const int i = base + lane;
+        const uint32_t k = i < n ? skeys[i] : 0u;
+        nv += k != 0u;
+        hist_add(hist, k >> 20, k != 0u);
+    }
+    uint32_t n_valid;
+    block_excl_scan(nv, tmp, &n_valid);
+    const uint32_t kk = min((uint32_t)a.topk, n_valid);
+    int32_t* out = a.out + (int64_t)t * a.topk;
+    if (kk == 0) {
+        for (int i = threadIdx.x; i < a.topk; i += PSEL_THREADS) out[i] = -1;
+        return;
+    }
+    int b1;
+    uint32_t above, T, need;
+    find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
+    refine_threshold(skeys, n, (uint32_t)b1, kk - above, hist, l0, l1, tmp, &T, &need);
+    emit_sorted(skeys, n, T, need, kk, a.topk, out, tmp, [](int i) { return (int32_t)i; });
 }
 
 // ============================================================================
@@ -760,6 +1129,7 @@ DecodeWs decode_ws_layout(int n, int64_t max_len) {
     l.blk_ctr = o; o = align256(o + (size_t)n * 8);
     l.blk_bnd_cnt = o; o = align256(o + (size_t)n * 4);
     l.tok_ctr = o; o = align256(o + (size_t)n * 4);
+    l.tok_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_thr = o; o = align256(o + (size_t)n * 16);
     l.tok_keys = o; o = align256(o + (size_t)n * kMaxCand * 4);
     if (nblk > kMaxKeep) {
@@ -779,20 +1149,53 @@ PrefillWs prefill_ws_layout(int T, int64_t n_entries) {
     return l;
 }
 
-static cudaError_t set_smem(const void* fn, size_t bytes) {
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+// Dynamic shared-memory opt-in, once per device.
+static cudaError_t ensure_smem(const void* fn, size_t bytes, bool* done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    return cudaSuccess;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+static int sm_count() {
+    static int n[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        n[dev] = v;
+    }
+    return n[dev];
 }
 
 cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, int keep, int32_t* out, int n, int64_t max_len, char* ws,
                               int32_t* err, cudaStream_t stream) {
-    static bool init = false;
-    if (!init) {
-        cudaError_t e = set_smem((const void*)block_score_kernel, K2_SMEM);
-        if (e == cudaSuccess) e = set_smem((const void*)block_select_kernel, K3_SMEM);
-        if (e != cudaSuccess) return e;
-        init = true;
-    }
+    static bool d2[64], d3[64];
+    cudaError_t e = ensure_smem((const void*)block_score_kernel, K2_SMEM, d2);
+    if (e == cudaSuccess) e = ensure_smem((const void*)block_select_kernel, K3_SMEM, d3);
+    if (e != cudaSuccess) return e;
+    if (n > K2_MAX_SEQS) return cudaErrorInvalidValue;
     const DecodeWs l = decode_ws_layout(n, max_len);
     BlockArgs a{};
     a.cache = cache;
@@ -810,11 +1213,29 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.err = err;
     a.nblk_pad = l.nblk_pad;
     a.max_len = max_len;
+    a.n = n;
     a.keep = keep;
+    a.page_shift = page_shift_of(cache);
+    a.box_rows = min(8, cache.page_size / kBlk);
     const int64_t nblk = (max_len + kBlk - 1) / kBlk;
-    LaunchCfg c2(dim3((unsigned)((nblk + K2_CHUNK - 1) / K2_CHUNK), n), dim3(K2_THREADS), K2_SMEM, stream);
-    cudaError_t e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, a);
-    if (e != cudaSuccess) return e;
+    if (nblk > keep) {
+        PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+        if (!enc) return cudaErrorNotSupported;
+        CUtensorMap map;
+        const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size / kBlk)};
+        const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kID, (cuuint32_t)a.box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k_pooled, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        const int64_t tiles = (int64_t)n * ((nblk + K2_TILE - 1) / K2_TILE);
+        const int grid = (int)std::min<int64_t>(tiles, sm_count());
+        LaunchCfg c2(dim3((unsigned)grid), dim3(K2_THREADS), K2_SMEM, stream);
+        e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, map, a);
+        if (e != cudaSuccess) return e;
+    }
     LaunchCfg c3(dim3((unsigned)((nblk + K3_CHUNK - 1) / K3_CHUNK), n), dim3(K3_THREADS), K3_SMEM, stream);
     return cudaLaunchKernelEx(&c3.cfg, block_select_kernel, a);
 }
@@ -822,13 +1243,21 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
 cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,
                               int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream) {
-    static bool init = false;
-    if (!init) {
-        cudaError_t e = set_smem((const void*)token_topk_kernel, K4_SMEM);
-        if (e != cudaSuccess) return e;
-        init = true;
-    }
-    const DecodeWs l = decode_ws_layout(n, max_len);
+    static bool d4[64];
+    cudaError_t e = ensure_smem((const void*)token_topk_kernel, TK_SMEM, d4);
+    if (e != cudaSuccess) return e;
+    (void)ws;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size)};
+    const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kID, (cuuint32_t)kBlk};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
     TokenArgs a{};
     a.cache = cache;
     a.q_idx = q_idx;
@@ -836,27 +1265,22 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.seq_lens = seq_lens;
     a.cand = cand_blocks;
     a.out = out;
-    a.keys = reinterpret_cast<uint32_t*>(ws + l.tok_keys);
-    a.ctr = reinterpret_cast<uint32_t*>(ws + l.tok_ctr);
     a.err = err;
     a.max_len = max_len;
     a.keep = keep;
     a.topk = topk;
-    const int nslots_max = keep * kBlk;
-    LaunchCfg c(dim3((unsigned)((nslots_max + K4_CHUNK - 1) / K4_CHUNK), n), dim3(K4_THREADS), K4_SMEM, stream);
-    return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, a);
+    a.page_shift = page_shift_of(cache);
+    LaunchCfg c(dim3((unsigned)n * TK_CL), dim3(TK_THREADS), TK_SMEM, stream);
+    return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, map, a);
 }
 
 cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                                 const int32_t* seq_lens, const int32_t* q_pos, int ratio, int topk, int32_t* out,
                                 int T, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream) {
-    static bool init = false;
-    if (!init) {
-        cudaError_t e = set_smem((const void*)prefill_select_kernel, PSEL_SMEM);
-        if (e == cudaSuccess) e = set_smem((const void*)prefill_score_kernel, PS_SMEM);
-        if (e != cudaSuccess) return e;
-        init = true;
-    }
+    static bool d1[64], d2[64];
+    cudaError_t e = ensure_smem((const void*)prefill_select_kernel, PSEL_SMEM, d1);
+    if (e == cudaSuccess) e = ensure_smem((const void*)prefill_score_kernel, PS_SMEM, d2);
+    if (e != cudaSuccess) return e;
     (void)seq_lens;
     const PrefillWs l = prefill_ws_layout(T, max_len);
     PrefillArgs a{};
@@ -872,8 +1296,9 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     a.ratio = ratio;
     a.topk = topk;
     a.n_entries = (int)max_len;
+    a.page_shift = page_shift_of(cache);
     LaunchCfg c1(dim3((unsigned)((T + PS_Q - 1) / PS_Q)), dim3(PS_THREADS), PS_SMEM, stream);
-    cudaError_t e = cudaLaunchKernelEx(&c1.cfg, prefill_score_kernel, a);
+    e = cudaLaunchKernelEx(&c1.cfg, prefill_score_kernel, a);
     if (e != cudaSuccess) return e;
     LaunchCfg c2(dim3((unsigned)T), dim3(PSEL_THREADS), PSEL_SMEM, stream);
     return cudaLaunchKernelEx(&c2.cfg, prefill_select_kernel, a);

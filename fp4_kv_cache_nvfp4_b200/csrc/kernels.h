@@ -9,6 +9,13 @@
 
 namespace csa2 {
 
+// log2 of a power-of-two page size (validated by the ABI layer)
+inline int page_shift_of(const csa2_kv_cache& c) {
+    int s = 0;
+    while ((1 << s) < c.page_size) ++s;
+    return s;
+}
+
 // Launch configuration with programmatic dependent launch enabled, and an
 // optional thread-block cluster.
 struct LaunchCfg {
@@ -38,7 +45,7 @@ struct LaunchCfg {
 // Workspace layout of the decode indexer (byte offsets; all 256-aligned).
 struct DecodeWs {
     size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt;
-    size_t tok_keys, tok_ctr;
+    size_t tok_keys, tok_ctr, tok_hist;
     size_t total;
     int64_t nblk_pad;  // per-sequence stride of block arrays
 };
@@ -79,6 +86,8 @@ struct AttnArgs {
     float* lse;
     int32_t* err;
     int rows, topk, window, swa_start, seq_len_prefill;
+    int page_shift;
+    int early;  // 1: index set, cache and SWA history may be read before the preceding kernel completes
 };
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
 

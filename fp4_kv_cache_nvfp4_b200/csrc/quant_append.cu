@@ -96,17 +96,30 @@ __global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
     if (!last_in_block) return;
     const int64_t s0 = slot & ~int64_t(7);
     const int cnt = int(slot - s0) + 1;
+    // all slot-mapping probes, then all row loads, issued together (two round trips)
+    int64_t probe[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int64_t er = e - (slot - (s0 + r));
+        probe[r] = (r < cnt && er >= 0) ? __ldg(a.slot_mapping + er) : -1;
+    }
+    uint32_t wr[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int64_t sr = s0 + r, er = e - (slot - sr);
+        wr[r] = 0u;
+        if (r < cnt) {
+            if (probe[r] == sr) wr[r] = __ldg(reinterpret_cast<const uint32_t*>(a.idx_src + er * kID) + lane);
+            else wr[r] = reinterpret_cast<const uint32_t*>(a.cache.idx_k + sr * kID)[lane];
+        }
+    }
     float acc0 = 0.f, acc1 = 0.f;
-    for (int r = 0; r < cnt; ++r) {
-        const int64_t sr = s0 + r;
-        const int64_t er = e - (slot - sr);
-        uint32_t w;
-        if (er >= 0 && a.slot_mapping[er] == sr)
-            w = __ldg(reinterpret_cast<const uint32_t*>(a.idx_src + er * kID) + lane);
-        else
-            w = reinterpret_cast<const uint32_t*>(a.cache.idx_k + sr * kID)[lane];
-        acc0 = __fadd_rn(acc0, bf16_lo(w));
-        acc1 = __fadd_rn(acc1, bf16_hi(w));
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        if (r < cnt) {
+            acc0 = __fadd_rn(acc0, bf16_lo(wr[r]));
+            acc1 = __fadd_rn(acc1, bf16_hi(wr[r]));
+        }
     }
     const float fc = (float)cnt;
     const __nv_bfloat16 m0 = __float2bfloat16_rn(__fdiv_rn(acc0, fc));

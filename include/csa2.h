@@ -67,6 +67,7 @@ typedef enum {
 #define CSA2_DEV_PAGE 0x2   /* page-table entry missing or outside the cache */
 #define CSA2_DEV_INDEX 0x4  /* a Top-K index >= the sequence length */
 #define CSA2_DEV_LEN 0x8    /* a sequence length outside [1, capacity] */
+#define CSA2_DEV_TIMEOUT 0x10 /* a bounded wait for an asynchronous copy gave up */
 
 typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
 typedef enum { CSA2_LEVEL_BLOCK = 0, CSA2_LEVEL_TOKEN = 1 } csa2_level;
@@ -95,9 +96,9 @@ typedef struct {
  *   idx_k        [n_slots][64]  bf16: indexer K of each entry
  *   idx_k_pooled [n_slots/8][64] bf16: mean of the rows present in each
  *                block of 8 (slot / 8); NULL if no hierarchical indexer is used
- * n_slots = n_phys_pages * page_size; page_size is a multiple of 8; every
- * array base is 16-byte aligned; page_table is [n_seqs][max_pages_per_seq]
- * int32 with -1 for unused pages. */
+ * n_slots = n_phys_pages * page_size; page_size is a power of two >= 8;
+ * every array base is 16-byte aligned; page_table is [n_seqs][max_pages_per_seq]
+ * int32 with -1 for unused pages; max_pages_per_seq * page_size <= 2^31. */
 typedef struct {
     uint8_t* codes;
     uint8_t* scales;
@@ -149,7 +150,7 @@ CSA2_API csa2_status csa2_kv_quant_append(const csa2_kv_cache* cache, const void
  * padded with -1.  The mode must be Full or Reindex (Reuse: INVALID_ARG).
  *
  * Decode (q_pos == NULL): n sequences, q_idx [n][4][64] bf16, w [n][4] fp32,
- * seq_lens [n] entries.
+ * seq_lens [n] entries (block level: n <= 1024, max_len <= 2^21 entries).
  *   level BLOCK: idx_out [n][keep_blocks] = the Top-keep blocks by the pooled
  *     indexer K score, or every block when ceil(L/8) <= keep_blocks.
  *   level TOKEN: idx_out [n][topk] = Top-min(topk, C) positions among the

@@ -174,7 +174,8 @@ def _swa(B, L_list, layer=0, window=128, seed=SEED):
     return s
 
 
-def test_attn_decode_parity(csa2, orc):
+@pytest.mark.parametrize("mode", [0, 2])  # Full (gathers after the wait) and Reuse (gathers before it)
+def test_attn_decode_parity(csa2, orc, mode):
     lens = [5000, 300, 100, 1]
     B = len(lens)
     ps = PagedSeqs(csa2, lens)
@@ -189,7 +190,7 @@ def test_attn_decode_parity(csa2, orc):
     swa = _swa(B, lens)
     out = torch.empty((B, 16, 128), dtype=torch.float32, device="cuda")
     lse = torch.empty((B, 16), dtype=torch.float32, device="cuda")
-    csa2.sparse_attn_decode(csa2.default_desc(), ps.cache, bits16(q), dev(idx), bits16(swa),
+    csa2.sparse_attn_decode(csa2.default_desc(mode), ps.cache, bits16(q), dev(idx), bits16(swa),
                             dev(np.array(lens, np.int32)), out, lse, B, err=ps.err)
     o, l = out.cpu().numpy(), lse.cpu().numpy()
     for b, L in enumerate(lens):
@@ -212,8 +213,6 @@ def test_attn_decode_swa_lens(csa2, orc):
     lse = torch.empty((2, 16), dtype=torch.float32, device="cuda")
     csa2.sparse_attn_decode(csa2.default_desc(), ps.cache, bits16(q), dev(idx), bits16(swa),
                             dev(np.array([L, L], np.int32)), out, lse, 2, swa_lens=dev(swl))
-    codes, scales = orc.quant_rows(kv)
-    ro, rl = orc.attend(q[1], idx[1], codes, scales, swa[1, :5])
     kv1 = synth.kv_rows(SEED, 1, 0, L)
     c1, s1 = orc.quant_rows(kv1)
     ro, rl = orc.attend(q[1], idx[1], c1, s1, swa[1, :5])
