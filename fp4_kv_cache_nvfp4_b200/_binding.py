@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
             for n in ("csa2_kv_quant_append", "csa2_indexer_topk", "csa2_sparse_attn_decode",
                       "csa2_sparse_attn_prefill", "csa2_decode_layers"):
                 getattr(L, n).restype = _I32
+            L.csa2_indexer_topk_noalloc.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_Cache), _I32, _P, _P,
+                                                    _P, _P, _P, _I32, _I64, _P, _P]
+            L.csa2_indexer_topk_noalloc.restype = _I32
             L.csa2_status_string.argtypes = [_I32]
             L.csa2_status_string.restype = ctypes.c_char_p
             L.csa2_abi_version.restype = _I32
@@ -181,3 +184,12 @@ def decode_layers(descs: list[LayerDesc], cache: KVCache, q_idx: list, w: list, 
                                     ctypes.cast(keep[4], _P), ctypes.cast(keep[5], _P), B, max_len,
                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
                                     _stream(stream)), "decode_layers")
+
+
+def indexer_topk_noalloc(desc: LayerDesc, cache: KVCache, level: int, q_idx, w, seq_lens, out, n: int, max_len: int,
+                         cand_blocks=None, err=None, stream=None) -> None:
+    """Decode indexer without a caller workspace (static 16 MiB library scratch);
+    for callers that cannot allocate device memory at this point."""
+    _check(lib().csa2_indexer_topk_noalloc(ctypes.byref(desc), ctypes.byref(cache.struct()), level, _ptr(q_idx),
+                                           _ptr(w), _ptr(seq_lens), _ptr(cand_blocks), _ptr(out), n, max_len,
+                                           _ptr(err), _stream(stream)), "indexer_topk_noalloc")

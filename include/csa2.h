@@ -218,6 +218,32 @@ CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc*
                                void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Allocation-free decode indexer.  The pages have no counterpart to this call:
+ * it is an integration convenience for callers that cannot allocate device
+ * memory where they run the indexer -- code being captured into a CUDA graph
+ * (cudaMalloc is not allowed while a stream captures), plug-ins whose host
+ * framework owns all device memory, serving loops that must not take the
+ * allocator's locks.  It does exactly what csa2_indexer_topk does for decode
+ * (q_pos = NULL, either level), but keeps its scratch in a 16 MiB array of
+ * static device memory inside the library instead of a caller workspace.
+ *   - allocates nothing (no cudaMalloc/cudaFree); every GPU that loads the
+ *     library holds the 16 MiB until the process exits;
+ *   - a call whose workspace layout (csa2_indexer_workspace_bytes for the same
+ *     desc, level, n and max_len) exceeds 16 MiB returns CSA2_ERR_WORKSPACE
+ *     (n = 8 sequences of 2^20 entries need about 13.5 MiB);
+ *   - the first call on a device looks up the array's device address (a
+ *     runtime call); make that first call before any stream capture;
+ *   - every call clears the counters it needs (a memset on `stream`) and
+ *     otherwise reuses the array as the previous call left it; all calls
+ *     share one array per device, so calls that overlap on the GPU (other
+ *     streams, other threads) race and must be serialised by the caller. */
+CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc* desc, const csa2_kv_cache* cache,
+                                               int32_t level, const uint16_t* q_idx, const float* w,
+                                               const int32_t* seq_lens, const int32_t* cand_blocks,
+                                               int32_t* idx_out, int32_t n, int64_t max_len, int32_t* err_word,
+                                               void* stream);
+
+/* ---------------------------------------------------------------------- */
 CSA2_API const char* csa2_status_string(csa2_status s);
 CSA2_API int32_t csa2_abi_version(void);
 
