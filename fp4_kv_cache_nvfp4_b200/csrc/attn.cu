@@ -22,12 +22,8 @@
 // The work per row is ~5 MFLOP against 136 KiB of gathered bytes, so the kernel
 // is bound by gather latency and HBM/L2 bandwidth; mma.sync keeps the math off
 // the critical path.
-#include <cooperative_groups.h>
-
 #include "common.cuh"
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace csa2 {
 
@@ -49,8 +45,8 @@ constexpr size_t ATT_OFF_OPART = 0;
 constexpr size_t ATT_END_OPART = ATT_OFF_OPART + (size_t)ATT_WARPS * kH * OACC_ROW * 4;
 constexpr size_t ATT_OFF_OACC = ATT_END_STAGE > ATT_END_OPART ? ATT_END_STAGE : ATT_END_OPART;
 constexpr size_t ATT_OFF_MS = ATT_OFF_OACC + kH * OACC_ROW * 4;
-constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;
-constexpr size_t ATT_OFF_MC = ATT_OFF_L + kH * 4;
+constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;  // receive (max, sum): 2 x 16 floats
+constexpr size_t ATT_OFF_MC = ATT_OFF_L + 2 * 2 * ATT_SPLIT * 4;
 constexpr size_t ATT_OFF_LPART = ATT_OFF_MC + kH * 4;
 constexpr size_t ATT_OFF_VALID = ATT_OFF_LPART + ATT_WARPS * kH * 4;
 constexpr size_t ATT_SMEM = ATT_OFF_VALID + ATT_WARPS * KPW * 4;
@@ -82,8 +78,7 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 
 __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    cg::cluster_group cluster = cg::this_cluster();
-    const int split = (int)cluster.block_rank();
+    const int split = blockIdx.x % ATT_SPLIT;  // rank in the cluster (cluster = 8 consecutive CTAs)
     const int row = blockIdx.x / ATT_SPLIT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -317,8 +312,8 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         }
     }
 
-    // ---- merge the 5 warps of this CTA: each writes its rescaled partial,
-    // then every thread sums the five for its share of the 16 x 128 outputs --
+    // ---- merge: the 5 warps of this CTA in shared memory, then each CTA sends
+    // its (max, sum, O) of heads 2c, 2c+1 to CTA c of the cluster ------------
     __syncthreads();  // ms complete
     float Mg = -INFINITY, Mg8 = -INFINITY;
 #pragma unroll
@@ -346,6 +341,10 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         }
     }
     __syncthreads();
+    // receive buffers (in this CTA): from CTA c, heads 2*split + hh
+    float* recv_o = oacc;                       // [ATT_SPLIT][2][kD]
+    float* recv_m = lacc;                       // [ATT_SPLIT][2]  (lacc/mc regions hold 16 floats each)
+    float* recv_l = recv_m + 2 * ATT_SPLIT;     // [ATT_SPLIT][2]
     for (int i = tid; i < kH * kD / 4; i += ATT_THREADS) {
         const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
         float4 acc = *reinterpret_cast<const float4*>(opart + h * OACC_ROW + d4);
@@ -357,25 +356,24 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             acc.z += v.z;
             acc.w += v.w;
         }
-        *reinterpret_cast<float4*>(oacc + h * OACC_ROW + d4) = acc;
+        const uint32_t dst = smem_u32(recv_o + (split * 2 + (h & 1)) * kD + d4);
+        st_cluster_f32x4(mapa_shared(dst, (uint32_t)(h >> 1)), acc);
     }
     if (tid < kH) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < ATT_WARPS; ++w) l += lpart[w * kH + tid];
-        lacc[tid] = l;
+        const uint32_t rank = (uint32_t)(tid >> 1), slot = (uint32_t)(split * 2 + (tid & 1));
+        st_cluster_u32(mapa_shared(smem_u32(recv_m + slot), rank), __float_as_uint(mc[tid]));
+        st_cluster_u32(mapa_shared(smem_u32(recv_l + slot), rank), __float_as_uint(l));
     }
+    cluster_sync_all();  // the only exchange: afterwards every CTA reads its own memory
 
-    // ---- merge the 8 CTAs of the cluster: CTA s writes heads 2s, 2s+1 ------
     __shared__ float fct[2][ATT_SPLIT], sden[2];
-    cluster.sync();
     if (warp == 0) {
-        const int hh = (lane >> 3) & 1, c = lane & 7, h = 2 * split + hh;
-        float mcv = -INFINITY, lv = 0.f;
-        if (lane < 2 * ATT_SPLIT) {
-            mcv = *cluster.map_shared_rank(mc + h, c);
-            lv = *cluster.map_shared_rank(lacc + h, c);
-        }
+        const int hh = (lane >> 3) & 1, c = lane & 7;
+        const float mcv = lane < 2 * ATT_SPLIT ? recv_m[c * 2 + hh] : -INFINITY;
+        const float lv = lane < 2 * ATT_SPLIT ? recv_l[c * 2 + hh] : 0.f;
         float M = mcv;
 #pragma unroll
         for (int o = 1; o < ATT_SPLIT; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -387,20 +385,29 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             fct[hh][c] = f;
             if (c == 0) {
                 sden[hh] = den;
-                a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+                a.lse[(int64_t)row * kH + 2 * split + hh] =
+                    den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
             }
         }
     }
     __syncthreads();
-    for (int i = tid; i < 2 * kD; i += ATT_THREADS) {
-        const int hh = i >> 7, h = 2 * split + hh, d = i & (kD - 1);
-        float num = 0.f;
+    for (int i = tid; i < 2 * kD / 4; i += ATT_THREADS) {
+        const int hh = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < ATT_SPLIT; ++c) num += *cluster.map_shared_rank(oacc + h * OACC_ROW + d, c) * fct[hh][c];
+        for (int c = 0; c < ATT_SPLIT; ++c) {
+            const float4 v = *reinterpret_cast<const float4*>(recv_o + (c * 2 + hh) * kD + d4);
+            const float f = fct[hh][c];
+            num.x += v.x * f;
+            num.y += v.y * f;
+            num.z += v.z * f;
+            num.w += v.w * f;
+        }
         const float den = sden[hh];
-        a.out[((int64_t)row * kH + h) * kD + d] = den > 0.f ? num / den : 0.f;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        *reinterpret_cast<float4*>(a.out + ((int64_t)row * kH + 2 * split + hh) * kD + d4) =
+            make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
     }
-    cluster.sync();
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {

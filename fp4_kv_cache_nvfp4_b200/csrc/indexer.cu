@@ -36,12 +36,8 @@
 
 #include <algorithm>
 
-#include <cooperative_groups.h>
-
 #include "common.cuh"
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace csa2 {
 
@@ -312,7 +308,7 @@ constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
 constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
 constexpr size_t K2_OFF_BAR = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
-constexpr size_t K2_SMEM = align16(K2_OFF_BAR + K2_STAGES * 8) + 1024;  // + alignment slack for the 1 KiB-aligned ring
+constexpr size_t K2_SMEM = align16(K2_OFF_BAR + K2_STAGES * 8);
 constexpr uint32_t kWaitLimit = 1u << 22;
 static_assert(K2_OFF_BAR % 8 == 0 && K2_OFF_QD % 16 == 0 && K2_OFF_HIST % 1024 == 0, "K2 shared-memory layout");
 
@@ -348,8 +344,7 @@ __device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int n, int
 
 __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                  BlockArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K2_OFF_HIST);
     float4* qd = reinterpret_cast<float4*>(smem + K2_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K2_OFF_TMP);
@@ -361,6 +356,10 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
 
     pdl_wait();
     pdl_trigger();
+    if (smem_u32(smem) & 1023u) {  // the swizzled ring needs a 1 KiB-aligned base
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
     // ---- tiles of every sequence (0 for sequences that keep all blocks) ------
     {
         const int per = (a.n + K2_THREADS - 1) / K2_THREADS;
@@ -680,16 +679,18 @@ constexpr int TK_BLKS = TK_SLOTS / kBlk;    // 256 candidate blocks per CTA
 constexpr size_t TK_STAGE_BYTES = (size_t)TK_ROUND * 128;
 constexpr size_t TK_OFF_KEYS = 2 * TK_STAGE_BYTES;
 constexpr size_t TK_OFF_HIST = align16(TK_OFF_KEYS + TK_SLOTS * 4);
-constexpr size_t TK_OFF_SLICE = align16(TK_OFF_HIST + kHistBins * 4);        // this CTA's reduced slice
-constexpr size_t TK_OFF_L0 = align16(TK_OFF_SLICE + (kHistBins / TK_CL) * 4);
+constexpr size_t TK_OFF_G1 = align16(TK_OFF_HIST + kHistBins * 4);
+constexpr size_t TK_OFF_G2 = align16(TK_OFF_G1 + kHistBins * 4);
+constexpr size_t TK_OFF_G3 = align16(TK_OFF_G2 + 1024 * 4);
+constexpr size_t TK_OFF_GCNT = align16(TK_OFF_G3 + 1024 * 4);
+constexpr size_t TK_OFF_L0 = align16(TK_OFF_GCNT + 2 * TK_CL * 4);
 constexpr size_t TK_OFF_L1 = align16(TK_OFF_L0 + TK_SLOTS * 2);
 constexpr size_t TK_OFF_BSLOT = align16(TK_OFF_L1 + TK_SLOTS * 2);
 constexpr size_t TK_OFF_BPOS = align16(TK_OFF_BSLOT + TK_BLKS * 8);
 constexpr size_t TK_OFF_QD = align16(TK_OFF_BPOS + TK_BLKS * 4);
 constexpr size_t TK_OFF_TMP = align16(TK_OFF_QD + kID * 16);
-constexpr size_t TK_OFF_X = align16(TK_OFF_TMP + (64 + kHistBins / TK_CL) * 4);  // exchanged words
-constexpr size_t TK_OFF_BAR = align16(TK_OFF_X + 16 * 4);
-constexpr size_t TK_SMEM = align16(TK_OFF_BAR + 2 * 8) + 1024;
+constexpr size_t TK_OFF_BAR = align16(TK_OFF_TMP + 64 * 4);
+constexpr size_t TK_SMEM = align16(TK_OFF_BAR + 2 * 8);
 static_assert(TK_OFF_BAR % 8 == 0 && TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0, "K4 shared-memory layout");
 
 // The earlier (non-cluster) layout constants are still used by the prefill select.
@@ -710,73 +711,50 @@ struct TokenArgs {
     int keep, topk, page_shift;
 };
 
-// Cluster-wide "which bin holds the need-th largest" over a histogram of
-// nbins bins split across the 8 CTAs (each CTA holds a full local histogram).
-// Returns the bin and the count of items in higher bins.  Whole CTA, all 8 CTAs.
-__device__ void cluster_kth_bin(cg::cluster_group& cl, const uint32_t* hist, int nbins, uint32_t need, uint32_t* slice,
-                                uint32_t* xw, uint32_t* tmp, int* bin_out, uint32_t* above_out) {
-    const int r = (int)cl.block_rank(), per = nbins / TK_CL;
-    cl.sync();  // local histograms complete
-    uint32_t tot = 0;
-    for (int i = threadIdx.x; i < per; i += blockDim.x) {
-        uint32_t v = 0;
+// Push this CTA's histogram (nonzero bins only) into the receive histogram of
+// every CTA of the cluster.  Whole CTA.
+__device__ __forceinline__ void push_hist(const uint32_t* lhist, int nbins, uint32_t* recv) {
+    const uint32_t base = smem_u32(recv);
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) {
+        const uint32_t v = lhist[i];
+        if (v) {
 #pragma unroll
-        for (int c = 0; c < TK_CL; ++c) v += *cl.map_shared_rank(hist + r * per + i, c);
-        slice[i] = v;
-        tot += v;
-    }
-    uint32_t sum;
-    block_excl_scan(tot, tmp, &sum);
-    if (threadIdx.x == 0) xw[0] = sum;
-    cl.sync();  // slices and their totals complete
-    // slices from the top: slice TK_CL-1 holds the highest bins
-    uint32_t above = 0;
-    int sstar = 0;
-    for (int c = TK_CL - 1; c >= 0; --c) {
-        const uint32_t t = *cl.map_shared_rank(xw, c);
-        if (above + t >= need) {
-            sstar = c;
-            break;
+            for (int c = 0; c < TK_CL; ++c) red_add_cluster(mapa_shared(base + 4u * i, c), v);
         }
-        above += t;
     }
-    const uint32_t* src = cl.map_shared_rank(slice, sstar);
-    for (int i = threadIdx.x; i < per; i += blockDim.x) tmp[64 + i] = src[i];  // tmp has room for a 512-bin slice
-    __syncthreads();
-    int b;
-    uint32_t ab;
-    find_kth_bin(tmp + 64, per, need - above, tmp, &b, &ab);
-    *bin_out = sstar * per + b;
-    *above_out = above + ab;
 }
 
 __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     token_topk_kernel(const __grid_constant__ CUtensorMap tmap, TokenArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem + TK_OFF_KEYS);
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);
-    uint32_t* slice = reinterpret_cast<uint32_t*>(smem + TK_OFF_SLICE);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);    // local histogram
+    uint32_t* g1 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G1);        // received, digit 1 (4096)
+    uint32_t* g2 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G2);        // received, digit 2 (1024)
+    uint32_t* g3 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G3);        // received, digit 3 (1024)
+    uint32_t* gcnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_GCNT);    // received per-CTA counts [8][2]
     uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L0);
     uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L1);
     int64_t* bslot = reinterpret_cast<int64_t*>(smem + TK_OFF_BSLOT);
     int32_t* bpos = reinterpret_cast<int32_t*>(smem + TK_OFF_BPOS);
     float4* qd = reinterpret_cast<float4*>(smem + TK_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
-    uint32_t* xw = reinterpret_cast<uint32_t*>(smem + TK_OFF_X);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + TK_OFF_BAR);
     __shared__ float4 s_w;
     __shared__ int s_timeout;
-    cg::cluster_group cl = cg::this_cluster();
-    const int r = (int)cl.block_rank();
+    __shared__ uint32_t s_cnt[2];
+    const int r = blockIdx.x % TK_CL;
     const int b = blockIdx.x / TK_CL;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
     pdl_trigger();
+    // the swizzled ring needs a 1 KiB-aligned base; uniform over the cluster
+    const bool misaligned = (smem_u32(smem) & 1023u) != 0;
     const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
     const int32_t cap = a.keep * kBlk;
-    const int nslots = a.cand ? cap : min(L, cap);
+    const int nslots = misaligned ? 0 : (a.cand ? cap : min(L, cap));
+    if (misaligned && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
     if (!a.cand && L > cap && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_LEN);
     const int s0 = r * TK_SLOTS, s1 = max(s0, min(s0 + TK_SLOTS, nslots));
 
@@ -803,8 +781,17 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
         mbar_init(&full[1], 1);
         mbar_init_fence();
     }
-    for (int i = tid; i < kHistBins; i += TK_THREADS) hist[i] = 0;
+    for (int i = tid; i < kHistBins; i += TK_THREADS) {
+        hist[i] = 0;
+        g1[i] = 0;
+    }
+    for (int i = tid; i < 1024; i += TK_THREADS) {
+        g2[i] = 0;
+        g3[i] = 0;
+    }
+    if (tid < 2 * TK_CL) gcnt[tid] = 0;
     __syncthreads();
+    cluster_arrive();  // receive buffers are zero; peers wait for this before pushing
 
     const int nrounds = (s1 - s0 + TK_ROUND - 1) / TK_ROUND;
     auto issue = [&](int k) {  // warp 0: round k into stage k & 1
@@ -846,28 +833,26 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     for (int i = nrounds * TK_ROUND + tid; i < TK_SLOTS; i += TK_THREADS) keys[i] = 0u;
     if (s_timeout && tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
 
-    // ---- cluster radix select ---------------------------------------------
+    // ---- cluster radix select: every CTA receives every CTA's histogram -----
+    cluster_wait();  // peers' receive buffers are zero
+    push_hist(hist, kHistBins, g1);
+    cluster_sync_all();
     uint32_t nv = 0;
-    for (int i = tid; i < kHistBins; i += TK_THREADS) nv += hist[i];
-    uint32_t mine_valid;
-    block_excl_scan(nv, tmp, &mine_valid);
-    if (tid == 0) xw[1] = mine_valid;
-    cl.sync();
-    uint32_t n_valid = 0;
-#pragma unroll
-    for (int c = 0; c < TK_CL; ++c) n_valid += *cl.map_shared_rank(xw + 1, c);
+    for (int i = tid; i < kHistBins; i += TK_THREADS) nv += g1[i];
+    uint32_t n_valid;
+    block_excl_scan(nv, tmp, &n_valid);
     const uint32_t kk = min((uint32_t)a.topk, n_valid);
     int32_t* out = a.out + (int64_t)b * a.topk;
     uint32_t T = 0xffffffffu, need = 0;
     if (kk > 0) {  // uniform across the cluster
         int b1, d2, d3;
         uint32_t above;
-        cluster_kth_bin(cl, hist, kHistBins, kk, slice, xw, tmp, &b1, &above);
+        find_kth_bin(g1, kHistBins, kk, tmp, &b1, &above);
         need = kk - above;
-        // survivors of digit 1, histogram of digit 2 (bits 19..10)
+        // digit 2 (bits 19..10) over this CTA's survivors of digit 1
         if (tid == 0) {
-            xw[2] = 0;
-            xw[3] = 0;
+            s_cnt[0] = 0;
+            s_cnt[1] = 0;
         }
         for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
         __syncthreads();
@@ -875,13 +860,15 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
             const int i = base + lane;
             const uint32_t k = keys[i];
             const bool in = k != 0u && (int)(k >> 20) == b1;
-            list_append(l0, &xw[2], (uint32_t)i, in);
+            list_append(l0, &s_cnt[0], (uint32_t)i, in);
             hist_add(hist, (k >> 10) & 1023u, in);
         }
         __syncthreads();
-        cluster_kth_bin(cl, hist, 1024, need, slice, xw + 4, tmp, &d2, &above);
+        push_hist(hist, 1024, g2);
+        cluster_sync_all();
+        find_kth_bin(g2, 1024, need, tmp, &d2, &above);
         need -= above;
-        const int n0 = (int)xw[2];
+        const int n0 = (int)s_cnt[0];
         for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
         __syncthreads();
         for (int base = wid * 32; base < n0; base += TK_THREADS) {
@@ -889,16 +876,18 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
             const int slot = i < n0 ? (int)l0[i] : 0;
             const uint32_t k = i < n0 ? keys[slot] : 0u;
             const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
-            list_append(l1, &xw[3], (uint32_t)slot, in);
+            list_append(l1, &s_cnt[1], (uint32_t)slot, in);
             hist_add(hist, k & 1023u, in);
         }
         __syncthreads();
-        cluster_kth_bin(cl, hist, 1024, need, slice, xw + 6, tmp, &d3, &above);
+        push_hist(hist, 1024, g3);
+        cluster_sync_all();
+        find_kth_bin(g3, 1024, need, tmp, &d3, &above);
         need -= above;
         T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
     }
 
-    // ---- ordered emission: counts per CTA, then each CTA writes at its offset
+    // ---- ordered emission: per-CTA counts to every CTA, then own offsets -----
     const unsigned lt = (1u << lane) - 1u;
     constexpr int SEG = TK_SLOTS / (TK_THREADS / 32);  // 128 slots per warp
     uint32_t n_gt = 0, n_eq = 0;
@@ -913,19 +902,19 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
         tmp[32 + wid] = n_gt;
     }
     __syncthreads();
-    if (tid == 0) {
+    if (tid < TK_CL) {  // lane c sends this CTA's totals to CTA c
         uint32_t e = 0, g = 0;
         for (int v = 0; v < TK_THREADS / 32; ++v) {
             e += tmp[v];
             g += tmp[32 + v];
         }
-        xw[8] = e;
-        xw[9] = g;
+        st_cluster_u32(mapa_shared(smem_u32(gcnt + 2 * r), tid), e);
+        st_cluster_u32(mapa_shared(smem_u32(gcnt + 2 * r + 1), tid), g);
     }
-    cl.sync();
+    cluster_sync_all();  // last exchange: no CTA touches another's memory after this
     uint32_t tie_base = 0, sel_base = 0;
     for (int c = 0; c < r; ++c) {
-        const uint32_t e = *cl.map_shared_rank(xw + 8, c), g = *cl.map_shared_rank(xw + 9, c);
+        const uint32_t e = gcnt[2 * c], g = gcnt[2 * c + 1];
         const uint32_t take = tie_base >= need ? 0u : min(e, need - tie_base);
         sel_base += g + take;
         tie_base += e;
@@ -948,7 +937,6 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     }
     if (r == 0)
         for (int i = (int)kk + tid; i < a.topk; i += TK_THREADS) out[i] = -1;
-    cl.sync();  // peers may still read this CTA's shared memory
 }
 
 // ============================================================================
