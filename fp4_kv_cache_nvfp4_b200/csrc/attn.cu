@@ -49,7 +49,8 @@ constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;  // receive (max, 
 constexpr size_t ATT_OFF_MC = ATT_OFF_L + 2 * 2 * ATT_SPLIT * 4;
 constexpr size_t ATT_OFF_LPART = ATT_OFF_MC + kH * 4;
 constexpr size_t ATT_OFF_VALID = ATT_OFF_LPART + ATT_WARPS * kH * 4;
-constexpr size_t ATT_SMEM = ATT_OFF_VALID + ATT_WARPS * KPW * 4;
+constexpr size_t ATT_OFF_FCT = ATT_OFF_VALID + ATT_WARPS * KPW * 4;  // merge factors [2][ATT_SPLIT] + sums [2]
+constexpr size_t ATT_SMEM = ATT_OFF_FCT + (2 * ATT_SPLIT + 2) * 4;
 static_assert(ATT_OFF_SWA % 16 == 0 && ATT_OFF_VT % 16 == 0 && ATT_OFF_OACC % 16 == 0 && ATT_OFF_MS % 16 == 0 &&
                   ATT_OFF_VALID % 16 == 0,
               "attention shared-memory layout");
@@ -95,6 +96,13 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     // A Reuse layer's index set, the cache and the SWA history come from kernels
     // at least two launches back, so they are gathered before waiting on the
     // preceding kernel; the query and the newest SWA row are read after it.
+    // every buffer offset below assumes a 16-byte-aligned dynamic shared base;
+    // the check is uniform over the grid, so no CTA waits on one that left
+    if (smem_u32(smem) & 15u) {
+        pdl_wait();
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
     const bool early = a.early != 0;
     if (!early) pdl_wait();
 
@@ -369,7 +377,8 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     }
     cluster_sync_all();  // the only exchange: afterwards every CTA reads its own memory
 
-    __shared__ float fct[2][ATT_SPLIT], sden[2];
+    float (*fct)[ATT_SPLIT] = reinterpret_cast<float (*)[ATT_SPLIT]>(smem + ATT_OFF_FCT);
+    float* sden = reinterpret_cast<float*>(smem + ATT_OFF_FCT) + 2 * ATT_SPLIT;
     if (warp == 0) {
         const int hh = (lane >> 3) & 1, c = lane & 7;
         const float mcv = lane < 2 * ATT_SPLIT ? recv_m[c * 2 + hh] : -INFINITY;

@@ -308,7 +308,8 @@ constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
 constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
 constexpr size_t K2_OFF_BAR = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
-constexpr size_t K2_SMEM = align16(K2_OFF_BAR + K2_STAGES * 8);
+constexpr size_t K2_OFF_MISC = align16(K2_OFF_BAR + K2_STAGES * 8);  // w (float4), last, timeout
+constexpr size_t K2_SMEM = align16(K2_OFF_MISC + 32);
 constexpr uint32_t kWaitLimit = 1u << 22;
 static_assert(K2_OFF_BAR % 8 == 0 && K2_OFF_QD % 16 == 0 && K2_OFF_HIST % 1024 == 0, "K2 shared-memory layout");
 
@@ -350,8 +351,9 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K2_OFF_TMP);
     int32_t* tile_start = reinterpret_cast<int32_t*>(smem + K2_OFF_TS);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + K2_OFF_BAR);
-    __shared__ float4 s_w;
-    __shared__ int s_last, s_timeout;
+    float4& s_w = *reinterpret_cast<float4*>(smem + K2_OFF_MISC);
+    int& s_last = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 16);
+    int& s_timeout = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 20);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
@@ -513,13 +515,18 @@ constexpr int K3_THREADS = 512;
 constexpr int K3_CHUNK = 8192;
 constexpr int K3_WORDS = (int)(kMaxBlockLevelLen / kBlk / 32);  // bitmap words for the largest context
 constexpr int K3_BND_CAP = 12288;                               // boundary entries held in shared memory
-constexpr size_t K3_SMEM = (size_t)2 * K3_WORDS * 4 + 1024 * 4 + 64 * 4 + (size_t)K3_BND_CAP * 8;
+constexpr size_t K3_OFF_LAST = (size_t)2 * K3_WORDS * 4 + 1024 * 4 + 64 * 4 + (size_t)K3_BND_CAP * 8;
+constexpr size_t K3_SMEM = K3_OFF_LAST + 16;
 
 __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_last;
+    int& s_last = *reinterpret_cast<int*>(smem + K3_OFF_LAST);
     pdl_wait();
     pdl_trigger();
+    if (smem_u32(smem) & 15u) {  // uniform over the grid
+        if (threadIdx.x == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
     const int b = blockIdx.y;
     const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
     const int32_t nblk = (L + kBlk - 1) / kBlk;
@@ -690,7 +697,8 @@ constexpr size_t TK_OFF_BPOS = align16(TK_OFF_BSLOT + TK_BLKS * 8);
 constexpr size_t TK_OFF_QD = align16(TK_OFF_BPOS + TK_BLKS * 4);
 constexpr size_t TK_OFF_TMP = align16(TK_OFF_QD + kID * 16);
 constexpr size_t TK_OFF_BAR = align16(TK_OFF_TMP + 64 * 4);
-constexpr size_t TK_SMEM = align16(TK_OFF_BAR + 2 * 8);
+constexpr size_t TK_OFF_MISC = align16(TK_OFF_BAR + 2 * 8);  // w (float4), timeout, two counters
+constexpr size_t TK_SMEM = align16(TK_OFF_MISC + 32);
 static_assert(TK_OFF_BAR % 8 == 0 && TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0, "K4 shared-memory layout");
 
 // The earlier (non-cluster) layout constants are still used by the prefill select.
@@ -740,21 +748,24 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     float4* qd = reinterpret_cast<float4*>(smem + TK_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + TK_OFF_BAR);
-    __shared__ float4 s_w;
-    __shared__ int s_timeout;
-    __shared__ uint32_t s_cnt[2];
+    float4& s_w = *reinterpret_cast<float4*>(smem + TK_OFF_MISC);
+    int& s_timeout = *reinterpret_cast<int*>(smem + TK_OFF_MISC + 16);
+    uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_MISC + 20);
     const int r = blockIdx.x % TK_CL;
     const int b = blockIdx.x / TK_CL;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
     pdl_trigger();
-    // the swizzled ring needs a 1 KiB-aligned base; uniform over the cluster
-    const bool misaligned = (smem_u32(smem) & 1023u) != 0;
+    // the swizzled ring needs a 1 KiB-aligned base; the check is uniform over
+    // the grid, so no CTA waits at a cluster barrier for one that left
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
     const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
     const int32_t cap = a.keep * kBlk;
-    const int nslots = misaligned ? 0 : (a.cand ? cap : min(L, cap));
-    if (misaligned && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+    const int nslots = a.cand ? cap : min(L, cap);
     if (!a.cand && L > cap && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_LEN);
     const int s0 = r * TK_SLOTS, s1 = max(s0, min(s0 + TK_SLOTS, nslots));
 
@@ -959,7 +970,9 @@ struct PrefillArgs {
 
 __device__ __forceinline__ int visible(int p, int ratio, int n) { return min((p + 1) / ratio, n); }
 
-constexpr size_t PS_SMEM = (size_t)kID * PS_E * 4 + (size_t)kID * PS_Q * kIH * 4;
+constexpr size_t PS_OFF_W = (size_t)kID * PS_E * 4 + (size_t)kID * PS_Q * kIH * 4;
+constexpr size_t PS_OFF_VIS = PS_OFF_W + PS_Q * kIH * 4;
+constexpr size_t PS_SMEM = PS_OFF_VIS + PS_Q * 4;
 
 // Thread (qi, ei) of a 16 x 16 grid computes queries 2qi, 2qi+1 against entries
 // 4ei .. 4ei+3 of the tile: 32 sequential fp32 FMA chains.
@@ -967,8 +980,8 @@ __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a
     extern __shared__ __align__(128) uint8_t smem[];
     float (*kt)[PS_E] = reinterpret_cast<float (*)[PS_E]>(smem);                                      // [d][entry]
     float (*qs)[PS_Q][kIH] = reinterpret_cast<float (*)[PS_Q][kIH]>(smem + (size_t)kID * PS_E * 4);  // [d][q][h]
-    __shared__ float ws_[PS_Q][kIH];
-    __shared__ int vis[PS_Q];
+    float (*ws_)[kIH] = reinterpret_cast<float (*)[kIH]>(smem + PS_OFF_W);
+    int* vis = reinterpret_cast<int*>(smem + PS_OFF_VIS);
     pdl_wait();
     pdl_trigger();
     const int q0 = blockIdx.x * PS_Q;
