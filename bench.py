@@ -45,7 +45,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    p.add_argument("--config", type=int, default=4, choices=[2, 4])
+    p.add_argument("--config", type=int, default=4, choices=[2, 3, 4])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--kernel-reps", type=int, default=300)
     p.add_argument("--contiguous-pages", action="store_true")
@@ -393,6 +393,131 @@ def whole_job_tokens_per_s(batch_per_rank: int, world: int, ms_per_step: float) 
     return world * batch_per_rank / (ms_per_step * 1e-3)
 
 
+def run_prefill(args, rank: int, world: int, local_rank: int):
+    """Encoder prefill chunk (config 3): 32,768 tokens of context (16,384
+    ratio-2 entries); the step appends the chunk's last 4096 tokens (2048
+    entries), runs the Full layer's indexer for the 4096 query tokens and the
+    attention of 6 layers (1 Full + 5 Reuse) over their Top-512 + window."""
+    import torch
+    import synth
+    import fp4_kv_cache_nvfp4_b200 as csa2
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    csa2.lib()
+    c = synth.CONFIGS[3]
+    tokens, T, layers, seed = c["tokens"], c["T"], c["layers"], c["seed"] + 100 * rank
+    n_ent, chunk_ent = tokens // 2, T // 2
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    table, n_phys = synth.page_table(seed, [n_ent], PAGE, shuffle=not args.contiguous_pages)
+    cache = csa2.KVCache(n_phys, PAGE, torch.from_numpy(table), device=dev, pooled=False)
+    gain = torch.from_numpy(synth.gain(seed)).to(dev)
+    tab = torch.from_numpy(table).to(dev).long()
+    pos = torch.arange(n_ent, device=dev)
+    slots = (tab[0, pos // PAGE] * PAGE + pos % PAGE).contiguous()
+    kv_all = (torch.randn((tokens, CH), generator=gen, device=dev) * gain).to(torch.bfloat16)
+    ik_all = torch.randn((n_ent, 64), generator=gen, device=dev).to(torch.bfloat16).view(torch.int16)
+    pre = n_ent - chunk_ent  # entries filled before the timed chunk
+    csa2.kv_quant_append(cache, kv_all[:2 * pre], ik_all[:pre], slots[:pre], ratio=2)
+    kv_chunk, ik_chunk, sl_chunk = kv_all[2 * pre:], ik_all[pre:], slots[pre:]
+    q_pos = torch.arange(tokens - T, tokens, dtype=torch.int32, device=dev)
+    bf = lambda shape: torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16)  # noqa: E731
+    q_idx, w = bf((T, 4, 64)), torch.rand((T, 4), generator=gen, device=dev)
+    qs = [bf((T, 16, 128)) for _ in range(layers)]
+    swa_start = tokens - T - 127
+    swas = [(torch.randn((tokens - swa_start, CH), generator=gen, device=dev) * gain).to(torch.bfloat16)
+            .view(torch.int16) for _ in range(layers)]
+    d_full = csa2.default_desc(csa2.FULL, 2)
+    d_reuse = csa2.default_desc(csa2.REUSE, 2)
+    ws = torch.zeros(csa2.workspace_bytes(d_full, csa2.TOKEN, T, n_ent, prefill=True), dtype=torch.uint8,
+                     device=dev)
+    sets = torch.empty((T, 512), dtype=torch.int32, device=dev)
+    outs = [torch.empty((T, 16, 128), device=dev) for _ in range(layers)]
+    lses = [torch.empty((T, 16), device=dev) for _ in range(layers)]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    nl = torch.tensor([n_ent], dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def append():
+        csa2.kv_quant_append(cache, kv_chunk, ik_chunk, sl_chunk, ratio=2, err=err, stream=stream)
+
+    def indexer():
+        csa2.indexer_topk(d_full, cache, csa2.TOKEN, q_idx, w, nl, sets, T, n_ent, ws, q_pos=q_pos, err=err,
+                          stream=stream)
+
+    def attn(l):
+        csa2.sparse_attn_prefill(d_full if l == 0 else d_reuse, cache, qs[l], sets, q_pos, swas[l], swa_start, n_ent,
+                                 outs[l], lses[l], T, err=err, stream=stream)
+
+    def step():
+        append()
+        indexer()
+        for l in range(layers):
+            attn(l)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    parts = {"append": append, "indexer": indexer, "attention layer (Full)": lambda: attn(0),
+             "attention layer (Reuse)": lambda: attn(1)}
+    pgraphs = {}
+    for name, fn in parts.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        pgraphs[name] = g
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                graph.replay()
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, 50))
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for k in range(steps):
+                flush.fill_(k & 0xFF)
+                ev[k][0].record(stream)
+                graph.replay()
+                ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / steps
+        part_us = {}
+        with torch.cuda.stream(stream):
+            for name, g in pgraphs.items():
+                pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+                for k in range(10):
+                    flush.fill_(k & 0xFF)
+                    pe[k][0].record(stream)
+                    g.replay()
+                    pe[k][1].record(stream)
+                torch.cuda.synchronize()
+                part_us[name] = round(statistics.mean(a.elapsed_time(b) for a, b in pe) * 1e3, 2)
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+    peaks = _peaks()
+    # tensor work of the attention layers (QK and PV over 512 selected + 128 window keys, 16 heads x 128)
+    att_flop = T * 16 * (512 + 128) * 128 * 2 * 2
+    idx_flop = sum(min((p + 1) // 2, n_ent) for p in range(tokens - T, tokens)) * 4 * 64 * 2
+    att_us = part_us["attention layer (Reuse)"]
+    return dict(metric="CSA2 encoder prefill tokens/s (4096-token chunk, 32K context, 1F+5R layers)",
+                value=world * T / (ms * 1e-3), unit="tokens/s", n_gpus=world, steps=steps, warmup=args.warmup,
+                ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="fp4 cache; f16 mma, f32 accumulate; exact f32 indexer", data="synthetic",
+                config=dict(workload=c["name"], context_tokens=tokens, chunk=T, entries=n_ent, ratio=2,
+                            layers=layers, l2="flushed before every timed step"),
+                breakdown_us=part_us,
+                tensor=dict(attention_tflops=att_flop / (att_us * 1e-6) / 1e12, attention_flop_per_layer=att_flop,
+                            indexer_gflop=idx_flop / 1e9,
+                            indexer_tflops=idx_flop / (part_us["indexer"] * 1e-6) / 1e12,
+                            peak_bf16_tflops=peaks.get("bf16_tflops")),
+                clocks=sampler.summary())
+
+
 def _cudart():
     import torch  # noqa: F401  (loads the runtime torch ships)
     for name in ("libcudart.so.12", "libcudart.so"):
@@ -480,6 +605,15 @@ def main():
         import torch
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.config == 3:
+        res = run_prefill(args, rank, world, local_rank)
+        if world > 1:
+            import torch
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res = run_cuda(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = oracle_sample(args.config, budget_s=15.0)

@@ -31,9 +31,6 @@
 //                              of a sequence refines and emits the Top-K.
 //   prefill_score_kernel / prefill_select_kernel: the same per query over the
 //                              entries visible to it.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 
 #include "common.cuh"
@@ -307,11 +304,11 @@ constexpr size_t K2_OFF_HIST = K2_STAGES * K2_STAGE_BYTES;
 constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
 constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
-constexpr size_t K2_OFF_BAR = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
-constexpr size_t K2_OFF_MISC = align16(K2_OFF_BAR + K2_STAGES * 8);  // w (float4), last, timeout
+constexpr size_t K2_OFF_NBLK = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
+constexpr size_t K2_OFF_MISC = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // w (float4), last
 constexpr size_t K2_SMEM = align16(K2_OFF_MISC + 32);
-constexpr uint32_t kWaitLimit = 1u << 22;
-static_assert(K2_OFF_BAR % 8 == 0 && K2_OFF_QD % 16 == 0 && K2_OFF_HIST % 1024 == 0, "K2 shared-memory layout");
+constexpr size_t K2_SLICE = 32 * 128;  // one warp's 32 rows of a stage
+static_assert(K2_OFF_QD % 16 == 0 && K2_OFF_MISC % 16 == 0, "K2 shared-memory layout");
 
 struct BlockArgs {
     csa2_kv_cache cache;
@@ -329,7 +326,7 @@ struct BlockArgs {
     int32_t* err;
     int64_t nblk_pad;
     int64_t max_len;
-    int n, keep, page_shift, box_rows;
+    int n, keep, page_shift;
 };
 
 // tile_start[b] = first tile of sequence b; returns the sequence of tile t
@@ -343,22 +340,20 @@ __device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int n, int
     return lo;
 }
 
-__global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_constant__ CUtensorMap tmap,
-                                                                 BlockArgs a) {
+__global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K2_OFF_HIST);
     float4* qd = reinterpret_cast<float4*>(smem + K2_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K2_OFF_TMP);
     int32_t* tile_start = reinterpret_cast<int32_t*>(smem + K2_OFF_TS);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K2_OFF_BAR);
+    int32_t* s_nblk = reinterpret_cast<int32_t*>(smem + K2_OFF_NBLK);
     float4& s_w = *reinterpret_cast<float4*>(smem + K2_OFF_MISC);
     int& s_last = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 16);
-    int& s_timeout = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 20);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
     pdl_trigger();
-    if (smem_u32(smem) & 1023u) {  // the swizzled ring needs a 1 KiB-aligned base
+    if (smem_u32(smem) & 15u) {  // 16-byte copies and vector reads need an aligned base
         if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
@@ -383,15 +378,11 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
                 tile_start[b] = (int32_t)base;
                 const int32_t L = a.seq_lens[b];
                 const int32_t nblk = (L >= 1 && L <= a.max_len) ? (L + kBlk - 1) / kBlk : 0;
+                s_nblk[b] = nblk;
                 base += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
             }
         }
         if (tid == 0) tile_start[a.n] = (int32_t)total;
-        if (tid < K2_STAGES) mbar_init(&full[tid], 1);
-        if (tid == 0) {
-            s_timeout = 0;
-            mbar_init_fence();
-        }
         for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
         __syncthreads();
     }
@@ -401,38 +392,57 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
     const int ntiles = t1 - t0;
     if (ntiles <= 0) return;
 
-    const int sh = a.page_shift, br = a.box_rows;
+    // Warp w owns rows [32 w, 32 w + 32) of every tile: it copies them into its
+    // own slice of the 3-stage ring with 16-byte cp.async (lane l moves chunk
+    // l & 7 of row 4 k + l / 8, so one instruction covers 512 contiguous bytes
+    // of a page) and scores them itself.  Warps therefore never wait for one
+    // another inside a sequence.  Each lane loads the physical page of its own
+    // row one tile before the copy needs it.
+    const int sh = a.page_shift;
     const int32_t emask = (1 << sh) - 1;
-    // warp 0: issue the boxes of tile t into stage s (lane-parallel)
-    auto issue = [&](int32_t t, int s) {
+    const uint8_t* pooled = reinterpret_cast<const uint8_t*>(a.cache.idx_k_pooled);
+    const int32_t mpps = a.cache.max_pages_per_seq;
+    struct RowPage {
+        int32_t j;     // row (block) index within its sequence; -1: past the end
+        int32_t phys;  // physical page of the row's entries
+    };
+    auto fetch = [&](int32_t t) {
         const int b = seq_of_tile(tile_start, a.n, t);
-        const int32_t L = a.seq_lens[b];
-        const int32_t nblk = (L + kBlk - 1) / kBlk;
-        const int32_t r0 = (t - tile_start[b]) * K2_TILE, r1 = min(r0 + K2_TILE, nblk);
-        const int nbox = (r1 - r0 + br - 1) / br;
-        uint8_t* stage = smem + (size_t)s * K2_STAGE_BYTES;
-        if (lane == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * br * 128));
-        }
-        __syncwarp();
-        for (int x = lane; x < nbox; x += 32) {
-            const int32_t e = (r0 + x * br) * kBlk;  // first entry of the box
-            const int32_t pg = e >> sh;
-            int32_t phys = pg < a.cache.max_pages_per_seq
-                               ? __ldg(a.cache.page_table + (int64_t)b * a.cache.max_pages_per_seq + pg)
-                               : -1;
+        RowPage r;
+        r.j = (t - tile_start[b]) * K2_TILE + 32 * wid + lane;
+        const int32_t pg = (r.j * kBlk) >> sh;
+        const bool in = r.j < s_nblk[b];
+        r.phys = (in && pg < mpps) ? __ldg(a.cache.page_table + (int64_t)b * mpps + pg) : -1;
+        if (!in) r.j = -1;
+        return r;
+    };
+    auto issue = [&](int s, RowPage r) {
+        int32_t prow = -1;
+        if (r.j >= 0) {
+            int32_t phys = r.phys;
             if (phys < 0 || phys >= a.cache.n_phys_pages) {
                 dev_error(a.err, CSA2_DEV_PAGE);
-                phys = 0;  // keep the byte count; results of this call are undefined
+                phys = 0;  // results of this call are undefined; the copy stays in bounds
             }
-            const int32_t prow = (int32_t)((((int64_t)phys << sh) | (e & emask)) >> 3);
-            tma_load_2d(stage + (size_t)x * br * 128, &tmap, 0, prow, &full[s]);
+            prow = (int32_t)((((int64_t)phys << sh) | ((r.j * kBlk) & emask)) >> 3);
         }
+        uint8_t* slice = smem + (size_t)s * K2_STAGE_BYTES + (size_t)wid * K2_SLICE;
+        const int c = lane & 7;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + (lane >> 3);
+            const int32_t pr = __shfl_sync(0xffffffffu, prow, rr);
+            if (pr >= 0) cp_async16(slice + rr * 128 + ((c ^ (rr & 7)) << 4), pooled + (int64_t)pr * 128 + c * 16);
+        }
+        cp_async_commit();
     };
-    if (wid == 0) {
-        for (int i = 0; i < min(2, ntiles); ++i) issue(t0 + i, i);
+    {
+        const RowPage r0 = fetch(t0);
+        const RowPage r1 = ntiles > 1 ? fetch(t0 + 1) : RowPage{-1, -1};
+        issue(0, r0);
+        issue(1, r1);  // an empty group when there is no second tile
     }
+    RowPage next = ntiles > 2 ? fetch(t0 + 2) : RowPage{-1, -1};
 
     int cur_b = -1, nloc = 0;
     auto flush = [&](int b, int nt) {
@@ -446,8 +456,7 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
         __threadfence();
         __syncthreads();
         if (tid == 0) {
-            const int32_t L = a.seq_lens[b];
-            const int32_t nblk = (L + kBlk - 1) / kBlk;
+            const int32_t nblk = s_nblk[b];
             const uint32_t need_t = (uint32_t)((nblk + K2_TILE - 1) / K2_TILE);
             s_last = atomicAdd(&a.ctr[2 * b], (uint32_t)nt) + (uint32_t)nt == need_t;
         }
@@ -474,7 +483,13 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
     for (int i = 0; i < ntiles; ++i) {
         const int32_t t = t0 + i;
         const int s = i % K2_STAGES;
-        if (wid == 0 && i + 2 < ntiles) issue(t + 2, (i + 2) % K2_STAGES);
+        __syncwarp();  // every lane has read the slice that is refilled next (tile i - 1's)
+        if (i + 2 < ntiles) {
+            issue((i + 2) % K2_STAGES, next);
+            if (i + 3 < ntiles) next = fetch(t + 3);
+        } else {
+            cp_async_commit();  // empty group: the wait below always leaves the two newest
+        }
         const int b = seq_of_tile(tile_start, a.n, t);
         if (b != cur_b) {
             if (cur_b >= 0) flush(cur_b, nloc);
@@ -484,26 +499,16 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(const __grid_co
             nloc = 0;
             __syncthreads();
         }
-        const int32_t L = a.seq_lens[b];
-        const int32_t nblk = (L + kBlk - 1) / kBlk;
-        const int32_t r0 = (t - tile_start[b]) * K2_TILE;
-        const int32_t j = r0 + tid;
-        if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, kWaitLimit)) s_timeout = 1;
+        const int32_t j = (t - tile_start[b]) * K2_TILE + 32 * wid + lane;
+        cp_async_wait<2>();
+        __syncwarp();  // the other lanes' copies of this warp's rows are visible
         uint32_t k[32];
-        read_row(smem + (size_t)s * K2_STAGE_BYTES, tid, k);
+        read_row(smem + (size_t)s * K2_STAGE_BYTES + (size_t)wid * K2_SLICE, lane, k);
         const float s0 = idx_score1(k, qd, s_w);
-        const bool act = j < nblk;
+        const bool act = j < s_nblk[b];
         if (act) a.scores[(int64_t)b * a.nblk_pad + j] = s0;
         hist_add(hist, score_key(s0) >> 20, act);
         ++nloc;
-        __syncthreads();
-        if (s_timeout) break;
-    }
-    if (s_timeout) {
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
-        // let every copy this CTA issued land before the shared memory goes away
-        for (int i = 0; i < K2_STAGES; ++i) mbar_wait(&full[i], 0u, kWaitLimit);
-        return;
     }
     if (cur_b >= 0) flush(cur_b, nloc);
 }
@@ -696,10 +701,9 @@ constexpr size_t TK_OFF_BSLOT = align16(TK_OFF_L1 + TK_SLOTS * 2);
 constexpr size_t TK_OFF_BPOS = align16(TK_OFF_BSLOT + TK_BLKS * 8);
 constexpr size_t TK_OFF_QD = align16(TK_OFF_BPOS + TK_BLKS * 4);
 constexpr size_t TK_OFF_TMP = align16(TK_OFF_QD + kID * 16);
-constexpr size_t TK_OFF_BAR = align16(TK_OFF_TMP + 64 * 4);
-constexpr size_t TK_OFF_MISC = align16(TK_OFF_BAR + 2 * 8);  // w (float4), timeout, two counters
+constexpr size_t TK_OFF_MISC = align16(TK_OFF_TMP + 64 * 4);  // w (float4), two counters
 constexpr size_t TK_SMEM = align16(TK_OFF_MISC + 32);
-static_assert(TK_OFF_BAR % 8 == 0 && TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0, "K4 shared-memory layout");
+static_assert(TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0 && TK_OFF_MISC % 16 == 0, "K4 shared-memory layout");
 
 // The earlier (non-cluster) layout constants are still used by the prefill select.
 constexpr size_t K4_OFF_HIST = (size_t)kMaxCand * 4;
@@ -733,7 +737,7 @@ __device__ __forceinline__ void push_hist(const uint32_t* lhist, int nbins, uint
 }
 
 __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
-    token_topk_kernel(const __grid_constant__ CUtensorMap tmap, TokenArgs a) {
+    token_topk_kernel(TokenArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem + TK_OFF_KEYS);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);    // local histogram
@@ -747,19 +751,17 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     int32_t* bpos = reinterpret_cast<int32_t*>(smem + TK_OFF_BPOS);
     float4* qd = reinterpret_cast<float4*>(smem + TK_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + TK_OFF_BAR);
     float4& s_w = *reinterpret_cast<float4*>(smem + TK_OFF_MISC);
-    int& s_timeout = *reinterpret_cast<int*>(smem + TK_OFF_MISC + 16);
-    uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_MISC + 20);
+    uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_MISC + 16);
     const int r = blockIdx.x % TK_CL;
     const int b = blockIdx.x / TK_CL;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
     pdl_trigger();
-    // the swizzled ring needs a 1 KiB-aligned base; the check is uniform over
-    // the grid, so no CTA waits at a cluster barrier for one that left
-    if (smem_u32(smem) & 1023u) {
+    // 16-byte copies and vector reads need an aligned base; the check is
+    // uniform over the grid, so no CTA waits at a cluster barrier for one that left
+    if (smem_u32(smem) & 15u) {
         if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
@@ -787,10 +789,6 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
     if (tid == 0) {
         s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
-        s_timeout = 0;
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init_fence();
     }
     for (int i = tid; i < kHistBins; i += TK_THREADS) {
         hist[i] = 0;
@@ -804,45 +802,48 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     __syncthreads();
     cluster_arrive();  // receive buffers are zero; peers wait for this before pushing
 
+    // Rows of round k: slot s0 + 512 k + 32 w + l belongs to lane l of warp w,
+    // which scores it.  The warp copies its 32 rows (4 candidate blocks of 8
+    // contiguous indexer-K rows) into its own slice of a 2-stage ring with
+    // 16-byte cp.async, lane l moving chunk l & 7 of row 4 j + l / 8, and
+    // waits only for its own copies.
     const int nrounds = (s1 - s0 + TK_ROUND - 1) / TK_ROUND;
-    auto issue = [&](int k) {  // warp 0: round k into stage k & 1
-        const int st = k & 1;
-        uint8_t* stage = smem + (size_t)st * TK_STAGE_BYTES;
-        uint32_t nvalid = 0;
-        for (int x = lane; x < TK_ROUND / kBlk; x += 32) nvalid += bslot[k * (TK_ROUND / kBlk) + x] >= 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
-        if (lane == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[st], nvalid * kBlk * 128);
-        }
-        __syncwarp();
-        for (int x = lane; x < TK_ROUND / kBlk; x += 32) {
-            const int64_t sl = bslot[k * (TK_ROUND / kBlk) + x];
-            if (sl >= 0) tma_load_2d(stage + (size_t)x * kBlk * 128, &tmap, 0, (int32_t)sl, &full[st]);
-        }
+    const uint8_t* idx_k = reinterpret_cast<const uint8_t*>(a.cache.idx_k);
+    auto row_src = [&](int k) {  // physical entry of this lane's row in round k, -1 if none
+        const int my = k * TK_ROUND + tid;
+        const int blk = my >> 3, e = my & 7;
+        return (s0 + my < s1 && bpos[blk] >= 0 && bpos[blk] + e < L) ? (int32_t)(bslot[blk] + e) : -1;
     };
-    if (wid == 0) {
-        for (int k = 0; k < min(2, nrounds); ++k) issue(k);
-    }
+    auto issue = [&](int k) {
+        const int32_t src = k < nrounds ? row_src(k) : -1;
+        uint8_t* slice = smem + (size_t)(k & 1) * TK_STAGE_BYTES + (size_t)wid * (32 * 128);
+        const int c = lane & 7;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int rr = 4 * j + (lane >> 3);
+            const int32_t ps = __shfl_sync(0xffffffffu, src, rr);
+            if (ps >= 0) cp_async16(slice + rr * 128 + ((c ^ (rr & 7)) << 4), idx_k + (int64_t)ps * 128 + c * 16);
+        }
+        cp_async_commit();  // possibly empty: the wait below always leaves the newest group
+    };
+    issue(0);
+    issue(1);
     for (int k = 0; k < nrounds; ++k) {
-        const int st = k & 1;
-        if (!mbar_wait(&full[st], (uint32_t)(k >> 1) & 1u, kWaitLimit)) s_timeout = 1;
-        const int blk = k * (TK_ROUND / kBlk) + (tid >> 3), e = tid & 7;
-        const bool valid = s0 + k * TK_ROUND + tid < s1 && bpos[blk] >= 0 && bpos[blk] + e < L;
+        cp_async_wait<1>();
+        __syncwarp();  // the other lanes' copies of this warp's rows are visible
         uint32_t key = 0u;
-        if (valid) {
+        if (row_src(k) >= 0) {
             uint32_t kr[32];
-            read_row(smem + (size_t)st * TK_STAGE_BYTES, tid, kr);
+            read_row(smem + (size_t)(k & 1) * TK_STAGE_BYTES + (size_t)wid * (32 * 128), lane, kr);
             key = score_key(idx_score1(kr, qd, s_w));
         }
         keys[k * TK_ROUND + tid] = key;
         hist_add(hist, key >> 20, key != 0u);
-        __syncthreads();
-        if (wid == 0 && k + 2 < nrounds) issue(k + 2);
+        __syncwarp();  // every lane has read the slice before it is refilled
+        issue(k + 2);
     }
     for (int i = nrounds * TK_ROUND + tid; i < TK_SLOTS; i += TK_THREADS) keys[i] = 0u;
-    if (s_timeout && tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+    __syncthreads();  // the local histogram is complete
 
     // ---- cluster radix select: every CTA receives every CTA's histogram -----
     cluster_wait();  // peers' receive buffers are zero
@@ -1164,19 +1165,6 @@ static cudaError_t ensure_smem(const void* fn, size_t bytes, bool* done) {
     return cudaSuccess;
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 static int sm_count() {
     static int n[64];
     int dev = 0;
@@ -1217,24 +1205,12 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.n = n;
     a.keep = keep;
     a.page_shift = page_shift_of(cache);
-    a.box_rows = min(8, cache.page_size / kBlk);
     const int64_t nblk = (max_len + kBlk - 1) / kBlk;
     if (nblk > keep) {
-        PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-        if (!enc) return cudaErrorNotSupported;
-        CUtensorMap map;
-        const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size / kBlk)};
-        const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kID, (cuuint32_t)a.box_rows};
-        const cuuint32_t estr[2] = {1, 1};
-        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k_pooled, dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
         const int64_t tiles = (int64_t)n * ((nblk + K2_TILE - 1) / K2_TILE);
         const int grid = (int)std::min<int64_t>(tiles, sm_count());
         LaunchCfg c2(dim3((unsigned)grid), dim3(K2_THREADS), K2_SMEM, stream);
-        e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, map, a);
+        e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, a);
         if (e != cudaSuccess) return e;
     }
     LaunchCfg c3(dim3((unsigned)((nblk + K3_CHUNK - 1) / K3_CHUNK), n), dim3(K3_THREADS), K3_SMEM, stream);
@@ -1248,17 +1224,6 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     cudaError_t e = ensure_smem((const void*)token_topk_kernel, TK_SMEM, d4);
     if (e != cudaSuccess) return e;
     (void)ws;
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map;
-    const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size)};
-    const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kID, (cuuint32_t)kBlk};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
     TokenArgs a{};
     a.cache = cache;
     a.q_idx = q_idx;
@@ -1272,7 +1237,7 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.topk = topk;
     a.page_shift = page_shift_of(cache);
     LaunchCfg c(dim3((unsigned)n * TK_CL), dim3(TK_THREADS), TK_SMEM, stream);
-    return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, map, a);
+    return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, a);
 }
 
 cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
