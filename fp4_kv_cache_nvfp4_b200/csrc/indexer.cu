@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
     // l & 7 of row 4 k + l / 8, so one instruction covers 512 contiguous bytes
     // of a page) and scores them itself.  Warps therefore never wait for one
     // another inside a sequence.  Each lane loads the physical page of its own
-    // row one tile before the copy needs it.
+    // row of every tile.
     const int sh = a.page_shift;
     const int32_t emask = (1 << sh) - 1;
     const uint8_t* pooled = reinterpret_cast<const uint8_t*>(a.cache.idx_k_pooled);
@@ -436,13 +436,18 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
         }
         cp_async_commit();
     };
+    // pages of tiles i + 2 and i + 3 are in registers while tile i is scored:
+    // a page load waits behind the copies already in flight, so it is issued
+    // two tiles before its copies
+    RowPage next0, next1;
     {
         const RowPage r0 = fetch(t0);
         const RowPage r1 = ntiles > 1 ? fetch(t0 + 1) : RowPage{-1, -1};
+        next0 = ntiles > 2 ? fetch(t0 + 2) : RowPage{-1, -1};
+        next1 = ntiles > 3 ? fetch(t0 + 3) : RowPage{-1, -1};
         issue(0, r0);
         issue(1, r1);  // an empty group when there is no second tile
     }
-    RowPage next = ntiles > 2 ? fetch(t0 + 2) : RowPage{-1, -1};
 
     int cur_b = -1, nloc = 0;
     auto flush = [&](int b, int nt) {
@@ -485,8 +490,9 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
         const int s = i % K2_STAGES;
         __syncwarp();  // every lane has read the slice that is refilled next (tile i - 1's)
         if (i + 2 < ntiles) {
-            issue((i + 2) % K2_STAGES, next);
-            if (i + 3 < ntiles) next = fetch(t + 3);
+            issue((i + 2) % K2_STAGES, next0);
+            next0 = next1;
+            if (i + 4 < ntiles) next1 = fetch(t + 4);
         } else {
             cp_async_commit();  // empty group: the wait below always leaves the two newest
         }
