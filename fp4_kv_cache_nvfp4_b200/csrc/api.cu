@@ -131,10 +131,13 @@ csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* 
                                        idx_out, n, max_len, ws, err_word, st));
 }
 
-csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
-                                    const int32_t* topk_idx, const uint16_t* swa_kv, const int32_t* seq_lens,
-                                    const int32_t* swa_lens, float* out, float* lse, int32_t B, int32_t* err_word,
-                                    void* stream) {
+}  // extern "C"
+
+// pre: what the kernel may read before the preceding kernel completes (kPre*)
+static csa2_status attn_decode(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
+                               const int32_t* topk_idx, const uint16_t* swa_kv, const int32_t* seq_lens,
+                               const int32_t* swa_lens, float* out, float* lse, int32_t B, int32_t* err_word,
+                               void* stream, int pre) {
     csa2_status s = check_desc(desc);
     if (s != CSA2_OK) return s;
     s = check_cache(cache, false, false);
@@ -161,8 +164,17 @@ csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const csa2_kv_c
     a.topk = desc->topk;
     a.window = desc->window;
     a.page_shift = page_shift_of(*cache);
-    a.early = desc->mode == CSA2_MODE_REUSE;
+    a.pre = pre;
     return from_cuda(launch_sparse_attn(a, (cudaStream_t)stream));
+}
+
+extern "C" {
+
+csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
+                                    const int32_t* topk_idx, const uint16_t* swa_kv, const int32_t* seq_lens,
+                                    const int32_t* swa_lens, float* out, float* lse, int32_t B, int32_t* err_word,
+                                    void* stream) {
+    return attn_decode(desc, cache, q, topk_idx, swa_kv, seq_lens, swa_lens, out, lse, B, err_word, stream, 0);
 }
 
 csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
@@ -197,7 +209,7 @@ csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_
     a.swa_start = swa_start;
     a.seq_len_prefill = seq_len;
     a.page_shift = page_shift_of(*cache);
-    a.early = 0;
+    a.pre = 0;
     return from_cuda(launch_sparse_attn(a, (cudaStream_t)stream));
 }
 
@@ -240,8 +252,11 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
             cur = set;
         }
         if (s != CSA2_OK) return s;
-        s = csa2_sparse_attn_decode(&d, cache, q[l], cur, swa_kv[l], seq_lens, swa_lens, out[l], lse[l], B,
-                                    err_word, stream);
+        // Not the call's first kernel: q, the SWA rows, the lengths and the
+        // cache were complete before that kernel passed its wait, and a Reuse
+        // layer's index set was written two or more launches back.
+        s = attn_decode(&d, cache, q[l], cur, swa_kv[l], seq_lens, swa_lens, out[l], lse[l], B, err_word, stream,
+                        kPreInputs | (d.mode == CSA2_MODE_REUSE ? kPreIdx : 0));
         if (s != CSA2_OK) return s;
     }
     return CSA2_OK;

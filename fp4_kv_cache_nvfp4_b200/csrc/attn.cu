@@ -93,18 +93,39 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     int* valid = reinterpret_cast<int*>(smem + ATT_OFF_VALID) + warp * KPW;
     uint8_t* vt = smem + ATT_OFF_VT + warp * KPW * VT_ROW;
 
-    // A Reuse layer's index set, the cache and the SWA history come from kernels
-    // at least two launches back, so they are gathered before waiting on the
-    // preceding kernel; the query and the newest SWA row are read after it.
-    // every buffer offset below assumes a 16-byte-aligned dynamic shared base;
-    // the check is uniform over the grid, so no CTA waits on one that left
+    // Inputs written before the launch sequence began (a.pre) are read before
+    // waiting on the preceding kernel, so their latency overlaps its tail.
+    // Every buffer offset below assumes a 16-byte-aligned dynamic shared base;
+    // the check is uniform over the grid, so no CTA waits on one that left.
     if (smem_u32(smem) & 15u) {
         pdl_wait();
         if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
-    const bool early = a.early != 0;
-    if (!early) pdl_wait();
+    const bool pre_idx = (a.pre & kPreIdx) != 0, pre_in = (a.pre & kPreInputs) != 0;
+    bool waited = false;
+    auto wait_once = [&]() {
+        if (!waited) {
+            pdl_wait();
+            waited = true;
+        }
+    };
+    if (!pre_idx && !pre_in) wait_once();
+
+    // Q (A operand rows: heads g and g + 8, bf16 pairs) of this row
+    uint32_t qraw[8][4];
+    auto load_q = [&]() {
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
+        const uint32_t* qg8 = qg + 8 * kD / 2;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            qraw[c][0] = __ldg(qg + 8 * c + t);
+            qraw[c][1] = __ldg(qg8 + 8 * c + t);
+            qraw[c][2] = __ldg(qg + 8 * c + 4 + t);
+            qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
+        }
+    };
+    if (pre_in) load_q();
 
     // ---- sequence, window --------------------------------------------------
     const int seq = prefill ? 0 : row;
@@ -121,7 +142,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         swa_base = a.swa + (int64_t)row * a.window * kCh;
         n_swa = a.swa_lens ? a.swa_lens[row] : (L < a.window ? L : a.window);
         n_swa = max(0, min(n_swa, a.window));
-        if (early && L > 0) newest = (L - 1) % a.window;
+        if (pre_idx && !pre_in && L > 0) newest = (L - 1) % a.window;  // the newest row waits
     }
 
     // ---- gather this warp's 16 keys into shared memory ---------------------
@@ -129,6 +150,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     uint8_t* st_swa = smem + ATT_OFF_SWA;
     const int k0 = warp < 4 ? split * 64 + warp * KPW : split * KPW;
     if (warp < 4) {
+        if (!pre_idx) wait_once();  // the index set comes from the preceding kernel
         int64_t slot = -1;
         if (lane < KPW) {
             const int kidx = k0 + lane;
@@ -173,8 +195,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     cp_async_commit();
 
     // B fragments of S = Q K^T (fp16) for the warp's two n8 tiles of keys, and
-    // the fp16 V tile [key][dim] in shared memory.  In a Reuse layer the four
-    // selected-key warps build both before waiting on the preceding kernel.
+    // the fp16 V tile [key][dim] in shared memory.
     uint32_t bk[2][8][2];
     auto build_kv = [&]() {
         const int key = lane >> 1, half = lane & 1;
@@ -219,41 +240,22 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
                                                                     bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
         }
     };
-    if (early) {
-        if (warp < 4) {
-            cp_async_wait<0>();
-            __syncwarp();
-            build_kv();
-            pdl_wait();
-        } else {
-            pdl_wait();
-            if (newest >= k0 && newest < k0 + KPW && newest < n_swa)
-                cp_async16(st_swa + (newest - k0) * SWA_ROW + lane * 16, swa_base + (int64_t)newest * kCh + lane * 8);
-            cp_async_commit();
-            cp_async_wait<0>();
-            __syncwarp();
-            build_kv();
-        }
-    } else {
-        cp_async_wait<0>();
-        __syncwarp();
-        build_kv();
+    if (warp == 4 && newest >= 0) {  // the newest window row is read after the wait
+        wait_once();
+        if (newest >= k0 && newest < k0 + KPW && newest < n_swa)
+            cp_async16(st_swa + (newest - k0) * SWA_ROW + lane * 16, swa_base + (int64_t)newest * kCh + lane * 8);
+        cp_async_commit();
     }
+    cp_async_wait<0>();
+    __syncwarp();
+    build_kv();
+    wait_once();  // every thread has waited before anything is written
     pdl_trigger();
+    if (!pre_in) load_q();
 
-    // ---- Q fragments (A operand, 16 heads x 128 dims, fp16) and S = Q K^T ---
+    // ---- S = Q K^T (A operand: 16 heads x 128 dims, fp16) -------------------
     float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     {
-        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
-        const uint32_t* qg8 = qg + 8 * kD / 2;
-        uint32_t qraw[8][4];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            qraw[c][0] = __ldg(qg + 8 * c + t);
-            qraw[c][1] = __ldg(qg8 + 8 * c + t);
-            qraw[c][2] = __ldg(qg + 8 * c + 4 + t);
-            qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
-        }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const uint32_t qa[4] = {bf2_to_h2(qraw[c][0]), bf2_to_h2(qraw[c][1]), bf2_to_h2(qraw[c][2]),

@@ -87,8 +87,14 @@ struct AttnArgs {
     int32_t* err;
     int rows, topk, window, swa_start, seq_len_prefill;
     int page_shift;
-    int early;  // 1: index set, cache and SWA history may be read before the preceding kernel completes
+    // What the kernel may read before the preceding kernel in the stream has
+    // completed (programmatic dependent launch).  Nothing is written before the
+    // wait.  kPreIdx: the index set and the cache; kPreInputs: q, the lengths
+    // and every SWA row.
+    int pre;
 };
+constexpr int kPreIdx = 1;
+constexpr int kPreInputs = 2;
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace csa2

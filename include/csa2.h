@@ -28,7 +28,8 @@
  *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and may be captured in a CUDA graph;
  *   - kernels are launched with programmatic dependent launch: each waits for
- *     the preceding kernel in the stream before touching memory;
+ *     the preceding kernel in the stream before touching memory (inside
+ *     csa2_decode_layers, see there);
  *   - host-side checks return a status and launch nothing; errors found on the
  *     device (a slot, page or index out of range) never fault: the access is
  *     skipped and a CSA2_DEV_* bit is OR-ed into *err_word (if non-NULL),
@@ -209,7 +210,12 @@ CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const
  * device pointers, one per layer: q_idx[l], w[l] (read for Full/Reindex
  * layers only), q[l], swa_kv[l], out[l], lse[l].  cand_blocks
  * [B][keep_blocks] and idx_sets [n_layers][B][topk] are device outputs; a
- * Reuse layer writes no set and reads the latest one.  Layer 0 must be Full. */
+ * Reuse layer writes no set and reads the latest one.  Layer 0 must be Full.
+ * Every input (q_idx, w, q, swa_kv, seq_lens, swa_lens, the cache) must be
+ * complete in stream order before the call, as usual; the attention kernels
+ * of the call rely on it and read them (and a Reuse layer's index set) before
+ * the preceding kernel of the call has finished, so no other stream may write
+ * them while the call runs. */
 CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, const csa2_kv_cache* cache,
                                const uint16_t* const* q_idx, const float* const* w, const uint16_t* const* q,
                                const uint16_t* const* swa_kv, const int32_t* seq_lens, const int32_t* swa_lens,
