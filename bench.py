@@ -77,6 +77,18 @@ def unique_bytes_per_seq(L: int, layers: int = 20) -> dict:
                 total=blk + tok + kv + swa + append + q + out)
 
 
+def attn_bytes_per_row(L: int) -> int:
+    """Algorithmic bytes of one decode row (sequence) of one attention launch:
+    the selected FP4 entries, the SWA window, q, the index set, out and lse."""
+    return min(512, L) * 144 + min(128, L) * 512 + 16 * 128 * 2 + 512 * 4 + 16 * 128 * 4 + 16 * 4
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one sparse_attn_kernel launch
+# (ncu --set full, first Full and Reuse launches of the eager step; the kernel
+# source has not changed since), keyed by (B, L)
+ATTN_TRAFFIC = {(8, 1 << 20): 1945088}
+
+
 class ClockSampler:
     def __init__(self, index: int):
         self.index = index
@@ -254,18 +266,29 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         total_ms = max_over_ranks(sum(step_ms), world, dev)
         ms_per_step = total_ms / args.steps
 
-        # ---- dominant kernel: block-level indexer (block scoring + select) ----
-        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.kernel_reps)]
-        with torch.cuda.stream(stream):
-            for k in range(args.kernel_reps):
-                flush.fill_(k & 0xFF)
-                kev[k][0].record(stream)
-                csa2.indexer_topk(descs[0], cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens, cand, B, L, ws,
-                                  err=err, stream=stream)
-                kev[k][1].record(stream)
-        torch.cuda.synchronize()
-        k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+        # ---- per-kernel rooflines: each launch timed alone between CUDA events,
+        # after an untimed L2 flush, on the stream it is launched on ------------
+        def time_launches(fn):
+            ev_ = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.kernel_reps)]
+            with torch.cuda.stream(stream):
+                for k in range(args.kernel_reps):
+                    flush.fill_(k & 0xFF)
+                    ev_[k][0].record(stream)
+                    fn()
+                    ev_[k][1].record(stream)
+            torch.cuda.synchronize()
+            return statistics.mean(a.elapsed_time(b) for a, b in ev_)
+
+        # dominant kernel by share of the step: sparse attention (20 launches a
+        # step); a Reuse layer's launch on the Full layer's index set
+        reuse = next(l for l, m in enumerate(modes) if m == csa2.REUSE)
+        a_ms = time_launches(lambda: csa2.sparse_attn_decode(descs[reuse], cache, q_all[reuse], sets[0], swa[reuse],
+                                                             seq_lens, outs[reuse], lses[reuse], B, err=err,
+                                                             stream=stream))
+        # largest single HBM stream: the block-level indexer (scoring + select)
+        k_ms = time_launches(lambda: csa2.indexer_topk(descs[0], cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens,
+                                                       cand, B, L, ws, err=err, stream=stream))
 
         # ---- end to end: pinned host inputs -> device, step, result -> host ----
         host_in = torch.empty(step_in.numel(), dtype=torch.uint8, pin_memory=True)
@@ -308,6 +331,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     hbm = peaks.get("hbm_gbs")
     k_bytes = B * ((L + 7) // 8) * 128
     k_gbs = k_bytes / (k_ms * 1e-3) / 1e9
+    a_bytes = B * attn_bytes_per_row(L)
+    a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
+    peak_src = "MEASURED_PEAKS.json hbm_gbs (measured, burst copy)" if hbm else "fallback 6650 GB/s"
     res = dict(metric=METRIC, value=whole_job_tokens_per_s(B, world, ms_per_step), unit=UNIT, n_gpus=world,
                steps=args.steps,
                warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
@@ -319,10 +345,14 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                            graph="one CUDA graph per step, programmatic dependent launch between kernels"),
                step_bytes_unique=B * ub["total"], step_gbs=B * ub["total"] / (ms_per_step * 1e-3) / 1e9,
                step_frac_of_hbm=(B * ub["total"] / (ms_per_step * 1e-3) / 1e9) / hbm if hbm else None,
-               roofline=dict(kernel="block-level indexer (block_score_kernel + block_select_kernel)", bound="hbm",
-                             achieved=k_gbs, peak=hbm, unit="GB/s", frac=k_gbs / hbm if hbm else None,
-                             traffic=None, bytes_per_launch=k_bytes, ms_per_launch=k_ms,
-                             peak_source="MEASURED_PEAKS.json hbm_gbs (measured)" if hbm else "fallback 6650"),
+               roofline=dict(kernel="sparse_attn_kernel (Reuse layer, B rows x 8 CTAs)", bound="hbm",
+                             achieved=a_gbs, peak=hbm, unit="GB/s", frac=a_gbs / hbm if hbm else None,
+                             traffic=ATTN_TRAFFIC.get((B, L)), bytes_per_launch=a_bytes, ms_per_launch=a_ms,
+                             peak_source=peak_src),
+               roofline_block_indexer=dict(kernel="block_score_kernel + block_select_kernel", bound="hbm",
+                                           achieved=k_gbs, peak=hbm, unit="GB/s",
+                                           frac=k_gbs / hbm if hbm else None, traffic=None,
+                                           bytes_per_launch=k_bytes, ms_per_launch=k_ms, peak_source=peak_src),
                e2e=dict(value=whole_job_tokens_per_s(B, world, max_over_ranks(e2e_ms, world, dev)), unit=UNIT,
                         h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                         ms_per_step=e2e_ms),
