@@ -81,6 +81,40 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// --- mbarriers (CTA scope) -------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued before has
+// landed (the barrier's expected count includes it).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Wait for the phase with the given parity; gives up after `limit` polls and
+// returns false (the caller records a timeout instead of hanging).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// Barrier over the first n threads of the block (named barrier `id`); id 0
+// with n = blockDim.x is the whole block.
+struct GroupBar {
+    int id, n;
+    __device__ __forceinline__ void sync() const { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+};
+
 // --- distributed shared memory (thread-block clusters) -----------------------------
 // Address of `local_addr` (a shared-memory address of this CTA) in the CTA of
 // the cluster with the given rank.
@@ -167,42 +201,46 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
     return v;
 }
 
-// Exclusive scan of one value per thread over the whole block (blockDim a
-// multiple of 32, <= 1024).  `tmp` holds >= 33 words of shared memory.
-// Returns the exclusive prefix; *total receives the block sum.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
-    int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Exclusive scan of one value per thread over the group's threads (a multiple
+// of 32, <= 1024; thread index = threadIdx.x).  `tmp` holds >= 33 words of
+// shared memory.  Returns the exclusive prefix; *total receives the sum.
+__device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total, GroupBar g) {
+    int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = g.n >> 5;
     uint32_t inc = warp_incl_scan(v);
     if (lane == 31) tmp[wid] = inc;
-    __syncthreads();
+    g.sync();
     if (wid == 0) {
         uint32_t s = lane < nw ? tmp[lane] : 0u;
         uint32_t si = warp_incl_scan(s);
         if (lane < nw) tmp[lane] = si - s;
         if (lane == 31) tmp[32] = si;
     }
-    __syncthreads();
+    g.sync();
     uint32_t r = tmp[wid] + inc - v;
     *total = tmp[32];
-    __syncthreads();
+    g.sync();
     return r;
+}
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+    return group_excl_scan(v, tmp, total, GroupBar{0, (int)blockDim.x});
 }
 
 // Given a histogram `hist[nbins]` in shared memory (descending rank = from the
 // top bin down) find the bin holding the k-th largest item (1-based k <= total):
-// *bin_out = that bin, *above_out = items in higher bins.  Whole block calls.
-__device__ __forceinline__ void find_kth_bin(const uint32_t* hist, int nbins, uint32_t k, uint32_t* tmp,
-                                             int* bin_out, uint32_t* above_out) {
+// *bin_out = that bin, *above_out = items in higher bins.  Every thread of the
+// group calls.
+__device__ __forceinline__ void group_find_kth_bin(const uint32_t* hist, int nbins, uint32_t k, uint32_t* tmp,
+                                                   int* bin_out, uint32_t* above_out, GroupBar g) {
     // each thread owns a contiguous run of bins counted from the top
-    int per = (nbins + blockDim.x - 1) / blockDim.x;
-    int hi = nbins - 1 - threadIdx.x * per;  // first (highest) bin of this thread
+    int per = (nbins + g.n - 1) / g.n;
+    int hi = nbins - 1 - (int)threadIdx.x * per;  // first (highest) bin of this thread
     uint32_t mine = 0;
     for (int i = 0; i < per; ++i) {
         int b = hi - i;
         if (b >= 0) mine += hist[b];
     }
     uint32_t total;
-    uint32_t before = block_excl_scan(mine, tmp, &total);
+    uint32_t before = group_excl_scan(mine, tmp, &total, g);
     if (before < k && before + mine >= k) {
         uint32_t acc = before;
         for (int i = 0; i < per; ++i) {
@@ -216,10 +254,14 @@ __device__ __forceinline__ void find_kth_bin(const uint32_t* hist, int nbins, ui
             acc += hist[b];
         }
     }
-    __syncthreads();
+    g.sync();
     *bin_out = (int)tmp[40];
     *above_out = tmp[41];
-    __syncthreads();
+    g.sync();
+}
+__device__ __forceinline__ void find_kth_bin(const uint32_t* hist, int nbins, uint32_t k, uint32_t* tmp,
+                                             int* bin_out, uint32_t* above_out) {
+    group_find_kth_bin(hist, nbins, k, tmp, bin_out, above_out, GroupBar{0, (int)blockDim.x});
 }
 
 }  // namespace csa2

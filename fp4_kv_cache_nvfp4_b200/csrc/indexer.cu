@@ -290,25 +290,35 @@ __device__ __forceinline__ void stage_pages(const csa2_kv_cache& c, int shift, i
 //
 // Persistent: one CTA per SM walks a contiguous range of the flattened list of
 // 512-row tiles of every sequence that needs block selection, so a ragged batch
-// balances across the SMs.  A 3-stage ring of 64 KiB tiles is filled by 2-D
-// bulk tensor copies (one box = the pooled rows of one page run, 128B swizzle:
-// chunk c of row r lands at chunk c ^ (r & 7), the layout read_row expects);
-// warp 0 runs two tiles ahead.  Each of the 512 threads scores one row.
+// balances across the SMs.  Warp-specialised around a 3-stage ring of 64 KiB
+// tiles: four producer warps only copy (16-byte cp.async; lane l moves chunk
+// l & 7 of row 4 k + l / 8, so one instruction covers 512 contiguous bytes of a
+// page; chunk c of row r lands at chunk c ^ (r & 7)) and signal a stage full
+// through an mbarrier once their copies land; eight consumer warps only score
+// (lane l takes rows l and l + 32 of its warp's 64: eight independent FMA
+// chains) and release the stage through a second mbarrier.  Copies and FMAs
+// therefore overlap instead of taking turns.
 // ============================================================================
-constexpr int K2_THREADS = 512;
-constexpr int K2_TILE = 512;                    // pooled rows per tile (one per thread)
+constexpr int K2_CWARPS = 8;                    // consumer (scoring) warps
+constexpr int K2_PWARPS = 4;                    // producer (copy) warps
+constexpr int K2_CTHREADS = K2_CWARPS * 32;
+constexpr int K2_THREADS = (K2_CWARPS + K2_PWARPS) * 32;
+constexpr int K2_TILE = 512;                    // pooled rows per tile
 constexpr int K2_STAGES = 3;
 constexpr size_t K2_STAGE_BYTES = (size_t)K2_TILE * 128;
 constexpr int K2_MAX_SEQS = 1024;
+constexpr int K2_PROWS = K2_TILE / K2_PWARPS;   // 128 rows copied per producer warp
+constexpr int K2_CROWS = K2_TILE / K2_CWARPS;   // 64 rows scored per consumer warp
 constexpr size_t K2_OFF_HIST = K2_STAGES * K2_STAGE_BYTES;
 constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
 constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
 constexpr size_t K2_OFF_NBLK = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
-constexpr size_t K2_OFF_MISC = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // w (float4), last
+constexpr size_t K2_OFF_BAR = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // full[3], empty[3]
+constexpr size_t K2_OFF_MISC = align16(K2_OFF_BAR + 2 * K2_STAGES * 8);  // w (float4), last, timeout
 constexpr size_t K2_SMEM = align16(K2_OFF_MISC + 32);
-constexpr size_t K2_SLICE = 32 * 128;  // one warp's 32 rows of a stage
-static_assert(K2_OFF_QD % 16 == 0 && K2_OFF_MISC % 16 == 0, "K2 shared-memory layout");
+constexpr uint32_t kWaitLimit = 1u << 22;
+static_assert(K2_OFF_QD % 16 == 0 && K2_OFF_BAR % 8 == 0 && K2_OFF_MISC % 16 == 0, "K2 shared-memory layout");
 
 struct BlockArgs {
     csa2_kv_cache cache;
@@ -340,15 +350,18 @@ __device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int n, int
     return lo;
 }
 
-__global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
+__global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K2_OFF_HIST);
     float4* qd = reinterpret_cast<float4*>(smem + K2_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + K2_OFF_TMP);
     int32_t* tile_start = reinterpret_cast<int32_t*>(smem + K2_OFF_TS);
     int32_t* s_nblk = reinterpret_cast<int32_t*>(smem + K2_OFF_NBLK);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K2_OFF_BAR);
+    uint64_t* empty = full + K2_STAGES;
     float4& s_w = *reinterpret_cast<float4*>(smem + K2_OFF_MISC);
     int& s_last = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 16);
+    int& s_timeout = *reinterpret_cast<int*>(smem + K2_OFF_MISC + 20);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     pdl_wait();
@@ -382,7 +395,14 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
                 base += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
             }
         }
-        if (tid == 0) tile_start[a.n] = (int32_t)total;
+        if (tid == 0) {
+            tile_start[a.n] = (int32_t)total;
+            for (int s = 0; s < K2_STAGES; ++s) {
+                mbar_init(&full[s], K2_PWARPS * 32);  // one cp.async arrival per producer thread
+                mbar_init(&empty[s], K2_CWARPS);      // one arrival per consumer warp
+            }
+            s_timeout = 0;
+        }
         for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
         __syncthreads();
     }
@@ -392,131 +412,138 @@ __global__ void __launch_bounds__(K2_THREADS) block_score_kernel(BlockArgs a) {
     const int ntiles = t1 - t0;
     if (ntiles <= 0) return;
 
-    // Warp w owns rows [32 w, 32 w + 32) of every tile: it copies them into its
-    // own slice of the 3-stage ring with 16-byte cp.async (lane l moves chunk
-    // l & 7 of row 4 k + l / 8, so one instruction covers 512 contiguous bytes
-    // of a page) and scores them itself.  Warps therefore never wait for one
-    // another inside a sequence.  Each lane loads the physical page of its own
-    // row of every tile.
-    const int sh = a.page_shift;
-    const int32_t emask = (1 << sh) - 1;
-    const uint8_t* pooled = reinterpret_cast<const uint8_t*>(a.cache.idx_k_pooled);
-    const int32_t mpps = a.cache.max_pages_per_seq;
-    struct RowPage {
-        int32_t j;     // row (block) index within its sequence; -1: past the end
-        int32_t phys;  // physical page of the row's entries
-    };
-    auto fetch = [&](int32_t t) {
-        const int b = seq_of_tile(tile_start, a.n, t);
-        RowPage r;
-        r.j = (t - tile_start[b]) * K2_TILE + 32 * wid + lane;
-        const int32_t pg = (r.j * kBlk) >> sh;
-        const bool in = r.j < s_nblk[b];
-        r.phys = (in && pg < mpps) ? __ldg(a.cache.page_table + (int64_t)b * mpps + pg) : -1;
-        if (!in) r.j = -1;
-        return r;
-    };
-    auto issue = [&](int s, RowPage r) {
-        int32_t prow = -1;
-        if (r.j >= 0) {
-            int32_t phys = r.phys;
-            if (phys < 0 || phys >= a.cache.n_phys_pages) {
-                dev_error(a.err, CSA2_DEV_PAGE);
-                phys = 0;  // results of this call are undefined; the copy stays in bounds
-            }
-            prow = (int32_t)((((int64_t)phys << sh) | ((r.j * kBlk) & emask)) >> 3);
-        }
-        uint8_t* slice = smem + (size_t)s * K2_STAGE_BYTES + (size_t)wid * K2_SLICE;
-        const int c = lane & 7;
+    if (wid >= K2_CWARPS) {
+        // ================= producers =================
+        const int pw = wid - K2_CWARPS;
+        const int sh = a.page_shift;
+        const int32_t emask = (1 << sh) - 1;
+        const uint8_t* pooled = reinterpret_cast<const uint8_t*>(a.cache.idx_k_pooled);
+        const int32_t mpps = a.cache.max_pages_per_seq;
+        // rows pw*128 + 32 h + lane of tile t: row index within the sequence
+        // (-1 past its end) and physical page, loaded one tile ahead
+        int32_t pj[4], pp[4];
+        auto fetch = [&](int32_t t) {
+            const int b = seq_of_tile(tile_start, a.n, t);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int rr = 4 * k + (lane >> 3);
-            const int32_t pr = __shfl_sync(0xffffffffu, prow, rr);
-            if (pr >= 0) cp_async16(slice + rr * 128 + ((c ^ (rr & 7)) << 4), pooled + (int64_t)pr * 128 + c * 16);
+            for (int h = 0; h < 4; ++h) {
+                const int32_t j = (t - tile_start[b]) * K2_TILE + K2_PROWS * pw + 32 * h + lane;
+                const int32_t pg = (j * kBlk) >> sh;
+                const bool in = j < s_nblk[b];
+                pp[h] = (in && pg < mpps) ? __ldg(a.cache.page_table + (int64_t)b * mpps + pg) : -1;
+                pj[h] = in ? j : -1;
+            }
+        };
+        fetch(t0);
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % K2_STAGES;
+            if (i >= K2_STAGES && !mbar_wait(&empty[s], (uint32_t)((i / K2_STAGES) - 1) & 1u, kWaitLimit))
+                s_timeout = 1;
+            int32_t prow[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                prow[h] = -1;
+                if (pj[h] >= 0) {
+                    int32_t phys = pp[h];
+                    if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                        dev_error(a.err, CSA2_DEV_PAGE);
+                        phys = 0;  // results of this call are undefined; the copy stays in bounds
+                    }
+                    prow[h] = (int32_t)((((int64_t)phys << sh) | ((pj[h] * kBlk) & emask)) >> 3);
+                }
+            }
+            if (i + 1 < ntiles) fetch(t0 + i + 1);  // loads overlap the copies below
+            uint8_t* dst0 = smem + (size_t)s * K2_STAGE_BYTES + (size_t)pw * K2_PROWS * 128;
+            const int c = lane & 7;
+#pragma unroll
+            for (int k = 0; k < K2_PROWS / 4; ++k) {
+                const int rr = 4 * k + (lane >> 3);  // register h = k / 8 of lane rr & 31 holds its page
+                const int32_t v = k < 8 ? prow[0] : k < 16 ? prow[1] : k < 24 ? prow[2] : prow[3];
+                const int32_t pr = __shfl_sync(0xffffffffu, v, rr & 31);
+                if (pr >= 0)
+                    cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), pooled + (int64_t)pr * 128 + c * 16);
+            }
+            cp_async_mbar_arrive(&full[s]);
         }
-        cp_async_commit();
-    };
-    // pages of tiles i + 2 and i + 3 are in registers while tile i is scored:
-    // a page load waits behind the copies already in flight, so it is issued
-    // two tiles before its copies
-    RowPage next0, next1;
-    {
-        const RowPage r0 = fetch(t0);
-        const RowPage r1 = ntiles > 1 ? fetch(t0 + 1) : RowPage{-1, -1};
-        next0 = ntiles > 2 ? fetch(t0 + 2) : RowPage{-1, -1};
-        next1 = ntiles > 3 ? fetch(t0 + 3) : RowPage{-1, -1};
-        issue(0, r0);
-        issue(1, r1);  // an empty group when there is no second tile
+        cp_async_wait<0>();  // every copy has landed before this thread leaves
+        if (s_timeout && lane == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
     }
 
+    // ================= consumers =================
+    const GroupBar cg{1, K2_CTHREADS};
     int cur_b = -1, nloc = 0;
     auto flush = [&](int b, int nt) {
-        __syncthreads();
+        cg.sync();
         uint32_t* gh = a.hist + (int64_t)b * kHistBins;
-        for (int i = tid; i < kHistBins; i += K2_THREADS) {
+        for (int i = tid; i < kHistBins; i += K2_CTHREADS) {
             const uint32_t v = hist[i];
             if (v) atomicAdd(&gh[i], v);
             hist[i] = 0;
         }
         __threadfence();
-        __syncthreads();
+        cg.sync();
         if (tid == 0) {
             const int32_t nblk = s_nblk[b];
             const uint32_t need_t = (uint32_t)((nblk + K2_TILE - 1) / K2_TILE);
             s_last = atomicAdd(&a.ctr[2 * b], (uint32_t)nt) + (uint32_t)nt == need_t;
         }
-        __syncthreads();
+        cg.sync();
         if (s_last) {  // the sequence's last tile is done: find the bin of the keep-th score
             __threadfence();
-            load_words(hist, gh, kHistBins);
-            __syncthreads();
-            for (int i = tid; i < kHistBins / 4; i += K2_THREADS)
+            for (int i = tid; i < kHistBins / 4; i += K2_CTHREADS)
+                reinterpret_cast<uint4*>(hist)[i] = __ldcg(reinterpret_cast<const uint4*>(gh) + i);
+            cg.sync();
+            for (int i = tid; i < kHistBins / 4; i += K2_CTHREADS)
                 reinterpret_cast<uint4*>(gh)[i] = make_uint4(0, 0, 0, 0);
             int bin;
             uint32_t above;
-            find_kth_bin(hist, kHistBins, (uint32_t)a.keep, tmp, &bin, &above);
+            group_find_kth_bin(hist, kHistBins, (uint32_t)a.keep, tmp, &bin, &above, cg);
             if (tid == 0) {
                 a.thr[4 * b] = bin;
                 a.thr[4 * b + 1] = (int32_t)above;
                 a.ctr[2 * b] = 0;
             }
-            for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
-            __syncthreads();
+            for (int i = tid; i < kHistBins; i += K2_CTHREADS) hist[i] = 0;
+            cg.sync();
         }
     };
 
     for (int i = 0; i < ntiles; ++i) {
         const int32_t t = t0 + i;
         const int s = i % K2_STAGES;
-        __syncwarp();  // every lane has read the slice that is refilled next (tile i - 1's)
-        if (i + 2 < ntiles) {
-            issue((i + 2) % K2_STAGES, next0);
-            next0 = next1;
-            if (i + 4 < ntiles) next1 = fetch(t + 4);
-        } else {
-            cp_async_commit();  // empty group: the wait below always leaves the two newest
-        }
         const int b = seq_of_tile(tile_start, a.n, t);
         if (b != cur_b) {
             if (cur_b >= 0) flush(cur_b, nloc);
-            load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
+            const uint16_t* qb = a.q_idx + (int64_t)b * kIH * kID;
+            for (int d = tid; d < kID; d += K2_CTHREADS)
+                qd[d] = make_float4(bf16_bits_to_f32(qb[d]), bf16_bits_to_f32(qb[kID + d]),
+                                    bf16_bits_to_f32(qb[2 * kID + d]), bf16_bits_to_f32(qb[3 * kID + d]));
             if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
             cur_b = b;
             nloc = 0;
-            __syncthreads();
+            cg.sync();
         }
-        const int32_t j = (t - tile_start[b]) * K2_TILE + 32 * wid + lane;
-        cp_async_wait<2>();
-        __syncwarp();  // the other lanes' copies of this warp's rows are visible
-        uint32_t k[32];
-        read_row(smem + (size_t)s * K2_STAGE_BYTES + (size_t)wid * K2_SLICE, lane, k);
-        const float s0 = idx_score1(k, qd, s_w);
-        const bool act = j < s_nblk[b];
-        if (act) a.scores[(int64_t)b * a.nblk_pad + j] = s0;
-        hist_add(hist, score_key(s0) >> 20, act);
+        if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, kWaitLimit)) s_timeout = 1;
+        const uint8_t* stage = smem + (size_t)s * K2_STAGE_BYTES;
+        const int r0 = K2_CROWS * wid + lane;  // rows r0 and r0 + 32 of the tile
+        uint32_t k[32], m[32];
+        read_row(stage, r0, k);
+        read_row(stage, r0 + 32, m);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // the stage's rows of this warp are in registers
+        float s0, s1;
+        idx_score2(k, m, qd, s_w, s0, s1);
+        const int32_t j = (t - tile_start[b]) * K2_TILE + r0;
+        const int32_t nblk = s_nblk[b];
+        float* sc = a.scores + (int64_t)b * a.nblk_pad;
+        if (j < nblk) sc[j] = s0;
+        if (j + 32 < nblk) sc[j + 32] = s1;
+        hist_add(hist, score_key(s0) >> 20, j < nblk);
+        hist_add(hist, score_key(s1) >> 20, j + 32 < nblk);
         ++nloc;
     }
     if (cur_b >= 0) flush(cur_b, nloc);
+    if (s_timeout && tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
 }
 
 // ============================================================================
