@@ -95,10 +95,15 @@ size_t csa2_indexer_workspace_bytes(const csa2_layer_desc* desc, int32_t level, 
     return decode_ws_layout(n, max_len).total;
 }
 
-csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
-                              const uint16_t* q_idx, const float* w, const int32_t* seq_lens, const int32_t* q_pos,
-                              const int32_t* cand_blocks, int32_t* idx_out, float* score_out, int32_t n,
-                              int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word, void* stream) {
+}  // extern "C"
+
+// pre: the token level may read cand_blocks, the lengths and the cache before
+// the preceding kernel completes (a Reindex layer inside the decode driver)
+static csa2_status indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
+                                const uint16_t* q_idx, const float* w, const int32_t* seq_lens, const int32_t* q_pos,
+                                const int32_t* cand_blocks, int32_t* idx_out, float* score_out, int32_t n,
+                                int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word, void* stream,
+                                int pre) {
     csa2_status s = check_desc(desc);
     if (s != CSA2_OK) return s;
     if (desc->mode == CSA2_MODE_REUSE) return CSA2_ERR_INVALID_ARG;
@@ -128,7 +133,17 @@ csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* 
         return from_cuda(launch_block_topk(*cache, q_idx, w, seq_lens, desc->keep_blocks, idx_out, n, max_len, ws,
                                            err_word, st));
     return from_cuda(launch_token_topk(*cache, q_idx, w, seq_lens, cand_blocks, desc->keep_blocks, desc->topk,
-                                       idx_out, n, max_len, ws, err_word, st));
+                                       idx_out, n, max_len, ws, err_word, st, pre));
+}
+
+extern "C" {
+
+csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
+                              const uint16_t* q_idx, const float* w, const int32_t* seq_lens, const int32_t* q_pos,
+                              const int32_t* cand_blocks, int32_t* idx_out, float* score_out, int32_t n,
+                              int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word, void* stream) {
+    return indexer_topk(desc, cache, level, q_idx, w, seq_lens, q_pos, cand_blocks, idx_out, score_out, n, max_len,
+                        workspace, ws_bytes, err_word, stream, 0);
 }
 
 }  // extern "C"
@@ -247,16 +262,17 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
                                       set, nullptr, B, max_len, workspace, ws_bytes, err_word, stream);
             cur = set;
         } else if (d.mode == CSA2_MODE_REINDEX) {
-            s = csa2_indexer_topk(&d, cache, CSA2_LEVEL_TOKEN, q_idx[l], w[l], seq_lens, nullptr, cand_blocks, set,
-                                  nullptr, B, max_len, workspace, ws_bytes, err_word, stream);
+            // the Full layer's candidates were written launches back
+            s = indexer_topk(&d, cache, CSA2_LEVEL_TOKEN, q_idx[l], w[l], seq_lens, nullptr, cand_blocks, set, nullptr,
+                             B, max_len, workspace, ws_bytes, err_word, stream, 1);
             cur = set;
         }
         if (s != CSA2_OK) return s;
-        // Not the call's first kernel: q, the SWA rows, the lengths and the
-        // cache were complete before that kernel passed its wait, and a Reuse
+        // Not the call's first kernel: the cache, the lengths and the SWA
+        // history were complete before that kernel passed its wait, and a Reuse
         // layer's index set was written two or more launches back.
         s = attn_decode(&d, cache, q[l], cur, swa_kv[l], seq_lens, swa_lens, out[l], lse[l], B, err_word, stream,
-                        kPreInputs | (d.mode == CSA2_MODE_REUSE ? kPreIdx : 0));
+                        kPreHist | (d.mode == CSA2_MODE_REUSE ? kPreIdx : 0));
         if (s != CSA2_OK) return s;
     }
     return CSA2_OK;

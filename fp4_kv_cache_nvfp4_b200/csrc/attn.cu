@@ -93,16 +93,18 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     int* valid = reinterpret_cast<int*>(smem + ATT_OFF_VALID) + warp * KPW;
     uint8_t* vt = smem + ATT_OFF_VT + warp * KPW * VT_ROW;
 
-    // Inputs written before the launch sequence began (a.pre) are read before
-    // waiting on the preceding kernel, so their latency overlaps its tail.
-    // Every buffer offset below assumes a 16-byte-aligned dynamic shared base;
-    // the check is uniform over the grid, so no CTA waits on one that left.
+    // Data that exists before the preceding layer finishes (a.pre: an earlier
+    // layer's index set, the cache, the SWA history) is gathered before waiting
+    // on the preceding kernel, so its latency overlaps that kernel's tail; q and
+    // the newest SWA row are read after the wait.  Every buffer offset below
+    // assumes a 16-byte-aligned dynamic shared base; the check is uniform over
+    // the grid, so no CTA waits on one that left.
     if (smem_u32(smem) & 15u) {
         pdl_wait();
         if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
-    const bool pre_idx = (a.pre & kPreIdx) != 0, pre_in = (a.pre & kPreInputs) != 0;
+    const bool pre_idx = (a.pre & kPreIdx) != 0, pre_hist = (a.pre & kPreHist) != 0;
     bool waited = false;
     auto wait_once = [&]() {
         if (!waited) {
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             waited = true;
         }
     };
-    if (!pre_idx && !pre_in) wait_once();
+    if (!pre_idx && !pre_hist) wait_once();
 
     // Q (A operand rows: heads g and g + 8, bf16 pairs) of this row
     uint32_t qraw[8][4];
@@ -125,7 +127,6 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
         }
     };
-    if (pre_in) load_q();
 
     // ---- sequence, window --------------------------------------------------
     const int seq = prefill ? 0 : row;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         swa_base = a.swa + (int64_t)row * a.window * kCh;
         n_swa = a.swa_lens ? a.swa_lens[row] : (L < a.window ? L : a.window);
         n_swa = max(0, min(n_swa, a.window));
-        if (pre_idx && !pre_in && L > 0) newest = (L - 1) % a.window;  // the newest row waits
+        if ((pre_idx || pre_hist) && L > 0) newest = (L - 1) % a.window;  // the newest row waits
     }
 
     // ---- gather this warp's 16 keys into shared memory ---------------------
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     build_kv();
     wait_once();  // every thread has waited before anything is written
     pdl_trigger();
-    if (!pre_in) load_q();
+    load_q();
 
     // ---- S = Q K^T (A operand: 16 heads x 128 dims, fp16) -------------------
     float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};

@@ -127,14 +127,12 @@ __device__ __forceinline__ void read_row(const uint8_t* tile, int r, uint32_t (&
 }
 
 // ----------------------------------------------------------------------------
-// Warp-aggregated shared-memory counters.  Every lane of the warp must call.
+// Shared-memory counters.  hist_add: plain shared atomics (on B200 the
+// hardware resolves same-bin collisions faster than a __match_any_sync
+// aggregation).  list_append: warp-aggregated; every lane of the warp calls.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-    const unsigned m = __ballot_sync(0xffffffffu, active);
-    if (active) {
-        const unsigned peers = __match_any_sync(m, bin);
-        if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-    }
+    if (active) atomicAdd(&hist[bin], 1u);
 }
 
 __device__ __forceinline__ void list_append(uint16_t* list, uint32_t* cnt, uint32_t v, bool pred) {
@@ -754,6 +752,7 @@ struct TokenArgs {
     int32_t* err;
     int64_t max_len;
     int keep, topk, page_shift;
+    int pre;  // 1: the lengths, cand and the cache may be read before the preceding kernel completes
 };
 
 // Push this CTA's histogram (nonzero bins only) into the receive histogram of
@@ -790,11 +789,20 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     const int b = blockIdx.x / TK_CL;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
-    pdl_wait();
-    pdl_trigger();
+    // With a.pre (a Reindex layer inside the decode driver: its candidates come
+    // from the Full layer, launches back) the candidates' slots are resolved
+    // and their first rows copied before waiting on the preceding kernel; q_idx
+    // and w, which a model computes from the previous layer's output, are read
+    // after the wait.
+    const bool pre = a.pre != 0;
+    if (!pre) {
+        pdl_wait();
+        pdl_trigger();
+    }
     // 16-byte copies and vector reads need an aligned base; the check is
     // uniform over the grid, so no CTA waits at a cluster barrier for one that left
     if (smem_u32(smem) & 15u) {
+        if (pre) pdl_wait();
         if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
@@ -818,10 +826,6 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
         }
         bpos[k] = sl >= 0 ? p : -1;
         bslot[k] = sl;
-    }
-    load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
-    if (tid == 0) {
-        s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
     }
     for (int i = tid; i < kHistBins; i += TK_THREADS) {
         hist[i] = 0;
@@ -861,6 +865,13 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     };
     issue(0);
     issue(1);
+    if (pre) {
+        pdl_wait();
+        pdl_trigger();
+    }
+    load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
+    if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
+    __syncthreads();  // qd and s_w
     for (int k = 0; k < nrounds; ++k) {
         cp_async_wait<1>();
         __syncwarp();  // the other lanes' copies of this warp's rows are visible
@@ -1252,7 +1263,8 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
 
 cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,
-                              int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream) {
+                              int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream,
+                              int pre) {
     static bool d4[64];
     cudaError_t e = ensure_smem((const void*)token_topk_kernel, TK_SMEM, d4);
     if (e != cudaSuccess) return e;
@@ -1269,6 +1281,7 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.keep = keep;
     a.topk = topk;
     a.page_shift = page_shift_of(cache);
+    a.pre = pre;
     LaunchCfg c(dim3((unsigned)n * TK_CL), dim3(TK_THREADS), TK_SMEM, stream);
     return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, a);
 }

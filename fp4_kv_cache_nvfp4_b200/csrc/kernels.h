@@ -67,7 +67,8 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
 
 cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,
-                              int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream);
+                              int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream,
+                              int pre = 0);
 
 cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                                 const int32_t* seq_lens, const int32_t* q_pos, int ratio, int topk, int32_t* out,
@@ -89,12 +90,14 @@ struct AttnArgs {
     int page_shift;
     // What the kernel may read before the preceding kernel in the stream has
     // completed (programmatic dependent launch).  Nothing is written before the
-    // wait.  kPreIdx: the index set and the cache; kPreInputs: q, the lengths
-    // and every SWA row.
+    // wait, and q and the newest SWA row (which a model computes from the
+    // previous layer's output) are always read after it.  kPreIdx: the index
+    // set and the cache; kPreHist: the lengths and the SWA rows other than the
+    // newest.
     int pre;
 };
 constexpr int kPreIdx = 1;
-constexpr int kPreInputs = 2;
+constexpr int kPreHist = 2;
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace csa2

@@ -211,11 +211,13 @@ CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const
  * layers only), q[l], swa_kv[l], out[l], lse[l].  cand_blocks
  * [B][keep_blocks] and idx_sets [n_layers][B][topk] are device outputs; a
  * Reuse layer writes no set and reads the latest one.  Layer 0 must be Full.
- * Every input (q_idx, w, q, swa_kv, seq_lens, swa_lens, the cache) must be
- * complete in stream order before the call, as usual; the attention kernels
- * of the call rely on it and read them (and a Reuse layer's index set) before
- * the preceding kernel of the call has finished, so no other stream may write
- * them while the call runs. */
+ * Every input must be complete in stream order before the call, as usual.
+ * Kernels of the call after the first read the cache, the lengths, the SWA
+ * rows other than the newest, a Reuse layer's index set and a Reindex layer's
+ * cand_blocks before the preceding kernel of the call has finished (a layer's
+ * q, q_idx, w and newest SWA row only after it, as a model computes them from
+ * the previous layer's output), so no other stream may write them while the
+ * call runs. */
 CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, const csa2_kv_cache* cache,
                                const uint16_t* const* q_idx, const float* const* w, const uint16_t* const* q,
                                const uint16_t* const* swa_kv, const int32_t* seq_lens, const int32_t* swa_lens,
