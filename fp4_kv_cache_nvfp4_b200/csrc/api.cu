@@ -203,7 +203,7 @@ csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_
     if (T < 0 || swa_start < 0 || seq_len < 1) return CSA2_ERR_INVALID_ARG;
     if (T == 0) return CSA2_OK;
     if (!q || !topk_idx || !q_pos || !swa_kv || !out || !lse) return CSA2_ERR_INVALID_ARG;
-    if (!aligned(q, 4) || !aligned(topk_idx, 4) || !aligned(q_pos, 4) || !aligned(swa_kv, 16) || !aligned(out, 4) ||
+    if (!aligned(q, 16) || !aligned(topk_idx, 4) || !aligned(q_pos, 4) || !aligned(swa_kv, 16) || !aligned(out, 16) ||
         !aligned(lse, 4))
         return CSA2_ERR_INVALID_ARG;
     if (err_word && !aligned(err_word, 4)) return CSA2_ERR_INVALID_ARG;

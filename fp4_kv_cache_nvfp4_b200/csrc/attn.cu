@@ -71,6 +71,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -422,6 +428,310 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     }
 }
 
+// ============================================================================
+// Prefill attention: one CTA per query, no cluster.  Warps 0..3 each take 16
+// of the query's selected entries and warp 4 takes 16 window tokens per chunk,
+// for 8 chunks (512 entries + 128 window tokens).  Each warp runs its own
+// double-buffered cp.async pipeline (gather chunk c + 2 while computing chunk
+// c), keeps the query's Q fragments in registers for all chunks, and carries an
+// online softmax (running max, sum and O) across its chunks; the five warps
+// merge once in shared memory at the end.  Work per query is the decode row's,
+// but without the per-query cluster barrier and with Q loaded once.
+// ============================================================================
+constexpr int PA_CHUNKS = 8;
+constexpr size_t PA_STAGE = 4 * KPW * FP4_ROW + KPW * SWA_ROW;  // 4 entry slices + 1 window slice
+constexpr size_t PA_OFF_VT = 2 * PA_STAGE;
+constexpr size_t PA_END_LOOP = PA_OFF_VT + (size_t)ATT_WARPS * KPW * VT_ROW;
+constexpr size_t PA_END_OPART = (size_t)ATT_WARPS * kH * OACC_ROW * 4;  // merge partials reuse the ring
+constexpr int PA_QROW = 272;  // fp16 Q tile row: 256 B + 16 B pad (ldmatrix without bank conflicts)
+constexpr size_t PA_OFF_MS = align16(PA_END_LOOP > PA_END_OPART ? PA_END_LOOP : PA_END_OPART);
+constexpr size_t PA_OFF_LP = PA_OFF_MS + ATT_WARPS * kH * 4;
+constexpr size_t PA_OFF_Q = align16(PA_OFF_LP + ATT_WARPS * kH * 4);          // [16][136] fp16
+constexpr size_t PA_OFF_SLOT = align16(PA_OFF_Q + (size_t)kH * PA_QROW);       // [4 warps][8 chunks][16] int32
+constexpr size_t PA_SMEM = align16(PA_OFF_SLOT + 4 * PA_CHUNKS * KPW * 4);
+static_assert(PA_STAGE % 16 == 0 && PA_OFF_VT % 16 == 0, "prefill attention shared-memory layout");
+
+__global__ void __launch_bounds__(ATT_THREADS, 3) prefill_attn_kernel(AttnArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int row = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    float* opart = reinterpret_cast<float*>(smem);
+    float* ms = reinterpret_cast<float*>(smem + PA_OFF_MS);
+    float* lpart = reinterpret_cast<float*>(smem + PA_OFF_LP);
+    uint8_t* qs = smem + PA_OFF_Q;
+    int32_t* s_slot = reinterpret_cast<int32_t*>(smem + PA_OFF_SLOT) + (warp < 4 ? warp : 0) * PA_CHUNKS * KPW;
+    uint8_t* vt = smem + PA_OFF_VT + warp * KPW * VT_ROW;
+
+    pdl_wait();
+    pdl_trigger();
+    if (smem_u32(smem) & 15u) {  // uniform over the grid
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
+    const int32_t L = a.seq_len_prefill;
+    const int p = a.q_pos[row];
+    const int lo = max(0, p - a.window + 1);
+    const uint16_t* swa_base = a.swa + (int64_t)(lo - a.swa_start) * kCh;
+    const int n_swa = (lo >= a.swa_start) ? p - lo + 1 : 0;
+    if (lo < a.swa_start && tid == 0) dev_error(a.err, CSA2_DEV_INDEX);
+
+    // physical slots of the entry warps' keys, chunk c key r at s_slot[16 c + r]
+    if (warp < 4 && lane < KPW) {
+        int32_t pos[PA_CHUNKS];
+#pragma unroll
+        for (int c = 0; c < PA_CHUNKS; ++c) {
+            const int kidx = c * 64 + warp * KPW + lane;
+            pos[c] = kidx < a.topk ? a.idx[(int64_t)row * a.topk + kidx] : -1;
+        }
+#pragma unroll
+        for (int c = 0; c < PA_CHUNKS; ++c) {
+            int32_t sl = -1;
+            if (pos[c] >= 0) {
+                if (pos[c] < L) sl = (int32_t)entry_slot(a.cache, a.page_shift, 0, pos[c], a.err);
+                else dev_error(a.err, CSA2_DEV_INDEX);
+            }
+            s_slot[c * KPW + lane] = sl;
+        }
+    }
+    __syncwarp();
+    auto stage_of = [&](int c) { return smem + (size_t)(c & 1) * PA_STAGE; };
+    auto gather = [&](int c) {  // chunk c of this warp into ring slot c & 1 (commits a group)
+        if (c < PA_CHUNKS) {
+            if (warp < 4) {
+                uint8_t* st = stage_of(c) + warp * KPW * FP4_ROW;
+#pragma unroll
+                for (int it = 0; it < (KPW * 9 + 31) / 32; ++it) {
+                    const int q = lane + 32 * it;
+                    const int r = min(q / 9, KPW - 1), ch = q % 9;
+                    const int32_t sl = s_slot[c * KPW + r];
+                    if (q < KPW * 9) {
+                        uint8_t* dst = st + r * FP4_ROW + ch * 16;
+                        if (sl >= 0) {
+                            if (ch < 8) cp_async16(dst, a.cache.codes + (int64_t)sl * kCodeBytes + ch * 16);
+                            else cp_async16(dst, a.cache.scales + (int64_t)sl * kScales);
+                        } else {
+                            *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+            } else {
+                uint8_t* st = stage_of(c) + 4 * KPW * FP4_ROW;
+                const int k0 = c * KPW;
+                for (int q = lane; q < KPW * 32; q += 32) {
+                    const int r = q >> 5, ch = q & 31;
+                    uint8_t* dst = st + r * SWA_ROW + ch * 16;
+                    if (k0 + r < n_swa) cp_async16(dst, swa_base + (int64_t)(k0 + r) * kCh + ch * 8);
+                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    gather(0);
+    gather(1);
+
+    // Q [16 heads][128] as an fp16 tile in shared memory (A operand via ldmatrix)
+    for (int i = tid; i < kH * kD / 8; i += ATT_THREADS) {
+        const int h = i >> 4, c8 = i & 15;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)row * kH + h) * kD) + c8);
+        *reinterpret_cast<uint4*>(qs + h * PA_QROW + c8 * 16) =
+            make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
+    }
+    __syncthreads();
+    // lane address of the A fragment of k-step cc: matrix m = lane / 8 holds
+    // heads (m & 1) * 8 + (lane & 7), dims 16 cc + (m >> 1) * 8
+    const uint32_t qa_base = smem_u32(qs) + (((lane >> 3) & 1) * 8 + (lane & 7)) * PA_QROW + (lane >> 4) * 16;
+
+    const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    float m_run = -INFINITY, m_run8 = -INFINITY, l_run = 0.f, l_run8 = 0.f;
+    float O[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+
+    for (int c = 0; c < PA_CHUNKS; ++c) {
+        cp_async_wait<1>();
+        __syncwarp();
+        const uint8_t* st = warp < 4 ? stage_of(c) + warp * KPW * FP4_ROW : stage_of(c) + 4 * KPW * FP4_ROW;
+        // validity of the 16 keys of this chunk (same rule as the gather)
+        uint32_t vmask;
+        if (warp < 4) {
+            vmask = __ballot_sync(0xffffffffu, lane < KPW && s_slot[c * KPW + (lane & (KPW - 1))] >= 0);
+        } else {
+            vmask = __ballot_sync(0xffffffffu, lane < KPW && c * KPW + lane < n_swa);
+        }
+        // S = Q K^T one n8 tile (8 keys) at a time, B fragments dequantised
+        // straight from the staged rows; then the fp16 V tile [key][dim]
+        float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint32_t bk[8][2];
+            if (warp < 4) {
+                const uint8_t* r = st + (8 * j + g) * FP4_ROW;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t sc = e4m3_to_h2(r[128 + cc]);
+                    const uint32_t wl = *reinterpret_cast<const uint32_t*>(r + 8 * cc);
+                    const uint32_t wh = *reinterpret_cast<const uint32_t*>(r + 8 * cc + 4);
+                    bk[cc][0] = hmul2(e2m1_low_byte_to_h2(wl >> (8 * t)), sc);
+                    bk[cc][1] = hmul2(e2m1_low_byte_to_h2(wh >> (8 * t)), sc);
+                }
+            } else {
+                const uint32_t* r = reinterpret_cast<const uint32_t*>(st + (8 * j + g) * SWA_ROW);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    bk[cc][0] = bf2_to_h2(r[8 * cc + t]);
+                    bk[cc][1] = bf2_to_h2(r[8 * cc + 4 + t]);
+                }
+            }
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint32_t qa[4];
+                ldsm_x4(qa_base + cc * 32, qa[0], qa[1], qa[2], qa[3]);
+                mma16816(S[j], qa, bk[cc][0], bk[cc][1]);
+            }
+        }
+        {
+            const int key = lane >> 1, half = lane & 1;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
+            if (warp < 4) {
+                const uint8_t* r = st + key * FP4_ROW;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(r + 64 + 32 * half + 4 * i);
+                    const uint32_t sc = e4m3_to_h2(r[128 + 8 + 4 * half + (i >> 1)]);
+                    uint32_t h0, h1, h2, h3;
+                    e2m1x8_to_h2x4(w, h0, h1, h2, h3);
+                    *reinterpret_cast<uint4*>(dst + 4 * i) =
+                        make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
+                }
+            } else {
+                const uint32_t* r = reinterpret_cast<const uint32_t*>(st + key * SWA_ROW) + 64 + 32 * half;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]),
+                                                                        bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+            }
+        }
+        __syncwarp();      // the staged rows are no longer read; the V tile is written
+        gather(c + 2);     // refill this ring slot while the chunk is finished
+
+        // online softmax (log2 domain) over this chunk's keys
+        float cm = -INFINITY, cm8 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const bool ok = (vmask >> (8 * j + 2 * t + e)) & 1u;
+                S[j][e] = ok ? S[j][e] * kScaleLog2 : -INFINITY;
+                S[j][2 + e] = ok ? S[j][2 + e] * kScaleLog2 : -INFINITY;
+                cm = fmaxf(cm, S[j][e]);
+                cm8 = fmaxf(cm8, S[j][2 + e]);
+            }
+        }
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+        cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 1));
+        cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 2));
+        const float mn = fmaxf(m_run, cm), mn8 = fmaxf(m_run8, cm8);
+        const float f = m_run == -INFINITY ? 0.f : exp2f(m_run - mn);
+        const float f8 = m_run8 == -INFINITY ? 0.f : exp2f(m_run8 - mn8);
+        m_run = mn;
+        m_run8 = mn8;
+        float lg = 0.f, lg8 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                S[j][e] = mn == -INFINITY ? 0.f : exp2f(S[j][e] - mn);
+                S[j][2 + e] = mn8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - mn8);
+                lg += S[j][e];
+                lg8 += S[j][2 + e];
+            }
+        }
+        lg += __shfl_xor_sync(0xffffffffu, lg, 1);
+        lg += __shfl_xor_sync(0xffffffffu, lg, 2);
+        lg8 += __shfl_xor_sync(0xffffffffu, lg8, 1);
+        lg8 += __shfl_xor_sync(0xffffffffu, lg8, 2);
+        l_run = l_run * f + lg;
+        l_run8 = l_run8 * f8 + lg8;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            O[j][0] *= f;
+            O[j][1] *= f;
+            O[j][2] *= f8;
+            O[j][3] *= f8;
+        }
+        const uint32_t pa[4] = {f2_to_h2(S[0][0], S[0][1]), f2_to_h2(S[0][2], S[0][3]), f2_to_h2(S[1][0], S[1][1]),
+                                f2_to_h2(S[1][2], S[1][3])};
+        {
+            const int m = lane >> 3, r = lane & 7;
+            const uint32_t base = smem_u32(vt) + ((m & 1) * 8 + r) * VT_ROW + (m >> 1) * 16;
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_trans(base + j * 16, b0, b1, b2, b3);
+                mma16816(O[j], pa, b0, b1);
+                mma16816(O[j + 1], pa, b2, b3);
+            }
+        }
+        __syncwarp();  // the V tile is read before the next chunk rewrites it
+    }
+    cp_async_wait<0>();
+
+    // ---- merge the five warps -------------------------------------------------
+    if (t == 0) {
+        ms[warp * kH + g] = m_run;
+        ms[warp * kH + g + 8] = m_run8;
+    }
+    __syncthreads();  // every warp is past its loop: the ring may hold the partials
+    float Mg = -INFINITY, Mg8 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < ATT_WARPS; ++w) {
+        Mg = fmaxf(Mg, ms[w * kH + g]);
+        Mg8 = fmaxf(Mg8, ms[w * kH + g + 8]);
+    }
+    const float fg = m_run == -INFINITY ? 0.f : exp2f(m_run - Mg);
+    const float fg8 = m_run8 == -INFINITY ? 0.f : exp2f(m_run8 - Mg8);
+    {
+        float* part = opart + warp * kH * OACC_ROW;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            *reinterpret_cast<float2*>(part + g * OACC_ROW + 8 * j + 2 * t) = make_float2(O[j][0] * fg, O[j][1] * fg);
+            *reinterpret_cast<float2*>(part + (g + 8) * OACC_ROW + 8 * j + 2 * t) =
+                make_float2(O[j][2] * fg8, O[j][3] * fg8);
+        }
+        if (t == 0) {
+            lpart[warp * kH + g] = l_run * fg;
+            lpart[warp * kH + g + 8] = l_run8 * fg8;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < kH * kD / 4; i += ATT_THREADS) {
+        const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
+        float4 acc = *reinterpret_cast<const float4*>(opart + h * OACC_ROW + d4);
+        float den = lpart[h];
+#pragma unroll
+        for (int w = 1; w < ATT_WARPS; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(opart + w * kH * OACC_ROW + h * OACC_ROW + d4);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+            den += lpart[w * kH + h];
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        *reinterpret_cast<float4*>(a.out + ((int64_t)row * kH + h) * kD + d4) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (d4 == 0) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < ATT_WARPS; ++w) M = fmaxf(M, ms[w * kH + h]);
+            a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+}
+
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
     static bool init[64];
     int dev = 0;
@@ -432,9 +742,20 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
         e = cudaFuncSetAttribute((const void*)sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ATT_SMEM);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute((const void*)prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PA_SMEM);
+        if (e != cudaSuccess) return e;
+        // several query CTAs per SM: ask for the largest shared-memory carveout
+        e = cudaFuncSetAttribute((const void*)prefill_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         init[dev] = true;
     }
     if (a.rows <= 0) return cudaSuccess;
+    if (a.q_pos) {  // prefill: one CTA per query
+        LaunchCfg c(dim3((unsigned)a.rows), dim3(ATT_THREADS), PA_SMEM, stream);
+        return cudaLaunchKernelEx(&c.cfg, prefill_attn_kernel, a);
+    }
     LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), ATT_SMEM, stream, ATT_SPLIT);
     return cudaLaunchKernelEx(&c.cfg, sparse_attn_kernel, a);
 }

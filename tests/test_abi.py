@@ -76,6 +76,10 @@ def test_host_validation_without_gpu(csa2):
     # misaligned pointers and bad cache geometry
     assert L.csa2_sparse_attn_decode(ctypes.byref(d), ctypes.byref(c), P(0x1000), P(0x1000), P(0x1001),
                                      P(0x1000), None, P(0x1000), P(0x1000), 1, None, None) == 1
+    # prefill attention loads q and writes out in 16-byte vectors: 4-byte alignment is rejected
+    for qp, op in ((0x1004, 0x1000), (0x1000, 0x1004)):
+        assert L.csa2_sparse_attn_prefill(ctypes.byref(d), ctypes.byref(c), P(qp), P(0x1000), P(0x1000), P(0x1000),
+                                          0, 1, P(op), P(0x1000), 1, None, None) == 1
     c2 = _cache_struct(csa2, page_size=12)
     assert L.csa2_kv_quant_append(ctypes.byref(c2), P(0x1000), 0, None, 1, 1, P(0x1000), None, None) == 1
     assert L.csa2_kv_quant_append(ctypes.byref(c), P(0x1000), 0, None, 1, 3, P(0x1000), None, None) == 1
