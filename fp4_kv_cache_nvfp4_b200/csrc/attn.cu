@@ -567,14 +567,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 3) prefill_attn_kernel(AttnArgs a
         for (int j = 0; j < 2; ++j) {
             uint32_t bk[8][2];
             if (warp < 4) {
+                // the row's K codes (64 B) and K scales (8 B) in five vector loads
                 const uint8_t* r = st + (8 * j + g) * FP4_ROW;
+                uint32_t w[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(r + 16 * v);
+                    w[4 * v] = x.x;
+                    w[4 * v + 1] = x.y;
+                    w[4 * v + 2] = x.z;
+                    w[4 * v + 3] = x.w;
+                }
+                const uint2 scs = *reinterpret_cast<const uint2*>(r + 128);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t sc = e4m3_to_h2(r[128 + cc]);
-                    const uint32_t wl = *reinterpret_cast<const uint32_t*>(r + 8 * cc);
-                    const uint32_t wh = *reinterpret_cast<const uint32_t*>(r + 8 * cc + 4);
-                    bk[cc][0] = hmul2(e2m1_low_byte_to_h2(wl >> (8 * t)), sc);
-                    bk[cc][1] = hmul2(e2m1_low_byte_to_h2(wh >> (8 * t)), sc);
+                    const uint32_t sc = e4m3_to_h2((uint8_t)(((cc < 4 ? scs.x : scs.y) >> (8 * (cc & 3))) & 0xffu));
+                    bk[cc][0] = hmul2(e2m1_low_byte_to_h2(w[2 * cc] >> (8 * t)), sc);
+                    bk[cc][1] = hmul2(e2m1_low_byte_to_h2(w[2 * cc + 1] >> (8 * t)), sc);
                 }
             } else {
                 const uint32_t* r = reinterpret_cast<const uint32_t*>(st + (8 * j + g) * SWA_ROW);
@@ -595,22 +604,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 3) prefill_attn_kernel(AttnArgs a
             const int key = lane >> 1, half = lane & 1;
             uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
             if (warp < 4) {
+                // half a row of V: 32 code bytes and 4 scale bytes in three vector loads
                 const uint8_t* r = st + key * FP4_ROW;
+                const uint4 v0 = *reinterpret_cast<const uint4*>(r + 64 + 32 * half);
+                const uint4 v1 = *reinterpret_cast<const uint4*>(r + 64 + 32 * half + 16);
+                const uint32_t scw = *reinterpret_cast<const uint32_t*>(r + 128 + 8 + 4 * half);
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(r + 64 + 32 * half + 4 * i);
-                    const uint32_t sc = e4m3_to_h2(r[128 + 8 + 4 * half + (i >> 1)]);
+                    const uint32_t sc = e4m3_to_h2((uint8_t)((scw >> (8 * (i >> 1))) & 0xffu));
                     uint32_t h0, h1, h2, h3;
-                    e2m1x8_to_h2x4(w, h0, h1, h2, h3);
+                    e2m1x8_to_h2x4(w[i], h0, h1, h2, h3);
                     *reinterpret_cast<uint4*>(dst + 4 * i) =
                         make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
                 }
             } else {
-                const uint32_t* r = reinterpret_cast<const uint32_t*>(st + key * SWA_ROW) + 64 + 32 * half;
+                const uint4* r = reinterpret_cast<const uint4*>(st + key * SWA_ROW + 256 + 128 * half);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]),
-                                                                        bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 x = r[i];
+                    *reinterpret_cast<uint4*>(dst + 4 * i) =
+                        make_uint4(bf2_to_h2(x.x), bf2_to_h2(x.y), bf2_to_h2(x.z), bf2_to_h2(x.w));
+                }
             }
         }
         __syncwarp();      // the staged rows are no longer read; the V tile is written
