@@ -1007,10 +1007,13 @@ struct PrefillArgs {
     const float* w;
     const int32_t* q_pos;
     int32_t* out;
-    uint32_t* keys;  // [T][stride]
+    uint32_t* keys;    // [T][stride] exact keys (fallback)
+    uint16_t* keys16;  // [T][stride] approximate keys (aliases `keys`)
+    int32_t* flags;    // [T]: null = every query takes the exact path
+    float* kmax;       // [kmax_parts]
     int32_t* err;
     int64_t stride;
-    int T, ratio, topk, n_entries, page_shift;
+    int T, ratio, topk, n_entries, page_shift, kmax_parts;
 };
 
 __device__ __forceinline__ int visible(int p, int ratio, int n) { return min((p + 1) / ratio, n); }
@@ -1031,6 +1034,10 @@ __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a
     pdl_trigger();
     const int q0 = blockIdx.x * PS_Q;
     const int tid = threadIdx.x;
+    if (a.flags) {  // exact fallback: only tiles holding a flagged query
+        const bool f = tid < PS_Q && q0 + tid < a.T && a.flags[q0 + tid] != 0;
+        if (!__syncthreads_or(f)) return;
+    }
     for (int i = tid; i < PS_Q * kIH * kID; i += PS_THREADS) {
         const int qq = i / (kIH * kID), h = (i / kID) % kIH, d = i % kID;
         const int t = q0 + qq;
@@ -1126,6 +1133,7 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
     pdl_wait();
     pdl_trigger();
     const int t = blockIdx.x;
+    if (a.flags && a.flags[t] == 0) return;  // exact fallback: flagged queries only
     const int n = (int)a.stride;
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K4_OFF_HIST);
@@ -1156,6 +1164,360 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
     find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
     refine_threshold(skeys, n, (uint32_t)b1, kk - above, hist, l0, l1, tmp, &T, &need);
     emit_sorted(skeys, n, T, need, kk, a.topk, out, tmp, [](int i) { return (int32_t)i; });
+}
+
+// ============================================================================
+// Prefill indexer on tensor cores, exact by verification
+//
+// K5a scores every (query, visible entry) pair with mma.sync bf16 x bf16 ->
+// fp32 (exact products, fp32 sums in the tensor core's order) and writes the
+// top 16 bits of each score's order-preserving key.  K5b, one CTA per query,
+// takes the approximate Top-1024 as candidates, rescores them with the exact
+// sequential-FMA chain and selects the exact Top-K among them; it then checks
+// that no other entry can reach that Top-K: every non-candidate's approximate
+// score lies below the candidates' 16-bit threshold B, and
+// |approximate - exact| <= delta = 2^-12 sum_h |w_h| ||q_h||_1 max|k|, a bound
+// several times above the rounding of either sum of 64 exact products.  If
+// B + delta >= the K-th exact score, the query is flagged and the exact
+// CUDA-core kernels recompute it.  The output is therefore the exact Top-K.
+// ============================================================================
+constexpr int PT_Q = 64;          // queries per CTA
+constexpr int PT_E = 64;          // entries per K tile
+constexpr int PT_SPLIT = 2048;    // entries per CTA (grid.y splits the entry range)
+constexpr int PT_THREADS = 256;
+constexpr int PT_CAND = 1024;     // approximate candidates per query
+constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit threshold) -> exact fallback
+constexpr size_t PT_OFF_K = 0;                                  // 2 x [64][64] bf16, 16 B chunks swizzled
+constexpr size_t PT_OFF_OUT = PT_OFF_K + 2 * PT_E * 128;        // [64 q][64 e] u16
+constexpr size_t PT_OFF_W = PT_OFF_OUT + PT_Q * PT_E * 2;       // [64][4] f32
+constexpr size_t PT_OFF_VIS = PT_OFF_W + PT_Q * kIH * 4;        // [64] int
+constexpr size_t PT_OFF_RED = PT_OFF_VIS + PT_Q * 4;            // [8] u32
+constexpr size_t PT_SMEM = PT_OFF_RED + 8 * 4;
+static_assert(PT_OFF_OUT % 16 == 0 && PT_OFF_W % 16 == 0, "K5a shared-memory layout");
+
+__device__ __forceinline__ void ldsm_x4_b16(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Warp w: queries 16 (w & 3) .. +16 of the CTA's 64, entries 32 (w >> 2) .. +32
+// of each 64-entry tile (four n8 tiles), all four heads (one K tile serves them).
+__global__ void __launch_bounds__(PT_THREADS) prefill_tc_score_kernel(PrefillArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* ktile = smem + PT_OFF_K;
+    uint16_t* otile = reinterpret_cast<uint16_t*>(smem + PT_OFF_OUT);
+    float* ws_ = reinterpret_cast<float*>(smem + PT_OFF_W);
+    int* vis = reinterpret_cast<int*>(smem + PT_OFF_VIS);
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem + PT_OFF_RED);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int g = lane >> 2, t = lane & 3, wq = wid & 3, we = wid >> 2;
+    const int q0 = blockIdx.x * PT_Q;
+    const int part = blockIdx.x + gridDim.x * blockIdx.y;
+    pdl_wait();
+    pdl_trigger();
+    if (tid < PT_Q) vis[tid] = q0 + tid < a.T ? visible(a.q_pos[q0 + tid], a.ratio, a.n_entries) : 0;
+    for (int i = tid; i < PT_Q * kIH; i += PT_THREADS) {
+        const int q = q0 + i / kIH;
+        ws_[i] = q < a.T ? a.w[(int64_t)q * kIH + i % kIH] : 0.f;
+    }
+    __syncthreads();
+    int max_vis = 0;
+    for (int i = 0; i < PT_Q; ++i) max_vis = max(max_vis, vis[i]);
+    const int e_beg = blockIdx.y * PT_SPLIT, e_end = min(e_beg + PT_SPLIT, max_vis);
+    if (e_beg >= e_end) {
+        if (tid == 0) a.kmax[part] = 0.f;
+        return;
+    }
+    // A fragments of Q_h (16 queries x 64 dims, bf16 pairs), all heads and k-steps
+    uint32_t qa[kIH][4][4];
+    {
+        const int qr0 = q0 + 16 * wq + g, qr1 = qr0 + 8;
+#pragma unroll
+        for (int h = 0; h < kIH; ++h)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int d = 16 * c + 2 * t;
+                auto ld = [&](int q, int dd) -> uint32_t {
+                    return q < a.T ? __ldg(reinterpret_cast<const uint32_t*>(a.q_idx + ((int64_t)q * kIH + h) * kID + dd))
+                                   : 0u;
+                };
+                qa[h][c][0] = ld(qr0, d);
+                qa[h][c][1] = ld(qr1, d);
+                qa[h][c][2] = ld(qr0, d + 8);
+                qa[h][c][3] = ld(qr1, d + 8);
+            }
+    }
+    const int sh = a.page_shift;
+    const int32_t emask = (1 << sh) - 1;
+    // tile copies: 64 rows x 8 chunks, two chunks per thread; chunk c of row r at c ^ (r & 7)
+    auto issue = [&](int e0, int buf) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int i = tid + PT_THREADS * k, r = i >> 3, c = i & 7;
+            const int e = e0 + r;
+            uint8_t* dst = ktile + (size_t)buf * PT_E * 128 + r * 128 + ((c ^ (r & 7)) << 4);
+            int32_t phys = -1;
+            if (e < e_end) {
+                const int32_t pg = e >> sh;
+                phys = pg < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + pg) : -1;
+                if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                    dev_error(a.err, CSA2_DEV_PAGE);
+                    phys = -1;
+                }
+            }
+            if (phys >= 0) {
+                const int64_t slot = ((int64_t)phys << sh) | (e & emask);
+                cp_async16(dst, a.cache.idx_k + slot * kID + c * 8);
+            } else {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        cp_async_commit();
+    };
+    uint32_t kmax_bits = 0;  // max |k| as bf16 bits (positive values order as integers)
+    const int ntile = (e_end - e_beg + PT_E - 1) / PT_E;
+    issue(e_beg, 0);
+    for (int it = 0; it < ntile; ++it) {
+        const int e0 = e_beg + it * PT_E, buf = it & 1;
+        if (it + 1 < ntile) issue(e0 + PT_E, buf ^ 1);
+        else cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();  // tile `it` is in shared memory for every warp
+        const uint8_t* kt = ktile + (size_t)buf * PT_E * 128;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {  // the chunks this thread copied
+            const int i = tid + PT_THREADS * k, r = i >> 3, c = i & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(kt + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                kmax_bits = max(kmax_bits, max(x[u] & 0x7fffu, (x[u] >> 16) & 0x7fffu));
+        }
+        float acc[kIH][4][4];
+#pragma unroll
+        for (int h = 0; h < kIH; ++h)
+#pragma unroll
+            for (int n = 0; n < 4; ++n) acc[h][n][0] = acc[h][n][1] = acc[h][n][2] = acc[h][n][3] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t b[4][2];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {  // n8 tiles 2 jj and 2 jj + 1
+                const int m = lane >> 3, n = 2 * jj + (m >> 1), kh = m & 1;
+                const int r = 32 * we + 8 * n + (lane & 7), ch = 2 * c + kh;
+                ldsm_x4_b16(smem_u32(kt + r * 128 + ((ch ^ (r & 7)) << 4)), b[2 * jj][0], b[2 * jj][1],
+                            b[2 * jj + 1][0], b[2 * jj + 1][1]);
+            }
+#pragma unroll
+            for (int h = 0; h < kIH; ++h)
+#pragma unroll
+                for (int n = 0; n < 4; ++n) mma_bf16_16816(acc[h][n], qa[h][c], b[n][0], b[n][1]);
+        }
+        // epilogue: score = sum_h w_h relu(q_h . k) (fp32, heads in order), 16-bit key
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int ql = 16 * wq + g + 8 * (i >> 1), el = 32 * we + 8 * n + 2 * t + (i & 1);
+                float s = 0.f;
+#pragma unroll
+                for (int h = 0; h < kIH; ++h) s = __fmaf_rn(ws_[ql * kIH + h], fmaxf(acc[h][n][i], 0.f), s);
+                otile[ql * PT_E + el] = e0 + el < vis[ql] ? (uint16_t)(score_key(s) >> 16) : (uint16_t)0;
+            }
+        __syncthreads();  // the out tile is complete; buffer `buf` may be refilled
+        for (int i = tid; i < PT_Q * PT_E / 8; i += PT_THREADS) {
+            const int ql = i >> 3, c = i & 7;
+            if (q0 + ql < a.T)
+                *reinterpret_cast<uint4*>(a.keys16 + (int64_t)(q0 + ql) * a.stride + e0 + c * 8) =
+                    *reinterpret_cast<const uint4*>(otile + ql * PT_E + c * 8);
+        }
+    }
+    // max |k| of the CTA's entries
+    for (int o = 16; o > 0; o >>= 1) kmax_bits = max(kmax_bits, __shfl_xor_sync(0xffffffffu, kmax_bits, o));
+    if (lane == 0) red[wid] = kmax_bits;
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t m = 0;
+        for (int i = 0; i < PT_THREADS / 32; ++i) m = max(m, red[i]);
+        a.kmax[part] = __uint_as_float(m << 16);
+    }
+}
+
+// float value of an order-preserving key (inverse of score_key)
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+constexpr int PC_THREADS = 512;
+constexpr size_t PC_OFF_K16 = 0;                                      // [16384] u16
+constexpr size_t PC_OFF_CK = PC_OFF_K16 + (size_t)kMaxCand * 2;        // [2048] u32 exact keys
+constexpr size_t PC_OFF_CAND = PC_OFF_CK + PT_CAND_MAX * 4;            // [2048] u16 entries
+constexpr size_t PC_OFF_HIST = PC_OFF_CAND + PT_CAND_MAX * 2;          // [4096]
+constexpr size_t PC_OFF_L0 = PC_OFF_HIST + kHistBins * 4;              // [2048] u16
+constexpr size_t PC_OFF_L1 = PC_OFF_L0 + PT_CAND_MAX * 2;              // [2048] u16
+constexpr size_t PC_OFF_QD = PC_OFF_L1 + PT_CAND_MAX * 2;              // [64] float4
+constexpr size_t PC_OFF_TMP = PC_OFF_QD + kID * 16;                    // [64] u32
+constexpr size_t PC_OFF_MISC = PC_OFF_TMP + 64 * 4;                    // w (float4), l1[4], kmax, thr, count
+constexpr size_t PC_SMEM = PC_OFF_MISC + 64;
+static_assert(PC_OFF_QD % 16 == 0 && PC_OFF_MISC % 16 == 0 && PC_OFF_HIST % 16 == 0, "K5b shared-memory layout");
+
+__global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint16_t* k16 = reinterpret_cast<uint16_t*>(smem + PC_OFF_K16);
+    uint32_t* ck = reinterpret_cast<uint32_t*>(smem + PC_OFF_CK);
+    uint16_t* cand = reinterpret_cast<uint16_t*>(smem + PC_OFF_CAND);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + PC_OFF_HIST);
+    uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + PC_OFF_L0);
+    uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + PC_OFF_L1);
+    float4* qd = reinterpret_cast<float4*>(smem + PC_OFF_QD);
+    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + PC_OFF_TMP);
+    float4& s_w = *reinterpret_cast<float4*>(smem + PC_OFF_MISC);
+    float* s_l1 = reinterpret_cast<float*>(smem + PC_OFF_MISC + 16);       // [4]
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(smem + PC_OFF_MISC + 32);  // kmax bits, count
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int t = blockIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    const int n_vis = visible(a.q_pos[t], a.ratio, a.n_entries);
+    int32_t* out = a.out + (int64_t)t * a.topk;
+    if (n_vis <= 0) {
+        for (int i = tid; i < a.topk; i += PC_THREADS) out[i] = -1;
+        if (tid == 0) a.flags[t] = 0;
+        return;
+    }
+    // query, weights, ||q_h||_1, max |k| over the scoring CTAs
+    const uint16_t* qb = a.q_idx + (int64_t)t * kIH * kID;
+    for (int d = tid; d < kID; d += PC_THREADS)
+        qd[d] = make_float4(bf16_bits_to_f32(qb[d]), bf16_bits_to_f32(qb[kID + d]), bf16_bits_to_f32(qb[2 * kID + d]),
+                            bf16_bits_to_f32(qb[3 * kID + d]));
+    if (wid < kIH) {
+        float v = fabsf(bf16_bits_to_f32(qb[wid * kID + lane])) + fabsf(bf16_bits_to_f32(qb[wid * kID + 32 + lane]));
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) s_l1[wid] = v;
+    }
+    if (wid == kIH) {
+        uint32_t m = 0;
+        for (int i = lane; i < a.kmax_parts; i += 32) m = max(m, __float_as_uint(a.kmax[i]));
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_u[0] = m;
+    }
+    if (tid == 0) {
+        s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)t * kIH);
+        s_u[1] = 0;
+    }
+    for (int i = tid; i < n_vis; i += PC_THREADS) k16[i] = a.keys16[(int64_t)t * a.stride + i];
+    for (int i = tid; i < 256; i += PC_THREADS) hist[i] = 0;
+    __syncthreads();
+
+    // ---- candidates: the entries whose 16-bit key is >= the PT_CAND-th largest
+    uint32_t thr16 = 0u;  // 0: every visible entry is a candidate
+    if (n_vis > PT_CAND) {
+        for (int i = tid; i < n_vis; i += PC_THREADS) hist_add(hist, k16[i] >> 8, true);
+        __syncthreads();
+        int b1, b2;
+        uint32_t above;
+        find_kth_bin(hist, 256, PT_CAND, tmp, &b1, &above);
+        for (int i = tid; i < 256; i += PC_THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n_vis; i += PC_THREADS) hist_add(hist, k16[i] & 255u, (int)(k16[i] >> 8) == b1);
+        __syncthreads();
+        find_kth_bin(hist, 256, PT_CAND - above, tmp, &b2, &above);
+        thr16 = ((uint32_t)b1 << 8) | (uint32_t)b2;
+    }
+    // compact in entry order (the output must come out ascending): warp v
+    // walks a contiguous segment, counts, then writes at its prefix offset
+    const int seg = ((n_vis + PC_THREADS / 32 - 1) / (PC_THREADS / 32) + 31) & ~31;
+    const int lo = wid * seg, hi = min(n_vis, lo + seg);
+    uint32_t mine = 0;
+    for (int b = lo; b < hi; b += 32) {
+        const int i = b + lane;
+        mine += __popc(__ballot_sync(0xffffffffu, i < hi && (uint32_t)k16[i] >= thr16));
+    }
+    __syncthreads();
+    if (lane == 0) tmp[wid] = mine;
+    __syncthreads();
+    uint32_t off = 0, m_total = 0;
+    for (int v = 0; v < PC_THREADS / 32; ++v) {
+        if (v < wid) off += tmp[v];
+        m_total += tmp[v];
+    }
+    const int m = (int)m_total;
+    if (m > PT_CAND_MAX) {  // too many ties at the 16-bit threshold: exact fallback
+        if (tid == 0) a.flags[t] = 1;
+        return;
+    }
+    for (int b = lo; b < hi; b += 32) {
+        const int i = b + lane;
+        const bool in = i < hi && (uint32_t)k16[i] >= thr16;
+        const unsigned bm = __ballot_sync(0xffffffffu, in);
+        if (in) cand[off + __popc(bm & ((1u << lane) - 1u))] = (uint16_t)i;
+        off += __popc(bm);
+    }
+    __syncthreads();
+
+    // ---- exact scores of the candidates (the oracle's sequential FMA chains)
+    const float4 w = s_w;
+    for (int i = tid; i < m; i += PC_THREADS) {
+        const int e = cand[i];
+        const int64_t slot = entry_slot(a.cache, a.page_shift, 0, e, a.err);
+        uint32_t kr[32];
+        if (slot >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.cache.idx_k + slot * kID);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = __ldg(src + c);
+                kr[4 * c] = v.x;
+                kr[4 * c + 1] = v.y;
+                kr[4 * c + 2] = v.z;
+                kr[4 * c + 3] = v.w;
+            }
+            ck[i] = score_key(idx_score1(kr, qd, w));
+        } else {
+            ck[i] = 0u;
+        }
+    }
+    for (int i = tid; i < kHistBins; i += PC_THREADS) hist[i] = 0;
+    __syncthreads();
+
+    // ---- exact Top-K among the candidates
+    uint32_t nv = 0;
+    for (int i = tid; i < m; i += PC_THREADS) {
+        nv += ck[i] != 0u;
+        hist_add(hist, ck[i] >> 20, ck[i] != 0u);
+    }
+    uint32_t n_valid;
+    block_excl_scan(nv, tmp, &n_valid);
+    const uint32_t kk = min((uint32_t)a.topk, n_valid);
+    if (kk == 0) {
+        for (int i = tid; i < a.topk; i += PC_THREADS) out[i] = -1;
+        if (tid == 0) a.flags[t] = 0;
+        return;
+    }
+    int b1;
+    uint32_t above, T, need;
+    find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
+    refine_threshold(ck, m, (uint32_t)b1, kk - above, hist, l0, l1, tmp, &T, &need);
+    // ---- no entry outside the candidates can reach the K-th exact score
+    if (thr16 != 0u) {
+        const double bound = (double)key_value(thr16 << 16);  // non-candidates score below this (approximately)
+        const double delta = 0x1p-12 * (fabs((double)w.x) * s_l1[0] + fabs((double)w.y) * s_l1[1] +
+                                        fabs((double)w.z) * s_l1[2] + fabs((double)w.w) * s_l1[3]) *
+                             (double)__uint_as_float(s_u[0]);
+        if (kk < (uint32_t)a.topk || !(bound + delta < (double)key_value(T))) {
+            if (tid == 0) a.flags[t] = 1;
+            return;
+        }
+    }
+    emit_sorted(ck, m, T, need, kk, a.topk, out, tmp, [&](int i) { return (int32_t)cand[i]; });
+    if (tid == 0) a.flags[t] = 0;
 }
 
 // ============================================================================
@@ -1190,8 +1552,12 @@ DecodeWs decode_ws_layout(int n, int64_t max_len) {
 PrefillWs prefill_ws_layout(int T, int64_t n_entries) {
     PrefillWs l{};
     l.stride = (n_entries + PS_E - 1) / PS_E * PS_E;
-    l.keys = 0;
-    l.total = align256((size_t)T * l.stride * 4);
+    l.kmax_parts = (int)(((T + PT_Q - 1) / PT_Q) * ((n_entries + PT_SPLIT - 1) / PT_SPLIT));
+    size_t o = 0;
+    l.keys = o; o = align256(o + (size_t)T * l.stride * 4);
+    l.flags = o; o = align256(o + (size_t)T * 4);
+    l.kmax = o; o = align256(o + (size_t)l.kmax_parts * 4);
+    l.total = o;
     return l;
 }
 
@@ -1289,9 +1655,11 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
 cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                                 const int32_t* seq_lens, const int32_t* q_pos, int ratio, int topk, int32_t* out,
                                 int T, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream) {
-    static bool d1[64], d2[64];
+    static bool d1[64], d2[64], d3[64], d4[64];
     cudaError_t e = ensure_smem((const void*)prefill_select_kernel, PSEL_SMEM, d1);
     if (e == cudaSuccess) e = ensure_smem((const void*)prefill_score_kernel, PS_SMEM, d2);
+    if (e == cudaSuccess) e = ensure_smem((const void*)prefill_tc_score_kernel, PT_SMEM, d3);
+    if (e == cudaSuccess) e = ensure_smem((const void*)prefill_candidates_kernel, PC_SMEM, d4);
     if (e != cudaSuccess) return e;
     (void)seq_lens;
     const PrefillWs l = prefill_ws_layout(T, max_len);
@@ -1302,6 +1670,10 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     a.q_pos = q_pos;
     a.out = out;
     a.keys = reinterpret_cast<uint32_t*>(ws + l.keys);
+    a.keys16 = reinterpret_cast<uint16_t*>(ws + l.keys);
+    a.flags = reinterpret_cast<int32_t*>(ws + l.flags);
+    a.kmax = reinterpret_cast<float*>(ws + l.kmax);
+    a.kmax_parts = l.kmax_parts;
     a.err = err;
     a.stride = l.stride;
     a.T = T;
@@ -1309,6 +1681,16 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     a.topk = topk;
     a.n_entries = (int)max_len;
     a.page_shift = page_shift_of(cache);
+    // tensor-core scores -> candidates, exact rescoring and verification; then
+    // the exact CUDA-core path for the queries that failed the check (it exits
+    // at once for the others)
+    LaunchCfg c0(dim3((unsigned)((T + PT_Q - 1) / PT_Q), (unsigned)((max_len + PT_SPLIT - 1) / PT_SPLIT)),
+                 dim3(PT_THREADS), PT_SMEM, stream);
+    e = cudaLaunchKernelEx(&c0.cfg, prefill_tc_score_kernel, a);
+    if (e != cudaSuccess) return e;
+    LaunchCfg cc(dim3((unsigned)T), dim3(PC_THREADS), PC_SMEM, stream);
+    e = cudaLaunchKernelEx(&cc.cfg, prefill_candidates_kernel, a);
+    if (e != cudaSuccess) return e;
     LaunchCfg c1(dim3((unsigned)((T + PS_Q - 1) / PS_Q)), dim3(PS_THREADS), PS_SMEM, stream);
     e = cudaLaunchKernelEx(&c1.cfg, prefill_score_kernel, a);
     if (e != cudaSuccess) return e;

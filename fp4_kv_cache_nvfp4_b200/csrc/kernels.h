@@ -52,8 +52,12 @@ struct DecodeWs {
 DecodeWs decode_ws_layout(int n, int64_t max_len);
 
 struct PrefillWs {
-    size_t keys, total;
+    size_t keys;   // [T][stride]: 16-bit approximate keys, later (aliased) 32-bit exact keys of the fallback
+    size_t flags;  // [T] int32: 1 = the query takes the exact fallback
+    size_t kmax;   // [tiles] float: max |indexer K| seen by each tensor-core scoring CTA
+    size_t total;
     int64_t stride;
+    int kmax_parts;
 };
 PrefillWs prefill_ws_layout(int T, int64_t n_entries);
 

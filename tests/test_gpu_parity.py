@@ -321,6 +321,34 @@ def test_prefill_parity(csa2, orc):
     assert ps.errors() == 0
 
 
+def test_prefill_indexer_exact_fallback_on_ties(csa2, orc):
+    # Entries 0..4999 share one indexer-K row, so their scores tie exactly.  A
+    # query that sees more than 2048 of them has too many candidates at the
+    # approximate threshold and must be recomputed by the exact fallback; the
+    # queries at the end of the context mix tied and distinct rows.  Either way
+    # the sets must equal the oracle's (ties to the lowest position).
+    seed = 1003
+    n_ent = 6000
+    tokens = 2 * n_ent
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 0, 0, tokens)
+    idx_k = synth.idx_k_rows(seed, 0, 0, n_ent).copy()
+    idx_k[:5000] = idx_k[0]
+    ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=999)
+    q_pos = np.concatenate([np.arange(6000, 6200), np.arange(tokens - 200, tokens)]).astype(np.int32)
+    T = len(q_pos)
+    q_idx = synth.q_idx(seed, 0, 0, T)
+    w = synth.w_idx(seed, 0, 0, T)
+    d = csa2.default_desc(csa2.FULL, 2)
+    ws = _ws(csa2, T, n_ent, prefill=True)
+    out_idx = torch.empty((T, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q_idx), dev(w), dev(np.array([n_ent], np.int32)), out_idx, T,
+                      n_ent, ws, q_pos=dev(q_pos), err=ps.err)
+    want = orc.prefill_indexer(q_pos, 2, n_ent, idx_k, q_idx, w)
+    check_sets(out_idx.cpu().numpy(), want, "prefill indexer with tied scores")
+    assert ps.errors() == 0
+
+
 # ---------------------------------------------------------------------------
 # device-side error reporting (bounds checks turn bad input into flags)
 # ---------------------------------------------------------------------------
