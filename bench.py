@@ -19,7 +19,6 @@ on the host cores on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
-import ctypes
 import json
 import math
 import os
@@ -188,8 +187,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     descs = [csa2.default_desc(m, 1) for m in modes]
     n_idx = sum(1 for m in modes if m != csa2.REUSE)
     # one packed device buffer holds every per-step input, so one H2D copy refreshes it
+    # (swa_new: every layer's newest SWA row; the end-to-end run scatters it into the rings)
     sizes = dict(q=layers * B * 16 * 128 * 2, qi=layers * B * 4 * 64 * 2, w=layers * B * 4 * 4, kv=B * CH * 4,
-                 ik=B * 64 * 2)
+                 ik=B * 64 * 2, swa_new=layers * B * CH * 2)
     offs, o = {}, 0
     for k, v in sizes.items():
         offs[k] = o
@@ -214,8 +214,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     seq_lens = torch.full((B,), L, dtype=torch.int32, device=dev)
     pos_new = torch.full((B,), L - 1, dtype=torch.int64, device=dev)  # the step (re)writes the newest entry
     slot_new = (tab_d[torch.arange(B, device=dev), pos_new // PAGE] * PAGE + pos_new % PAGE).contiguous()
-    outs = [torch.empty((B, 16, 128), dtype=torch.float32, device=dev) for _ in range(layers)]
-    lses = [torch.empty((B, 16), dtype=torch.float32, device=dev) for _ in range(layers)]
+    outs = [torch.empty((B, 16, 128), dtype=torch.float32, device=dev) for _ in range(layers - 1)]
+    lses = [torch.empty((B, 16), dtype=torch.float32, device=dev) for _ in range(layers - 1)]
+    # the step's result (last layer's out and lse) in one buffer: one device-to-host copy
+    result = torch.empty(B * 16 * 128 + B * 16, dtype=torch.float32, device=dev)
+    outs.append(result[:B * 16 * 128].view(B, 16, 128))
+    lses.append(result[B * 16 * 128:].view(B, 16))
     cand = torch.empty((B, 2048), dtype=torch.int32, device=dev)
     sets = torch.empty((layers, B, 512), dtype=torch.int32, device=dev)
     ws = torch.zeros(csa2.workspace_bytes(descs[0], csa2.BLOCK, B, L), dtype=torch.uint8, device=dev)
@@ -291,14 +295,15 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                                                        cand, B, L, ws, err=err, stream=stream))
 
         # ---- end to end: pinned host inputs -> device, step, result -> host ----
+        # one H2D copy of the packed inputs (q, q_idx, w, the appended entry and
+        # every layer's newest SWA row), one strided device copy of those rows
+        # into their ring slots, the step, one D2H copy of out and lse
+        ring = (L - 1) % 128
+        view("swa_new", (layers, B, CH), torch.int16).copy_(swa[:, :, ring, :])
         host_in = torch.empty(step_in.numel(), dtype=torch.uint8, pin_memory=True)
         host_in.copy_(step_in.cpu())
-        host_swa = torch.empty((layers, B, CH), dtype=torch.int16, pin_memory=True)
-        host_swa.copy_(swa[:, :, (L - 1) % 128, :].cpu())
-        host_out = torch.empty((B, 16, 128), dtype=torch.float32, pin_memory=True)
-        host_lse = torch.empty((B, 16), dtype=torch.float32, pin_memory=True)
-        cudart = _cudart()
-        ring = (L - 1) % 128
+        host_res = torch.empty(result.numel(), dtype=torch.float32, pin_memory=True)
+        swa_new = view("swa_new", (layers, B, CH), torch.int16)
         e2e_steps = max(10, min(args.steps, 100))
         eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
         with torch.cuda.stream(stream):
@@ -306,16 +311,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                 flush.fill_(k & 0xFF)
                 eev[k][0].record(stream)
                 step_in.copy_(host_in, non_blocking=True)
-                for l in range(layers):  # the new token's SWA row of every layer into its ring slot
-                    dst = swa[l, :, ring, :]
-                    rc = cudart.cudaMemcpy2DAsync(ctypes.c_void_p(dst.data_ptr()), ctypes.c_size_t(128 * CH * 2),
-                                                  ctypes.c_void_p(host_swa[l].data_ptr()), ctypes.c_size_t(CH * 2),
-                                                  ctypes.c_size_t(CH * 2), ctypes.c_size_t(B), 1,
-                                                  ctypes.c_void_p(stream.cuda_stream))
-                    assert rc == 0
+                swa[:, :, ring, :].copy_(swa_new)
                 graph.replay()
-                host_out.copy_(outs[-1], non_blocking=True)
-                host_lse.copy_(lses[-1], non_blocking=True)
+                host_res.copy_(result, non_blocking=True)
                 eev[k][1].record(stream)
         torch.cuda.synchronize()
         e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in eev)
@@ -324,8 +322,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     breakdown = _breakdown(csa2, cache, descs, modes, qi_all, w_all, q_all, swa, seq_lens, cand, sets, outs, lses,
                            kv_new, ik_new, slot_new, ws, err, flush, stream, B, L) if args.breakdown else None
 
-    h2d = step_in.numel() + layers * B * CH * 2
-    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+    h2d = step_in.numel()
+    d2h = host_res.numel() * 4
     ub = unique_bytes_per_seq(L, layers)
     peaks = _peaks()
     hbm = peaks.get("hbm_gbs")
@@ -546,18 +544,6 @@ def run_prefill(args, rank: int, world: int, local_rank: int):
                             indexer_tflops=idx_flop / (part_us["indexer"] * 1e-6) / 1e12,
                             peak_bf16_tflops=peaks.get("bf16_tflops")),
                 clocks=sampler.summary())
-
-
-def _cudart():
-    import torch  # noqa: F401  (loads the runtime torch ships)
-    for name in ("libcudart.so.12", "libcudart.so"):
-        try:
-            lib = ctypes.CDLL(name)
-            lib.cudaMemcpy2DAsync.restype = ctypes.c_int
-            return lib
-        except OSError:
-            continue
-    raise RuntimeError("libcudart not found")
 
 
 def _peaks() -> dict:

@@ -229,8 +229,11 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
 // top bin down) find the bin holding the k-th largest item (1-based k <= total):
 // *bin_out = that bin, *above_out = items in higher bins.  Every thread of the
 // group calls.
+// *total_out (if given) receives the histogram total; the bin is defined only
+// when k <= total.
 __device__ __forceinline__ void group_find_kth_bin(const uint32_t* hist, int nbins, uint32_t k, uint32_t* tmp,
-                                                   int* bin_out, uint32_t* above_out, GroupBar g) {
+                                                   int* bin_out, uint32_t* above_out, GroupBar g,
+                                                   uint32_t* total_out = nullptr) {
     // each thread owns a contiguous run of bins counted from the top
     int per = (nbins + g.n - 1) / g.n;
     int hi = nbins - 1 - (int)threadIdx.x * per;  // first (highest) bin of this thread
@@ -241,6 +244,7 @@ __device__ __forceinline__ void group_find_kth_bin(const uint32_t* hist, int nbi
     }
     uint32_t total;
     uint32_t before = group_excl_scan(mine, tmp, &total, g);
+    if (total_out) *total_out = total;
     if (before < k && before + mine >= k) {
         uint32_t acc = before;
         for (int i = 0; i < per; ++i) {

@@ -1126,14 +1126,10 @@ __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a
 }
 
 constexpr int PSEL_THREADS = 512;
-constexpr size_t PSEL_SMEM = K4_OFF_CB + 64 * 4;  // keys | hist | list0 | list1 | tmp
+constexpr size_t PSEL_SMEM = K4_OFF_CB + 64 * 4 + (PSEL_THREADS / 32) * 4;  // keys | hist | list0 | list1 | tmp | flag words
 
-__global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    pdl_wait();
-    pdl_trigger();
-    const int t = blockIdx.x;
-    if (a.flags && a.flags[t] == 0) return;  // exact fallback: flagged queries only
+__device__ void prefill_select_one(const PrefillArgs& a, int t, uint8_t* smem) {
+    __syncthreads();  // the previous trip's shared memory is no longer read
     const int n = (int)a.stride;
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K4_OFF_HIST);
@@ -1166,6 +1162,37 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
     emit_sorted(skeys, n, T, need, kk, a.topk, out, tmp, [](int i) { return (int32_t)i; });
 }
 
+// One query per loop trip (grid-stride: with flags the grid is a few CTAs per
+// SM and almost every trip ends at the flag).
+__global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    if (!a.flags) {
+        for (int t = blockIdx.x; t < a.T; t += gridDim.x) prefill_select_one(a, t, smem);
+        return;
+    }
+    // exact fallback: this CTA's queries t = blockIdx.x + j gridDim.x, their flags
+    // read side by side, chunks of PSEL_THREADS trips
+    for (int j0 = 0; blockIdx.x + (int64_t)j0 * gridDim.x < a.T; j0 += PSEL_THREADS) {
+        const int64_t tj = blockIdx.x + (int64_t)(j0 + threadIdx.x) * gridDim.x;
+        const bool f = tj < a.T && a.flags[tj] != 0;
+        const unsigned m = __ballot_sync(0xffffffffu, f);
+        __syncthreads();  // the previous chunk's trips no longer read the words below
+        uint32_t* words = reinterpret_cast<uint32_t*>(smem + K4_OFF_CB + 64 * 4);
+        if ((threadIdx.x & 31) == 0) words[threadIdx.x >> 5] = m;
+        __syncthreads();
+        for (int w = 0; w < PSEL_THREADS / 32; ++w) {
+            uint32_t bits = words[w];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1;
+                prefill_select_one(a, (int)(blockIdx.x + (int64_t)(j0 + 32 * w + b) * gridDim.x), smem);
+            }
+        }
+    }
+}
+
 // ============================================================================
 // Prefill indexer on tensor cores, exact by verification
 //
@@ -1185,11 +1212,13 @@ constexpr int PT_Q = 64;          // queries per CTA
 constexpr int PT_E = 64;          // entries per K tile
 constexpr int PT_SPLIT = 2048;    // entries per CTA (grid.y splits the entry range)
 constexpr int PT_THREADS = 256;
-constexpr int PT_CAND = 1024;     // approximate candidates per query
+constexpr int PT_CAND = 768;      // approximate candidates per query
 constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit threshold) -> exact fallback
+constexpr int PT_OROW = PT_E + 8;                               // out-tile row (u16): 144 B, rows on distinct banks
 constexpr size_t PT_OFF_K = 0;                                  // 2 x [64][64] bf16, 16 B chunks swizzled
-constexpr size_t PT_OFF_OUT = PT_OFF_K + 2 * PT_E * 128;        // [64 q][64 e] u16
-constexpr size_t PT_OFF_W = PT_OFF_OUT + PT_Q * PT_E * 2;       // [64][4] f32
+constexpr size_t PT_OFF_Q = PT_OFF_K + 2 * PT_E * 128;          // [64 q][4 h][64] bf16, chunks swizzled by q
+constexpr size_t PT_OFF_OUT = PT_OFF_Q + (size_t)PT_Q * kIH * kID * 2;  // [64 q][72] u16
+constexpr size_t PT_OFF_W = PT_OFF_OUT + PT_Q * PT_OROW * 2;    // [64][4] f32
 constexpr size_t PT_OFF_VIS = PT_OFF_W + PT_Q * kIH * 4;        // [64] int
 constexpr size_t PT_OFF_RED = PT_OFF_VIS + PT_Q * 4;            // [8] u32
 constexpr size_t PT_SMEM = PT_OFF_RED + 8 * 4;
@@ -1210,9 +1239,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 
 // Warp w: queries 16 (w & 3) .. +16 of the CTA's 64, entries 32 (w >> 2) .. +32
 // of each 64-entry tile (four n8 tiles), all four heads (one K tile serves them).
-__global__ void __launch_bounds__(PT_THREADS) prefill_tc_score_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(PT_THREADS, 2) prefill_tc_score_kernel(PrefillArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* ktile = smem + PT_OFF_K;
+    uint8_t* qtile = smem + PT_OFF_Q;
     uint16_t* otile = reinterpret_cast<uint16_t*>(smem + PT_OFF_OUT);
     float* ws_ = reinterpret_cast<float*>(smem + PT_OFF_W);
     int* vis = reinterpret_cast<int*>(smem + PT_OFF_VIS);
@@ -1236,25 +1266,23 @@ __global__ void __launch_bounds__(PT_THREADS) prefill_tc_score_kernel(PrefillArg
         if (tid == 0) a.kmax[part] = 0.f;
         return;
     }
-    // A fragments of Q_h (16 queries x 64 dims, bf16 pairs), all heads and k-steps
-    uint32_t qa[kIH][4][4];
-    {
-        const int qr0 = q0 + 16 * wq + g, qr1 = qr0 + 8;
-#pragma unroll
-        for (int h = 0; h < kIH; ++h)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int d = 16 * c + 2 * t;
-                auto ld = [&](int q, int dd) -> uint32_t {
-                    return q < a.T ? __ldg(reinterpret_cast<const uint32_t*>(a.q_idx + ((int64_t)q * kIH + h) * kID + dd))
-                                   : 0u;
-                };
-                qa[h][c][0] = ld(qr0, d);
-                qa[h][c][1] = ld(qr1, d);
-                qa[h][c][2] = ld(qr0, d + 8);
-                qa[h][c][3] = ld(qr1, d + 8);
-            }
+    // Q of the 64 queries in shared memory: query row r holds 32 chunks of 16 B
+    // (head h, dims 8c2..8c2+7 at chunk 8 h + c2), stored at chunk ^ (r & 7) so
+    // ldmatrix reads 8 rows on 8 distinct bank groups
+    for (int i = tid; i < PT_Q * 32; i += PT_THREADS) {
+        const int r = i >> 5, ch = i & 31;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (q0 + r < a.T) v = __ldg(reinterpret_cast<const uint4*>(a.q_idx + (int64_t)(q0 + r) * kIH * kID) + ch);
+        *reinterpret_cast<uint4*>(qtile + r * 512 + ((ch ^ (r & 7)) << 4)) = v;
     }
+    // lane address of the A fragment (16 queries x 16 dims) of head h, k-step c:
+    // matrix m = lane / 8 holds queries (m & 1) * 8 + lane % 8, dims 16 c + (m >> 1) * 8
+    const int qrow = 16 * wq + ((lane >> 3) & 1) * 8 + (lane & 7);
+    const uint32_t qa_row = smem_u32(qtile + qrow * 512);
+    auto qa_addr = [&](int h, int c) {
+        const int ch = 8 * h + 2 * c + (lane >> 4);
+        return qa_row + (uint32_t)((ch ^ (qrow & 7)) << 4);
+    };
     const int sh = a.page_shift;
     const int32_t emask = (1 << sh) - 1;
     // tile copies: 64 rows x 8 chunks, two chunks per thread; chunk c of row r at c ^ (r & 7)
@@ -1317,9 +1345,12 @@ __global__ void __launch_bounds__(PT_THREADS) prefill_tc_score_kernel(PrefillArg
                             b[2 * jj + 1][0], b[2 * jj + 1][1]);
             }
 #pragma unroll
-            for (int h = 0; h < kIH; ++h)
+            for (int h = 0; h < kIH; ++h) {
+                uint32_t qa[4];
+                ldsm_x4_b16(qa_addr(h, c), qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
-                for (int n = 0; n < 4; ++n) mma_bf16_16816(acc[h][n], qa[h][c], b[n][0], b[n][1]);
+                for (int n = 0; n < 4; ++n) mma_bf16_16816(acc[h][n], qa, b[n][0], b[n][1]);
+            }
         }
         // epilogue: score = sum_h w_h relu(q_h . k) (fp32, heads in order), 16-bit key
 #pragma unroll
@@ -1330,14 +1361,14 @@ __global__ void __launch_bounds__(PT_THREADS) prefill_tc_score_kernel(PrefillArg
                 float s = 0.f;
 #pragma unroll
                 for (int h = 0; h < kIH; ++h) s = __fmaf_rn(ws_[ql * kIH + h], fmaxf(acc[h][n][i], 0.f), s);
-                otile[ql * PT_E + el] = e0 + el < vis[ql] ? (uint16_t)(score_key(s) >> 16) : (uint16_t)0;
+                otile[ql * PT_OROW + el] = e0 + el < vis[ql] ? (uint16_t)(score_key(s) >> 16) : (uint16_t)0;
             }
         __syncthreads();  // the out tile is complete; buffer `buf` may be refilled
         for (int i = tid; i < PT_Q * PT_E / 8; i += PT_THREADS) {
             const int ql = i >> 3, c = i & 7;
             if (q0 + ql < a.T)
                 *reinterpret_cast<uint4*>(a.keys16 + (int64_t)(q0 + ql) * a.stride + e0 + c * 8) =
-                    *reinterpret_cast<const uint4*>(otile + ql * PT_E + c * 8);
+                    *reinterpret_cast<const uint4*>(otile + ql * PT_OROW + c * 8);
         }
     }
     // max |k| of the CTA's entries
@@ -1356,7 +1387,7 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-constexpr int PC_THREADS = 512;
+constexpr int PC_THREADS = 256;
 constexpr size_t PC_OFF_K16 = 0;                                      // [16384] u16
 constexpr size_t PC_OFF_CK = PC_OFF_K16 + (size_t)kMaxCand * 2;        // [2048] u32 exact keys
 constexpr size_t PC_OFF_CAND = PC_OFF_CK + PT_CAND_MAX * 4;            // [2048] u16 entries
@@ -1413,24 +1444,42 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
         s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)t * kIH);
         s_u[1] = 0;
     }
-    for (int i = tid; i < n_vis; i += PC_THREADS) k16[i] = a.keys16[(int64_t)t * a.stride + i];
-    for (int i = tid; i < 256; i += PC_THREADS) hist[i] = 0;
+    {  // the visible entries' 16-bit keys, 16 B at a time (rows are 128 B aligned)
+        const uint4* src = reinterpret_cast<const uint4*>(a.keys16 + (int64_t)t * a.stride);
+        for (int i = tid; i < (n_vis + 7) / 8; i += PC_THREADS) reinterpret_cast<uint4*>(k16)[i] = __ldcg(src + i);
+    }
+    for (int i = tid; i < 1024; i += PC_THREADS) hist[i] = 0;
     __syncthreads();
 
-    // ---- candidates: the entries whose 16-bit key is >= the PT_CAND-th largest
-    uint32_t thr16 = 0u;  // 0: every visible entry is a candidate
-    if (n_vis > PT_CAND) {
-        for (int i = tid; i < n_vis; i += PC_THREADS) hist_add(hist, k16[i] >> 8, true);
+    // ---- candidates: entries whose 16-bit key is >= that of the PT_CAND-th
+    // largest.  The histogram counts each key's distance below the row's
+    // largest key (one bin per key value, 1024 values = 8 binades); distances
+    // beyond are not counted, and a row whose PT_CAND-th key lies beyond takes
+    // the exact fallback.
+    const bool limited = n_vis > PT_CAND;
+    uint32_t thr16 = 0u;
+    if (limited) {
+        uint32_t mx = 0;
+        for (int i = tid; i < n_vis; i += PC_THREADS) mx = max(mx, (uint32_t)k16[i]);
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) tmp[wid] = mx;
         __syncthreads();
-        int b1, b2;
-        uint32_t above;
-        find_kth_bin(hist, 256, PT_CAND, tmp, &b1, &above);
-        for (int i = tid; i < 256; i += PC_THREADS) hist[i] = 0;
+        mx = 0;
+        for (int v = 0; v < PC_THREADS / 32; ++v) mx = max(mx, tmp[v]);
         __syncthreads();
-        for (int i = tid; i < n_vis; i += PC_THREADS) hist_add(hist, k16[i] & 255u, (int)(k16[i] >> 8) == b1);
+        for (int i = tid; i < n_vis; i += PC_THREADS) {
+            const uint32_t dist = mx - (uint32_t)k16[i];
+            hist_add(hist, 1023u - dist, dist < 1024u);
+        }
         __syncthreads();
-        find_kth_bin(hist, 256, PT_CAND - above, tmp, &b2, &above);
-        thr16 = ((uint32_t)b1 << 8) | (uint32_t)b2;
+        int b;
+        uint32_t above, counted;
+        group_find_kth_bin(hist, 1024, PT_CAND, tmp, &b, &above, GroupBar{0, PC_THREADS}, &counted);
+        if (counted < (uint32_t)PT_CAND) {  // the threshold lies more than 8 binades below the maximum
+            if (tid == 0) a.flags[t] = 1;
+            return;
+        }
+        thr16 = mx - (1023u - (uint32_t)b);
     }
     // compact in entry order (the output must come out ascending): warp v
     // walks a contiguous segment, counts, then writes at its prefix offset
@@ -1439,7 +1488,7 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
     uint32_t mine = 0;
     for (int b = lo; b < hi; b += 32) {
         const int i = b + lane;
-        mine += __popc(__ballot_sync(0xffffffffu, i < hi && (uint32_t)k16[i] >= thr16));
+        mine += __popc(__ballot_sync(0xffffffffu, i < hi && (!limited || (uint32_t)k16[i] >= thr16)));
     }
     __syncthreads();
     if (lane == 0) tmp[wid] = mine;
@@ -1456,7 +1505,7 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
     }
     for (int b = lo; b < hi; b += 32) {
         const int i = b + lane;
-        const bool in = i < hi && (uint32_t)k16[i] >= thr16;
+        const bool in = i < hi && (!limited || (uint32_t)k16[i] >= thr16);
         const unsigned bm = __ballot_sync(0xffffffffu, in);
         if (in) cand[off + __popc(bm & ((1u << lane) - 1u))] = (uint16_t)i;
         off += __popc(bm);
@@ -1506,7 +1555,7 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
     find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
     refine_threshold(ck, m, (uint32_t)b1, kk - above, hist, l0, l1, tmp, &T, &need);
     // ---- no entry outside the candidates can reach the K-th exact score
-    if (thr16 != 0u) {
+    if (limited) {
         const double bound = (double)key_value(thr16 << 16);  // non-candidates score below this (approximately)
         const double delta = 0x1p-12 * (fabs((double)w.x) * s_l1[0] + fabs((double)w.y) * s_l1[1] +
                                         fabs((double)w.z) * s_l1[2] + fabs((double)w.w) * s_l1[3]) *
@@ -1694,7 +1743,7 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     LaunchCfg c1(dim3((unsigned)((T + PS_Q - 1) / PS_Q)), dim3(PS_THREADS), PS_SMEM, stream);
     e = cudaLaunchKernelEx(&c1.cfg, prefill_score_kernel, a);
     if (e != cudaSuccess) return e;
-    LaunchCfg c2(dim3((unsigned)T), dim3(PSEL_THREADS), PSEL_SMEM, stream);
+    LaunchCfg c2(dim3((unsigned)std::min(T, 2 * sm_count())), dim3(PSEL_THREADS), PSEL_SMEM, stream);
     return cudaLaunchKernelEx(&c2.cfg, prefill_select_kernel, a);
 }
 
