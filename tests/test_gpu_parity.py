@@ -256,10 +256,11 @@ def run_decode_layers(csa2, ps, lens, q_idx, w, q, swa, max_len, ws=None):
                 lse=[x.cpu().numpy() for x in lse], modes=modes)
 
 
-def test_decode_layers_vs_oracle(csa2, orc):
+@pytest.mark.parametrize("page_size", [64, 8, 1024])
+def test_decode_layers_vs_oracle(csa2, orc, page_size):
     lens = [20000, 9000, 130]
     B, max_len = len(lens), max(lens)
-    ps = PagedSeqs(csa2, lens)
+    ps = PagedSeqs(csa2, lens, page_size=page_size)
     data = [_fill(ps, b, L) for b, L in enumerate(lens)]
     q_idx, w, q, swa = _decode_layer_inputs(B, lens)
     snap = [t.clone() for t in (ps.cache.codes, ps.cache.scales, ps.cache.idx_k, ps.cache.pooled)]
@@ -318,6 +319,43 @@ def test_prefill_parity(csa2, orc):
                              T, err=ps.err)
     ro, rl = orc.prefill_attn(q_pos, q, want, codes, scales, swa, swa_start)
     check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, "prefill attention")
+    assert ps.errors() == 0
+
+
+def test_prefill_scattered_queries(csa2, orc):
+    # queries at non-consecutive positions, in no particular order: the window
+    # branch walks the union of 16 queries' windows, the indexer's query tiles
+    # and the per-query kernels see unrelated neighbours
+    seed = 1003
+    tokens = 4096 + 62
+    n_ent = tokens // 2
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 0, 0, tokens)
+    idx_k = synth.idx_k_rows(seed, 0, 0, n_ent)
+    ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=999)
+    kvb = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+    codes, scales = orc.quant_rows(kvb, ratio=2)
+    rng = np.random.default_rng(5)
+    q_pos = rng.choice(np.arange(700, tokens), size=96, replace=False).astype(np.int32)
+    T = len(q_pos)
+    q_idx = synth.q_idx(seed, 0, 0, T)
+    w = synth.w_idx(seed, 0, 0, T)
+    d = csa2.default_desc(csa2.FULL, 2)
+    ws = _ws(csa2, T, n_ent, prefill=True)
+    out_idx = torch.empty((T, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q_idx), dev(w), dev(np.array([n_ent], np.int32)), out_idx, T,
+                      n_ent, ws, q_pos=dev(q_pos), err=ps.err)
+    want = orc.prefill_indexer(q_pos, 2, n_ent, idx_k, q_idx, w)
+    check_sets(out_idx.cpu().numpy(), want, "prefill indexer, scattered queries")
+    swa_start = int(q_pos.min()) - 127
+    swa = synth.swa_rows(seed, 0, 0, tokens - swa_start)
+    q = synth.q_heads(seed, 0, 0, T)
+    out = torch.empty((T, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_prefill(d, ps.cache, bits16(q), out_idx, dev(q_pos), bits16(swa), swa_start, n_ent, out, lse,
+                             T, err=ps.err)
+    ro, rl = orc.prefill_attn(q_pos, q, want, codes, scales, swa, swa_start)
+    check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, "prefill attention, scattered queries")
     assert ps.errors() == 0
 
 
