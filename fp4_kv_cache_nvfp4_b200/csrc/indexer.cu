@@ -905,42 +905,54 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
         uint32_t above;
         find_kth_bin(g1, kHistBins, kk, tmp, &b1, &above);
         need = kk - above;
-        // digit 2 (bits 19..10) over this CTA's survivors of digit 1
-        if (tid == 0) {
-            s_cnt[0] = 0;
-            s_cnt[1] = 0;
+        // A bin whose keys are all taken ends the search: T just below it, no
+        // ties (the histograms are the cluster's, so every CTA decides alike).
+        if (b1 > 0 && g1[b1] == need) {
+            T = ((uint32_t)b1 << 20) - 1u;
+            need = 0;
+        } else {
+            // digit 2 (bits 19..10) over this CTA's survivors of digit 1
+            if (tid == 0) {
+                s_cnt[0] = 0;
+                s_cnt[1] = 0;
+            }
+            for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
+            __syncthreads();
+            for (int base = wid * 32; base < TK_SLOTS; base += TK_THREADS) {
+                const int i = base + lane;
+                const uint32_t k = keys[i];
+                const bool in = k != 0u && (int)(k >> 20) == b1;
+                list_append(l0, &s_cnt[0], (uint32_t)i, in);
+                hist_add(hist, (k >> 10) & 1023u, in);
+            }
+            __syncthreads();
+            push_hist(hist, 1024, g2);
+            cluster_sync_all();
+            find_kth_bin(g2, 1024, need, tmp, &d2, &above);
+            need -= above;
+            if (g2[d2] == need) {
+                T = (((uint32_t)b1 << 20) | ((uint32_t)d2 << 10)) - 1u;
+                need = 0;
+            } else {
+                const int n0 = (int)s_cnt[0];
+                for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
+                __syncthreads();
+                for (int base = wid * 32; base < n0; base += TK_THREADS) {
+                    const int i = base + lane;
+                    const int slot = i < n0 ? (int)l0[i] : 0;
+                    const uint32_t k = i < n0 ? keys[slot] : 0u;
+                    const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
+                    list_append(l1, &s_cnt[1], (uint32_t)slot, in);
+                    hist_add(hist, k & 1023u, in);
+                }
+                __syncthreads();
+                push_hist(hist, 1024, g3);
+                cluster_sync_all();
+                find_kth_bin(g3, 1024, need, tmp, &d3, &above);
+                need -= above;
+                T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+            }
         }
-        for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
-        __syncthreads();
-        for (int base = wid * 32; base < TK_SLOTS; base += TK_THREADS) {
-            const int i = base + lane;
-            const uint32_t k = keys[i];
-            const bool in = k != 0u && (int)(k >> 20) == b1;
-            list_append(l0, &s_cnt[0], (uint32_t)i, in);
-            hist_add(hist, (k >> 10) & 1023u, in);
-        }
-        __syncthreads();
-        push_hist(hist, 1024, g2);
-        cluster_sync_all();
-        find_kth_bin(g2, 1024, need, tmp, &d2, &above);
-        need -= above;
-        const int n0 = (int)s_cnt[0];
-        for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
-        __syncthreads();
-        for (int base = wid * 32; base < n0; base += TK_THREADS) {
-            const int i = base + lane;
-            const int slot = i < n0 ? (int)l0[i] : 0;
-            const uint32_t k = i < n0 ? keys[slot] : 0u;
-            const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
-            list_append(l1, &s_cnt[1], (uint32_t)slot, in);
-            hist_add(hist, k & 1023u, in);
-        }
-        __syncthreads();
-        push_hist(hist, 1024, g3);
-        cluster_sync_all();
-        find_kth_bin(g3, 1024, need, tmp, &d3, &above);
-        need -= above;
-        T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
     }
 
     // ---- ordered emission: per-CTA counts to every CTA, then own offsets -----
