@@ -198,6 +198,13 @@ __device__ void refine_threshold(const uint32_t* keys, int nslots, uint32_t b1, 
     uint32_t above;
     find_kth_bin(hist, 1024, need, tmp, &d2, &above);
     need -= above;
+    const uint32_t base22 = (b1 << 20) | ((uint32_t)d2 << 10);
+    if (base22 > 0u && hist[d2] == need) {  // the bin is taken whole: T just below it, no ties
+        *T_out = base22 - 1u;
+        *need_out = 0;
+        return;
+    }
+    __syncthreads();  // every thread has read hist[d2]
     for (int i = tid; i < 1024; i += nt) hist[i] = 0;
     __syncthreads();
     for (int base = wid * 32; base < n0; base += nt) {
