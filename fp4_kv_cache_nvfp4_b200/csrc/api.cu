@@ -120,6 +120,7 @@ static csa2_status indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache
     if (level == CSA2_LEVEL_BLOCK && (max_len > kMaxBlockLevelLen || n > 1024)) return CSA2_ERR_UNSUPPORTED;
     if (level == CSA2_LEVEL_BLOCK && cache->n_phys_pages * cache->page_size / 8 > 0x7fffffff) return CSA2_ERR_UNSUPPORTED;
     if (prefill && max_len > kMaxCand) return CSA2_ERR_UNSUPPORTED;
+    if (prefill && !aligned(q_idx, 16)) return CSA2_ERR_INVALID_ARG;  // read in 16-byte rows by the tensor-core tiles
     if (max_len > (int64_t)cache->max_pages_per_seq * cache->page_size) return CSA2_ERR_INVALID_ARG;
     const size_t need = csa2_indexer_workspace_bytes(desc, level, n, max_len, prefill ? 1 : 0);
     if (!workspace || !aligned(workspace, 256) || ws_bytes < need) return CSA2_ERR_WORKSPACE;

@@ -1227,178 +1227,264 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
 // B + delta >= the K-th exact score, the query is flagged and the exact
 // CUDA-core kernels recompute it.  The output is therefore the exact Top-K.
 // ============================================================================
-constexpr int PT_Q = 64;          // queries per CTA
-constexpr int PT_E = 64;          // entries per K tile
 constexpr int PT_SPLIT = 2048;    // entries per CTA (grid.y splits the entry range)
-constexpr int PT_THREADS = 256;
 constexpr int PT_CAND = 768;      // approximate candidates per query
 constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit threshold) -> exact fallback
-constexpr int PT_OROW = PT_E + 8;                               // out-tile row (u16): 144 B, rows on distinct banks
-constexpr size_t PT_OFF_K = 0;                                  // 2 x [64][64] bf16, 16 B chunks swizzled
-constexpr size_t PT_OFF_Q = PT_OFF_K + 2 * PT_E * 128;          // [64 q][4 h][64] bf16, chunks swizzled by q
-constexpr size_t PT_OFF_OUT = PT_OFF_Q + (size_t)PT_Q * kIH * kID * 2;  // [64 q][72] u16
-constexpr size_t PT_OFF_W = PT_OFF_OUT + PT_Q * PT_OROW * 2;    // [64][4] f32
-constexpr size_t PT_OFF_VIS = PT_OFF_W + PT_Q * kIH * 4;        // [64] int
-constexpr size_t PT_OFF_RED = PT_OFF_VIS + PT_Q * 4;            // [8] u32
-constexpr size_t PT_SMEM = PT_OFF_RED + 8 * 4;
-static_assert(PT_OFF_OUT % 16 == 0 && PT_OFF_W % 16 == 0, "K5a shared-memory layout");
 
-__device__ __forceinline__ void ldsm_x4_b16(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
+// ---- tcgen05 helpers (5th-generation tensor cores, accumulators in TMEM) ----
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand tile
+// (rows of 128 B, 8-row groups 1024 B apart, chunk c of row r at c ^ (r & 7);
+// the tile starts on a 1024-byte boundary).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+// D[128 x n] (+)= A[128 x 16] . B[n x 16]^T, bf16 inputs, fp32 accumulators in TMEM
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
 }
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(addr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Warp w: queries 16 (w & 3) .. +16 of the CTA's 64, entries 32 (w >> 2) .. +32
-// of each 64-entry tile (four n8 tiles), all four heads (one K tile serves them).
-__global__ void __launch_bounds__(PT_THREADS, 2) prefill_tc_score_kernel(PrefillArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* ktile = smem + PT_OFF_K;
-    uint8_t* qtile = smem + PT_OFF_Q;
-    uint16_t* otile = reinterpret_cast<uint16_t*>(smem + PT_OFF_OUT);
-    float* ws_ = reinterpret_cast<float*>(smem + PT_OFF_W);
-    int* vis = reinterpret_cast<int*>(smem + PT_OFF_VIS);
-    uint32_t* red = reinterpret_cast<uint32_t*>(smem + PT_OFF_RED);
+// K5a on tcgen05: a CTA scores 128 queries (MMA M, one TMEM lane each) against
+// its range of entries, 64 at a time (MMA N), all four heads (4 accumulators
+// of 64 columns, double-buffered: 512 TMEM columns).
+//   warps 0-3  epilogue: thread q reads lane q of the four accumulators with
+//              tcgen05.ld, computes sum_h w_h relu(.) and writes 16-bit keys
+//   warp 4     producer: K tiles by cp.async into a 4-stage ring (chunk
+//              swizzle of the canonical 128-byte layout); it waits for its
+//              own copies two tiles behind, fences them for the tensor core
+//              (generic -> async proxy) and marks the stage full
+//   warp 5     MMA: one thread issues 16 tcgen05.mma per tile and commits to
+//              the tile's "done" and the stage's "empty" barriers
+//   warp 6     max |k| of every staged tile (the verification bound)
+constexpr int TC_Q = 128;
+constexpr int TC_E = 64;
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 7 * 32;
+constexpr size_t TC_OFF_Q = 0;                                          // 4 heads x [128][128 B]
+constexpr size_t TC_OFF_K = TC_OFF_Q + (size_t)kIH * TC_Q * 128;        // 4 stages x [64][128 B]
+constexpr size_t TC_OFF_BAR = TC_OFF_K + (size_t)TC_STAGES * TC_E * 128;  // full[4] empty[4] done[2] free[2]
+constexpr size_t TC_OFF_MISC = TC_OFF_BAR + 12 * 8;                     // tmem base, timeout
+constexpr size_t TC_SMEM = 120 * 1024;                                  // one CTA per SM: it owns all of TMEM
+static_assert(TC_OFF_MISC + 16 <= TC_SMEM && TC_OFF_K % 1024 == 0, "K5a (tcgen05) shared-memory layout");
+
+__global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(PrefillArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
+    uint64_t* empty = full + TC_STAGES;
+    uint64_t* done = empty + TC_STAGES;
+    uint64_t* tfree = done + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
+    int* s_timeout = reinterpret_cast<int*>(smem + TC_OFF_MISC + 4);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int g = lane >> 2, t = lane & 3, wq = wid & 3, we = wid >> 2;
-    const int q0 = blockIdx.x * PT_Q;
+    const int q0 = blockIdx.x * TC_Q;
     const int part = blockIdx.x + gridDim.x * blockIdx.y;
     pdl_wait();
     pdl_trigger();
-    if (tid < PT_Q) vis[tid] = q0 + tid < a.T ? visible(a.q_pos[q0 + tid], a.ratio, a.n_entries) : 0;
-    for (int i = tid; i < PT_Q * kIH; i += PT_THREADS) {
-        const int q = q0 + i / kIH;
-        ws_[i] = q < a.T ? a.w[(int64_t)q * kIH + i % kIH] : 0.f;
+    if (smem_u32(smem) & 1023u) {  // the swizzled operand tiles need a 1 KiB-aligned base (uniform)
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
     }
-    __syncthreads();
+    // entry range of this CTA: the split, cut at the largest visibility of its queries
     int max_vis = 0;
-    for (int i = 0; i < PT_Q; ++i) max_vis = max(max_vis, vis[i]);
+    for (int i = lane; i < TC_Q; i += 32)
+        if (q0 + i < a.T) max_vis = max(max_vis, visible(a.q_pos[q0 + i], a.ratio, a.n_entries));
+    for (int o = 16; o > 0; o >>= 1) max_vis = max(max_vis, __shfl_xor_sync(0xffffffffu, max_vis, o));
     const int e_beg = blockIdx.y * PT_SPLIT, e_end = min(e_beg + PT_SPLIT, max_vis);
     if (e_beg >= e_end) {
         if (tid == 0) a.kmax[part] = 0.f;
         return;
     }
-    // Q of the 64 queries in shared memory: query row r holds 32 chunks of 16 B
-    // (head h, dims 8c2..8c2+7 at chunk 8 h + c2), stored at chunk ^ (r & 7) so
-    // ldmatrix reads 8 rows on 8 distinct bank groups
-    for (int i = tid; i < PT_Q * 32; i += PT_THREADS) {
-        const int r = i >> 5, ch = i & 31;
+    const int ntile = (e_end - e_beg + TC_E - 1) / TC_E;
+    // Q of the 128 queries, one 128-byte-swizzled tile per head
+    for (int i = tid; i < TC_Q * kIH * 8; i += TC_THREADS) {
+        const int q = i >> 5, h = (i >> 3) & 3, c = i & 7;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (q0 + r < a.T) v = __ldg(reinterpret_cast<const uint4*>(a.q_idx + (int64_t)(q0 + r) * kIH * kID) + ch);
-        *reinterpret_cast<uint4*>(qtile + r * 512 + ((ch ^ (r & 7)) << 4)) = v;
+        if (q0 + q < a.T) v = __ldg(reinterpret_cast<const uint4*>(a.q_idx + ((int64_t)(q0 + q) * kIH + h) * kID) + c);
+        *reinterpret_cast<uint4*>(smem + TC_OFF_Q + (size_t)h * TC_Q * 128 + q * 128 + ((c ^ (q & 7)) << 4)) = v;
     }
-    // lane address of the A fragment (16 queries x 16 dims) of head h, k-step c:
-    // matrix m = lane / 8 holds queries (m & 1) * 8 + lane % 8, dims 16 c + (m >> 1) * 8
-    const int qrow = 16 * wq + ((lane >> 3) & 1) * 8 + (lane & 7);
-    const uint32_t qa_row = smem_u32(qtile + qrow * 512);
-    auto qa_addr = [&](int h, int c) {
-        const int ch = 8 * h + 2 * c + (lane >> 4);
-        return qa_row + (uint32_t)((ch ^ (qrow & 7)) << 4);
-    };
-    const int sh = a.page_shift;
-    const int32_t emask = (1 << sh) - 1;
-    // tile copies: 64 rows x 8 chunks, two chunks per thread; chunk c of row r at c ^ (r & 7)
-    auto issue = [&](int e0, int buf) {
+    if (tid == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 2);  // the MMA commit and the max-|k| warp
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&done[b], 1);
+            mbar_init(&tfree[b], 4);  // one arrival per epilogue warp
+        }
+        *s_timeout = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    fence_proxy_async_smem();  // the Q tiles are read by the tensor core
+    if (wid == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(512)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (wid == 4) {
+        // ================= producer =================
+        const int sh = a.page_shift;
+        const int32_t emask = (1 << sh) - 1;
+        auto issue = [&](int i) {
+            const int s = i % TC_STAGES, e0 = e_beg + i * TC_E;
+            uint8_t* st = smem + TC_OFF_K + (size_t)s * TC_E * 128;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int i = tid + PT_THREADS * k, r = i >> 3, c = i & 7;
-            const int e = e0 + r;
-            uint8_t* dst = ktile + (size_t)buf * PT_E * 128 + r * 128 + ((c ^ (r & 7)) << 4);
-            int32_t phys = -1;
-            if (e < e_end) {
-                const int32_t pg = e >> sh;
-                phys = pg < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + pg) : -1;
-                if (phys < 0 || phys >= a.cache.n_phys_pages) {
-                    dev_error(a.err, CSA2_DEV_PAGE);
-                    phys = -1;
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = lane + 32 * rr, e = e0 + r;
+                int32_t phys = -1;
+                if (e < e_end) {
+                    const int32_t pg = e >> sh;
+                    phys = pg < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + pg) : -1;
+                    if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                        dev_error(a.err, CSA2_DEV_PAGE);
+                        phys = -1;
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint8_t* dst = st + r * 128 + ((c ^ (r & 7)) << 4);
+                    if (phys >= 0) cp_async16(dst, a.cache.idx_k + (((int64_t)phys << sh) | (e & emask)) * kID + c * 8);
+                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
                 }
             }
-            if (phys >= 0) {
-                const int64_t slot = ((int64_t)phys << sh) | (e & emask);
-                cp_async16(dst, a.cache.idx_k + slot * kID + c * 8);
-            } else {
-                *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        };
+        auto publish = [&](int i) {  // tile i's copies have landed: make them visible to the tensor core
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[i % TC_STAGES]);
+        };
+        for (int i = 0; i < ntile + 2; ++i) {
+            if (i < ntile) {
+                if (i >= TC_STAGES &&
+                    !mbar_wait(&empty[i % TC_STAGES], (uint32_t)((i / TC_STAGES) - 1) & 1u, kWaitLimit))
+                    *s_timeout = 1;
+                issue(i);
+            }
+            cp_async_commit();
+            if (i >= 2) {
+                cp_async_wait<2>();  // tile i - 2 is in shared memory
+                publish(i - 2);
             }
         }
-        cp_async_commit();
-    };
-    uint32_t kmax_bits = 0;  // max |k| as bf16 bits (positive values order as integers)
-    const int ntile = (e_end - e_beg + PT_E - 1) / PT_E;
-    issue(e_beg, 0);
-    for (int it = 0; it < ntile; ++it) {
-        const int e0 = e_beg + it * PT_E, buf = it & 1;
-        if (it + 1 < ntile) issue(e0 + PT_E, buf ^ 1);
-        else cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();  // tile `it` is in shared memory for every warp
-        const uint8_t* kt = ktile + (size_t)buf * PT_E * 128;
+    } else if (wid == 5) {
+        // ================= MMA issue =================
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_E >> 3) << 17) |
+                                   ((uint32_t)(TC_Q >> 4) << 24);  // bf16 x bf16 -> f32, K-major, M 128, N 64
+            for (int i = 0; i < ntile; ++i) {
+                const int s = i % TC_STAGES, buf = i & 1;
+                if (!mbar_wait(&full[s], (uint32_t)(i / TC_STAGES) & 1u, kWaitLimit)) *s_timeout = 1;
+                if (i >= 2 && !mbar_wait(&tfree[buf], (uint32_t)((i >> 1) - 1) & 1u, kWaitLimit)) *s_timeout = 1;
+                tc_fence_after();
+                const uint64_t db = umma_desc_sw128(smem_u32(smem + TC_OFF_K + (size_t)s * TC_E * 128));
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {  // the chunks this thread copied
-            const int i = tid + PT_THREADS * k, r = i >> 3, c = i & 7;
-            const uint4 v = *reinterpret_cast<const uint4*>(kt + r * 128 + ((c ^ (r & 7)) << 4));
-            const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+                for (int h = 0; h < kIH; ++h) {
+                    const uint64_t da = umma_desc_sw128(smem_u32(smem + TC_OFF_Q + (size_t)h * TC_Q * 128));
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                kmax_bits = max(kmax_bits, max(x[u] & 0x7fffu, (x[u] >> 16) & 0x7fffu));
-        }
-        float acc[kIH][4][4];
-#pragma unroll
-        for (int h = 0; h < kIH; ++h)
-#pragma unroll
-            for (int n = 0; n < 4; ++n) acc[h][n][0] = acc[h][n][1] = acc[h][n][2] = acc[h][n][3] = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t b[4][2];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {  // n8 tiles 2 jj and 2 jj + 1
-                const int m = lane >> 3, n = 2 * jj + (m >> 1), kh = m & 1;
-                const int r = 32 * we + 8 * n + (lane & 7), ch = 2 * c + kh;
-                ldsm_x4_b16(smem_u32(kt + r * 128 + ((ch ^ (r & 7)) << 4)), b[2 * jj][0], b[2 * jj][1],
-                            b[2 * jj + 1][0], b[2 * jj + 1][1]);
-            }
-#pragma unroll
-            for (int h = 0; h < kIH; ++h) {
-                uint32_t qa[4];
-                ldsm_x4_b16(qa_addr(h, c), qa[0], qa[1], qa[2], qa[3]);
-#pragma unroll
-                for (int n = 0; n < 4; ++n) mma_bf16_16816(acc[h][n], qa, b[n][0], b[n][1]);
+                    for (int kk = 0; kk < kID / 16; ++kk)  // +32 B per k-step of 16
+                        umma_bf16(tmem + (uint32_t)(buf * kIH * TC_E + h * TC_E), da + 2u * kk, db + 2u * kk, idesc,
+                                  kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&done[buf]);
+                umma_commit(&empty[s]);
             }
         }
-        // epilogue: score = sum_h w_h relu(q_h . k) (fp32, heads in order), 16-bit key
+        __syncwarp();
+    } else if (wid == 6) {
+        // ================= max |k| of the staged tiles =================
+        uint32_t kmax_bits = 0;
+        for (int i = 0; i < ntile; ++i) {
+            const int s = i % TC_STAGES, e0 = e_beg + i * TC_E;
+            if (!mbar_wait(&full[s], (uint32_t)(i / TC_STAGES) & 1u, kWaitLimit)) *s_timeout = 1;
+            const uint8_t* st = smem + TC_OFF_K + (size_t)s * TC_E * 128;
+            for (int j = lane; j < TC_E * 8; j += 32) {
+                if (e0 + (j >> 3) >= e_end) continue;
+                const uint4 v = *reinterpret_cast<const uint4*>(st + j * 16);
+                const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int ql = 16 * wq + g + 8 * (i >> 1), el = 32 * we + 8 * n + 2 * t + (i & 1);
-                float s = 0.f;
-#pragma unroll
-                for (int h = 0; h < kIH; ++h) s = __fmaf_rn(ws_[ql * kIH + h], fmaxf(acc[h][n][i], 0.f), s);
-                otile[ql * PT_OROW + el] = e0 + el < vis[ql] ? (uint16_t)(score_key(s) >> 16) : (uint16_t)0;
+                for (int u = 0; u < 4; ++u) kmax_bits = max(kmax_bits, max(x[u] & 0x7fffu, (x[u] >> 16) & 0x7fffu));
             }
-        __syncthreads();  // the out tile is complete; buffer `buf` may be refilled
-        for (int i = tid; i < PT_Q * PT_E / 8; i += PT_THREADS) {
-            const int ql = i >> 3, c = i & 7;
-            if (q0 + ql < a.T)
-                *reinterpret_cast<uint4*>(a.keys16 + (int64_t)(q0 + ql) * a.stride + e0 + c * 8) =
-                    *reinterpret_cast<const uint4*>(otile + ql * PT_OROW + c * 8);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        for (int o = 16; o > 0; o >>= 1) kmax_bits = max(kmax_bits, __shfl_xor_sync(0xffffffffu, kmax_bits, o));
+        if (lane == 0) a.kmax[part] = __uint_as_float(kmax_bits << 16);
+    } else {
+        // ================= epilogue: thread = query = TMEM lane =================
+        const int ql = tid, t = q0 + ql;
+        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+        int vis = 0;
+        if (t < a.T) {
+            w = *reinterpret_cast<const float4*>(a.w + (int64_t)t * kIH);
+            vis = visible(a.q_pos[t], a.ratio, a.n_entries);
+        }
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * wid) << 16);
+        for (int i = 0; i < ntile; ++i) {
+            const int buf = i & 1, e0 = e_beg + i * TC_E;
+            if (!mbar_wait(&done[buf], (uint32_t)(i >> 1) & 1u, kWaitLimit)) *s_timeout = 1;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < TC_E / 16; ++c) {
+                uint32_t v0[16], v1[16], v2[16], v3[16];
+                const uint32_t col = lane_base + (uint32_t)(buf * kIH * TC_E + 16 * c);
+                tmem_ld16(col, v0);
+                tmem_ld16(col + TC_E, v1);
+                tmem_ld16(col + 2 * TC_E, v2);
+                tmem_ld16(col + 3 * TC_E, v3);
+                tmem_wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float s = 0.f;
+                    s = __fmaf_rn(w.x, fmaxf(__uint_as_float(v0[j]), 0.f), s);
+                    s = __fmaf_rn(w.y, fmaxf(__uint_as_float(v1[j]), 0.f), s);
+                    s = __fmaf_rn(w.z, fmaxf(__uint_as_float(v2[j]), 0.f), s);
+                    s = __fmaf_rn(w.w, fmaxf(__uint_as_float(v3[j]), 0.f), s);
+                    const uint32_t k16 = e0 + 16 * c + j < vis ? score_key(s) >> 16 : 0u;
+                    if (j & 1) pk[j >> 1] |= k16 << 16;
+                    else pk[j >> 1] = k16;
+                }
+                if (t < a.T) {
+                    uint4* dst = reinterpret_cast<uint4*>(a.keys16 + (int64_t)t * a.stride + e0 + 16 * c);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tfree[buf]);
         }
     }
-    // max |k| of the CTA's entries
-    for (int o = 16; o > 0; o >>= 1) kmax_bits = max(kmax_bits, __shfl_xor_sync(0xffffffffu, kmax_bits, o));
-    if (lane == 0) red[wid] = kmax_bits;
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t m = 0;
-        for (int i = 0; i < PT_THREADS / 32; ++i) m = max(m, red[i]);
-        a.kmax[part] = __uint_as_float(m << 16);
+    tc_fence_before();
+    __syncthreads();  // every accumulator has been read
+    if (wid == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
+    if (tid == 0 && *s_timeout) dev_error(a.err, CSA2_DEV_TIMEOUT);
 }
 
 // float value of an order-preserving key (inverse of score_key)
@@ -1620,7 +1706,7 @@ DecodeWs decode_ws_layout(int n, int64_t max_len) {
 PrefillWs prefill_ws_layout(int T, int64_t n_entries) {
     PrefillWs l{};
     l.stride = (n_entries + PS_E - 1) / PS_E * PS_E;
-    l.kmax_parts = (int)(((T + PT_Q - 1) / PT_Q) * ((n_entries + PT_SPLIT - 1) / PT_SPLIT));
+    l.kmax_parts = (int)(((T + TC_Q - 1) / TC_Q) * ((n_entries + PT_SPLIT - 1) / PT_SPLIT));
     size_t o = 0;
     l.keys = o; o = align256(o + (size_t)T * l.stride * 4);
     l.flags = o; o = align256(o + (size_t)T * 4);
@@ -1726,7 +1812,7 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     static bool d1[64], d2[64], d3[64], d4[64];
     cudaError_t e = ensure_smem((const void*)prefill_select_kernel, PSEL_SMEM, d1);
     if (e == cudaSuccess) e = ensure_smem((const void*)prefill_score_kernel, PS_SMEM, d2);
-    if (e == cudaSuccess) e = ensure_smem((const void*)prefill_tc_score_kernel, PT_SMEM, d3);
+    if (e == cudaSuccess) e = ensure_smem((const void*)prefill_tc_score_kernel, TC_SMEM, d3);
     if (e == cudaSuccess) e = ensure_smem((const void*)prefill_candidates_kernel, PC_SMEM, d4);
     if (e != cudaSuccess) return e;
     (void)seq_lens;
@@ -1752,8 +1838,8 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     // tensor-core scores -> candidates, exact rescoring and verification; then
     // the exact CUDA-core path for the queries that failed the check (it exits
     // at once for the others)
-    LaunchCfg c0(dim3((unsigned)((T + PT_Q - 1) / PT_Q), (unsigned)((max_len + PT_SPLIT - 1) / PT_SPLIT)),
-                 dim3(PT_THREADS), PT_SMEM, stream);
+    LaunchCfg c0(dim3((unsigned)((T + TC_Q - 1) / TC_Q), (unsigned)((max_len + PT_SPLIT - 1) / PT_SPLIT)),
+                 dim3(TC_THREADS), TC_SMEM, stream);
     e = cudaLaunchKernelEx(&c0.cfg, prefill_tc_score_kernel, a);
     if (e != cudaSuccess) return e;
     LaunchCfg cc(dim3((unsigned)T), dim3(PC_THREADS), PC_SMEM, stream);

@@ -160,9 +160,13 @@ CSA2_API csa2_status csa2_kv_quant_append(const csa2_kv_cache* cache, const void
  *     the Full layer of this step), or all L positions if cand_blocks is NULL
  *     (then L <= 8 * keep_blocks).
  * Prefill (q_pos != NULL, level TOKEN): n queries of sequence 0 of the page
- *   table, q_idx [n][4][64], w [n][4], q_pos [n] absolute token positions,
- *   seq_lens [1] = entries in the cache (<= 16384); entry j is visible to the
- *   query at p iff (j+1)*ratio - 1 <= p; idx_out [n][topk].
+ *   table, q_idx [n][4][64] (16-byte aligned), w [n][4], q_pos [n] absolute
+ *   token positions, seq_lens [1] = entries in the cache (<= 16384); entry j
+ *   is visible to the query at p iff (j+1)*ratio - 1 <= p; idx_out [n][topk].
+ *   The result is the same exact Top-K: approximate tensor-core scores pick
+ *   candidates, which are rescored with the sequential FMA chains and checked
+ *   against a bound on the approximation; a query that fails the check is
+ *   recomputed exactly.
  * score_out is reserved (pass NULL).
  * workspace: device memory of csa2_indexer_workspace_bytes() bytes, 256-byte
  * aligned, zero-filled before its first use; every call leaves it zero-filled

@@ -76,6 +76,10 @@ def test_host_validation_without_gpu(csa2):
     # misaligned pointers and bad cache geometry
     assert L.csa2_sparse_attn_decode(ctypes.byref(d), ctypes.byref(c), P(0x1000), P(0x1000), P(0x1001),
                                      P(0x1000), None, P(0x1000), P(0x1000), 1, None, None) == 1
+    # the prefill indexer reads q_idx in 16-byte rows: 4-byte alignment is rejected
+    assert L.csa2_indexer_topk(ctypes.byref(csa2.default_desc(csa2.FULL, 2)), ctypes.byref(c), 1, P(0x1004),
+                               P(0x1000), P(0x1000), P(0x1000), None, P(0x1000), None, 1, 1000, P(ws), 1 << 30, None,
+                               None) == 1
     # prefill attention loads q and writes out in 16-byte vectors: 4-byte alignment is rejected
     for qp, op in ((0x1004, 0x1000), (0x1000, 0x1004)):
         assert L.csa2_sparse_attn_prefill(ctypes.byref(d), ctypes.byref(c), P(qp), P(0x1000), P(0x1000), P(0x1000),
