@@ -1265,25 +1265,29 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 // K5a on tcgen05: a CTA scores 128 queries (MMA M, one TMEM lane each) against
 // its range of entries, 64 at a time (MMA N), all four heads (4 accumulators
 // of 64 columns, double-buffered: 512 TMEM columns).
-//   warps 0-3  epilogue: thread q reads lane q of the four accumulators with
-//              tcgen05.ld, computes sum_h w_h relu(.) and writes 16-bit keys
-//   warp 4     producer: K tiles by cp.async into a 4-stage ring (chunk
+//   warps 0-7  epilogue: warps w and w + 4 read lane quarter w of the four
+//              accumulators (one query per thread, half of the 64 entries
+//              each) with tcgen05.ld, compute sum_h w_h relu(.), write keys
+//   warp 8     producer: K tiles by cp.async into a 4-stage ring (chunk
 //              swizzle of the canonical 128-byte layout); it waits for its
 //              own copies two tiles behind, fences them for the tensor core
 //              (generic -> async proxy) and marks the stage full
-//   warp 5     MMA: one thread issues 16 tcgen05.mma per tile and commits to
+//   warp 9     MMA: one thread issues 16 tcgen05.mma per tile and commits to
 //              the tile's "done" and the stage's "empty" barriers
-//   warp 6     max |k| of every staged tile (the verification bound)
+//   warp 10    max |k| of every staged tile (the verification bound)
 constexpr int TC_Q = 128;
 constexpr int TC_E = 64;
 constexpr int TC_STAGES = 4;
-constexpr int TC_THREADS = 7 * 32;
+constexpr int TC_THREADS = 11 * 32;
+constexpr int TC_EPI_WARPS = 8;
 constexpr size_t TC_OFF_Q = 0;                                          // 4 heads x [128][128 B]
 constexpr size_t TC_OFF_K = TC_OFF_Q + (size_t)kIH * TC_Q * 128;        // 4 stages x [64][128 B]
 constexpr size_t TC_OFF_BAR = TC_OFF_K + (size_t)TC_STAGES * TC_E * 128;  // full[4] empty[4] done[2] free[2]
 constexpr size_t TC_OFF_MISC = TC_OFF_BAR + 12 * 8;                     // tmem base, timeout
+constexpr size_t TC_OFF_PG = TC_OFF_MISC + 16;                          // physical pages of the entry range
+constexpr int TC_MAX_PG = PT_SPLIT / kBlk;                              // pages are >= 8 entries
 constexpr size_t TC_SMEM = 120 * 1024;                                  // one CTA per SM: it owns all of TMEM
-static_assert(TC_OFF_MISC + 16 <= TC_SMEM && TC_OFF_K % 1024 == 0, "K5a (tcgen05) shared-memory layout");
+static_assert(TC_OFF_PG + TC_MAX_PG * 4 <= TC_SMEM && TC_OFF_K % 1024 == 0, "K5a (tcgen05) shared-memory layout");
 
 __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1293,6 +1297,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     uint64_t* tfree = done + 2;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
     int* s_timeout = reinterpret_cast<int*>(smem + TC_OFF_MISC + 4);
+    int32_t* s_pg = reinterpret_cast<int32_t*>(smem + TC_OFF_PG);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int q0 = blockIdx.x * TC_Q;
     const int part = blockIdx.x + gridDim.x * blockIdx.y;
@@ -1313,6 +1318,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
         return;
     }
     const int ntile = (e_end - e_beg + TC_E - 1) / TC_E;
+    // physical pages of the entries [e_beg, e_end), loaded once (-1: outside the cache)
+    const int sh = a.page_shift;
+    const int pg0 = e_beg >> sh, npg = ((e_end - 1) >> sh) - pg0 + 1;
+    for (int i = tid; i < npg; i += TC_THREADS) {
+        const int pg = pg0 + i;
+        int32_t phys = pg < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + pg) : -1;
+        if (phys < 0 || phys >= a.cache.n_phys_pages) {
+            dev_error(a.err, CSA2_DEV_PAGE);
+            phys = -1;
+        }
+        s_pg[i] = phys;
+    }
     // Q of the 128 queries, one 128-byte-swizzled tile per head
     for (int i = tid; i < TC_Q * kIH * 8; i += TC_THREADS) {
         const int q = i >> 5, h = (i >> 3) & 3, c = i & 7;
@@ -1327,13 +1344,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&done[b], 1);
-            mbar_init(&tfree[b], 4);  // one arrival per epilogue warp
+            mbar_init(&tfree[b], TC_EPI_WARPS);  // one arrival per epilogue warp
         }
         *s_timeout = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     fence_proxy_async_smem();  // the Q tiles are read by the tensor core
-    if (wid == 5) {
+    if (wid == 9) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                      "r"(512)
                      : "memory");
@@ -1344,9 +1361,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (wid == 4) {
+    if (wid == 8) {
         // ================= producer =================
-        const int sh = a.page_shift;
         const int32_t emask = (1 << sh) - 1;
         auto issue = [&](int i) {
             const int s = i % TC_STAGES, e0 = e_beg + i * TC_E;
@@ -1354,15 +1370,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = lane + 32 * rr, e = e0 + r;
-                int32_t phys = -1;
-                if (e < e_end) {
-                    const int32_t pg = e >> sh;
-                    phys = pg < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + pg) : -1;
-                    if (phys < 0 || phys >= a.cache.n_phys_pages) {
-                        dev_error(a.err, CSA2_DEV_PAGE);
-                        phys = -1;
-                    }
-                }
+                const int32_t phys = e < e_end ? s_pg[(e >> sh) - pg0] : -1;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint8_t* dst = st + r * 128 + ((c ^ (r & 7)) << 4);
@@ -1389,7 +1397,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
                 publish(i - 2);
             }
         }
-    } else if (wid == 5) {
+    } else if (wid == 9) {
         // ================= MMA issue =================
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_E >> 3) << 17) |
@@ -1413,7 +1421,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
             }
         }
         __syncwarp();
-    } else if (wid == 6) {
+    } else if (wid == 10) {
         // ================= max |k| of the staged tiles =================
         uint32_t kmax_bits = 0;
         for (int i = 0; i < ntile; ++i) {
@@ -1434,20 +1442,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
         if (lane == 0) a.kmax[part] = __uint_as_float(kmax_bits << 16);
     } else {
         // ================= epilogue: thread = query = TMEM lane =================
-        const int ql = tid, t = q0 + ql;
+        const int quarter = wid & 3, half = wid >> 2;
+        const int ql = 32 * quarter + lane, t = q0 + ql;
         float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
         int vis = 0;
         if (t < a.T) {
             w = *reinterpret_cast<const float4*>(a.w + (int64_t)t * kIH);
             vis = visible(a.q_pos[t], a.ratio, a.n_entries);
         }
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * wid) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
         for (int i = 0; i < ntile; ++i) {
             const int buf = i & 1, e0 = e_beg + i * TC_E;
             if (!mbar_wait(&done[buf], (uint32_t)(i >> 1) & 1u, kWaitLimit)) *s_timeout = 1;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < TC_E / 16; ++c) {
+            for (int c = 2 * half; c < 2 * half + 2; ++c) {  // this warp's 32 of the 64 entries
                 uint32_t v0[16], v1[16], v2[16], v3[16];
                 const uint32_t col = lane_base + (uint32_t)(buf * kIH * TC_E + 16 * c);
                 tmem_ld16(col, v0);
@@ -1480,7 +1489,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     }
     tc_fence_before();
     __syncthreads();  // every accumulator has been read
-    if (wid == 5) {
+    if (wid == 9) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
@@ -1504,6 +1513,8 @@ constexpr size_t PC_OFF_TMP = PC_OFF_QD + kID * 16;                    // [64] u
 constexpr size_t PC_OFF_MISC = PC_OFF_TMP + 64 * 4;                    // w (float4), l1[4], kmax, thr, count
 constexpr size_t PC_SMEM = PC_OFF_MISC + 64;
 static_assert(PC_OFF_QD % 16 == 0 && PC_OFF_MISC % 16 == 0 && PC_OFF_HIST % 16 == 0, "K5b shared-memory layout");
+// the visible entries' page ids (pages hold >= 8 entries) fit in the l0/l1 lists' space
+static_assert((kMaxCand / 8) * 4 <= PC_OFF_QD - PC_OFF_L0, "K5b page-id staging");
 
 __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
