@@ -1,6 +1,6 @@
 """Benchmark: CSA2 decode over an NVFP4 main-KV cache at 1M context, batch 8.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--config 2|4]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--config 2|3|4|6]
 
 One step = one FP4 quant-append of the new token of every sequence + the 20
 decoder layers (Full + 3 Reuse, then 4 x (Reindex + 3 Reuse)), each layer
@@ -12,6 +12,10 @@ step.  Prints one JSON line (rank 0).
 Multi-GPU: one process per GPU (torchrun), each rank runs its own batch of 8
 sequences (weak scaling, no collective on the data path); the step time is the
 max over ranks.
+
+--config 3 times a prefill chunk instead; --config 6 the encoder side of one
+generated token: 18 ratio-2 layers (3 x (Full + 5 Reuse)) whose Full layers
+select over every entry (8 x 524,288 entries = 1M tokens each).
 
 --impl reference times the CPU oracle (the plain C restatement of the method)
 on the host cores on a bounded sample of the same workload.
@@ -33,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "CSA2 decode attn tokens/s @1M ctx & achieved HBM GB/s (fraction of roofline)"
+METRIC_ENC = "CSA2 encoder-side decode tokens/s @1M ctx (18 ratio-2 layers, flat indexer)"
 UNIT = "tokens/s"
 PAGE = 64
 CH = 256
@@ -44,7 +49,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    p.add_argument("--config", type=int, default=4, choices=[2, 3, 4])
+    p.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 6])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--kernel-reps", type=int, default=300)
     p.add_argument("--contiguous-pages", action="store_true")
@@ -57,7 +62,8 @@ def parse():
 def workload(cfg_id: int) -> dict:
     import synth
     c = synth.CONFIGS[cfg_id]
-    return dict(workload=c["name"], L=c["L"], B=c["B"], layers=c["layers"], seed=c["seed"])
+    return dict(workload=c["name"], L=c["L"], B=c["B"], layers=c["layers"], seed=c["seed"],
+                ratio=c.get("ratio", 1), decoder=c.get("decoder", True))
 
 
 def unique_bytes_per_seq(L: int, layers: int = 20) -> dict:
@@ -74,6 +80,19 @@ def unique_bytes_per_seq(L: int, layers: int = 20) -> dict:
     out = layers * (16 * 128 * 4 + 16 * 4)
     return dict(block=blk, token=tok, kv=kv, swa=swa, append=append, q=q, out=out,
                 total=blk + tok + kv + swa + append + q + out)
+
+
+def unique_bytes_per_seq_flat(L: int, layers: int, n_full: int, ratio: int = 2) -> dict:
+    """Algorithmic bytes of one encoder-side decode step for one sequence:
+    every Full layer reads the whole indexer K (it does not fit in L2, so each
+    of the n_full passes counts), then gathers its 512 FP4 entries."""
+    idx = n_full * L * 128
+    kv = n_full * min(512, L) * 144
+    swa = layers * min(128, L) * 512
+    append = ratio * 256 * 4 + 64 * 2 + 144 + 128
+    q = layers * 16 * 128 * 2 + n_full * (4 * 64 * 2 + 16)
+    out = layers * (16 * 128 * 4 + 16 * 4)
+    return dict(index=idx, kv=kv, swa=swa, append=append, q=q, out=out, total=idx + kv + swa + append + q + out)
 
 
 def attn_bytes_per_row(L: int) -> int:
@@ -162,6 +181,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     if args.batch or args.seq_len:
         W["workload"] += f"-override-b{W['B']}-l{W['L']}"
     B, L, layers, seed = W["B"], W["L"], W["layers"], W["seed"] + 100 * rank
+    ratio, flat = W["ratio"], not W["decoder"]  # flat: the encoder's layers (no block level)
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
 
@@ -177,18 +197,18 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
             m = min(chunk, L - s0)
             pos = torch.arange(s0, s0 + m, device=dev)
             slots = (tab_d[b, pos // PAGE] * PAGE + pos % PAGE).contiguous()
-            kv = torch.randn((m, CH), generator=gen, device=dev) * gain
+            kv = torch.randn((m * ratio, CH), generator=gen, device=dev) * gain
             ik = torch.randn((m, 64), generator=gen, device=dev).to(torch.bfloat16).view(torch.int16)
-            csa2.kv_quant_append(cache, kv, ik, slots)
+            csa2.kv_quant_append(cache, kv, ik, slots, ratio=ratio)
     torch.cuda.synchronize()
 
     # ---- per-layer inputs -------------------------------------------------------
-    modes = csa2.schedule(True)[:layers]
-    descs = [csa2.default_desc(m, 1) for m in modes]
+    modes = csa2.schedule(not flat)[:layers]
+    descs = [csa2.default_desc(m, ratio, **({"keep_blocks": 0} if flat else {})) for m in modes]
     n_idx = sum(1 for m in modes if m != csa2.REUSE)
     # one packed device buffer holds every per-step input, so one H2D copy refreshes it
     # (swa_new: every layer's newest SWA row; the end-to-end run scatters it into the rings)
-    sizes = dict(q=layers * B * 16 * 128 * 2, qi=layers * B * 4 * 64 * 2, w=layers * B * 4 * 4, kv=B * CH * 4,
+    sizes = dict(q=layers * B * 16 * 128 * 2, qi=layers * B * 4 * 64 * 2, w=layers * B * 4 * 4, kv=B * ratio * CH * 4,
                  ik=B * 64 * 2, swa_new=layers * B * CH * 2)
     offs, o = {}, 0
     for k, v in sizes.items():
@@ -202,7 +222,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     q_all = view("q", (layers, B, 16, 128), torch.int16)
     qi_all = view("qi", (layers, B, 4, 64), torch.int16)
     w_all = view("w", (layers, B, 4), torch.float32)
-    kv_new = view("kv", (B, CH), torch.float32)
+    kv_new = view("kv", (B * ratio, CH), torch.float32)  # ratio source rows per appended entry
     ik_new = view("ik", (B, 64), torch.int16)
     q_all.copy_(torch.randn(q_all.shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16))
     qi_all.copy_(torch.randn(qi_all.shape, generator=gen, device=dev).to(torch.bfloat16).view(torch.int16))
@@ -220,16 +240,17 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     result = torch.empty(B * 16 * 128 + B * 16, dtype=torch.float32, device=dev)
     outs.append(result[:B * 16 * 128].view(B, 16, 128))
     lses.append(result[B * 16 * 128:].view(B, 16))
-    cand = torch.empty((B, 2048), dtype=torch.int32, device=dev)
+    cand = None if flat else torch.empty((B, 2048), dtype=torch.int32, device=dev)
     sets = torch.empty((layers, B, 512), dtype=torch.int32, device=dev)
-    ws = torch.zeros(csa2.workspace_bytes(descs[0], csa2.BLOCK, B, L), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(csa2.workspace_bytes(descs[0], csa2.TOKEN if flat else csa2.BLOCK, B, L), dtype=torch.uint8,
+                     device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     stream = torch.cuda.Stream(device=dev)
 
     def step():
-        csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, err=err, stream=stream)
+        csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, ratio=ratio, err=err, stream=stream)
         csa2.decode_layers(descs, cache, [qi_all[l] for l in range(layers)], [w_all[l] for l in range(layers)],
                            [q_all[l] for l in range(layers)], [swa[l] for l in range(layers)], seq_lens, cand, sets,
                            outs, lses, B, L, ws, err=err, stream=stream)
@@ -242,7 +263,10 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    launches_per_step = 1 + sum({csa2.FULL: 4, csa2.REINDEX: 2, csa2.REUSE: 1}[m] for m in modes)
+    if flat:  # Full: block_score + block_select over entries (token kernel at <= 16,384), then attention
+        launches_per_step = 1 + sum((3 if L > 16384 else 2) if m != csa2.REUSE else 1 for m in modes)
+    else:
+        launches_per_step = 1 + sum({csa2.FULL: 4, csa2.REINDEX: 2, csa2.REUSE: 1}[m] for m in modes)
 
     def barrier():
         if world > 1:
@@ -290,9 +314,14 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         a_ms = time_launches(lambda: csa2.sparse_attn_decode(descs[reuse], cache, q_all[reuse], sets[0], swa[reuse],
                                                              seq_lens, outs[reuse], lses[reuse], B, err=err,
                                                              stream=stream))
-        # largest single HBM stream: the block-level indexer (scoring + select)
-        k_ms = time_launches(lambda: csa2.indexer_topk(descs[0], cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens,
-                                                       cand, B, L, ws, err=err, stream=stream))
+        # largest single HBM stream: the block-level indexer (scoring + select),
+        # or the flat indexer over every entry of the encoder's Full layers
+        if flat:
+            k_ms = time_launches(lambda: csa2.indexer_topk(descs[0], cache, csa2.TOKEN, qi_all[0], w_all[0],
+                                                           seq_lens, sets[0], B, L, ws, err=err, stream=stream))
+        else:
+            k_ms = time_launches(lambda: csa2.indexer_topk(descs[0], cache, csa2.BLOCK, qi_all[0], w_all[0],
+                                                           seq_lens, cand, B, L, ws, err=err, stream=stream))
 
         # ---- end to end: pinned host inputs -> device, step, result -> host ----
         # one H2D copy of the packed inputs (q, q_idx, w, the appended entry and
@@ -320,69 +349,76 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     clocks = sampler.summary()
     assert int(err.item()) == 0, f"device error flags {int(err.item())}"
     breakdown = _breakdown(csa2, cache, descs, modes, qi_all, w_all, q_all, swa, seq_lens, cand, sets, outs, lses,
-                           kv_new, ik_new, slot_new, ws, err, flush, stream, B, L) if args.breakdown else None
+                           kv_new, ik_new, slot_new, ws, err, flush, stream, B, L, ratio,
+                           flat) if args.breakdown else None
 
     h2d = step_in.numel()
     d2h = host_res.numel() * 4
-    ub = unique_bytes_per_seq(L, layers)
+    n_full = sum(1 for m in modes if m != csa2.REUSE)
+    ub = unique_bytes_per_seq_flat(L, layers, n_full, ratio) if flat else unique_bytes_per_seq(L, layers)
     peaks = _peaks()
     hbm = peaks.get("hbm_gbs")
-    k_bytes = B * ((L + 7) // 8) * 128
+    k_bytes = B * (L if flat else (L + 7) // 8) * 128
     k_gbs = k_bytes / (k_ms * 1e-3) / 1e9
     a_bytes = B * attn_bytes_per_row(L)
     a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
     peak_src = "MEASURED_PEAKS.json hbm_gbs (measured, burst copy)" if hbm else "fallback 6650 GB/s"
-    res = dict(metric=METRIC, value=whole_job_tokens_per_s(B, world, ms_per_step), unit=UNIT, n_gpus=world,
-               steps=args.steps,
+    attn_roof = dict(kernel="sparse_attn_kernel (Reuse layer, B rows x 8 CTAs)", bound="hbm", achieved=a_gbs,
+                     peak=hbm, unit="GB/s", frac=a_gbs / hbm if hbm else None, traffic=ATTN_TRAFFIC.get((B, L)),
+                     bytes_per_launch=a_bytes, ms_per_launch=a_ms, peak_source=peak_src)
+    idx_roof = dict(kernel="block_score_kernel + block_select_kernel" + (" over entries (flat indexer)" if flat else ""),
+                    bound="hbm", achieved=k_gbs, peak=hbm, unit="GB/s", frac=k_gbs / hbm if hbm else None,
+                    traffic=None, bytes_per_launch=k_bytes, ms_per_launch=k_ms, peak_source=peak_src)
+    schedule = "encoder: 3 x (F+5R), ratio 2, flat indexer" if flat else "decoder: F+3R, 4x(RI+3R)"
+    res = dict(metric=METRIC_ENC if flat else METRIC, value=whole_job_tokens_per_s(B, world, ms_per_step), unit=UNIT,
+               n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
                vs_baseline=None, dtype="fp4(e2m1)+e4m3 cache; bf16 q/idx; fp32 accumulate", data="synthetic",
-               config=dict(workload=W["workload"], seq_len=L, batch_per_gpu=B, global_batch=world * B,
-                           layers=layers, schedule="decoder: F+3R, 4x(RI+3R)", page_size=PAGE,
+               config=dict(workload=W["workload"], seq_len=L * ratio, entries=L, ratio=ratio, batch_per_gpu=B,
+                           global_batch=world * B, layers=layers, schedule=schedule, page_size=PAGE,
                            pages="contiguous" if args.contiguous_pages else "random permutation",
                            l2="flushed before every timed step (256 MiB write, not timed)", parallelism=f"dp{world}",
                            graph="one CUDA graph per step, programmatic dependent launch between kernels"),
                step_bytes_unique=B * ub["total"], step_gbs=B * ub["total"] / (ms_per_step * 1e-3) / 1e9,
                step_frac_of_hbm=(B * ub["total"] / (ms_per_step * 1e-3) / 1e9) / hbm if hbm else None,
-               roofline=dict(kernel="sparse_attn_kernel (Reuse layer, B rows x 8 CTAs)", bound="hbm",
-                             achieved=a_gbs, peak=hbm, unit="GB/s", frac=a_gbs / hbm if hbm else None,
-                             traffic=ATTN_TRAFFIC.get((B, L)), bytes_per_launch=a_bytes, ms_per_launch=a_ms,
-                             peak_source=peak_src),
-               roofline_block_indexer=dict(kernel="block_score_kernel + block_select_kernel", bound="hbm",
-                                           achieved=k_gbs, peak=hbm, unit="GB/s",
-                                           frac=k_gbs / hbm if hbm else None, traffic=None,
-                                           bytes_per_launch=k_bytes, ms_per_launch=k_ms, peak_source=peak_src),
                e2e=dict(value=whole_job_tokens_per_s(B, world, max_over_ranks(e2e_ms, world, dev)), unit=UNIT,
                         h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                         ms_per_step=e2e_ms),
                gpu_launches=launches_per_step * args.steps, launches_per_step=launches_per_step,
                clocks=clocks)
+    if flat:  # the flat indexer's full scans dominate the encoder's step
+        res["roofline"], res["roofline_attention"] = idx_roof, attn_roof
+    else:
+        res["roofline"], res["roofline_block_indexer"] = attn_roof, idx_roof
     if breakdown is not None:
         res["breakdown_us"] = breakdown
     return res
 
 
 def _breakdown(csa2, cache, descs, modes, qi_all, w_all, q_all, swa, seq_lens, cand, sets, outs, lses, kv_new,
-               ik_new, slot_new, ws, err, flush, stream, B, L, reps=50):
+               ik_new, slot_new, ws, err, flush, stream, B, L, ratio=1, flat=False, reps=50):
     """Every call of the step timed on its own with CUDA events (mean over
     reps), once after an L2 flush (cold) and once right after the same call
     (warm)."""
     import torch
     full = descs[0]
-    rei = next(d for d, m in zip(descs, modes) if m == csa2.REINDEX)
     reuse = next(d for d, m in zip(descs, modes) if m == csa2.REUSE)
-    calls = {
-        "quant_append (B entries)": lambda: csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, err=err,
-                                                                  stream=stream),
-        "indexer block level (block_score + block_select)": lambda: csa2.indexer_topk(
-            full, cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens, cand, B, L, ws, err=err, stream=stream),
-        "indexer token level (token_topk)": lambda: csa2.indexer_topk(
+    calls = {"quant_append (B entries)": lambda: csa2.kv_quant_append(cache, kv_new, ik_new, slot_new, ratio=ratio,
+                                                                       err=err, stream=stream)}
+    if flat:
+        calls["indexer, flat over every entry"] = lambda: csa2.indexer_topk(
+            full, cache, csa2.TOKEN, qi_all[0], w_all[0], seq_lens, sets[0], B, L, ws, err=err, stream=stream)
+    else:
+        rei = next(d for d, m in zip(descs, modes) if m == csa2.REINDEX)
+        calls["indexer block level (block_score + block_select)"] = lambda: csa2.indexer_topk(
+            full, cache, csa2.BLOCK, qi_all[0], w_all[0], seq_lens, cand, B, L, ws, err=err, stream=stream)
+        calls["indexer token level (token_topk)"] = lambda: csa2.indexer_topk(
             rei, cache, csa2.TOKEN, qi_all[4], w_all[4], seq_lens, sets[4], B, L, ws, cand_blocks=cand, err=err,
-            stream=stream),
-        "attention, Full/Reindex layer": lambda: csa2.sparse_attn_decode(
-            full, cache, q_all[0], sets[0], swa[0], seq_lens, outs[0], lses[0], B, err=err, stream=stream),
-        "attention, Reuse layer": lambda: csa2.sparse_attn_decode(
-            reuse, cache, q_all[1], sets[0], swa[1], seq_lens, outs[1], lses[1], B, err=err, stream=stream),
-    }
+            stream=stream)
+    calls["attention, Full/Reindex layer"] = lambda: csa2.sparse_attn_decode(
+        full, cache, q_all[0], sets[0], swa[0], seq_lens, outs[0], lses[0], B, err=err, stream=stream)
+    calls["attention, Reuse layer"] = lambda: csa2.sparse_attn_decode(
+        reuse, cache, q_all[1], sets[0], swa[1], seq_lens, outs[1], lses[1], B, err=err, stream=stream)
     res = {}
     with torch.cuda.stream(stream):
         for name, fn in calls.items():
@@ -564,15 +600,18 @@ def oracle_sample(cfg_id: int, budget_s: float = 15.0, max_steps: int = 1000):
     import oracle
     import synth
     W = workload(cfg_id)
-    L, layers, seed = W["L"], W["layers"], W["seed"]
+    L, layers, seed, ratio, flat = W["L"], W["layers"], W["seed"], W["ratio"], not W["decoder"]
     n_seq = min(W["B"], os.cpu_count() or 1)
     # one sequence's cache, built by the oracle itself (not timed), shared by the sampled sequences
-    kv = synth.kv_rows(seed, 0, 0, L)
-    codes, scales = oracle.quant_rows(kv)
-    del kv
+    codes = np.empty((L, 128), np.uint8)
+    scales = np.empty((L, 16), np.uint8)
+    for e0 in range(0, L, 1 << 16):
+        m = min(1 << 16, L - e0)
+        codes[e0:e0 + m], scales[e0:e0 + m] = oracle.quant_rows(synth.kv_rows(seed, 0, e0 * ratio, m * ratio),
+                                                                ratio=ratio)
     idx = synth.idx_k_rows(seed, 0, 0, L)
     pooled = oracle.pool_blocks(idx)
-    modes = oracle.schedule(True)[:layers]
+    modes = oracle.schedule(not flat)[:layers]
     q_idx = np.stack([np.concatenate([synth.q_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
     w = np.stack([np.concatenate([synth.w_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
     q = np.stack([np.concatenate([synth.q_heads(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
@@ -580,7 +619,7 @@ def oracle_sample(cfg_id: int, budget_s: float = 15.0, max_steps: int = 1000):
     steps, t0 = 0, time.perf_counter()
     while steps < max_steps:
         oracle.decode_batch(modes, [L] * n_seq, [codes] * n_seq, [scales] * n_seq, [idx] * n_seq,
-                            [pooled] * n_seq, q_idx, w, q, swa)
+                            [pooled] * n_seq, q_idx, w, q, swa, keep=0 if flat else 2048)
         steps += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -596,11 +635,12 @@ def run_reference(args, rank: int, world: int):
         return None
     W = workload(args.config)
     cb = oracle_sample(args.config, budget_s=max(10.0, min(60.0, 2.0 * args.steps)), max_steps=max(args.steps, 1))
-    return dict(metric=METRIC, value=cb["value"], unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+    return dict(metric=METRIC if W["decoder"] else METRIC_ENC, value=cb["value"], unit=UNIT, n_gpus=world,
+                steps=args.steps, warmup=args.warmup,
                 ms_per_step=W["B"] / cb["value"] * 1e3 if cb["value"] else None, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f32 decisions / f64 attention (oracle)", data="synthetic",
-                config=dict(workload=W["workload"], seq_len=W["L"], batch_per_gpu=W["B"], layers=W["layers"],
-                            parallelism="host cores"),
+                config=dict(workload=W["workload"], seq_len=W["L"] * W["ratio"], entries=W["L"], ratio=W["ratio"],
+                            batch_per_gpu=W["B"], layers=W["layers"], parallelism="host cores"),
                 impl="reference", cpu_baseline=cb,
                 e2e=dict(value=cb["value"], unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 

@@ -18,7 +18,7 @@ csa2_status check_desc(const csa2_layer_desc* d) {
         return CSA2_ERR_UNSUPPORTED;
     if (d->ratio != 1 && d->ratio != 2) return CSA2_ERR_INVALID_ARG;
     if (d->topk < 1 || d->topk > kMaxTopk) return CSA2_ERR_INVALID_ARG;
-    if (d->keep_blocks < 1 || d->keep_blocks > kMaxKeep) return CSA2_ERR_INVALID_ARG;
+    if (d->keep_blocks < 0 || d->keep_blocks > kMaxKeep) return CSA2_ERR_INVALID_ARG;  // 0: flat indexer
     if (d->window < 1 || d->window > kMaxWindow) return CSA2_ERR_INVALID_ARG;
     if (d->mode < CSA2_MODE_FULL || d->mode > CSA2_MODE_REUSE) return CSA2_ERR_INVALID_ARG;
     return CSA2_OK;
@@ -92,7 +92,7 @@ size_t csa2_indexer_workspace_bytes(const csa2_layer_desc* desc, int32_t level, 
     if (!desc || n < 1 || max_len < 1) return 0;
     if (prefill) return prefill_ws_layout(n, max_len).total;
     (void)level;
-    return decode_ws_layout(n, max_len).total;
+    return decode_ws_layout(n, max_len, desc->keep_blocks == 0).total;
 }
 
 }  // extern "C"
@@ -109,7 +109,9 @@ static csa2_status indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache
     if (desc->mode == CSA2_MODE_REUSE) return CSA2_ERR_INVALID_ARG;
     if (level != CSA2_LEVEL_BLOCK && level != CSA2_LEVEL_TOKEN) return CSA2_ERR_INVALID_ARG;
     const bool prefill = q_pos != nullptr;
+    const bool flat = desc->keep_blocks == 0;  // no block level: Top-K over every entry
     if (prefill && level != CSA2_LEVEL_TOKEN) return CSA2_ERR_INVALID_ARG;
+    if (flat && (level != CSA2_LEVEL_TOKEN || cand_blocks)) return CSA2_ERR_INVALID_ARG;
     s = check_cache(cache, true, level == CSA2_LEVEL_BLOCK);
     if (s != CSA2_OK) return s;
     if (score_out) return CSA2_ERR_UNSUPPORTED;
@@ -119,6 +121,9 @@ static csa2_status indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache
     if (cand_blocks && (!aligned(cand_blocks, 4) || prefill || level != CSA2_LEVEL_TOKEN)) return CSA2_ERR_INVALID_ARG;
     if (level == CSA2_LEVEL_BLOCK && (max_len > kMaxBlockLevelLen || n > 1024)) return CSA2_ERR_UNSUPPORTED;
     if (level == CSA2_LEVEL_BLOCK && cache->n_phys_pages * cache->page_size / 8 > 0x7fffffff) return CSA2_ERR_UNSUPPORTED;
+    const bool flat_rows = flat && !prefill && max_len > kMaxCand;  // scored by the block-level kernels, row = entry
+    if (flat_rows && (max_len > kMaxBlockLevelLen || n > 1024)) return CSA2_ERR_UNSUPPORTED;
+    if (flat_rows && cache->n_phys_pages * cache->page_size > 0x7fffffff) return CSA2_ERR_UNSUPPORTED;
     if (prefill && max_len > kMaxCand) return CSA2_ERR_UNSUPPORTED;
     if (prefill && !aligned(q_idx, 16)) return CSA2_ERR_INVALID_ARG;  // read in 16-byte rows by the tensor-core tiles
     if (max_len > (int64_t)cache->max_pages_per_seq * cache->page_size) return CSA2_ERR_INVALID_ARG;
@@ -133,8 +138,12 @@ static csa2_status indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache
     if (level == CSA2_LEVEL_BLOCK)
         return from_cuda(launch_block_topk(*cache, q_idx, w, seq_lens, desc->keep_blocks, idx_out, n, max_len, ws,
                                            err_word, st));
-    return from_cuda(launch_token_topk(*cache, q_idx, w, seq_lens, cand_blocks, desc->keep_blocks, desc->topk,
-                                       idx_out, n, max_len, ws, err_word, st, pre));
+    if (flat_rows)
+        return from_cuda(launch_block_topk(*cache, q_idx, w, seq_lens, desc->topk, idx_out, n, max_len, ws, err_word,
+                                           st, true));
+    // a flat selection over at most 16,384 entries runs as one candidate set
+    return from_cuda(launch_token_topk(*cache, q_idx, w, seq_lens, cand_blocks, flat ? kMaxKeep : desc->keep_blocks,
+                                       desc->topk, idx_out, n, max_len, ws, err_word, st, pre));
 }
 
 extern "C" {
@@ -235,9 +244,11 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
                                int32_t* cand_blocks, int32_t* idx_sets, float* const* out, float* const* lse,
                                int32_t B, int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word,
                                void* stream) {
-    if (n_layers < 1 || !descs || !q_idx || !w || !q || !swa_kv || !out || !lse || !cand_blocks || !idx_sets)
+    if (n_layers < 1 || !descs || !q_idx || !w || !q || !swa_kv || !out || !lse || !idx_sets)
         return CSA2_ERR_INVALID_ARG;
     if (descs[0].mode != CSA2_MODE_FULL) return CSA2_ERR_INVALID_ARG;
+    const bool flat = descs[0].keep_blocks == 0;  // every indexer layer selects over all entries
+    if (!flat && !cand_blocks) return CSA2_ERR_INVALID_ARG;
     // validate every layer before launching anything
     for (int l = 0; l < n_layers; ++l) {
         csa2_status s = check_desc(&descs[l]);
@@ -247,7 +258,8 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
         if (!q[l] || !swa_kv[l] || !out[l] || !lse[l]) return CSA2_ERR_INVALID_ARG;
         if (descs[l].mode != CSA2_MODE_REUSE && (!q_idx[l] || !w[l])) return CSA2_ERR_INVALID_ARG;
     }
-    const size_t need = csa2_indexer_workspace_bytes(&descs[0], CSA2_LEVEL_BLOCK, B, max_len, 0);
+    const size_t need =
+        csa2_indexer_workspace_bytes(&descs[0], flat ? CSA2_LEVEL_TOKEN : CSA2_LEVEL_BLOCK, B, max_len, 0);
     if (!workspace || ws_bytes < need) return CSA2_ERR_WORKSPACE;
     const int topk = descs[0].topk;
     const int32_t* cur = nullptr;
@@ -255,7 +267,12 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
         const csa2_layer_desc& d = descs[l];
         int32_t* set = idx_sets + (int64_t)l * B * topk;
         csa2_status s = CSA2_OK;
-        if (d.mode == CSA2_MODE_FULL) {
+        if (flat && d.mode != CSA2_MODE_REUSE) {
+            // no candidate set: Full and Reindex layers both select over every entry
+            s = csa2_indexer_topk(&d, cache, CSA2_LEVEL_TOKEN, q_idx[l], w[l], seq_lens, nullptr, nullptr, set,
+                                  nullptr, B, max_len, workspace, ws_bytes, err_word, stream);
+            cur = set;
+        } else if (d.mode == CSA2_MODE_FULL) {
             s = csa2_indexer_topk(&d, cache, CSA2_LEVEL_BLOCK, q_idx[l], w[l], seq_lens, nullptr, nullptr,
                                   cand_blocks, nullptr, B, max_len, workspace, ws_bytes, err_word, stream);
             if (s == CSA2_OK)

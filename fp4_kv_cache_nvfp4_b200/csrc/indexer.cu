@@ -338,10 +338,13 @@ struct BlockArgs {
     uint32_t* bitmap;  // [n][nblk_pad/32]
     uint64_t* bnd;     // [n][nblk_pad]
     uint32_t* bnd_cnt; // [n]
+    uint32_t* tie;     // [n][nblk_pad/32] (flat only: the finalize's tie bitmap)
+    const uint8_t* rows;  // scored rows: pooled indexer K (rshift 3) or indexer K (rshift 0)
     int32_t* err;
     int64_t nblk_pad;
     int64_t max_len;
     int n, keep, page_shift;
+    int rshift;        // log2 entries per scored row
 };
 
 // tile_start[b] = first tile of sequence b; returns the sequence of tile t
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
             const int b = tid * per + i;
             if (b < a.n) {
                 const int32_t L = a.seq_lens[b];
-                const int32_t nblk = (L >= 1 && L <= a.max_len) ? (L + kBlk - 1) / kBlk : 0;
+                const int32_t nblk = (L >= 1 && L <= a.max_len) ? ((L - 1) >> a.rshift) + 1 : 0;
                 if (L < 1 || L > a.max_len) dev_error(a.err, CSA2_DEV_LEN);
                 mine += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
             }
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
             if (b < a.n) {
                 tile_start[b] = (int32_t)base;
                 const int32_t L = a.seq_lens[b];
-                const int32_t nblk = (L >= 1 && L <= a.max_len) ? (L + kBlk - 1) / kBlk : 0;
+                const int32_t nblk = (L >= 1 && L <= a.max_len) ? ((L - 1) >> a.rshift) + 1 : 0;
                 s_nblk[b] = nblk;
                 base += nblk > a.keep ? (nblk + K2_TILE - 1) / K2_TILE : 0;
             }
@@ -422,7 +425,8 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
         const int pw = wid - K2_CWARPS;
         const int sh = a.page_shift;
         const int32_t emask = (1 << sh) - 1;
-        const uint8_t* pooled = reinterpret_cast<const uint8_t*>(a.cache.idx_k_pooled);
+        const uint8_t* rows = a.rows;
+        const int rsh = a.rshift;
         const int32_t mpps = a.cache.max_pages_per_seq;
         // rows pw*128 + 32 h + lane of tile t: row index within the sequence
         // (-1 past its end) and physical page, loaded one tile ahead
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 const int32_t j = (t - tile_start[b]) * K2_TILE + K2_PROWS * pw + 32 * h + lane;
-                const int32_t pg = (j * kBlk) >> sh;
+                const int32_t pg = (j << rsh) >> sh;
                 const bool in = j < s_nblk[b];
                 pp[h] = (in && pg < mpps) ? __ldg(a.cache.page_table + (int64_t)b * mpps + pg) : -1;
                 pj[h] = in ? j : -1;
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
                         dev_error(a.err, CSA2_DEV_PAGE);
                         phys = 0;  // results of this call are undefined; the copy stays in bounds
                     }
-                    prow[h] = (int32_t)((((int64_t)phys << sh) | ((pj[h] * kBlk) & emask)) >> 3);
+                    prow[h] = (int32_t)((((int64_t)phys << sh) | ((pj[h] << rsh) & emask)) >> rsh);
                 }
             }
             if (i + 1 < ntiles) fetch(t0 + i + 1);  // loads overlap the copies below
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
                 const int32_t v = k < 8 ? prow[0] : k < 16 ? prow[1] : k < 24 ? prow[2] : prow[3];
                 const int32_t pr = __shfl_sync(0xffffffffu, v, rr & 31);
                 if (pr >= 0)
-                    cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), pooled + (int64_t)pr * 128 + c * 16);
+                    cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), rows + (int64_t)pr * 128 + c * 16);
             }
             cp_async_mbar_arrive(&full[s]);
         }
@@ -572,7 +576,7 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     }
     const int b = blockIdx.y;
     const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
-    const int32_t nblk = (L + kBlk - 1) / kBlk;
+    const int32_t nblk = L >= 1 ? ((L - 1) >> a.rshift) + 1 : 0;
     int32_t* out = a.out + (int64_t)b * a.keep;
     if (nblk <= a.keep) {
         if (blockIdx.x == 0)
@@ -626,19 +630,24 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     __threadfence();
 
     // ---- finalize: exact threshold inside the boundary bin -----------------
+    // The row bitmap and the tie bitmap live in shared memory when they fit
+    // (every block-level context); a flat selection over more rows works on
+    // the sequence's bitmap in global memory and a tie bitmap beside it.
     const int nwords = (nblk + 31) >> 5;
-    uint32_t* bm = reinterpret_cast<uint32_t*>(smem);
-    uint32_t* tie = bm + K3_WORDS;
-    uint32_t* hist = tie + K3_WORDS;
+    const bool gm = nwords > K3_WORDS;
+    uint32_t* sm_bm = reinterpret_cast<uint32_t*>(smem);
+    uint32_t* hist = sm_bm + 2 * K3_WORDS;
     uint32_t* tmp = hist + 1024;
     uint64_t* sbnd = reinterpret_cast<uint64_t*>(tmp + 64);
+    uint32_t* bm = gm ? bitmap : sm_bm;
+    uint32_t* tie = gm ? a.tie + (int64_t)b * (a.nblk_pad >> 5) : sm_bm + K3_WORDS;
     const uint32_t n_bnd = __ldcg(&a.bnd_cnt[b]);
     const uint64_t* B = bnd;
     if (n_bnd <= (uint32_t)K3_BND_CAP) {  // stage the boundary list (the common case)
         load_words(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd), 2 * (int)n_bnd);
         B = sbnd;
     }
-    load_words(bm, bitmap, nwords);
+    if (!gm) load_words(bm, bitmap, nwords);
     for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
     uint32_t need = (uint32_t)a.keep - (uint32_t)__ldcg(&a.thr[4 * b + 1]);
     int d2, d3;
@@ -675,12 +684,13 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     const int per = (nwords + K3_THREADS - 1) / K3_THREADS;
     const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
     uint32_t my_ties = 0;
-    for (int i = w0; i < w1; ++i) my_ties += __popc(tie[i]);
+    auto ld = [gm](const uint32_t* p, int i) { return gm ? __ldcg(p + i) : p[i]; };
+    for (int i = w0; i < w1; ++i) my_ties += __popc(ld(tie, i));
     uint32_t tot;
     uint32_t rank = block_excl_scan(my_ties, tmp, &tot);
     uint32_t my_sel = 0;
     for (int i = w0; i < w1; ++i) {
-        uint32_t t = tie[i], kept = 0;
+        uint32_t t = ld(tie, i), kept = 0;
         while (t && rank < need) {
             const uint32_t lb = t & (0u - t);
             kept |= lb;
@@ -688,12 +698,13 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
             ++rank;
         }
         rank += __popc(t);
-        bm[i] |= kept;
-        my_sel += __popc(bm[i]);
+        const uint32_t v = ld(bm, i) | kept;
+        bm[i] = v;
+        my_sel += __popc(v);
     }
     uint32_t base = block_excl_scan(my_sel, tmp, &tot);
     for (int i = w0; i < w1; ++i) {
-        uint32_t m = bm[i];
+        uint32_t m = ld(bm, i);
         while (m) {
             const int bit = __ffs(m) - 1;
             m &= m - 1;
@@ -1693,11 +1704,11 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // One layout for both levels: the small arrays that must start at zero come
 // first, so a workspace zero-filled once stays valid for any mix of calls with
 // the same (n, max_len).
-DecodeWs decode_ws_layout(int n, int64_t max_len) {
+DecodeWs decode_ws_layout(int n, int64_t max_len, bool flat) {
     DecodeWs l{};
     size_t o = 0;
-    const int64_t nblk = (max_len + kBlk - 1) / kBlk;
-    l.nblk_pad = (nblk + K3_CHUNK - 1) / K3_CHUNK * K3_CHUNK;
+    const int64_t nrows = flat ? max_len : (max_len + kBlk - 1) / kBlk;  // rows scored per sequence
+    l.nblk_pad = (nrows + K3_CHUNK - 1) / K3_CHUNK * K3_CHUNK;
     l.blk_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_ctr = o; o = align256(o + (size_t)n * 8);
     l.blk_bnd_cnt = o; o = align256(o + (size_t)n * 4);
@@ -1705,10 +1716,12 @@ DecodeWs decode_ws_layout(int n, int64_t max_len) {
     l.tok_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_thr = o; o = align256(o + (size_t)n * 16);
     l.tok_keys = o; o = align256(o + (size_t)n * kMaxCand * 4);
-    if (nblk > kMaxKeep) {
-        l.blk_scores = o; o = align256(o + (size_t)n * l.nblk_pad * 4);
-        l.blk_bitmap = o; o = align256(o + (size_t)n * (l.nblk_pad / 32) * 4);
-        l.blk_bnd = o; o = align256(o + (size_t)n * l.nblk_pad * 8);
+    // the scored rows' arrays (any keep below the row count needs them)
+    l.blk_scores = o; o = align256(o + (size_t)n * l.nblk_pad * 4);
+    l.blk_bitmap = o; o = align256(o + (size_t)n * (l.nblk_pad / 32) * 4);
+    l.blk_bnd = o; o = align256(o + (size_t)n * l.nblk_pad * 8);
+    if (flat) {
+        l.blk_tie = o; o = align256(o + (size_t)n * (l.nblk_pad / 32) * 4);
     }
     l.total = o;
     return l;
@@ -1754,13 +1767,13 @@ static int sm_count() {
 
 cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, int keep, int32_t* out, int n, int64_t max_len, char* ws,
-                              int32_t* err, cudaStream_t stream) {
+                              int32_t* err, cudaStream_t stream, bool flat) {
     static bool d2[64], d3[64];
     cudaError_t e = ensure_smem((const void*)block_score_kernel, K2_SMEM, d2);
     if (e == cudaSuccess) e = ensure_smem((const void*)block_select_kernel, K3_SMEM, d3);
     if (e != cudaSuccess) return e;
     if (n > K2_MAX_SEQS) return cudaErrorInvalidValue;
-    const DecodeWs l = decode_ws_layout(n, max_len);
+    const DecodeWs l = decode_ws_layout(n, max_len, flat);
     BlockArgs a{};
     a.cache = cache;
     a.q_idx = q_idx;
@@ -1774,13 +1787,16 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.bitmap = reinterpret_cast<uint32_t*>(ws + l.blk_bitmap);
     a.bnd = reinterpret_cast<uint64_t*>(ws + l.blk_bnd);
     a.bnd_cnt = reinterpret_cast<uint32_t*>(ws + l.blk_bnd_cnt);
+    a.tie = flat ? reinterpret_cast<uint32_t*>(ws + l.blk_tie) : nullptr;
+    a.rows = reinterpret_cast<const uint8_t*>(flat ? cache.idx_k : cache.idx_k_pooled);
+    a.rshift = flat ? 0 : 3;
     a.err = err;
     a.nblk_pad = l.nblk_pad;
     a.max_len = max_len;
     a.n = n;
     a.keep = keep;
     a.page_shift = page_shift_of(cache);
-    const int64_t nblk = (max_len + kBlk - 1) / kBlk;
+    const int64_t nblk = flat ? max_len : (max_len + kBlk - 1) / kBlk;
     if (nblk > keep) {
         const int64_t tiles = (int64_t)n * ((nblk + K2_TILE - 1) / K2_TILE);
         const int grid = (int)std::min<int64_t>(tiles, sm_count());

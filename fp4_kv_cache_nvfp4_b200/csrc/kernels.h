@@ -44,12 +44,13 @@ struct LaunchCfg {
 
 // Workspace layout of the decode indexer (byte offsets; all 256-aligned).
 struct DecodeWs {
-    size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt;
+    size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt, blk_tie;
     size_t tok_keys, tok_ctr, tok_hist;
     size_t total;
     int64_t nblk_pad;  // per-sequence stride of block arrays
 };
-DecodeWs decode_ws_layout(int n, int64_t max_len);
+// flat: rows are entries (the indexer without a block level), not blocks of 8
+DecodeWs decode_ws_layout(int n, int64_t max_len, bool flat = false);
 
 struct PrefillWs {
     size_t keys;   // [T][stride]: 16-bit approximate keys, later (aliased) 32-bit exact keys of the fallback
@@ -67,7 +68,7 @@ cudaError_t launch_quant_append(const csa2_kv_cache& cache, const void* src, boo
 
 cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, int keep, int32_t* out, int n, int64_t max_len,
-                              char* ws, int32_t* err, cudaStream_t stream);
+                              char* ws, int32_t* err, cudaStream_t stream, bool flat = false);
 
 cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
                               const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,

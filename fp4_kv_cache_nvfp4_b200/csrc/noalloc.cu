@@ -66,7 +66,7 @@ extern "C" CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc*
     // The kernels expect their counters and histograms at zero.  The previous
     // call may have used another (n, max_len) and so another layout: clear the
     // zero-state head of this call's layout first (a memset, no allocation).
-    const DecodeWs l = decode_ws_layout(n, max_len);
+    const DecodeWs l = decode_ws_layout(n, max_len, desc->keep_blocks == 0);
     if (cudaMemsetAsync(scratch, 0, l.blk_thr, (cudaStream_t)stream) != cudaSuccess) {
         (void)cudaGetLastError();
         return CSA2_ERR_CUDA;

@@ -75,14 +75,20 @@ typedef enum { CSA2_LEVEL_BLOCK = 0, CSA2_LEVEL_TOKEN = 1 } csa2_level;
 typedef enum { CSA2_SRC_F32 = 0, CSA2_SRC_BF16 = 1 } csa2_src_dtype;
 
 /* Per-layer descriptor.  Supported values: ratio 1 or 2; 1 <= topk <= 512;
- * block 8; 1 <= keep_blocks <= 2048; 1 <= window <= 128; n_heads 16;
- * head_dim 128; idx_heads 4; idx_dim 64. */
+ * block 8; 0 <= keep_blocks <= 2048; 1 <= window <= 128; n_heads 16;
+ * head_dim 128; idx_heads 4; idx_dim 64.
+ * keep_blocks = 0 means no block level (a flat indexer over every entry).
+ * The pages place the hierarchical indexer in the decoder only ("Como
+ * funciona" of e-cogni.com.br, CSA2 paragraph of conexaotc.com.br), so the
+ * encoder's layers (ratio 2, 3 x (Full + 5 Reuse)) select their Top-512 among
+ * all entries; csa2_layer_desc_default leaves keep_blocks at 2048, and a
+ * caller running the encoder side of a decode step sets it to 0. */
 typedef struct {
     int32_t mode;        /* csa2_mode */
     int32_t ratio;       /* tokens per main-KV entry: 1 decoder, 2 encoder */
     int32_t topk;        /* indices kept per Full/Reindex layer (512) */
     int32_t block;       /* positions per indexer block (8) */
-    int32_t keep_blocks; /* blocks kept by the Full layer (2048) */
+    int32_t keep_blocks; /* blocks kept by the Full layer (2048); 0: flat */
     int32_t window;      /* SWA window in tokens (128) */
     int32_t n_heads;     /* 16 */
     int32_t head_dim;    /* 128 */
@@ -159,6 +165,11 @@ CSA2_API csa2_status csa2_kv_quant_append(const csa2_kv_cache* cache, const void
  *     [n][keep_blocks] (ascending, -1 padded; normally the BLOCK output of
  *     the Full layer of this step), or all L positions if cand_blocks is NULL
  *     (then L <= 8 * keep_blocks).
+ *   keep_blocks = 0 (flat): level TOKEN only (BLOCK: INVALID_ARG), with
+ *     cand_blocks NULL (else INVALID_ARG); idx_out [n][topk] = Top-min(topk,
+ *     L) of all L positions, n <= 1024 and max_len <= 2^21 (UNSUPPORTED
+ *     otherwise); above 16,384 entries the cache must hold at most 2^31 - 1
+ *     slots.  The pooled indexer K is not read.
  * Prefill (q_pos != NULL, level TOKEN): n queries of sequence 0 of the page
  *   table, q_idx [n][4][64] (16-byte aligned), w [n][4], q_pos [n] absolute
  *   token positions, seq_lens [1] = entries in the cache (<= 16384); entry j
@@ -168,9 +179,11 @@ CSA2_API csa2_status csa2_kv_quant_append(const csa2_kv_cache* cache, const void
  *   against a bound on the approximation; a query that fails the check is
  *   recomputed exactly.
  * score_out is reserved (pass NULL).
- * workspace: device memory of csa2_indexer_workspace_bytes() bytes, 256-byte
- * aligned, zero-filled before its first use; every call leaves it zero-filled
- * again.  Calls sharing one workspace must not overlap on the GPU. */
+ * workspace: device memory of csa2_indexer_workspace_bytes() bytes (for the
+ * same desc: a flat desc needs one row per entry, a hierarchical one per
+ * block), 256-byte aligned, zero-filled before its first use; every call
+ * leaves its counters and histograms zero again.  Calls sharing one workspace
+ * must not overlap on the GPU. */
 CSA2_API size_t csa2_indexer_workspace_bytes(const csa2_layer_desc* desc, int32_t level, int32_t n, int64_t max_len,
                                     int32_t prefill);
 CSA2_API csa2_status csa2_indexer_topk(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
@@ -216,6 +229,10 @@ CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const
  * layers only), q[l], swa_kv[l], out[l], lse[l].  cand_blocks
  * [B][keep_blocks] and idx_sets [n_layers][B][topk] are device outputs; a
  * Reuse layer writes no set and reads the latest one.  Layer 0 must be Full.
+ * With keep_blocks = 0 in descs (the encoder's layers: every desc must carry
+ * the same keep_blocks), Full and Reindex layers take the flat TOKEN indexer
+ * over all entries, cand_blocks may be NULL and is not written, and the
+ * workspace is sized by csa2_indexer_workspace_bytes(descs[0], TOKEN, ...).
  * Every input must be complete in stream order before the call, as usual.
  * Kernels of the call after the first read the cache, the lengths, the SWA
  * rows other than the newest, a Reuse layer's index set and a Reindex layer's

@@ -254,7 +254,8 @@ def schedule(decoder: bool = True) -> np.ndarray:
 def decode_step(modes, L: int, codes, scales, idx_k, pooled, q_idx, w, q, swa, window=128, keep=2048, topk_=512):
     """One decode step of one sequence.  Per-layer arrays have a leading layer
     axis: q_idx [n,4,64], w [n,4], q [n,16,128], swa [n,window,256] (rows beyond
-    min(window, L) ignored)."""
+    min(window, L) ignored).  keep=0: flat indexer over all L entries (the
+    encoder's layers), pooled unused."""
     modes = _c(modes, np.int32)
     n = modes.size
     codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)

@@ -49,6 +49,11 @@
  *   R10 decode window = last min(128, L) tokens including the current one;
  *       prefill window of the query at p = tokens [max(0, p-127), p]; entry j
  *       is visible to query p iff (j+1)*ratio - 1 <= p.
+ *   R11 the pages place the hierarchical indexer in the decoder only; the
+ *       encoder's Full layers (ratio 2) select their Top-512 over every entry
+ *       of the context ("flat"), as its prefill does.  A decode step with
+ *       keep = 0 has no block level: a Full (or Reindex) layer takes the
+ *       Top-K over all L entries.
  *
  * Floating point: where a float decides an integer (codes, scales, pooled
  * bf16, scores deciding Top-K membership) the oracle works in fp32, the
@@ -434,7 +439,8 @@ int orc_schedule(int decoder, int32_t* modes) {
 
 /* One decode step of one sequence through n_layers layers of the given modes.
  * The cache (codes, scales, idx_k, pooled) already holds the L entries,
- * including the current token.  Per layer l: q[l] [16][128] bf16, swa[l]
+ * including the current token.  keep = 0 selects the flat indexer (R11):
+ * pooled and blocks are not used.  Per layer l: q[l] [16][128] bf16, swa[l]
  * [n_swa][256] bf16 (n_swa = min(window, L)); indexer layers also read
  * q_idx[l] [4][64] bf16 and w[l] [4].  Outputs: idx_sets[l] [topk],
  * out[l] [16][128], lse[l] [16], blocks [keep] (the Full layer's set). */
@@ -449,7 +455,9 @@ void orc_decode_step(int n_layers, const int32_t* modes, int64_t L, const uint8_
         int32_t* set = idx_sets + (int64_t)l * topk;
         const uint16_t* qi = q_idx + (int64_t)l * ORC_IH * ORC_ID;
         const float* wl = w + (int64_t)l * ORC_IH;
-        if (modes[l] == ORC_FULL) {
+        if (modes[l] != ORC_REUSE && keep == 0) {
+            orc_select_tokens(idx_k, L, NULL, 0, qi, wl, topk, set, NULL, NULL, NULL);
+        } else if (modes[l] == ORC_FULL) {
             orc_select_blocks(pooled, L, qi, wl, keep, blocks, NULL);
             have_blocks = 1;
             orc_select_tokens(idx_k, L, blocks, keep, qi, wl, topk, set, NULL, NULL, NULL);

@@ -36,6 +36,8 @@ CONFIGS = {
     3: dict(name="encoder-prefill-32k-t4096-6l", seed=1003, tokens=32768, T=4096, ratio=2, layers=6),
     4: dict(name="decoder-20l-1m-b8", seed=1004, L=1 << 20, B=8, ratio=1, layers=20),
     5: dict(name="ragged-64seq-paged", seed=1005, B=64, lo=4096, hi=1 << 20, page=64, burst=16384, layers=20),
+    # the encoder's 18 CSA2 layers per generated token: 1M tokens at ratio 2
+    6: dict(name="encoder-decode-18l-1m-b8", seed=1006, L=1 << 19, B=8, ratio=2, layers=18, decoder=False),
 }
 
 

@@ -83,3 +83,50 @@ def check_sets(got, want, what=""):
     if not np.array_equal(got, want):
         bad = np.nonzero(got != want)
         raise AssertionError(f"{what}: {bad[0].size} index mismatches, first at {tuple(b[0] for b in bad)}")
+
+
+# ---------------------------------------------------------------------------
+# the encoder side of a decode step (flat indexer)
+# ---------------------------------------------------------------------------
+
+def encoder_layer_inputs(seed, B, lens, n_layers):
+    q_idx = np.stack([np.concatenate([synth.q_idx(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    w = np.stack([np.concatenate([synth.w_idx(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    q = np.stack([np.concatenate([synth.q_heads(seed, l, b) for l in range(n_layers)]) for b in range(B)])
+    swa = np.zeros((B, n_layers, 128, 256), np.uint16)
+    for b, L in enumerate(lens):
+        for l in range(n_layers):
+            swa[b, l, :min(128, L)] = synth.swa_rows(seed, l, b, min(128, L))
+    return q_idx, w, q, swa
+
+
+def run_encoder_step(csa2, ps, lens, q_idx, w, q, swa):
+    """The encoder's 18 CSA2 layers (3 x (Full + 5 Reuse), ratio 2, flat
+    indexer) through the schedule driver; no candidate-block buffer."""
+    B, max_len = len(lens), int(max(lens))
+    modes = csa2.schedule(False)
+    n = len(modes)
+    descs = [csa2.default_desc(m, 2, keep_blocks=0) for m in modes]
+    t16 = lambda a: bits16(np.ascontiguousarray(a))  # noqa: E731
+    out = [torch.empty((B, 16, 128), device="cuda") for _ in range(n)]
+    lse = [torch.empty((B, 16), device="cuda") for _ in range(n)]
+    sets = torch.full((n, B, 512), -9, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(csa2.workspace_bytes(descs[0], csa2.TOKEN, B, max_len), dtype=torch.uint8, device="cuda")
+    csa2.decode_layers(descs, ps.cache, [t16(q_idx[:, l]) for l in range(n)],
+                       [dev(np.ascontiguousarray(w[:, l])) for l in range(n)], [t16(q[:, l]) for l in range(n)],
+                       [t16(swa[:, l]) for l in range(n)], dev(np.asarray(lens, np.int32)), None, sets, out, lse, B,
+                       max_len, ws, err=ps.err)
+    torch.cuda.synchronize()
+    return dict(sets=sets.cpu().numpy(), out=[o.cpu().numpy() for o in out], lse=[x.cpu().numpy() for x in lse],
+                modes=modes)
+
+
+def compare_encoder_seq(orc, r, b, L, codes, scales, idx, q_idx, w, q, swa, what):
+    modes = np.array(r["modes"], np.int32)
+    ref = orc.decode_step(modes, int(L), codes, scales, idx, orc.pool_blocks(idx), q_idx, w, q, swa, keep=0)
+    last = 0
+    for l, m in enumerate(modes):
+        if m != 2:
+            last = l
+        check_sets(r["sets"][last, b], ref["idx"][l], f"{what} layer {l} set")
+        check_attn(r["out"][l][b], r["lse"][l][b], ref["out"][l], ref["lse"][l], f"{what} layer {l}")

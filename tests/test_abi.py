@@ -110,3 +110,44 @@ def test_workspace_sizes(csa2):
     # block arrays: scores + bitmap + boundary list per sequence at 131,072 blocks
     assert big >= 8 * (131072 * (4 + 8) + 131072 // 8)
     assert csa2.workspace_bytes(d, csa2.TOKEN, 4096, 16384, prefill=True) >= 4096 * 16384 * 4
+
+
+def test_flat_indexer_arguments(csa2):
+    """keep_blocks = 0 removes the block level (the encoder's layers): the
+    indexer then runs at TOKEN level over every entry, with no candidates, up
+    to 2^21 entries, and its workspace holds one row per entry."""
+    L = csa2.lib()
+    c = _cache_struct(csa2)
+    P = ctypes.c_void_p
+    ws = 0x100000
+    flat = csa2.default_desc(csa2.FULL, 2, keep_blocks=0)
+    # no BLOCK level without blocks
+    assert L.csa2_indexer_topk(ctypes.byref(flat), ctypes.byref(c), csa2.BLOCK, P(0x1000), P(0x1000), P(0x1000),
+                               None, None, P(0x1000), None, 1, 1000, P(ws), 1 << 30, None, None) == 1
+    # no candidate blocks for a flat layer
+    assert L.csa2_indexer_topk(ctypes.byref(flat), ctypes.byref(c), csa2.TOKEN, P(0x1000), P(0x1000), P(0x1000),
+                               None, P(0x1000), P(0x1000), None, 1, 1000, P(ws), 1 << 30, None, None) == 1
+    # above the compiled limit of 2^21 entries
+    assert L.csa2_indexer_topk(ctypes.byref(flat), ctypes.byref(c), csa2.TOKEN, P(0x1000), P(0x1000), P(0x1000),
+                               None, None, P(0x1000), None, 1, (1 << 21) + 1, P(ws), 1 << 40, None, None) == 2
+    # within the limits the call gets as far as the workspace check
+    assert L.csa2_indexer_topk(ctypes.byref(flat), ctypes.byref(c), csa2.TOKEN, P(0x1000), P(0x1000), P(0x1000),
+                               None, None, P(0x1000), None, 1, 1000, P(ws), 16, None, None) == 4
+    # a negative keep_blocks is still rejected
+    bad = csa2.default_desc(csa2.FULL, 2, keep_blocks=-1)
+    assert L.csa2_indexer_topk(ctypes.byref(bad), ctypes.byref(c), csa2.TOKEN, P(0x1000), P(0x1000), P(0x1000),
+                               None, None, P(0x1000), None, 1, 1000, P(ws), 1 << 30, None, None) == 1
+    # workspace: scores, boundary list and two bitmaps per entry, not per block
+    hier = csa2.workspace_bytes(csa2.default_desc(csa2.FULL, 2), csa2.BLOCK, 8, 1 << 20)
+    fl = csa2.workspace_bytes(flat, csa2.TOKEN, 8, 1 << 20)
+    assert fl > hier and fl % 256 == 0
+    assert fl >= 8 * ((1 << 20) * (4 + 8) + 2 * (1 << 20) // 8)
+    # the decode driver takes flat layers without a cand_blocks buffer (and
+    # still needs its workspace)
+    descs = (csa2.LayerDesc * 2)(flat, csa2.default_desc(csa2.REUSE, 2, keep_blocks=0))
+    ptrs = (ctypes.c_void_p * 2)(0x1000, 0x1000)
+    assert L.csa2_decode_layers(2, descs, ctypes.byref(c), ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
+                                P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 16, None, None) == 4
+    hdesc = (csa2.LayerDesc * 2)(csa2.default_desc(csa2.FULL, 1), csa2.default_desc(csa2.REUSE, 1))
+    assert L.csa2_decode_layers(2, hdesc, ctypes.byref(c), ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
+                                P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 1 << 30, None, None) == 1

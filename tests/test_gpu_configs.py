@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import synth
-from _gpu_util import PagedSeqs, bits16, check_attn, check_sets, dev
+from _gpu_util import (PagedSeqs, bits16, check_attn, check_sets, compare_encoder_seq, dev, encoder_layer_inputs,
+                       run_encoder_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -235,4 +236,28 @@ def test_config3_encoder_prefill_sampled(csa2, orc):
     for l, (q, swa, o, lse) in enumerate(outs):
         ro, rl = orc.prefill_attn(q_pos[pick], q[pick], want, codes, scales, swa, swa_start)
         check_attn(o[pick], lse[pick], ro, rl, f"config 3 layer {l}")
+    assert ps.errors() == 0
+
+
+def test_config6_encoder_decode_1m_b8_sampled(csa2, orc):
+    """The encoder side of one generated token at 1M tokens: B = 8 sequences of
+    524,288 entries at ratio 2 through the 18 encoder layers (3 x (Full + 5
+    Reuse), flat indexer), the launch configuration bench.py --config 6 times.
+    Sequences 0 and 3 are checked against the oracle; the rest of the batch
+    holds seeded device-side data."""
+    c = synth.CONFIGS[6]
+    L, B, seed = c["L"], c["B"], c["seed"]
+    ps = PagedSeqs(csa2, [L] * B)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    sampled = {0: None, 3: None}
+    for b in range(B):
+        if b in sampled:
+            sampled[b] = fill_synth(ps, orc, b, L, seed, ratio=2)
+        else:
+            fill_device(ps, csa2, b, L, gen)
+    q_idx, w, q, swa = encoder_layer_inputs(seed, B, [L] * B, 18)
+    r = run_encoder_step(csa2, ps, [L] * B, q_idx, w, q, swa)
+    for b, (codes, scales, idx) in sampled.items():
+        compare_encoder_seq(orc, r, b, L, codes, scales, idx, q_idx[b], w[b], q[b], swa[b], f"config 6 seq {b}")
     assert ps.errors() == 0

@@ -136,6 +136,40 @@ def test_decode_step_schedule_invariants(orc):
     assert changed == [6, 7]
 
 
+def test_encoder_decode_step_is_flat(orc):
+    # keep = 0 (the encoder's layers): each Full layer's set is the Top-512 of
+    # ALL L scores by (score desc, index asc), here ranked by numpy; a planted
+    # entry whose block pools to ~0 is found by the flat selection and missed
+    # by the decoder's hierarchy on the same context.
+    L = 8 * 2048 + 8 * 300 + 5
+    codes, scales, k, pooled, q_idx, w, q, swa = _decode_inputs(L, n_layers=18, seed=1003)
+    modes = orc.schedule(False)
+    u = np.random.default_rng(11).standard_normal((4, 64)).astype(np.float32)
+    q_idx[0] = bf(u)
+    w[0] = 1.0
+    e = 8 * 1234 + 3
+    v = 8.0 * u.sum(0)                    # positive dot with every head
+    kf = np.tile(-v * (3.0 / 7.0), (8, 1))
+    kf[3] = v                             # the block pools to -v/4: score 0
+    k[8 * 1234:8 * 1235] = bf(kf)
+    pooled = orc.pool_blocks(k)
+    r = orc.decode_step(modes, L, codes, scales, k, pooled, q_idx, w, q, swa, keep=0)
+    for l, m in enumerate(modes):
+        if m == 2:
+            np.testing.assert_array_equal(r["idx"][l], r["idx"][l - 1])
+        else:
+            s = orc.score_rows(q_idx[l], w[l], k).astype(np.float64)
+            order = np.lexsort((np.arange(L), -s))[:512]
+            assert sorted(order.tolist()) == r["idx"][l].tolist()
+        o, lse = orc.attend(q[l], r["idx"][l], codes, scales, swa[l, :128])
+        np.testing.assert_array_equal(o, r["out"][l])
+        np.testing.assert_array_equal(lse, r["lse"][l])
+    assert e in r["idx"][0].tolist()
+    rh = orc.decode_step(modes, L, codes, scales, k, pooled, q_idx, w, q, swa, keep=2048)
+    assert e not in rh["idx"][0].tolist()
+    assert 1234 not in orc.select_blocks(pooled, L, q_idx[0], w[0]).tolist()  # pruned by the hierarchy
+
+
 def test_decode_window_boundary(orc):
     # L < 128: only the first L SWA rows take part (a sentinel in row L must not count)
     L = 50
