@@ -41,32 +41,45 @@ namespace csa2 {
 // ----------------------------------------------------------------------------
 // score of one indexer-K row held as 32 bf16x2 words; qd[d] = (q_0..q_3)[d]
 // ----------------------------------------------------------------------------
+// Two rows at once with packed fp32 arithmetic: fma.rn.f32x2 performs one
+// fused multiply-add, rounded to nearest, in each 32-bit half, so the low half
+// follows row k's scalar FMA chain and the high half row m's, bit for bit.
+// qp[2 d + j] holds ((q_2j, q_2j), (q_2j+1, q_2j+1)) of dimension d, j = 0, 1.
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
 __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32_t (&m)[32],
-                                           const float4* __restrict__ qd, float4 w, float& s_k, float& s_m) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+                                           const ulonglong2* __restrict__ qp, float4 w, float& s_k, float& s_m) {
+    uint64_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;  // (row k, row m) dot of head h; zero bits are (+0, +0)
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const float k0 = bf16_lo(k[i]), k1 = bf16_hi(k[i]);
-        const float m0 = bf16_lo(m[i]), m1 = bf16_hi(m[i]);
-        const float4 q0 = qd[2 * i], q1 = qd[2 * i + 1];
-        a0 = __fmaf_rn(q0.x, k0, a0);
-        a1 = __fmaf_rn(q0.y, k0, a1);
-        a2 = __fmaf_rn(q0.z, k0, a2);
-        a3 = __fmaf_rn(q0.w, k0, a3);
-        b0 = __fmaf_rn(q0.x, m0, b0);
-        b1 = __fmaf_rn(q0.y, m0, b1);
-        b2 = __fmaf_rn(q0.z, m0, b2);
-        b3 = __fmaf_rn(q0.w, m0, b3);
-        a0 = __fmaf_rn(q1.x, k1, a0);
-        a1 = __fmaf_rn(q1.y, k1, a1);
-        a2 = __fmaf_rn(q1.z, k1, a2);
-        a3 = __fmaf_rn(q1.w, k1, a3);
-        b0 = __fmaf_rn(q1.x, m1, b0);
-        b1 = __fmaf_rn(q1.y, m1, b1);
-        b2 = __fmaf_rn(q1.z, m1, b2);
-        b3 = __fmaf_rn(q1.w, m1, b3);
+        const uint64_t x0 = pack2(bf16_lo(k[i]), bf16_lo(m[i]));  // dimension 2i
+        const uint64_t x1 = pack2(bf16_hi(k[i]), bf16_hi(m[i]));  // dimension 2i + 1
+        const ulonglong2 q01a = qp[4 * i], q23a = qp[4 * i + 1], q01b = qp[4 * i + 2], q23b = qp[4 * i + 3];
+        c0 = ffma2(q01a.x, x0, c0);
+        c1 = ffma2(q01a.y, x0, c1);
+        c2 = ffma2(q23a.x, x0, c2);
+        c3 = ffma2(q23a.y, x0, c3);
+        c0 = ffma2(q01b.x, x1, c0);
+        c1 = ffma2(q01b.y, x1, c1);
+        c2 = ffma2(q23b.x, x1, c2);
+        c3 = ffma2(q23b.y, x1, c3);
     }
+    float a0, a1, a2, a3, b0, b1, b2, b3;
+    unpack2(c0, a0, b0);
+    unpack2(c1, a1, b1);
+    unpack2(c2, a2, b2);
+    unpack2(c3, a3, b3);
     float s = 0.f, t = 0.f;
     s = __fmaf_rn(w.x, a0 > 0.f ? a0 : 0.f, s);
     t = __fmaf_rn(w.x, b0 > 0.f ? b0 : 0.f, t);
@@ -78,6 +91,16 @@ __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32
     t = __fmaf_rn(w.w, b3 > 0.f ? b3 : 0.f, t);
     s_k = s;
     s_m = t;
+}
+
+// Load q_idx [4][64] bf16 of one row into the duplicated layout idx_score2 reads.
+__device__ __forceinline__ void load_q_pairs(const uint16_t* q, float4* qp, int tid, int nt) {
+    for (int d = tid; d < kID; d += nt) {
+        const float q0 = bf16_bits_to_f32(q[d]), q1 = bf16_bits_to_f32(q[kID + d]);
+        const float q2 = bf16_bits_to_f32(q[2 * kID + d]), q3 = bf16_bits_to_f32(q[3 * kID + d]);
+        qp[2 * d] = make_float4(q0, q0, q1, q1);
+        qp[2 * d + 1] = make_float4(q2, q2, q3, q3);
+    }
 }
 
 __device__ __forceinline__ float idx_score1(const uint32_t (&k)[32], const float4* __restrict__ qd, float4 w) {
@@ -316,7 +339,7 @@ constexpr int K2_PROWS = K2_TILE / K2_PWARPS;   // 128 rows copied per producer 
 constexpr int K2_CROWS = K2_TILE / K2_CWARPS;   // 64 rows scored per consumer warp
 constexpr size_t K2_OFF_HIST = K2_STAGES * K2_STAGE_BYTES;
 constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
-constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);
+constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 32);  // q in pairs: 64 x 32 B
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
 constexpr size_t K2_OFF_NBLK = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
 constexpr size_t K2_OFF_BAR = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // full[3], empty[3]
@@ -345,6 +368,7 @@ struct BlockArgs {
     int64_t max_len;
     int n, keep, page_shift;
     int rshift;        // log2 entries per scored row
+    int span;          // rows filtered per select CTA (a multiple of 8192)
 };
 
 // tile_start[b] = first tile of sequence b; returns the sequence of tile t
@@ -523,10 +547,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
         const int b = seq_of_tile(tile_start, a.n, t);
         if (b != cur_b) {
             if (cur_b >= 0) flush(cur_b, nloc);
-            const uint16_t* qb = a.q_idx + (int64_t)b * kIH * kID;
-            for (int d = tid; d < kID; d += K2_CTHREADS)
-                qd[d] = make_float4(bf16_bits_to_f32(qb[d]), bf16_bits_to_f32(qb[kID + d]),
-                                    bf16_bits_to_f32(qb[2 * kID + d]), bf16_bits_to_f32(qb[3 * kID + d]));
+            load_q_pairs(a.q_idx + (int64_t)b * kIH * kID, qd, tid, K2_CTHREADS);
             if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
             cur_b = b;
             nloc = 0;
@@ -541,7 +562,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // the stage's rows of this warp are in registers
         float s0, s1;
-        idx_score2(k, m, qd, s_w, s0, s1);
+        idx_score2(k, m, reinterpret_cast<const ulonglong2*>(qd), s_w, s0, s1);
         const int32_t j = (t - tile_start[b]) * K2_TILE + r0;
         const int32_t nblk = s_nblk[b];
         float* sc = a.scores + (int64_t)b * a.nblk_pad;
@@ -565,6 +586,9 @@ constexpr int K3_BND_CAP = 12288;                               // boundary entr
 constexpr size_t K3_OFF_LAST = (size_t)2 * K3_WORDS * 4 + 1024 * 4 + 64 * 4 + (size_t)K3_BND_CAP * 8;
 constexpr size_t K3_SMEM = K3_OFF_LAST + 16;
 
+// kFlat: rows are entries (several chunks per CTA, bitmaps possibly in global
+// memory); otherwise blocks of 8 (one chunk per CTA, bitmaps in shared memory).
+template <bool kFlat>
 __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     int& s_last = *reinterpret_cast<int*>(smem + K3_OFF_LAST);
@@ -583,15 +607,16 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
             for (int i = threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = i < nblk ? i : -1;
         return;
     }
-    const int32_t c0 = blockIdx.x * K3_CHUNK;
+    const int32_t span = kFlat ? a.span : K3_CHUNK;
+    const int32_t c0 = blockIdx.x * span;
     if (c0 >= nblk) return;
-    const int32_t c1 = min(c0 + K3_CHUNK, nblk);
+    const int32_t c1 = min(c0 + span, nblk);
     const uint32_t bstar = (uint32_t)__ldcg(&a.thr[4 * b]);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const float* scores = a.scores + (int64_t)b * a.nblk_pad;
     uint32_t* bitmap = a.bitmap + (int64_t)b * (a.nblk_pad >> 5);
     uint64_t* bnd = a.bnd + (int64_t)b * a.nblk_pad;
-    constexpr int U = 4;  // loads in flight per thread
+    constexpr int U = kFlat ? 8 : 4;  // loads in flight per thread
     for (int32_t base = c0 + wid * 32; base < c1; base += U * K3_THREADS) {
         float v[U];
 #pragma unroll
@@ -622,7 +647,7 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        const uint32_t nch = (uint32_t)((nblk + K3_CHUNK - 1) / K3_CHUNK);
+        const uint32_t nch = (uint32_t)((nblk + span - 1) / span);
         s_last = atomicAdd(&a.ctr[2 * b + 1], 1u) == nch - 1;
     }
     __syncthreads();
@@ -634,7 +659,7 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     // (every block-level context); a flat selection over more rows works on
     // the sequence's bitmap in global memory and a tie bitmap beside it.
     const int nwords = (nblk + 31) >> 5;
-    const bool gm = nwords > K3_WORDS;
+    const bool gm = kFlat && nwords > K3_WORDS;
     uint32_t* sm_bm = reinterpret_cast<uint32_t*>(smem);
     uint32_t* hist = sm_bm + 2 * K3_WORDS;
     uint32_t* tmp = hist + 1024;
@@ -647,8 +672,13 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
         load_words(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd), 2 * (int)n_bnd);
         B = sbnd;
     }
-    if (!gm) load_words(bm, bitmap, nwords);
-    for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
+    if (!gm) {
+        load_words(bm, bitmap, nwords);
+        for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
+    } else {  // 16-byte groups: a sequence's bitmaps are 1 KiB aligned, padded to 256 words
+        for (int i = threadIdx.x; i < (nwords + 3) / 4; i += K3_THREADS)
+            reinterpret_cast<uint4*>(tie)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     uint32_t need = (uint32_t)a.keep - (uint32_t)__ldcg(&a.thr[4 * b + 1]);
     int d2, d3;
     uint32_t above;
@@ -680,38 +710,118 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
         else if (key == T) atomicOr(&tie[j >> 5], 1u << (j & 31));
     }
     __syncthreads();
-    // ordered scan over words: thread t owns words [t*per, (t+1)*per)
-    const int per = (nwords + K3_THREADS - 1) / K3_THREADS;
-    const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
-    uint32_t my_ties = 0;
-    auto ld = [gm](const uint32_t* p, int i) { return gm ? __ldcg(p + i) : p[i]; };
-    for (int i = w0; i < w1; ++i) my_ties += __popc(ld(tie, i));
-    uint32_t tot;
-    uint32_t rank = block_excl_scan(my_ties, tmp, &tot);
-    uint32_t my_sel = 0;
-    for (int i = w0; i < w1; ++i) {
-        uint32_t t = ld(tie, i), kept = 0;
-        while (t && rank < need) {
-            const uint32_t lb = t & (0u - t);
-            kept |= lb;
-            t ^= lb;
-            ++rank;
+    // Ordered emission, K3_WORDS words at a time: global bitmaps are staged
+    // into shared memory chunk by chunk with coalesced loads (the bitmaps that
+    // live in shared memory are one chunk).  Ties are taken lowest index first
+    // across chunks.
+    uint32_t rank0 = 0, base0 = 0;  // ties and selected entries of the chunks before
+    for (int c0w = 0; c0w < nwords; c0w += K3_WORDS) {
+        const int cn = min(K3_WORDS, nwords - c0w);
+        uint32_t* cbm = sm_bm;
+        uint32_t* ctie = sm_bm + K3_WORDS;
+        if (gm) {
+            __syncthreads();  // the previous chunk is no longer read
+            constexpr int V = K3_WORDS / 4 / K3_THREADS;  // 16-byte loads per thread and bitmap
+            const uint4* gb = reinterpret_cast<const uint4*>(bm + c0w);
+            const uint4* gt = reinterpret_cast<const uint4*>(tie + c0w);
+            uint4 vb[V], vt[V];
+#pragma unroll
+            for (int k = 0; k < V; ++k) {  // all loads in flight at once
+                const int i = threadIdx.x + k * K3_THREADS;
+                vb[k] = 4 * i < cn ? __ldcg(gb + i) : make_uint4(0u, 0u, 0u, 0u);
+                vt[k] = 4 * i < cn ? __ldcg(gt + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const int i = threadIdx.x + k * K3_THREADS;
+                reinterpret_cast<uint4*>(cbm)[i] = vb[k];
+                reinterpret_cast<uint4*>(ctie)[i] = vt[k];
+            }
+            __syncthreads();
         }
-        rank += __popc(t);
-        const uint32_t v = ld(bm, i) | kept;
-        bm[i] = v;
-        my_sel += __popc(v);
-    }
-    uint32_t base = block_excl_scan(my_sel, tmp, &tot);
-    for (int i = w0; i < w1; ++i) {
-        uint32_t m = ld(bm, i);
-        while (m) {
-            const int bit = __ffs(m) - 1;
-            m &= m - 1;
-            if (base < (uint32_t)a.keep) out[base] = i * 32 + bit;
-            ++base;
+        uint32_t n_ties, n_sel;
+        if (gm) {  // long chunks (flat selections): warp-ordered, conflict-free reads
+            // warp v owns words [lo, hi) of the chunk; lane l takes words lo + 32 k + l,
+            // so shared-memory reads are conflict-free and warp scans give the order
+            const int pw = ((cn + K3_THREADS / 32 - 1) / (K3_THREADS / 32) + 31) & ~31;
+            const int lo = wid * pw, hi = min(cn, lo + pw);
+            uint32_t w_ties = 0;
+            for (int i0 = lo; i0 < hi; i0 += 32) {
+                const int i = i0 + lane;
+                w_ties += __popc(i < hi ? ctie[i] : 0u);
+            }
+            for (int o = 16; o > 0; o >>= 1) w_ties += __shfl_xor_sync(0xffffffffu, w_ties, o);
+            uint32_t rank = rank0 + __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? w_ties : 0u, tmp, &n_ties), 0);
+            uint32_t w_sel = 0;
+            for (int i0 = lo; i0 < hi; i0 += 32) {
+                const int i = i0 + lane;
+                uint32_t t = i < hi ? ctie[i] : 0u;
+                const uint32_t c = __popc(t);
+                const uint32_t incl = warp_incl_scan(c);
+                const uint32_t r = rank + incl - c;  // ties before this word, in entry order
+                uint32_t take = r >= need ? 0u : min(c, need - r), kept = 0;
+                while (take--) {  // the lowest-index ties of the word
+                    const uint32_t lb = t & (0u - t);
+                    kept |= lb;
+                    t ^= lb;
+                }
+                if (i < hi) {
+                    cbm[i] |= kept;
+                    w_sel += __popc(cbm[i]);
+                }
+                rank += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            for (int o = 16; o > 0; o >>= 1) w_sel += __shfl_xor_sync(0xffffffffu, w_sel, o);
+            uint32_t base = base0 + __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? w_sel : 0u, tmp, &n_sel), 0);
+            for (int i0 = lo; i0 < hi; i0 += 32) {
+                const int i = i0 + lane;
+                uint32_t m = i < hi ? cbm[i] : 0u;
+                const uint32_t c = __popc(m);
+                const uint32_t incl = warp_incl_scan(c);
+                uint32_t pos = base + incl - c;
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (pos < (uint32_t)a.keep) out[pos] = (c0w + i) * 32 + bit;
+                    ++pos;
+                }
+                base += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        } else {  // the block level's short chunk
+            // thread t owns words [t*per, (t+1)*per) of the chunk
+            const int per = (cn + K3_THREADS - 1) / K3_THREADS;
+            const int w0 = threadIdx.x * per, w1 = min(cn, w0 + per);
+            uint32_t my_ties = 0;
+            for (int i = w0; i < w1; ++i) my_ties += __popc(ctie[i]);
+            uint32_t rank = rank0 + block_excl_scan(my_ties, tmp, &n_ties);
+            uint32_t my_sel = 0;
+            for (int i = w0; i < w1; ++i) {
+                uint32_t t = ctie[i], kept = 0;
+                while (t && rank < need) {  // the lowest-index ties
+                    const uint32_t lb = t & (0u - t);
+                    kept |= lb;
+                    t ^= lb;
+                    ++rank;
+                }
+                rank += __popc(t);
+                cbm[i] |= kept;
+                my_sel += __popc(cbm[i]);
+            }
+            uint32_t base = base0 + block_excl_scan(my_sel, tmp, &n_sel);
+            for (int i = w0; i < w1; ++i) {
+                uint32_t m = cbm[i];
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (base < (uint32_t)a.keep) out[base] = (c0w + i) * 32 + bit;
+                    ++base;
+                }
+            }
         }
+        rank0 += n_ties;
+        base0 += n_sel;
     }
+    const uint32_t tot = base0;
     for (int i = (int)tot + threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = -1;
     if (threadIdx.x == 0) {
         a.bnd_cnt[b] = 0;
@@ -1770,7 +1880,9 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
                               int32_t* err, cudaStream_t stream, bool flat) {
     static bool d2[64], d3[64];
     cudaError_t e = ensure_smem((const void*)block_score_kernel, K2_SMEM, d2);
-    if (e == cudaSuccess) e = ensure_smem((const void*)block_select_kernel, K3_SMEM, d3);
+    static bool d3f[64];
+    if (e == cudaSuccess) e = ensure_smem((const void*)block_select_kernel<false>, K3_SMEM, d3);
+    if (e == cudaSuccess) e = ensure_smem((const void*)block_select_kernel<true>, K3_SMEM, d3f);
     if (e != cudaSuccess) return e;
     if (n > K2_MAX_SEQS) return cudaErrorInvalidValue;
     const DecodeWs l = decode_ws_layout(n, max_len, flat);
@@ -1804,8 +1916,14 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
         e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, a);
         if (e != cudaSuccess) return e;
     }
-    LaunchCfg c3(dim3((unsigned)((nblk + K3_CHUNK - 1) / K3_CHUNK), n), dim3(K3_THREADS), K3_SMEM, stream);
-    return cudaLaunchKernelEx(&c3.cfg, block_select_kernel, a);
+    // one CTA per SM holds the select's shared memory: give each CTA several
+    // 8192-row chunks when the batch has more chunks than one wave
+    const int64_t chunks = (nblk + K3_CHUNK - 1) / K3_CHUNK;
+    const int64_t cpb = flat ? std::max<int64_t>(1, (chunks * n + sm_count() - 1) / sm_count()) : 1;
+    a.span = (int)(K3_CHUNK * cpb);
+    LaunchCfg c3(dim3((unsigned)((nblk + a.span - 1) / a.span), n), dim3(K3_THREADS), K3_SMEM, stream);
+    return flat ? cudaLaunchKernelEx(&c3.cfg, block_select_kernel<true>, a)
+                : cudaLaunchKernelEx(&c3.cfg, block_select_kernel<false>, a);
 }
 
 cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
