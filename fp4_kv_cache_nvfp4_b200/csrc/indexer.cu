@@ -31,7 +31,11 @@
 //                              of a sequence refines and emits the Top-K.
 //   prefill_score_kernel / prefill_select_kernel: the same per query over the
 //                              entries visible to it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -369,6 +373,7 @@ struct BlockArgs {
     int n, keep, page_shift;
     int rshift;        // log2 entries per scored row
     int span;          // rows filtered per select CTA (a multiple of 8192)
+    int tma;           // 1: rows arrive as 64-row tensor boxes (entry rows, pages of >= 64 entries)
 };
 
 // tile_start[b] = first tile of sequence b; returns the sequence of tile t
@@ -382,7 +387,8 @@ __device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int n, int
     return lo;
 }
 
-__global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a) {
+__global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                     BlockArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + K2_OFF_HIST);
     float4* qd = reinterpret_cast<float4*>(smem + K2_OFF_QD);
@@ -398,7 +404,9 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
 
     pdl_wait();
     pdl_trigger();
-    if (smem_u32(smem) & 15u) {  // 16-byte copies and vector reads need an aligned base
+    // 16-byte copies and vector reads need an aligned base; 128-byte-swizzled
+    // tensor boxes a 1 KiB aligned one (uniform over the grid)
+    if (smem_u32(smem) & (a.tma ? 1023u : 15u)) {
         if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
         return;
     }
@@ -430,9 +438,11 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
         if (tid == 0) {
             tile_start[a.n] = (int32_t)total;
             for (int s = 0; s < K2_STAGES; ++s) {
-                mbar_init(&full[s], K2_PWARPS * 32);  // one cp.async arrival per producer thread
-                mbar_init(&empty[s], K2_CWARPS);      // one arrival per consumer warp
+                // one cp.async arrival per producer thread, or one expect-tx arrival per producer warp
+                mbar_init(&full[s], a.tma ? K2_PWARPS : K2_PWARPS * 32);
+                mbar_init(&empty[s], K2_CWARPS);  // one arrival per consumer warp
             }
+            fence_mbar_init();
             s_timeout = 0;
         }
         for (int i = tid; i < kHistBins; i += K2_THREADS) hist[i] = 0;
@@ -444,6 +454,50 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(BlockArgs a)
     const int ntiles = t1 - t0;
     if (ntiles <= 0) return;
 
+    if (wid >= K2_CWARPS && a.tma) {
+        // ============ producers, tensor boxes (entry rows) ============
+        // Lanes 0 and 1 of producer warp pw copy the two 64-row boxes of the
+        // warp's 128 rows; a box lies in one page (pages hold >= 64 entries,
+        // boxes start at multiples of 64) and lands 128-byte swizzled, chunk c
+        // of row r at c ^ (r & 7), the layout the consumers read.
+        const int pw = wid - K2_CWARPS;
+        const int sh = a.page_shift;
+        const int32_t emask = (1 << sh) - 1;
+        const int32_t mpps = a.cache.max_pages_per_seq;
+        auto box_slot = [&](int32_t t) -> int32_t {  // first slot of this lane's box of tile t, -1 past the end
+            const int b = seq_of_tile(tile_start, a.n, t);
+            const int32_t j = (t - tile_start[b]) * K2_TILE + K2_PROWS * pw + 64 * lane;
+            if (lane >= 2 || j >= s_nblk[b]) return -1;
+            const int32_t pg = j >> sh;
+            int32_t phys = pg < mpps ? __ldg(a.cache.page_table + (int64_t)b * mpps + pg) : -1;
+            if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                dev_error(a.err, CSA2_DEV_PAGE);
+                phys = 0;  // results of this call are undefined; the copy stays in bounds
+            }
+            return (int32_t)(((int64_t)phys << sh) | (j & emask));
+        };
+        int32_t nxt = box_slot(t0);
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % K2_STAGES;
+            if (i >= K2_STAGES && !mbar_wait(&empty[s], (uint32_t)((i / K2_STAGES) - 1) & 1u, kWaitLimit))
+                s_timeout = 1;
+            const int32_t slot = nxt;
+            if (i + 1 < ntiles) nxt = box_slot(t0 + i + 1);  // the page lookup overlaps the copies
+            const unsigned m = __ballot_sync(0xffffffffu, slot >= 0);
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], 64u * 128u * (uint32_t)__popc(m));
+            __syncwarp();
+            if (slot >= 0)
+                tma_load_2d(smem + (size_t)s * K2_STAGE_BYTES + (size_t)(K2_PROWS * pw + 64 * lane) * 128, &tmap, 0,
+                            slot, &full[s]);
+        }
+        // the last stages' copies have landed before this warp leaves (bounded)
+        for (int i = max(0, ntiles - K2_STAGES); i < ntiles; ++i)
+            if (lane == 0 && !mbar_wait(&full[i % K2_STAGES], (uint32_t)(i / K2_STAGES) & 1u, kWaitLimit))
+                s_timeout = 1;
+        __syncwarp();
+        if (s_timeout && lane == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;
+    }
     if (wid >= K2_CWARPS) {
         // ================= producers =================
         const int pw = wid - K2_CWARPS;
@@ -1863,6 +1917,35 @@ static cudaError_t ensure_smem(const void* fn, size_t bytes, bool* done) {
     return cudaSuccess;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+// The indexer-K rows as a 2-D tensor [n_slots][64] bf16 read in 64-row boxes,
+// 128-byte swizzled.  Returns false when the map cannot be made.
+static bool entry_row_map(const csa2_kv_cache& cache, CUtensorMap* map) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size)};
+    const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kID, 64u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int sm_count() {
     static int n[64];
     int dev = 0;
@@ -1909,11 +1992,14 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.keep = keep;
     a.page_shift = page_shift_of(cache);
     const int64_t nblk = flat ? max_len : (max_len + kBlk - 1) / kBlk;
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    a.tma = flat && cache.page_size >= 64 && entry_row_map(cache, &map) ? 1 : 0;
     if (nblk > keep) {
         const int64_t tiles = (int64_t)n * ((nblk + K2_TILE - 1) / K2_TILE);
         const int grid = (int)std::min<int64_t>(tiles, sm_count());
         LaunchCfg c2(dim3((unsigned)grid), dim3(K2_THREADS), K2_SMEM, stream);
-        e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, a);
+        e = cudaLaunchKernelEx(&c2.cfg, block_score_kernel, map, a);
         if (e != cudaSuccess) return e;
     }
     // one CTA per SM holds the select's shared memory: give each CTA several
