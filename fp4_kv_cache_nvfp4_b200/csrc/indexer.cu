@@ -366,6 +366,8 @@ struct BlockArgs {
     uint64_t* bnd;     // [n][nblk_pad]
     uint32_t* bnd_cnt; // [n]
     uint32_t* tie;     // [n][nblk_pad/32] (flat only: the finalize's tie bitmap)
+    int32_t* abv;      // [n][512] (flat only: rows whose first digit is above the K-th's)
+    uint32_t* abv_cnt; // [n]
     const uint8_t* rows;  // scored rows: pooled indexer K (rshift 3) or indexer K (rshift 0)
     int32_t* err;
     int64_t nblk_pad;
@@ -688,6 +690,14 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
             const unsigned mgt = __ballot_sync(0xffffffffu, j < c1 && bin > bstar);
             const unsigned meq = __ballot_sync(0xffffffffu, j < c1 && bin == bstar);
             if (lane == 0) bitmap[wbase >> 5] = mgt;
+            if (kFlat && mgt) {  // fewer than keep rows lie above the K-th's bin: list them too
+                const int leader = __ffs(mgt) - 1;
+                uint32_t pos = 0;
+                if (lane == leader) pos = atomicAdd(&a.abv_cnt[b], (uint32_t)__popc(mgt));
+                pos = __shfl_sync(0xffffffffu, pos, leader);
+                const uint32_t at = pos + __popc(mgt & ((1u << lane) - 1u));
+                if (((mgt >> lane) & 1u) && at < (uint32_t)kMaxTopk) a.abv[(int64_t)b * kMaxTopk + at] = j;
+            }
             if (meq) {
                 const int leader = __ffs(meq) - 1;
                 uint32_t pos = 0;
@@ -757,6 +767,74 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     find_kth_bin(hist, 1024, need, tmp, &d3, &above);
     need -= above;
     const uint32_t T = (bstar << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+    if (kFlat) {
+        // A flat selection takes keep (<= 512) of up to 2^21 rows: list them
+        // (the rows above the K-th's bin, the boundary rows above T and the
+        // `need` lowest-index ties) and sort the list, instead of scanning the
+        // row bitmap.  More than 256 ties take the bitmap scan below.
+        uint32_t my_t = 0;
+        for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) my_t += (uint32_t)(B[i] >> 32) == T ? 1u : 0u;
+        uint32_t n_tie;
+        (void)block_excl_scan(my_t, tmp, &n_tie);
+        const uint32_t n_abv = __ldcg(&a.abv_cnt[b]);
+        if (n_tie <= 256u && n_abv < (uint32_t)a.keep) {  // uniform over the CTA
+            uint32_t* s_sel = sm_bm;         // [1024] selected rows, then the sort's padding
+            uint32_t* s_tie = sm_bm + 1024;  // [256] rows tied at T
+            uint32_t* s_cnt = sm_bm + 1280;  // boundary rows above T, ties
+            if (threadIdx.x == 0) {
+                s_cnt[0] = 0;
+                s_cnt[1] = 0;
+            }
+            for (uint32_t i = threadIdx.x; i < n_abv; i += K3_THREADS)
+                s_sel[i] = (uint32_t)__ldcg(a.abv + (int64_t)b * kMaxTopk + i);
+            __syncthreads();
+            for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) {
+                const uint64_t v = B[i];
+                const uint32_t key = (uint32_t)(v >> 32), j = (uint32_t)v;
+                if (key > T) {
+                    const uint32_t p = atomicAdd(&s_cnt[0], 1u);
+                    if (n_abv + p < 1024u) s_sel[n_abv + p] = j;
+                } else if (key == T) {
+                    s_tie[atomicAdd(&s_cnt[1], 1u)] = j;
+                }
+            }
+            __syncthreads();
+            const uint32_t n_gt = s_cnt[0];
+            for (uint32_t t = threadIdx.x; t < n_tie; t += K3_THREADS) {  // rank of a tie among the ties
+                const uint32_t j = s_tie[t];
+                uint32_t r = 0;
+                for (uint32_t u = 0; u < n_tie; ++u) r += s_tie[u] < j ? 1u : 0u;
+                if (r < need && n_abv + n_gt + r < 1024u) s_sel[n_abv + n_gt + r] = j;
+            }
+            const uint32_t m = min(n_abv + n_gt + min(need, n_tie), 1024u);
+            uint32_t P = 1;
+            while (P < m) P <<= 1;
+            for (uint32_t i = m + threadIdx.x; i < P; i += K3_THREADS) s_sel[i] = 0xffffffffu;
+            __syncthreads();
+            for (uint32_t k = 2; k <= P; k <<= 1) {  // bitonic sort, ascending
+                for (uint32_t jj = k >> 1; jj > 0; jj >>= 1) {
+                    for (uint32_t i = threadIdx.x; i < P; i += K3_THREADS) {
+                        const uint32_t ixj = i ^ jj;
+                        if (ixj > i) {
+                            const uint32_t x = s_sel[i], y = s_sel[ixj];
+                            if ((x > y) == ((i & k) == 0)) {
+                                s_sel[i] = y;
+                                s_sel[ixj] = x;
+                            }
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+            for (int i = threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = (uint32_t)i < m ? (int32_t)s_sel[i] : -1;
+            if (threadIdx.x == 0) {
+                a.bnd_cnt[b] = 0;
+                a.abv_cnt[b] = 0;
+                a.ctr[2 * b + 1] = 0;
+            }
+            return;
+        }
+    }
     for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) {
         const uint64_t v = B[i];
         const uint32_t key = (uint32_t)(v >> 32), j = (uint32_t)v;
@@ -879,6 +957,7 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     for (int i = (int)tot + threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = -1;
     if (threadIdx.x == 0) {
         a.bnd_cnt[b] = 0;
+        if (kFlat) a.abv_cnt[b] = 0;
         a.ctr[2 * b + 1] = 0;
     }
 }
@@ -1876,6 +1955,7 @@ DecodeWs decode_ws_layout(int n, int64_t max_len, bool flat) {
     l.blk_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_ctr = o; o = align256(o + (size_t)n * 8);
     l.blk_bnd_cnt = o; o = align256(o + (size_t)n * 4);
+    l.blk_abv_cnt = o; o = align256(o + (size_t)n * 4);
     l.tok_ctr = o; o = align256(o + (size_t)n * 4);
     l.tok_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_thr = o; o = align256(o + (size_t)n * 16);
@@ -1886,6 +1966,7 @@ DecodeWs decode_ws_layout(int n, int64_t max_len, bool flat) {
     l.blk_bnd = o; o = align256(o + (size_t)n * l.nblk_pad * 8);
     if (flat) {
         l.blk_tie = o; o = align256(o + (size_t)n * (l.nblk_pad / 32) * 4);
+        l.blk_abv = o; o = align256(o + (size_t)n * kMaxTopk * 4);
     }
     l.total = o;
     return l;
@@ -1983,6 +2064,8 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.bnd = reinterpret_cast<uint64_t*>(ws + l.blk_bnd);
     a.bnd_cnt = reinterpret_cast<uint32_t*>(ws + l.blk_bnd_cnt);
     a.tie = flat ? reinterpret_cast<uint32_t*>(ws + l.blk_tie) : nullptr;
+    a.abv = flat ? reinterpret_cast<int32_t*>(ws + l.blk_abv) : nullptr;
+    a.abv_cnt = reinterpret_cast<uint32_t*>(ws + l.blk_abv_cnt);
     a.rows = reinterpret_cast<const uint8_t*>(flat ? cache.idx_k : cache.idx_k_pooled);
     a.rshift = flat ? 0 : 3;
     a.err = err;

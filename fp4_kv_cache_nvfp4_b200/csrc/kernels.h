@@ -45,6 +45,7 @@ struct LaunchCfg {
 // Workspace layout of the decode indexer (byte offsets; all 256-aligned).
 struct DecodeWs {
     size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt, blk_tie;
+    size_t blk_abv, blk_abv_cnt;  // flat: rows above the K-th's bin, and their count
     size_t tok_keys, tok_ctr, tok_hist;
     size_t total;
     int64_t nblk_pad;  // per-sequence stride of block arrays

@@ -134,3 +134,26 @@ def test_encoder_decode_layers_vs_oracle(csa2, orc):
         codes, scales = orc.quant_rows(data[b][0], ratio=2)
         compare_encoder_seq(orc, r, b, L, codes, scales, data[b][1], q_idx[b], w[b], q[b], swa[b], f"seq {b}")
     assert ps.errors() == 0
+
+
+def test_flat_indexer_few_ties_at_the_boundary(csa2, orc):
+    """500 high rows and 30 identical rows just below them: the K-th score is
+    shared by the 30, and the 12 lowest-index ones complete the set (the
+    selection's list-and-sort path, which handles up to 256 ties)."""
+    L = 300000
+    ps = PagedSeqs(csa2, [L])
+    rng = np.random.default_rng(4)
+    kf = np.zeros((L, 64), np.float32)
+    picks = rng.choice(L, 530, replace=False)
+    hot, tied = picks[:500], np.sort(picks[500:])
+    kf[hot, 5] = 2.0 + rng.random(500).astype(np.float32)
+    kf[tied, 5] = 1.5
+    idx = synth.to_bf16_bits(kf)
+    _fill(ps, 0, L, keep_kv=False, idx=idx)
+    qf = np.zeros((1, 4, 64), np.float32)
+    qf[0, :, 5] = 1.0
+    q, w = synth.to_bf16_bits(qf), np.ones((1, 4), np.float32)
+    got = _run_flat(csa2, ps, [L], q, w)[0]
+    check_sets(got, orc.select_tokens(idx, L, None, q[0], w[0]), "ties")
+    assert set(tied[:12].tolist()) <= set(got.tolist()) and not set(tied[12:].tolist()) & set(got.tolist())
+    assert ps.errors() == 0
