@@ -806,26 +806,34 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
                 for (uint32_t u = 0; u < n_tie; ++u) r += s_tie[u] < j ? 1u : 0u;
                 if (r < need && n_abv + n_gt + r < 1024u) s_sel[n_abv + n_gt + r] = j;
             }
-            const uint32_t m = min(n_abv + n_gt + min(need, n_tie), 1024u);
+            const uint32_t m = min(n_abv + n_gt + min(need, n_tie), (uint32_t)K3_THREADS);
             uint32_t P = 1;
             while (P < m) P <<= 1;
-            for (uint32_t i = m + threadIdx.x; i < P; i += K3_THREADS) s_sel[i] = 0xffffffffu;
             __syncthreads();
-            for (uint32_t k = 2; k <= P; k <<= 1) {  // bitonic sort, ascending
+            // Bitonic sort, ascending, one value per thread (P <= 512 threads; the
+            // rest sort padding among themselves): partners closer than 32 are
+            // exchanged by shuffles, farther ones through two alternating
+            // shared-memory buffers, one barrier per such stage.
+            const uint32_t tid_u = threadIdx.x;
+            uint32_t v = tid_u < m ? s_sel[tid_u] : 0xffffffffu;
+            uint32_t* xb = sm_bm + 2048;  // [2][512]
+            int par = 0;
+            for (uint32_t k = 2; k <= P; k <<= 1) {
                 for (uint32_t jj = k >> 1; jj > 0; jj >>= 1) {
-                    for (uint32_t i = threadIdx.x; i < P; i += K3_THREADS) {
-                        const uint32_t ixj = i ^ jj;
-                        if (ixj > i) {
-                            const uint32_t x = s_sel[i], y = s_sel[ixj];
-                            if ((x > y) == ((i & k) == 0)) {
-                                s_sel[i] = y;
-                                s_sel[ixj] = x;
-                            }
-                        }
+                    uint32_t o;
+                    if (jj >= 32) {
+                        xb[par * K3_THREADS + tid_u] = v;
+                        __syncthreads();
+                        o = xb[par * K3_THREADS + (tid_u ^ jj)];
+                        par ^= 1;
+                    } else {
+                        o = __shfl_xor_sync(0xffffffffu, v, (int)jj);
                     }
-                    __syncthreads();
+                    v = (((tid_u & jj) == 0) == ((tid_u & k) == 0)) ? min(v, o) : max(v, o);
                 }
             }
+            s_sel[tid_u] = v;
+            __syncthreads();
             for (int i = threadIdx.x; i < a.keep; i += K3_THREADS) out[i] = (uint32_t)i < m ? (int32_t)s_sel[i] : -1;
             if (threadIdx.x == 0) {
                 a.bnd_cnt[b] = 0;
