@@ -105,6 +105,10 @@ def attn_bytes_per_row(L: int) -> int:
 # (ncu --set full, first Full and Reuse launches of the eager step; the kernel
 # source has not changed since), keyed by (B, L)
 ATTN_TRAFFIC = {(8, 1 << 20): 1944320}
+# dram__bytes_read.sum + dram__bytes_write.sum of one flat indexer launch
+# (block_score_kernel + block_select_kernel<1>) keyed by (B, entries), taken at
+# B = 2 (139,576,576 B) and scaled by the rows scored
+FLAT_TRAFFIC = {(8, 1 << 19): 558306304}
 
 
 class ClockSampler:
@@ -368,7 +372,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      bytes_per_launch=a_bytes, ms_per_launch=a_ms, peak_source=peak_src)
     idx_roof = dict(kernel="block_score_kernel + block_select_kernel" + (" over entries (flat indexer)" if flat else ""),
                     bound="hbm", achieved=k_gbs, peak=hbm, unit="GB/s", frac=k_gbs / hbm if hbm else None,
-                    traffic=None, bytes_per_launch=k_bytes, ms_per_launch=k_ms, peak_source=peak_src)
+                    traffic=FLAT_TRAFFIC.get((B, L)) if flat else None, bytes_per_launch=k_bytes, ms_per_launch=k_ms,
+                    peak_source=peak_src)
     schedule = "encoder: 3 x (F+5R), ratio 2, flat indexer" if flat else "decoder: F+3R, 4x(RI+3R)"
     res = dict(metric=METRIC_ENC if flat else METRIC, value=whole_job_tokens_per_s(B, world, ms_per_step), unit=UNIT,
                n_gpus=world, steps=args.steps,
