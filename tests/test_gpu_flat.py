@@ -67,7 +67,7 @@ def _run_flat(csa2, ps, lens, q, w, ws=None):
 
 # 300,000 entries: more than 262,144 rows, so the selection's final pass works
 # on the bitmaps in global memory; 20,001 and 70,000 keep them in shared memory.
-@pytest.mark.parametrize("page_size", [64, 8])
+@pytest.mark.parametrize("page_size", [64, 8, 1024])  # 64, 1024: rows as tensor boxes; 8: 16-byte copies
 def test_flat_indexer_bitexact(csa2, orc, page_size):
     lens = [20001, 70000, 300000, 3000, 400, 1]
     B = len(lens)

@@ -86,3 +86,26 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(csa2):
     st = L.csa2_indexer_topk_noalloc(ctypes.byref(d), ctypes.byref(cache), csa2.BLOCK, P(0x1000), P(0x1000),
                                      P(0x1000), None, P(0x1000), 64, 1 << 20, None, None)
     assert st == 4  # CSA2_ERR_WORKSPACE
+
+
+def test_noalloc_flat_indexer_matches_workspace_indexer(csa2):
+    """The flat indexer (keep_blocks = 0, Top-512 over every entry) through the
+    static scratch, twice, against the workspace entry point."""
+    lens = [70000, 300, 40000]
+    B, max_len = len(lens), max(lens)
+    ps = PagedSeqs(csa2, lens)
+    for b, L in enumerate(lens):
+        _fill(ps, b, L)
+    sl = dev(np.array(lens, np.int32))
+    d = csa2.default_desc(csa2.FULL, 2, keep_blocks=0)
+    ws = torch.zeros(csa2.workspace_bytes(d, csa2.TOKEN, B, max_len), dtype=torch.uint8, device="cuda")
+    q = bits16(np.concatenate([synth.q_idx(SEED, 6, b) for b in range(B)]))
+    w = dev(np.concatenate([synth.w_idx(SEED, 6, b) for b in range(B)]))
+    ref = torch.empty((B, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, q, w, sl, ref, B, max_len, ws, err=ps.err)
+    for call in range(2):
+        got = torch.full((B, 512), -5, dtype=torch.int32, device="cuda")
+        csa2.indexer_topk_noalloc(d, ps.cache, csa2.TOKEN, q, w, sl, got, B, max_len, err=ps.err)
+        torch.cuda.synchronize()
+        check_sets(got.cpu().numpy(), ref.cpu().numpy(), f"flat, call {call}")
+    assert ps.errors() == 0
