@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
     p.add_argument("--seq-len", type=int, default=0, help="override the context (profiling runs)")
     p.add_argument("--breakdown", action="store_true", help="also time every call of the step on its own")
+    p.add_argument("--kv-host", action="store_true",
+                   help="main KV (codes, scales) in pinned host memory, read in place (decode configs)")
     return p.parse_args()
 
 
@@ -192,7 +194,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     # ---- cache: B sequences of L entries, pages permuted ----------------------
     lens = np.full(B, L, np.int64)
     table, n_phys = synth.page_table(seed, lens, PAGE, shuffle=not args.contiguous_pages)
-    cache = csa2.KVCache(n_phys, PAGE, torch.from_numpy(table), device=dev)
+    cache = csa2.KVCache(n_phys, PAGE, torch.from_numpy(table), device=dev, main_kv_on_host=args.kv_host)
     gain = torch.from_numpy(synth.gain(seed)).to(dev)
     tab_d = torch.from_numpy(table).to(dev).long()
     chunk = 1 << 16
@@ -344,7 +346,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                 flush.fill_(k & 0xFF)
                 eev[k][0].record(stream)
                 step_in.copy_(host_in, non_blocking=True)
-                swa[:, :, ring, :].copy_(swa_new)
+                swa[:, :, ring, :].copy_(swa_new, non_blocking=True)
                 graph.replay()
                 host_res.copy_(result, non_blocking=True)
                 eev[k][1].record(stream)
@@ -383,6 +385,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                            global_batch=world * B, layers=layers, schedule=schedule, page_size=PAGE,
                            pages="contiguous" if args.contiguous_pages else "random permutation",
                            l2="flushed before every timed step (256 MiB write, not timed)", parallelism=f"dp{world}",
+                           kv_placement=("main KV (FP4 codes, E4M3 scales) in pinned host memory, read in "
+                                         "place; indexer K and SWA rows in device memory"
+                                         if args.kv_host else "device memory"),
                            graph="one CUDA graph per step, programmatic dependent launch between kernels"),
                step_bytes_unique=B * ub["total"], step_gbs=B * ub["total"] / (ms_per_step * 1e-3) / 1e9,
                step_frac_of_hbm=(B * ub["total"] / (ms_per_step * 1e-3) / 1e9) / hbm if hbm else None,

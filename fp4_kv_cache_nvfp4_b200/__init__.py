@@ -13,6 +13,6 @@ import os
 
 from ._binding import (  # noqa: F401
     BLOCK, BF16, CSA2Error, F32, FULL, KVCache, LayerDesc, REINDEX, REUSE, TOKEN, abi_version, decode_layers,
-    default_desc, indexer_topk, indexer_topk_noalloc, kv_quant_append, lib, lib_path, schedule, sparse_attn_decode, sparse_attn_prefill,
-    workspace_bytes,
+    default_desc, device_accessible, indexer_topk, indexer_topk_noalloc, kv_quant_append, lib, lib_path, schedule,
+    sparse_attn_decode, sparse_attn_prefill, workspace_bytes,
 )

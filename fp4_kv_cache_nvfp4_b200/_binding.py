@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             L.csa2_status_string.argtypes = [_I32]
             L.csa2_status_string.restype = ctypes.c_char_p
             L.csa2_abi_version.restype = _I32
+            L.csa2_device_accessible.argtypes = [_P]
+            L.csa2_device_accessible.restype = _I32
             _lib = L
     return _lib
 
@@ -100,6 +102,11 @@ def abi_version() -> int:
     return int(lib().csa2_abi_version())
 
 
+def device_accessible(t) -> int:
+    """1 if kernels can read the tensor (or raw address) in place, 0 if not, -1 on a CUDA error."""
+    return int(lib().csa2_device_accessible(_ptr(t)))
+
+
 def default_desc(mode: int = FULL, ratio: int = 1, **over) -> LayerDesc:
     d = LayerDesc()
     lib().csa2_layer_desc_default(ctypes.byref(d), mode, ratio)
@@ -118,14 +125,23 @@ class KVCache:
     """Paged FP4 main-KV cache + indexer K (+ pooled indexer K) in device memory.
 
     page_table: int32 [n_seqs, max_pages] (host or device tensor) mapping the
-    entry pages of each sequence to physical pages (-1 = none)."""
+    entry pages of each sequence to physical pages (-1 = none).
+    main_kv_on_host: keep codes and scales (the main KV) in pinned host memory
+    that the device reads in place; the indexer K stays in device memory."""
 
     def __init__(self, n_phys_pages: int, page_size: int, page_table: torch.Tensor, device="cuda",
-                 pooled: bool = True):
+                 pooled: bool = True, main_kv_on_host: bool = False):
         n = n_phys_pages * page_size
         self.page_size, self.n_phys_pages = page_size, n_phys_pages
-        self.codes = torch.zeros((n, 128), dtype=torch.uint8, device=device)
-        self.scales = torch.zeros((n, 16), dtype=torch.uint8, device=device)
+        if main_kv_on_host:
+            self.codes = torch.zeros((n, 128), dtype=torch.uint8, pin_memory=True)
+            self.scales = torch.zeros((n, 16), dtype=torch.uint8, pin_memory=True)
+            for t in (self.codes, self.scales):
+                if device_accessible(t) != 1:
+                    raise RuntimeError("pinned host memory is not mapped into the device address space")
+        else:
+            self.codes = torch.zeros((n, 128), dtype=torch.uint8, device=device)
+            self.scales = torch.zeros((n, 16), dtype=torch.uint8, device=device)
         self.idx_k = torch.zeros((n, 64), dtype=torch.int16, device=device)
         self.pooled = torch.zeros((n // 8, 64), dtype=torch.int16, device=device) if pooled else None
         self.page_table = page_table.to(device=device, dtype=torch.int32).contiguous()

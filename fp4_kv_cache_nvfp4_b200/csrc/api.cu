@@ -309,4 +309,24 @@ const char* csa2_status_string(csa2_status s) {
 
 int32_t csa2_abi_version(void) { return CSA2_ABI_VERSION; }
 
+int32_t csa2_device_accessible(const void* p) {
+    if (!p) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    switch (at.type) {
+        case cudaMemoryTypeDevice: return at.device == dev ? 1 : 0;
+        case cudaMemoryTypeManaged: return 1;
+        case cudaMemoryTypeHost: return at.devicePointer == p ? 1 : 0;
+        default: return 0;
+    }
+}
+
 }  // extern "C"

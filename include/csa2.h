@@ -96,8 +96,15 @@ typedef struct {
     int32_t idx_dim;     /* 64 */
 } csa2_layer_desc;
 
-/* Paged global-KV cache (caller-owned device memory).  Entry e of sequence b
+/* Paged global-KV cache (caller-owned memory).  Entry e of sequence b
  * lives in slot page_table[b][e / page_size] * page_size + e % page_size.
+ * Every array must be device-accessible (see csa2_device_accessible).  codes
+ * and scales (the main KV) may live in pinned host memory mapped into the
+ * device address space: attention then gathers only its selected 144-byte
+ * entries over the host link.  This is the global-KV tiering of the
+ * deployment paragraph of conexaotc.com.br, "FP4 KV, repeticion limitada..."
+ * (7minutos.es).  The indexer K arrays, which the indexer streams, belong in
+ * device memory.
  *   codes        [n_slots][128] u8  : channel 2j in the low nibble of byte j
  *   scales       [n_slots][16]  u8  : E4M3 bits, scale i covers channels 16i..16i+15
  *   idx_k        [n_slots][64]  bf16: indexer K of each entry
@@ -276,6 +283,12 @@ CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc* desc, cons
 /* ---------------------------------------------------------------------- */
 CSA2_API const char* csa2_status_string(csa2_status s);
 CSA2_API int32_t csa2_abi_version(void);
+
+/* 1 if kernels on the current device may dereference p at that same address:
+ * device or managed memory, or host memory allocated or registered with CUDA
+ * and mapped at p.  0 for pageable host memory or another device's memory, -1
+ * if CUDA reports an error.  The library does not call it on its own paths. */
+CSA2_API int32_t csa2_device_accessible(const void* p);
 
 #ifdef __cplusplus
 }

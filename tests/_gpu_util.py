@@ -24,13 +24,15 @@ def bits16(x: np.ndarray) -> torch.Tensor:
 class PagedSeqs:
     """A paged cache holding B sequences of the given entry lengths."""
 
-    def __init__(self, csa2, lens, page_size=64, shuffle=True, seed=7, pooled=True, extra_pages=0):
+    def __init__(self, csa2, lens, page_size=64, shuffle=True, seed=7, pooled=True, extra_pages=0,
+                 main_kv_on_host=False):
         self.csa2 = csa2
         self.lens = np.asarray(lens, np.int64)
         self.page = page_size
         cap = self.lens + extra_pages * page_size
         self.table, n_phys = synth.page_table(seed, cap, page_size, shuffle)
-        self.cache = csa2.KVCache(n_phys, page_size, torch.from_numpy(self.table), pooled=pooled)
+        self.cache = csa2.KVCache(n_phys, page_size, torch.from_numpy(self.table), pooled=pooled,
+                                  main_kv_on_host=main_kv_on_host)
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def slots(self, seq, positions):
@@ -55,7 +57,8 @@ class PagedSeqs:
         if c.pooled is not None:
             ps = torch.from_numpy(self.slots(seq, np.arange(0, L, 8)) // 8).cuda()
             pooled = c.pooled[ps].cpu().numpy().view(np.uint16)
-        return (c.codes[s].cpu().numpy(), c.scales[s].cpu().numpy(), c.idx_k[s].cpu().numpy().view(np.uint16),
+        sm = s.to(c.codes.device)  # the main KV may sit in pinned host memory
+        return (c.codes[sm].cpu().numpy(), c.scales[sm].cpu().numpy(), c.idx_k[s].cpu().numpy().view(np.uint16),
                 pooled)
 
     def errors(self):

@@ -35,6 +35,7 @@ def test_every_declared_symbol_is_exported(csa2):
     for n in _declared():
         assert hasattr(L, n), n
     assert csa2.abi_version() == 1
+    assert csa2.device_accessible(None) == 0  # answered before any CUDA call
 
 
 def test_schedule_and_defaults(csa2):
