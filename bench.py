@@ -273,6 +273,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         launches_per_step = 1 + sum((3 if L > 16384 else 2) if m != csa2.REUSE else 1 for m in modes)
     else:
         launches_per_step = 1 + sum({csa2.FULL: 4, csa2.REINDEX: 2, csa2.REUSE: 1}[m] for m in modes)
+    if args.kv_host:  # each new index set's rows are staged on the device once
+        launches_per_step += n_idx
 
     def barrier():
         if world > 1:

@@ -38,6 +38,22 @@ csa2_status check_cache(const csa2_kv_cache* c, bool need_idx, bool need_pooled)
     return CSA2_OK;
 }
 
+// Whether p is host memory (pinned and mapped, as the cache requires); the
+// answer for the last pointer asked is kept, so repeated calls (and calls
+// under stream capture) do not query the driver again.
+bool in_host_memory(const void* p) {
+    static thread_local const void* last = nullptr;
+    static thread_local bool last_host = false;
+    if (p == last) return last_host;
+    cudaPointerAttributes at{};
+    bool host = false;
+    if (cudaPointerGetAttributes(&at, p) == cudaSuccess) host = at.type == cudaMemoryTypeHost;
+    else (void)cudaGetLastError();
+    last = p;
+    last_host = host;
+    return host;
+}
+
 csa2_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return CSA2_OK;
     (void)cudaGetLastError();
@@ -263,6 +279,33 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
     if (!workspace || ws_bytes < need) return CSA2_ERR_WORKSPACE;
     const int topk = descs[0].topk;
     const int32_t* cur = nullptr;
+    // A main KV in host memory: each new index set's rows are copied once into
+    // the workspace's staged cache, and every attention layer reads them there.
+    const bool host_kv = in_host_memory(cache->codes);
+    const DecodeWs wl = decode_ws_layout(B, max_len, flat);
+    char* wsb = static_cast<char*>(workspace);
+    StageArgs sa{};
+    csa2_kv_cache staged{};
+    if (host_kv) {
+        sa.cache = *cache;
+        sa.seq_lens = seq_lens;
+        sa.stage_codes = reinterpret_cast<uint8_t*>(wsb + wl.stage_codes);
+        sa.stage_scales = reinterpret_cast<uint8_t*>(wsb + wl.stage_scales);
+        sa.stage_idx = reinterpret_cast<int32_t*>(wsb + wl.stage_idx);
+        sa.stage_pt = reinterpret_cast<int32_t*>(wsb + wl.stage_pt);
+        sa.err = err_word;
+        sa.topk = topk;
+        sa.stage_rows = wl.stage_rows;
+        sa.page_shift = page_shift_of(*cache);
+        staged.codes = sa.stage_codes;
+        staged.scales = sa.stage_scales;
+        staged.idx_k = cache->idx_k;
+        staged.idx_k_pooled = nullptr;
+        staged.page_table = sa.stage_pt;
+        staged.page_size = wl.stage_rows;
+        staged.max_pages_per_seq = 1;
+        staged.n_phys_pages = B;
+    }
     for (int l = 0; l < n_layers; ++l) {
         const csa2_layer_desc& d = descs[l];
         int32_t* set = idx_sets + (int64_t)l * B * topk;
@@ -286,10 +329,17 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
             cur = set;
         }
         if (s != CSA2_OK) return s;
+        if (host_kv && d.mode != CSA2_MODE_REUSE) {  // stage the new set's rows
+            sa.idx = cur;
+            s = from_cuda(launch_stage_rows(sa, B, (cudaStream_t)stream));
+            if (s != CSA2_OK) return s;
+        }
         // Not the call's first kernel: the cache, the lengths and the SWA
         // history were complete before that kernel passed its wait, and a Reuse
-        // layer's index set was written two or more launches back.
-        s = attn_decode(&d, cache, q[l], cur, swa_kv[l], seq_lens, swa_lens, out[l], lse[l], B, err_word, stream,
+        // layer's index set (and its staged rows) were written two or more
+        // launches back.
+        s = attn_decode(&d, host_kv ? &staged : cache, q[l], host_kv ? sa.stage_idx : cur, swa_kv[l], seq_lens,
+                        swa_lens, out[l], lse[l], B, err_word, stream,
                         kPreHist | (d.mode == CSA2_MODE_REUSE ? kPreIdx : 0));
         if (s != CSA2_OK) return s;
     }

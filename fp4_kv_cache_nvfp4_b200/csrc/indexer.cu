@@ -1968,6 +1968,11 @@ DecodeWs decode_ws_layout(int n, int64_t max_len, bool flat) {
     l.tok_hist = o; o = align256(o + (size_t)n * kHistBins * 4);
     l.blk_thr = o; o = align256(o + (size_t)n * 16);
     l.tok_keys = o; o = align256(o + (size_t)n * kMaxCand * 4);
+    l.stage_rows = kMaxTopk;
+    l.stage_codes = o; o = align256(o + (size_t)n * l.stage_rows * kCodeBytes);
+    l.stage_scales = o; o = align256(o + (size_t)n * l.stage_rows * kScales);
+    l.stage_idx = o; o = align256(o + (size_t)n * kMaxTopk * 4);
+    l.stage_pt = o; o = align256(o + (size_t)n * 4);
     // the scored rows' arrays (any keep below the row count needs them)
     l.blk_scores = o; o = align256(o + (size_t)n * l.nblk_pad * 4);
     l.blk_bitmap = o; o = align256(o + (size_t)n * (l.nblk_pad / 32) * 4);

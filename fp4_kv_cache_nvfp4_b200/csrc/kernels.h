@@ -46,6 +46,9 @@ struct LaunchCfg {
 struct DecodeWs {
     size_t blk_scores, blk_hist, blk_thr, blk_ctr, blk_bitmap, blk_bnd, blk_bnd_cnt, blk_tie;
     size_t blk_abv, blk_abv_cnt;  // flat: rows above the K-th's bin, and their count
+    // staged rows of one index set when the main KV is in host memory
+    size_t stage_codes, stage_scales, stage_idx, stage_pt;
+    int stage_rows;               // rows per sequence in the staged cache (a power of two >= topk)
     size_t tok_keys, tok_ctr, tok_hist;
     size_t total;
     int64_t nblk_pad;  // per-sequence stride of block arrays
@@ -105,5 +108,19 @@ struct AttnArgs {
 constexpr int kPreIdx = 1;
 constexpr int kPreHist = 2;
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+
+// Copies the FP4 rows of a decode index set into the staged cache (stage.cu).
+struct StageArgs {
+    csa2_kv_cache cache;   // the main KV (host memory)
+    const int32_t* idx;    // [B][topk]
+    const int32_t* seq_lens;
+    uint8_t* stage_codes;  // [B * stage_rows][128]
+    uint8_t* stage_scales; // [B * stage_rows][16]
+    int32_t* stage_idx;    // [B][topk]: i for a staged row, -1 otherwise
+    int32_t* stage_pt;     // [B]: page b of the staged cache is sequence b's
+    int32_t* err;
+    int topk, stage_rows, page_shift;
+};
+cudaError_t launch_stage_rows(const StageArgs& a, int B, cudaStream_t stream);
 
 }  // namespace csa2

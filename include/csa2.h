@@ -240,6 +240,11 @@ CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const
  * the same keep_blocks), Full and Reindex layers take the flat TOKEN indexer
  * over all entries, cand_blocks may be NULL and is not written, and the
  * workspace is sized by csa2_indexer_workspace_bytes(descs[0], TOKEN, ...).
+ * With the main KV (cache->codes, scales) in host memory, each Full or
+ * Reindex layer's set is followed by one kernel that copies its selected rows
+ * into a staged cache in the workspace, and every attention layer reads them
+ * there: the rows of a set cross the host link once, not once per layer.
+ * Results are bit-identical to a device-resident cache.
  * Every input must be complete in stream order before the call, as usual.
  * Kernels of the call after the first read the cache, the lengths, the SWA
  * rows other than the newest, a Reuse layer's index set and a Reindex layer's
