@@ -646,7 +646,7 @@ constexpr size_t K3_SMEM = K3_OFF_LAST + 16;
 // memory); otherwise blocks of 8 (one chunk per CTA, bitmaps in shared memory).
 template <bool kFlat>
 __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     int& s_last = *reinterpret_cast<int*>(smem + K3_OFF_LAST);
     pdl_wait();
     pdl_trigger();
@@ -1306,7 +1306,7 @@ constexpr size_t PS_SMEM = PS_OFF_VIS + PS_Q * 4;
 // Thread (qi, ei) of a 16 x 16 grid computes queries 2qi, 2qi+1 against entries
 // 4ei .. 4ei+3 of the tile: 32 sequential fp32 FMA chains.
 __global__ void __launch_bounds__(PS_THREADS) prefill_score_kernel(PrefillArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     float (*kt)[PS_E] = reinterpret_cast<float (*)[PS_E]>(smem);                                      // [d][entry]
     float (*qs)[PS_Q][kIH] = reinterpret_cast<float (*)[PS_Q][kIH]>(smem + (size_t)kID * PS_E * 4);  // [d][q][h]
     float (*ws_)[kIH] = reinterpret_cast<float (*)[kIH]>(smem + PS_OFF_W);
@@ -1446,7 +1446,7 @@ __device__ void prefill_select_one(const PrefillArgs& a, int t, uint8_t* smem) {
 // One query per loop trip (grid-stride: with flags the grid is a few CTAs per
 // SM and almost every trip ends at the flag).
 __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     pdl_wait();
     pdl_trigger();
     if (!a.flags) {
@@ -1779,7 +1779,7 @@ static_assert(PC_OFF_QD % 16 == 0 && PC_OFF_MISC % 16 == 0 && PC_OFF_HIST % 16 =
 static_assert((kMaxCand / 8) * 4 <= PC_OFF_QD - PC_OFF_L0, "K5b page-id staging");
 
 __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     uint16_t* k16 = reinterpret_cast<uint16_t*>(smem + PC_OFF_K16);
     uint32_t* ck = reinterpret_cast<uint32_t*>(smem + PC_OFF_CK);
     uint16_t* cand = reinterpret_cast<uint16_t*>(smem + PC_OFF_CAND);
