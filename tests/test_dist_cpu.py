@@ -50,3 +50,15 @@ def test_single_rank_passthrough():
     import bench
     assert bench.max_over_ranks(4.25, 1) == 4.25
     assert bench.whole_job_tokens_per_s(8, 1, 2.0) == pytest.approx(4000.0)
+
+
+def test_encoder_workload_and_bytes():
+    import bench
+    W = bench.workload(6)
+    assert (W["ratio"], W["decoder"], W["layers"], W["B"], W["L"]) == (2, False, 18, 8, 1 << 19)
+    ub = bench.unique_bytes_per_seq_flat(W["L"], W["layers"], 3, W["ratio"])
+    assert ub["index"] == 3 * (1 << 19) * 128  # every Full layer streams the whole indexer K
+    assert ub["kv"] == 3 * 512 * 144 and ub["swa"] == 18 * 128 * 512
+    assert ub["total"] == sum(v for k, v in ub.items() if k != "total")
+    dec = bench.workload(4)
+    assert (dec["ratio"], dec["decoder"], dec["layers"]) == (1, True, 20)

@@ -148,3 +148,31 @@ def test_short_contexts(orc):
         assert (sel[:m] >= 0).all() and (sel[m:] == -1).all()
         if L <= 512:
             assert sel[:m].tolist() == list(range(L))
+
+
+def test_flat_selection_is_the_prefill_selection_of_a_query_that_sees_everything(orc):
+    # The flat reading (no block level) selects exactly what the prefill
+    # indexer selects for a query at the last token: every entry is visible to it.
+    for ratio, L in [(2, 3000), (1, 777), (2, 513)]:
+        k = synth.idx_k_rows(1006, 3, 0, L)
+        qi, w = synth.q_idx(1006, 0, 3)[0], synth.w_idx(1006, 0, 3)[0]
+        flat = orc.select_tokens(k, L, None, qi, w)
+        assert orc.visible_entries(ratio * L - 1, ratio, L) == L
+        pre = orc.prefill_indexer(np.array([ratio * L - 1], np.int32), ratio, L, k, qi[None], w[None])[0]
+        np.testing.assert_array_equal(flat, pre)
+        # one token earlier at ratio 2 the last entry is not complete yet
+        if ratio == 2:
+            assert orc.visible_entries(ratio * L - 2, ratio, L) == L - 1
+
+
+def test_flat_selection_brute_force_small(orc):
+    # Top-512 of all L scores by (score desc, index asc), ascending: a Python sort
+    # of the oracle's per-row scores, with ties planted by duplicated rows.
+    rng = np.random.default_rng(9)
+    L = 1500
+    k = bf(rng.standard_normal((L, 64)))
+    k[700:760] = k[5]  # 61 equal scores
+    qi, w = bf(rng.standard_normal((4, 64))), rng.uniform(0, 1, 4).astype(np.float32)
+    s = orc.score_rows(qi, w, k)
+    order = sorted(range(L), key=lambda j: (-float(s[j]), j))[:512]
+    assert orc.select_tokens(k, L, None, qi, w).tolist() == sorted(order)
