@@ -38,20 +38,25 @@ csa2_status check_cache(const csa2_kv_cache* c, bool need_idx, bool need_pooled)
     return CSA2_OK;
 }
 
-// Whether p is host memory (pinned and mapped, as the cache requires); the
-// answer for the last pointer asked is kept, so repeated calls (and calls
+// Where p lives: 0 device (or managed) memory, 1 host memory mapped into the
+// device address space at p, -1 host memory the device cannot read in place.
+// The answer for the last pointer asked is kept, so repeated calls (and calls
 // under stream capture) do not query the driver again.
-bool in_host_memory(const void* p) {
+int memory_kind(const void* p) {
     static thread_local const void* last = nullptr;
-    static thread_local bool last_host = false;
-    if (p == last) return last_host;
+    static thread_local int last_kind = 0;
+    if (p == last) return last_kind;
     cudaPointerAttributes at{};
-    bool host = false;
-    if (cudaPointerGetAttributes(&at, p) == cudaSuccess) host = at.type == cudaMemoryTypeHost;
-    else (void)cudaGetLastError();
+    int kind = 0;
+    if (cudaPointerGetAttributes(&at, p) == cudaSuccess) {
+        if (at.type == cudaMemoryTypeHost) kind = at.devicePointer == p ? 1 : -1;
+        else if (at.type == cudaMemoryTypeUnregistered) kind = -1;
+    } else {
+        (void)cudaGetLastError();
+    }
     last = p;
-    last_host = host;
-    return host;
+    last_kind = kind;
+    return kind;
 }
 
 csa2_status from_cuda(cudaError_t e) {
@@ -260,7 +265,7 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
                                int32_t* cand_blocks, int32_t* idx_sets, float* const* out, float* const* lse,
                                int32_t B, int64_t max_len, void* workspace, size_t ws_bytes, int32_t* err_word,
                                void* stream) {
-    if (n_layers < 1 || !descs || !q_idx || !w || !q || !swa_kv || !out || !lse || !idx_sets)
+    if (n_layers < 1 || !descs || !cache || !q_idx || !w || !q || !swa_kv || !out || !lse || !idx_sets)
         return CSA2_ERR_INVALID_ARG;
     if (descs[0].mode != CSA2_MODE_FULL) return CSA2_ERR_INVALID_ARG;
     const bool flat = descs[0].keep_blocks == 0;  // every indexer layer selects over all entries
@@ -281,7 +286,9 @@ csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc* descs, c
     const int32_t* cur = nullptr;
     // A main KV in host memory: each new index set's rows are copied once into
     // the workspace's staged cache, and every attention layer reads them there.
-    const bool host_kv = in_host_memory(cache->codes);
+    const int kind = memory_kind(cache->codes);
+    if (kind < 0) return CSA2_ERR_INVALID_ARG;  // host memory the kernels cannot read in place
+    const bool host_kv = kind == 1;
     const DecodeWs wl = decode_ws_layout(B, max_len, flat);
     char* wsb = static_cast<char*>(workspace);
     StageArgs sa{};

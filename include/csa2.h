@@ -244,7 +244,9 @@ CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const
  * Reindex layer's set is followed by one kernel that copies its selected rows
  * into a staged cache in the workspace, and every attention layer reads them
  * there: the rows of a set cross the host link once, not once per layer.
- * Results are bit-identical to a device-resident cache.
+ * Results are bit-identical to a device-resident cache.  A main KV in host
+ * memory that the device cannot read in place (pageable, or mapped at another
+ * address) is rejected with INVALID_ARG before anything is launched.
  * Every input must be complete in stream order before the call, as usual.
  * Kernels of the call after the first read the cache, the lengths, the SWA
  * rows other than the newest, a Reuse layer's index set and a Reindex layer's

@@ -149,6 +149,8 @@ def test_flat_indexer_arguments(csa2):
     ptrs = (ctypes.c_void_p * 2)(0x1000, 0x1000)
     assert L.csa2_decode_layers(2, descs, ctypes.byref(c), ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
                                 P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 16, None, None) == 4
+    assert L.csa2_decode_layers(2, descs, None, ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
+                                P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 1 << 30, None, None) == 1  # no cache
     hdesc = (csa2.LayerDesc * 2)(csa2.default_desc(csa2.FULL, 1), csa2.default_desc(csa2.REUSE, 1))
     assert L.csa2_decode_layers(2, hdesc, ctypes.byref(c), ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
                                 P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 1 << 30, None, None) == 1
