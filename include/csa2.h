@@ -291,7 +291,8 @@ CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc* desc, cons
 CSA2_API const char* csa2_status_string(csa2_status s);
 CSA2_API int32_t csa2_abi_version(void);
 
-/* 1 if kernels on the current device may dereference p at that same address:
+/* A helper with no counterpart on the pages, for the tiered main KV.
+ * 1 if kernels on the current device may dereference p at that same address:
  * device or managed memory, or host memory allocated or registered with CUDA
  * and mapped at p.  0 for pageable host memory or another device's memory, -1
  * if CUDA reports an error.  The library does not call it on its own paths. */
