@@ -1,5 +1,6 @@
-"""The five benchmark configurations at full size, in the launch configuration
-bench.py times (decode: quant-append + the 20-layer schedule driver), checked
+"""The benchmark configurations at full size (five of the decoder and prefill,
+and the encoder side of a decode step), in the launch configuration bench.py
+times (decode: quant-append + the schedule driver), checked
 against the oracle: every sequence where the oracle can afford it, sampled
 sequences or queries otherwise (the rest of the batch is filled with seeded
 device-side data of the same distribution, so the GPU still runs the full
