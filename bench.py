@@ -15,7 +15,9 @@ max over ranks.
 
 --config 3 times a prefill chunk instead; --config 6 the encoder side of one
 generated token: 18 ratio-2 layers (3 x (Full + 5 Reuse)) whose Full layers
-select over every entry (8 x 524,288 entries = 1M tokens each).
+select over every entry (8 x 524,288 entries = 1M tokens each).  --kv-host keeps
+the main KV in pinned host memory (the decode driver stages each index set's
+rows on the device once).
 
 --impl reference times the CPU oracle (the plain C restatement of the method)
 on the host cores on a bounded sample of the same workload.
