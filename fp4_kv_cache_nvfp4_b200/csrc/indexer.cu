@@ -974,14 +974,15 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
 // K4: token scores over the candidates + Top-K, one 8-CTA cluster per sequence
 //
 // CTA r of a sequence's cluster scores candidate slots [2048 r, 2048 r + 2048):
-// the indexer-K rows of its 256 candidate blocks (one 1 KiB box each) arrive by
-// 2-D bulk tensor copies into a 2-stage ring; every thread scores one row per
-// round.  The radix select then runs across the cluster: each CTA histograms
-// its own keys, CTA r sums slice r of the histogram over the 8 CTAs through
-// distributed shared memory, every CTA locates the slice and bin holding the
-// K-th key, and the next digit repeats this on the survivors only.  The
-// ordered emission exchanges per-CTA counts the same way, so every CTA writes
-// its selected positions at its own offset, ascending.
+// each warp copies the indexer-K rows of its candidate blocks (a block's 8 rows
+// are one 1 KiB run) with 16-byte cp.async into its own slice of a 2-stage
+// ring, and every thread scores one row per round.  The radix select then runs
+// across the cluster: each CTA adds its digit histogram into every CTA's
+// receive buffer (red.shared::cluster), one cluster barrier follows, every CTA
+// locates the bin holding the K-th key, and the next digit repeats this on the
+// survivors only; a bin whose keys are all taken ends the search.  The ordered
+// emission exchanges per-CTA counts the same way, so every CTA writes its
+// selected positions at its own offset, ascending.
 // ============================================================================
 constexpr int TK_CL = 8;
 constexpr int TK_THREADS = 512;
