@@ -18,19 +18,24 @@
 // emission (ballots in slot order) that keeps ties at the lowest index.
 //
 // Kernels
-//   block_score_kernel  (K2)  stream the pooled indexer K of every block,
-//                              write fp32 scores and a per-sequence histogram
-//                              of the first digit; the last CTA of a sequence
-//                              finds the bin holding the keep-th score.
-//                              HBM-bound: 128 B per block.
-//   block_select_kernel (K3)  mark blocks above that bin in a bitmap and
+//   block_score_kernel  (K2)  stream the pooled indexer K of every block (or,
+//                              for a flat selection, the indexer K of every
+//                              entry), write fp32 scores and a per-sequence
+//                              histogram of the first digit; the last CTA of a
+//                              sequence finds the bin holding the keep-th
+//                              score.  HBM-bound: 128 B per row.
+//   block_select_kernel (K3)  mark rows above that bin in a bitmap and
 //                              collect the bin's members; the last CTA refines
-//                              the boundary and emits the kept blocks in order.
-//   token_topk_kernel   (K4)  score the <= 16,384 candidates (1 KiB runs of 8
-//                              indexer-K rows) and histogram them; the last CTA
-//                              of a sequence refines and emits the Top-K.
-//   prefill_score_kernel / prefill_select_kernel: the same per query over the
-//                              entries visible to it.
+//                              the boundary and emits the kept rows in order
+//                              (a flat selection lists and sorts them).
+//   token_topk_kernel   (K4)  one 8-CTA cluster per sequence scores the
+//                              <= 16,384 candidates (1 KiB runs of 8 indexer-K
+//                              rows) and selects the Top-K across the cluster.
+//   prefill_tc_score_kernel / prefill_candidates_kernel: prefill, approximate
+//                              scores on tcgen05, exact rescoring of the
+//                              candidates and a verified exact Top-K per query;
+//   prefill_score_kernel / prefill_select_kernel: the exact fallback for the
+//                              queries that fail the verification.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -329,7 +334,8 @@ __device__ __forceinline__ void stage_pages(const csa2_kv_cache& c, int shift, i
 // through an mbarrier once their copies land; eight consumer warps only score
 // (lane l takes rows l and l + 32 of its warp's 64: eight independent FMA
 // chains) and release the stage through a second mbarrier.  Copies and FMAs
-// therefore overlap instead of taking turns.
+// therefore overlap instead of taking turns.  Entry rows in pages of >= 64
+// entries arrive instead as 64-row tensor boxes (one 8 KiB run each).
 // ============================================================================
 constexpr int K2_CWARPS = 8;                    // consumer (scoring) warps
 constexpr int K2_PWARPS = 4;                    // producer (copy) warps
