@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     p.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 6])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-prefill", action="store_true", help="skip the prefill chunk timed beside the decode step")
+    p.add_argument("--launch-floor", action="store_true",
+                   help="time chains of empty dependent kernels in one CUDA graph (the launch floor)")
     p.add_argument("--kernel-reps", type=int, default=300)
     p.add_argument("--contiguous-pages", action="store_true")
     p.add_argument("--batch", type=int, default=0, help="override the batch (profiling runs)")
@@ -591,6 +594,7 @@ def run_prefill(args, rank: int, world: int, local_rank: int):
                             layers=layers, l2="flushed before every timed step"),
                 breakdown_us=part_us,
                 tensor=dict(attention_tflops=att_flop / (att_us * 1e-6) / 1e12, attention_flop_per_layer=att_flop,
+                            chunk_flop=idx_flop + layers * att_flop,
                             indexer_gflop=idx_flop / 1e9,
                             indexer_tflops=idx_flop / (part_us["indexer"] * 1e-6) / 1e12,
                             peak_bf16_tflops=peaks.get("bf16_tflops")),
@@ -609,40 +613,186 @@ def _peaks() -> dict:
 # CPU oracle (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(cfg_id: int, budget_s: float = 15.0, max_steps: int = 1000):
-    """Time the oracle's decode step on the host cores: the same 20-layer step
-    on sequences of the workload's length, one OpenMP thread per sequence."""
-    import oracle
+def cpu_model() -> str:
+    """The host CPU's model name (lscpu's "Model name")."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_cache(orc, seed: int, L: int, ratio: int):
+    """One sequence's cache built by the oracle from the seeded generators."""
     import synth
-    W = workload(cfg_id)
-    L, layers, seed, ratio, flat = W["L"], W["layers"], W["seed"], W["ratio"], not W["decoder"]
-    n_seq = min(W["B"], os.cpu_count() or 1)
-    # one sequence's cache, built by the oracle itself (not timed), shared by the sampled sequences
     codes = np.empty((L, 128), np.uint8)
     scales = np.empty((L, 16), np.uint8)
     for e0 in range(0, L, 1 << 16):
         m = min(1 << 16, L - e0)
-        codes[e0:e0 + m], scales[e0:e0 + m] = oracle.quant_rows(synth.kv_rows(seed, 0, e0 * ratio, m * ratio),
-                                                                ratio=ratio)
-    idx = synth.idx_k_rows(seed, 0, 0, L)
-    pooled = oracle.pool_blocks(idx)
-    modes = oracle.schedule(not flat)[:layers]
+        codes[e0:e0 + m], scales[e0:e0 + m] = orc.quant_rows(synth.kv_rows(seed, 0, e0 * ratio, m * ratio),
+                                                             ratio=ratio)
+    return codes, scales, synth.idx_k_rows(seed, 0, 0, L)
+
+
+def _layer_inputs(seed: int, layers: int, n_seq: int):
+    import synth
     q_idx = np.stack([np.concatenate([synth.q_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
     w = np.stack([np.concatenate([synth.w_idx(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
     q = np.stack([np.concatenate([synth.q_heads(seed, l, b) for l in range(layers)]) for b in range(n_seq)])
     swa = np.stack([np.stack([synth.swa_rows(seed, l, b, 128) for l in range(layers)]) for b in range(n_seq)])
+    return q_idx, w, q, swa
+
+
+def oracle_sample(cfg_id: int, budget_s: float = 15.0, max_steps: int = 1000, max_threads: int = 32):
+    """Time the oracle's decode step on the host cores: the same step on
+    sequences of the workload's length, one sequence per host thread (OpenMP),
+    each with a cache of its own."""
+    import oracle
+    W = workload(cfg_id)
+    L, layers, seed, ratio, flat = W["L"], W["layers"], W["seed"], W["ratio"], not W["decoder"]
+    n_seq = max(1, min(os.cpu_count() or 1, max_threads))
+    # Sequence 0's cache comes from the seeded generators; sequence b's is that
+    # cache rotated by b * L / n_seq entries (a multiple of 8, so blocks stay
+    # whole), so no two sampled sequences share an entry at any position.
+    codes0, scales0, idx0 = _oracle_cache(oracle, seed, L, ratio)
+    caches = []
+    for b in range(n_seq):
+        sh = (b * (L // max(n_seq, 1))) // 8 * 8
+        c, s_, k = (np.roll(a, sh, axis=0) for a in (codes0, scales0, idx0))
+        caches.append((c, s_, k, oracle.pool_blocks(k)))
+    del codes0, scales0, idx0
+    modes = oracle.schedule(not flat)[:layers]
+    q_idx, w, q, swa = _layer_inputs(seed, layers, n_seq)
     steps, t0 = 0, time.perf_counter()
     while steps < max_steps:
-        oracle.decode_batch(modes, [L] * n_seq, [codes] * n_seq, [scales] * n_seq, [idx] * n_seq,
-                            [pooled] * n_seq, q_idx, w, q, swa, keep=0 if flat else 2048)
+        oracle.decode_batch(modes, [L] * n_seq, [c[0] for c in caches], [c[1] for c in caches],
+                            [c[2] for c in caches], [c[3] for c in caches], q_idx, w, q, swa,
+                            keep=0 if flat else 2048)
         steps += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return dict(value=steps * n_seq / dt, unit=UNIT, cores=n_seq, kind="oracle",
+    return dict(value=steps * n_seq / dt, unit=UNIT, cores=n_seq, kind="oracle", cpu_model=cpu_model(),
+                host_threads=os.cpu_count(),
                 sample=f"{steps} decode step(s) x {n_seq} sequences of the {W['workload']} workload "
-                       f"({layers} layers, L={L}); the quant-append of the step is not in the sample; "
-                       f"{dt:.1f} s on {n_seq} of {os.cpu_count()} host threads (one per sequence)")
+                       f"({layers} layers, L={L}, a distinct cache per sequence); the quant-append of the step "
+                       f"is not in the sample; {dt:.1f} s on {n_seq} of {os.cpu_count()} host threads "
+                       f"(one OpenMP thread per sequence)")
+
+
+def oracle_single_core(cfg_id: int, budget_s: float = 3.0) -> dict:
+    """The oracle's decode step of one sequence on one core (no OpenMP)."""
+    import oracle
+    W = workload(cfg_id)
+    L, layers, seed, ratio = W["L"], W["layers"], W["seed"], W["ratio"]
+    codes, scales, idx = _oracle_cache(oracle, seed, L, ratio)
+    pooled = oracle.pool_blocks(idx)
+    modes = oracle.schedule(True)[:layers]
+    q_idx, w, q, swa = (a[0] for a in _layer_inputs(seed, layers, 1))
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(modes, L, codes, scales, idx, pooled, q_idx, w, q, swa)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return dict(value=steps / dt, unit=UNIT, cores=1, kind="oracle", ms_per_step=dt / steps * 1e3,
+                sample=f"{steps} decode step(s) of one sequence of the {W['workload']} workload ({layers} "
+                       f"layer(s), L={L}) on one core")
+
+
+def oracle_prefill_sample(budget_s: float = 8.0) -> dict:
+    """The oracle's prefill (indexer + 6 attention layers) on the host cores,
+    timed on a sample of the chunk's queries spread over its positions."""
+    import oracle
+    import synth
+    c = synth.CONFIGS[3]
+    tokens, T, layers, seed = c["tokens"], c["T"], c["layers"], c["seed"]
+    n_ent = tokens // 2
+    codes, scales, idx = _oracle_cache(oracle, seed, n_ent, 2)
+    swa_start = tokens - T - 127
+    swas = [synth.swa_rows(seed, l, 0, tokens - swa_start) for l in range(layers)]
+    done, t0, rounds = 0, time.perf_counter(), 0
+    per = 64
+    while True:
+        lo = (rounds * 997) % (T - per)  # a different slice of the chunk each round
+        q_pos = np.arange(tokens - T + lo, tokens - T + lo + per, dtype=np.int32)
+        q_idx = synth.q_idx(seed, 0, rounds, per)
+        w = synth.w_idx(seed, 0, rounds, per)
+        sets = oracle.prefill_indexer(q_pos, 2, n_ent, idx, q_idx, w)
+        for l in range(layers):
+            oracle.prefill_attn(q_pos, synth.q_heads(seed, l, rounds, per), sets, codes, scales, swas[l], swa_start)
+        done += per
+        rounds += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    n_thr = min(os.cpu_count() or 1, per)
+    return dict(value=done / dt, unit="tokens/s", cores=n_thr, kind="oracle", cpu_model=cpu_model(),
+                sample=f"{done} query tokens of the {c['name']} chunk ({rounds} slices of {per}); indexer over "
+                       f"the visible entries plus {layers} attention layers each; {dt:.1f} s on {n_thr} of "
+                       f"{os.cpu_count()} host threads (OpenMP over the slice's queries)")
+
+
+def W_DECODER(cfg_id: int) -> bool:
+    return bool(workload(cfg_id)["decoder"])
+
+
+def prefill_summary(p: dict) -> dict:
+    """The prefill run's line, condensed into the decode line's "prefill" object."""
+    peaks = _peaks()
+    sus = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    flop = p["tensor"]["chunk_flop"]
+    ach = flop / (p["ms_per_step"] * 1e-3) / 1e12
+    return dict(metric=p["metric"], value=p["value"], unit=p["unit"], ms_per_chunk=p["ms_per_step"],
+                steps=p["steps"], config=p["config"], breakdown_us=p["breakdown_us"],
+                tensor=dict(p["tensor"], chunk_tflops=ach, peak_tflops=sus,
+                            peak_source="MEASURED_PEAKS.json bf16_tflops_sustained (cuBLAS bf16, seconds-long loop)"
+                            if peaks.get("bf16_tflops_sustained") else "bf16 burst peak",
+                            frac_of_peak=ach / sus if sus else None),
+                clocks=p["clocks"])
+
+
+def run_launch_floor(args, local_rank: int) -> dict:
+    """Floor that kernel boundaries alone put under a step: chains of empty
+    kernels with programmatic dependent launch, each chain captured in one CUDA
+    graph and replayed, timed with CUDA events on the launching stream."""
+    import torch
+    import fp4_kv_cache_nvfp4_b200 as csa2
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+    for n, ctas in ((28, 64), (28, 148), (28, 296), (20, 148), (1, 148)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            csa2.test_empty_chain(n, ctas, 160, sink, stream=stream)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            csa2.test_empty_chain(n, ctas, 160, sink, stream=stream)
+        reps = max(args.steps, 50)
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                g.replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for k in range(reps):
+                ev[k][0].record(stream)
+                g.replay()
+                ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        us = [a.elapsed_time(b) * 1e3 for a, b in ev]
+        out[f"{n}x{ctas}"] = dict(kernels=n, ctas=ctas, us_per_graph=statistics.median(us),
+                                  us_per_kernel=statistics.median(us) / n, reps=reps)
+        del g
+    return dict(metric="launch-chain floor: empty dependent kernels (programmatic dependent launch) in one CUDA "
+                       "graph", unit="us", chains=out)
 
 
 def run_reference(args, rank: int, world: int):
@@ -685,9 +835,22 @@ def main():
         if rank == 0:
             print(json.dumps(res), flush=True)
         return
+    if args.launch_floor:
+        res = run_launch_floor(args, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res = run_cuda(args, rank, world, local_rank)
+    if args.config == 4 and not args.no_prefill:
+        # the prefill chunk (configuration 3) timed in the same process: the
+        # north star asks for decode and prefill tokens/s side by side
+        res["prefill"] = prefill_summary(run_prefill(args, rank, world, local_rank))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = oracle_sample(args.config, budget_s=15.0)
+        if W_DECODER(args.config):
+            res["cpu_baseline"]["single_core"] = {f"config{c}": oracle_single_core(c) for c in (1, 2)}
+        if "prefill" in res:
+            res["prefill"]["cpu_baseline"] = oracle_prefill_sample()
     if world > 1:
         import torch
         torch.distributed.barrier()

@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
             L.csa2_abi_version.restype = _I32
             L.csa2_device_accessible.argtypes = [_P]
             L.csa2_device_accessible.restype = _I32
+            L.csa2_test_empty_chain.argtypes = [_I32, _I32, _I32, _P, _P]
+            L.csa2_test_empty_chain.restype = _I32
+            L.csa2_test_set_wait_limit.argtypes = [ctypes.c_uint32]
+            L.csa2_test_set_wait_limit.restype = ctypes.c_uint32
             _lib = L
     return _lib
 
@@ -105,6 +109,18 @@ def abi_version() -> int:
 def device_accessible(t) -> int:
     """1 if kernels can read the tensor (or raw address) in place, 0 if not, -1 on a CUDA error."""
     return int(lib().csa2_device_accessible(_ptr(t)))
+
+
+def test_set_wait_limit(polls: int) -> int:
+    """Test hook: poll limit of the block-level indexer's cp.async copy-ring
+    waits (returns the previous limit)."""
+    return int(lib().csa2_test_set_wait_limit(polls))
+
+
+def test_empty_chain(n_kernels: int, ctas: int, threads: int = 128, sink=None, stream=None) -> None:
+    """Measurement helper: n_kernels empty dependent kernels (programmatic
+    dependent launch) on the stream."""
+    _check(lib().csa2_test_empty_chain(n_kernels, ctas, threads, _ptr(sink), _stream(stream)), "test_empty_chain")
 
 
 def default_desc(mode: int = FULL, ratio: int = 1, **over) -> LayerDesc:

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     // the grid, so no CTA waits on one that left.
     if (smem_u32(smem) & 15u) {
         pdl_wait();
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     const bool pre_idx = (a.pre & kPreIdx) != 0, pre_hist = (a.pre & kPreHist) != 0;
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(PA_THREADS, 3) prefill_attn_kernel(AttnArgs a)
     pdl_wait();
     pdl_trigger();
     if (smem_u32(smem) & 15u) {  // uniform over the grid
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     const int32_t L = a.seq_len_prefill;
@@ -757,7 +757,7 @@ __global__ void __launch_bounds__(PW_THREADS, 1) prefill_swa_kernel(AttnArgs a) 
     pdl_wait();
     pdl_trigger();
     if (smem_u32(smem) & 15u) {  // uniform over the grid
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     // window [lo, p] of each query (empty: lo > p)

@@ -40,6 +40,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -356,6 +357,9 @@ constexpr size_t K2_OFF_BAR = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // full[3
 constexpr size_t K2_OFF_MISC = align16(K2_OFF_BAR + 2 * K2_STAGES * 8);  // w (float4), last, timeout
 constexpr size_t K2_SMEM = align16(K2_OFF_MISC + 32);
 constexpr uint32_t kWaitLimit = 1u << 22;
+// Poll limit of the block-scoring copy ring's waits (cp.async rows only): the
+// default above, lowered only by csa2_test_set_wait_limit.
+static std::atomic<uint32_t> g_copy_wait_limit{kWaitLimit};
 static_assert(K2_OFF_QD % 16 == 0 && K2_OFF_BAR % 8 == 0 && K2_OFF_MISC % 16 == 0, "K2 shared-memory layout");
 
 struct BlockArgs {
@@ -382,6 +386,7 @@ struct BlockArgs {
     int rshift;        // log2 entries per scored row
     int span;          // rows filtered per select CTA (a multiple of 8192)
     int tma;           // 1: rows arrive as 64-row tensor boxes (entry rows, pages of >= 64 entries)
+    uint32_t wait_limit;  // polls before a wait of the copy ring gives up (cp.async rows)
 };
 
 // tile_start[b] = first tile of sequence b; returns the sequence of tile t
@@ -415,7 +420,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid
     // 16-byte copies and vector reads need an aligned base; 128-byte-swizzled
     // tensor boxes a 1 KiB aligned one (uniform over the grid)
     if (smem_u32(smem) & (a.tma ? 1023u : 15u)) {
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     // ---- tiles of every sequence (0 for sequences that keep all blocks) ------
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid
         fetch(t0);
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % K2_STAGES;
-            if (i >= K2_STAGES && !mbar_wait(&empty[s], (uint32_t)((i / K2_STAGES) - 1) & 1u, kWaitLimit))
+            if (i >= K2_STAGES && !mbar_wait(&empty[s], (uint32_t)((i / K2_STAGES) - 1) & 1u, a.wait_limit))
                 s_timeout = 1;
             int32_t prow[4];
 #pragma unroll
@@ -615,7 +620,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid
             nloc = 0;
             cg.sync();
         }
-        if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, kWaitLimit)) s_timeout = 1;
+        if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, a.wait_limit)) s_timeout = 1;
         const uint8_t* stage = smem + (size_t)s * K2_STAGE_BYTES;
         const int r0 = K2_CROWS * wid + lane;  // rows r0 and r0 + 32 of the tile
         uint32_t k[32], m[32];
@@ -657,7 +662,7 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     pdl_wait();
     pdl_trigger();
     if (smem_u32(smem) & 15u) {  // uniform over the grid
-        if (threadIdx.x == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (threadIdx.x == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     const int b = blockIdx.y;
@@ -1079,7 +1084,7 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
     // uniform over the grid, so no CTA waits at a cluster barrier for one that left
     if (smem_u32(smem) & 15u) {
         if (pre) pdl_wait();
-        if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
@@ -1573,7 +1578,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     pdl_wait();
     pdl_trigger();
     if (smem_u32(smem) & 1023u) {  // the swizzled operand tiles need a 1 KiB-aligned base (uniform)
-        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
     // entry range of this CTA: the split, cut at the largest visibility of its queries
@@ -2098,6 +2103,11 @@ cudaError_t launch_block_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     CUtensorMap map;
     memset(&map, 0, sizeof(map));
     a.tma = flat && cache.page_size >= 64 && entry_row_map(cache, &map) ? 1 : 0;
+    // A tensor-box ring keeps the fixed limit: a wait that gave up there could
+    // leave bulk copies in flight into the CTA's shared memory when it exits.
+    // The cp.async ring's producers drain their own copies before they leave,
+    // so its limit may be lowered (csa2_test_set_wait_limit).
+    a.wait_limit = a.tma ? kWaitLimit : g_copy_wait_limit.load(std::memory_order_relaxed);
     if (nblk > keep) {
         const int64_t tiles = (int64_t)n * ((nblk + K2_TILE - 1) / K2_TILE);
         const int grid = (int)std::min<int64_t>(tiles, sm_count());
@@ -2187,3 +2197,8 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
 }
 
 }  // namespace csa2
+
+extern "C" CSA2_API uint32_t csa2_test_set_wait_limit(uint32_t polls) {
+    if (polls > csa2::kWaitLimit) polls = csa2::kWaitLimit;
+    return csa2::g_copy_wait_limit.exchange(polls);
+}

@@ -1,13 +1,14 @@
 // Allocation-free variant of the decode indexer (csa2_indexer_topk_noalloc).
 //
 // Some callers cannot allocate device memory at the point where they run the
-// indexer: code that is being captured into a CUDA graph (cudaMalloc is not
-// allowed while a stream is capturing), plug-ins whose host framework owns all
-// device memory and hands them only the tensors they work on, and latency-
-// critical serving loops that must not take the allocator's locks or
-// synchronise.  For them this entry point keeps its scratch in a fixed array
-// inside the library's own device memory instead of a caller workspace.
+// indexer: plug-ins whose host framework owns all device memory and hands them
+// only the tensors they work on, and latency-critical serving loops that must
+// not call cudaMalloc (it can synchronise the device and takes the driver's
+// allocation locks).  For them this entry point keeps its scratch in a fixed
+// array inside the library's own device memory instead of a caller workspace.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -23,19 +24,22 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // Device address of the scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
 // per device with that device current.
+// Host threads making their first call on one device at the same time both
+// look the address up and store the same value; the slots are atomic, so
+// that is not a data race.
 static cudaError_t noalloc_scratch(void** out) {
-    static void* addr[64];
+    static std::atomic<void*> addr[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!addr[dev]) {
-        void* p = nullptr;
+    void* p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
-    *out = addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -63,13 +67,20 @@ extern "C" CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc*
         (void)cudaGetLastError();
         return CSA2_ERR_CUDA;
     }
-    // The kernels expect their counters and histograms at zero.  The previous
-    // call may have used another (n, max_len) and so another layout: clear the
-    // zero-state head of this call's layout first (a memset, no allocation).
-    const DecodeWs l = decode_ws_layout(n, max_len, desc->keep_blocks == 0);
-    if (cudaMemsetAsync(scratch, 0, l.blk_thr, (cudaStream_t)stream) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return CSA2_ERR_CUDA;
+    // The block-level and flat-row kernels expect their counters and
+    // histograms at zero.  The previous call may have used another (n, max_len)
+    // and so another layout: clear the zero-state head of this call's layout
+    // first (a memset, no allocation).  The token-level kernel (a hierarchical
+    // Reindex/Full token call, or a flat call over at most 16,384 entries)
+    // keeps all its state on chip and reads no scratch, so it needs no clear.
+    const bool flat = desc->keep_blocks == 0;
+    const bool uses_scratch = level == CSA2_LEVEL_BLOCK || (flat && max_len > kMaxCand);
+    if (uses_scratch) {
+        const DecodeWs l = decode_ws_layout(n, max_len, flat);
+        if (cudaMemsetAsync(scratch, 0, l.blk_thr, (cudaStream_t)stream) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return CSA2_ERR_CUDA;
+        }
     }
     return csa2_indexer_topk(desc, cache, level, q_idx, w, seq_lens, nullptr, cand_blocks, idx_out, nullptr, n,
                              max_len, scratch, kNoAllocScratchBytes, err_word, stream);

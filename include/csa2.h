@@ -69,6 +69,8 @@ typedef enum {
 #define CSA2_DEV_INDEX 0x4  /* a Top-K index >= the sequence length */
 #define CSA2_DEV_LEN 0x8    /* a sequence length outside [1, capacity] */
 #define CSA2_DEV_TIMEOUT 0x10 /* a bounded wait for an asynchronous copy gave up */
+#define CSA2_DEV_ALIGN 0x20   /* a kernel's dynamic shared memory was not aligned as its
+                               * layout needs; the kernel returned without computing */
 
 typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
 typedef enum { CSA2_LEVEL_BLOCK = 0, CSA2_LEVEL_TOKEN = 1 } csa2_level;
@@ -264,23 +266,32 @@ CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc*
 /* ---------------------------------------------------------------------- */
 /* Allocation-free decode indexer.  The pages have no counterpart to this call:
  * it is an integration convenience for callers that cannot allocate device
- * memory where they run the indexer -- code being captured into a CUDA graph
- * (cudaMalloc is not allowed while a stream captures), plug-ins whose host
- * framework owns all device memory, serving loops that must not take the
- * allocator's locks.  It does exactly what csa2_indexer_topk does for decode
- * (q_pos = NULL, either level), but keeps its scratch in a 16 MiB array of
- * static device memory inside the library instead of a caller workspace.
+ * memory where they run the indexer -- plug-ins whose host framework owns all
+ * device memory and hands them only the tensors they work on, and serving
+ * loops that must not call cudaMalloc (it may synchronise the device and takes
+ * the driver's allocation locks).  It does exactly what csa2_indexer_topk does
+ * for decode (q_pos = NULL, either level), but keeps its scratch in a 16 MiB
+ * array of static device memory inside the library instead of a caller
+ * workspace.
  *   - allocates nothing (no cudaMalloc/cudaFree); every GPU that loads the
  *     library holds the 16 MiB until the process exits;
  *   - a call whose workspace layout (csa2_indexer_workspace_bytes for the same
- *     desc, level, n and max_len) exceeds 16 MiB returns CSA2_ERR_WORKSPACE
- *     (n = 8 sequences of 2^20 entries need about 13.5 MiB);
- *   - the first call on a device looks up the array's device address (a
- *     runtime call); make that first call before any stream capture;
- *   - every call clears the counters it needs (a memset on `stream`) and
- *     otherwise reuses the array as the previous call left it; all calls
- *     share one array per device, so calls that overlap on the GPU (other
- *     streams, other threads) race and must be serialised by the caller. */
+ *     desc, level, n and max_len) exceeds 16 MiB returns CSA2_ERR_WORKSPACE.
+ *     The limit depends on the mode: the hierarchical indexer (keep_blocks >
+ *     0) scores one row per block of 8, so n = 8 sequences of 2^20 entries fit
+ *     (about 13.5 MiB); the flat indexer (keep_blocks = 0) above 16,384
+ *     entries scores one row per entry, so n * max_len may reach only about
+ *     1.3 * 2^20 entries (one sequence of 2^20 needs about 12.4 MiB, two need
+ *     about 24.8 MiB);
+ *   - the first call on a device looks up the array's device address, and the
+ *     first call of each level and mode runs the kernels' one-time set-up
+ *     (shared-memory attributes, and for flat rows the tensor-map entry
+ *     point); make those first calls before any stream capture;
+ *   - block-level and flat-row calls clear the counters they need (a memset on
+ *     `stream`); token-level calls read no scratch.  Otherwise the array keeps
+ *     what the previous call left; all calls share one array per device, so
+ *     calls that overlap on the GPU (other streams, other threads) race and
+ *     must be serialised by the caller. */
 CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc* desc, const csa2_kv_cache* cache,
                                                int32_t level, const uint16_t* q_idx, const float* w,
                                                const int32_t* seq_lens, const int32_t* cand_blocks,
@@ -288,6 +299,25 @@ CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc* desc, cons
                                                void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Test hook with no counterpart on the pages: the poll limit of the bounded
+ * waits in the block-level indexer's cp.async copy ring (the hierarchical
+ * indexer's pooled rows), which otherwise give up after 2^22 polls.  A wait
+ * that gives up sets CSA2_DEV_TIMEOUT in err_word; the kernel still drains its
+ * own copies, reaches every barrier and returns, and that call's results are
+ * undefined.  Lowering the limit (0 = every wait gives up at once) lets a test
+ * drive that path; polls above 2^22 are clamped.  Process-wide, read when a
+ * call is launched; returns the previous limit.  Not for production use. */
+CSA2_API uint32_t csa2_test_set_wait_limit(uint32_t polls);
+
+/* Measurement helper with no counterpart on the pages: launches n_kernels
+ * empty kernels of `ctas` CTAs x `threads` threads on `stream`, each waiting on
+ * its predecessor with programmatic dependent launch exactly as the decode
+ * step's kernels do (the first CTA of each adds 1 to *sink, if non-NULL, a
+ * device int32).  Captured in a CUDA graph it gives the floor that kernel
+ * boundaries alone put under a step of that many kernels. */
+CSA2_API csa2_status csa2_test_empty_chain(int32_t n_kernels, int32_t ctas, int32_t threads, int32_t* sink,
+                                           void* stream);
+
 CSA2_API const char* csa2_status_string(csa2_status s);
 CSA2_API int32_t csa2_abi_version(void);
 

@@ -154,3 +154,17 @@ def test_flat_indexer_arguments(csa2):
     hdesc = (csa2.LayerDesc * 2)(csa2.default_desc(csa2.FULL, 1), csa2.default_desc(csa2.REUSE, 1))
     assert L.csa2_decode_layers(2, hdesc, ctypes.byref(c), ptrs, ptrs, ptrs, ptrs, P(0x1000), None, None,
                                 P(0x1000), ptrs, ptrs, 1, 1000, P(ws), 1 << 30, None, None) == 1
+
+
+def test_noalloc_scratch_limits_per_mode(csa2):
+    """The allocation-free indexer's 16 MiB scratch holds the hierarchical
+    layout of 8 sequences of 2^20 entries, the flat layout of one such
+    sequence, but not the flat layout of two (flat rows are entries, not
+    blocks of 8)."""
+    lim = 16 << 20
+    hier = csa2.default_desc(csa2.FULL, 1)
+    flat = csa2.default_desc(csa2.FULL, 2, keep_blocks=0)
+    assert csa2.workspace_bytes(hier, csa2.BLOCK, 8, 1 << 20) <= lim
+    assert csa2.workspace_bytes(flat, csa2.TOKEN, 1, 1 << 20) <= lim
+    assert csa2.workspace_bytes(flat, csa2.TOKEN, 2, 1 << 20) > lim
+    assert csa2.workspace_bytes(hier, csa2.BLOCK, 64, 1 << 20) > lim

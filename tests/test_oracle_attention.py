@@ -217,14 +217,59 @@ def test_prefill_window_and_visibility(orc):
 
 
 def test_cache_accounting(orc):
-    with open(os.path.join(GOLD, "pages_facts.json")) as f:
-        facts = json.load(f)
     # Full layers carry the cache: 3 encoder Full layers at ratio 2, 1 decoder Full at ratio 1
     ratios = [2, 2, 2, 1]
     main = 256 * 0.5 + 16  # FP4 codes + one E4M3 byte per 16 channels
     ours = orc.cache_bytes_per_token(ratios, main, 64 * 2)
-    assert ours == 680.0
-    # consistency report against the pages' 890 B/token: same structure, other dims
-    assert abs(orc.cache_bytes_per_token(ratios, 512 * 0.5 + 32, 64 + 4) - facts["kv_bytes_per_token"]["value"]) < 1
+    # closed form with these dimensions: 3 x (144 + 128) / 2 + (144 + 128)
+    assert ours == 3 * (144 + 128) / 2 + (144 + 128) == 680.0
+    # one Full layer at ratio 1 alone is one entry per token
+    assert orc.cache_bytes_per_token([1], main, 128) == 272.0
     # FP4 + E4M3/16 is 4.5 bits per channel: a bit over half of 8-bit storage
     assert main / 256 * 8 == 4.5
+    # consistency report (not an assertion): the pages' 890 B/token over the
+    # same 2.5 Full entries per token is 356 B per entry, against our 272
+    with open(os.path.join(GOLD, "pages_facts.json")) as f:
+        facts = json.load(f)
+    pages = facts["kv_bytes_per_token"]["value"]
+    print(f"cache bytes/token: ours {ours:.0f} with 256-ch FP4 main + 64-d bf16 indexer K; pages {pages} "
+          f"(= {pages / 2.5:.0f} B per Full entry at 2.5 entries/token)")
+
+
+def _batch_case(keep, lens, modes, seed):
+    """Per-sequence caches and per-layer inputs for decode_batch / decode_step."""
+    n = len(modes)
+    caches, q_idx, w, q, swa = [], [], [], [], []
+    for b, L in enumerate(lens):
+        codes, scales, k, pooled, qi, wi, qh, sw = _decode_inputs(int(L), n_layers=n, seed=seed, seq=b)
+        caches.append((codes, scales, k, pooled))
+        q_idx.append(qi)
+        w.append(wi)
+        q.append(qh)
+        swa.append(sw)
+    return caches, np.stack(q_idx), np.stack(w), np.stack(q), np.stack(swa)
+
+
+def test_decode_batch_equals_per_sequence_steps(orc):
+    # decode_batch (the CPU baseline's entry point) runs decode_step on every
+    # sequence with its own per-sequence strides: ragged lengths, a distinct
+    # cache per sequence (different seq seeds), both indexer modes.  A wrong
+    # offset of q, q_idx, w, swa, the outputs or the block list would mix
+    # sequences and fail the bit-exact comparison.
+    lens = [8 * 2048 + 8 * 37 + 3, 130, 5000, 8 * 2048 + 1]
+    for keep, decoder, seed in ((2048, True, 1002), (0, False, 1006)):
+        modes = orc.schedule(decoder)[:8]
+        caches, q_idx, w, q, swa = _batch_case(keep, lens, modes, seed)
+        r = orc.decode_batch(modes, lens, [c[0] for c in caches], [c[1] for c in caches],
+                             [c[2] for c in caches], [c[3] for c in caches], q_idx, w, q, swa, keep=keep)
+        for b, L in enumerate(lens):
+            codes, scales, k, pooled = caches[b]
+            one = orc.decode_step(modes, L, codes, scales, k, pooled, q_idx[b], w[b], q[b], swa[b], keep=keep)
+            np.testing.assert_array_equal(r["idx"][b], one["idx"])
+            np.testing.assert_array_equal(r["out"][b], one["out"])
+            np.testing.assert_array_equal(r["lse"][b], one["lse"])
+            if keep:
+                np.testing.assert_array_equal(r["blocks"][b], one["blocks"])
+        # the sequences really differ (distinct caches and queries)
+        assert not np.array_equal(r["out"][0], r["out"][3])
+        assert not np.array_equal(r["idx"][0], r["idx"][3])
