@@ -109,10 +109,10 @@ def attn_bytes_per_row(L: int) -> int:
     return min(512, L) * 144 + min(128, L) * 512 + 16 * 128 * 2 + 512 * 4 + 16 * 128 * 4 + 16 * 4
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one sparse_attn_kernel launch
-# (ncu --set full, first Full and Reuse launches of the eager step; the kernel
-# source has not changed since), keyed by (B, L)
-ATTN_TRAFFIC = {(8, 1 << 20): 1944320}
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode_attn_kernel launch
+# from an ncu capture of the current kernel source, keyed by (B, L); empty
+# until such a capture exists (the line then reports traffic null)
+ATTN_TRAFFIC: dict = {}
 # dram__bytes_read.sum + dram__bytes_write.sum of one flat indexer launch
 # (block_score_kernel + block_select_kernel<1>) keyed by (B, entries), taken at
 # B = 2 (139,576,576 B) and scaled by the rows scored
@@ -377,7 +377,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     a_bytes = B * attn_bytes_per_row(L)
     a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
     peak_src = "MEASURED_PEAKS.json hbm_gbs (measured, burst copy)" if hbm else "fallback 6650 GB/s"
-    attn_roof = dict(kernel="sparse_attn_kernel (Reuse layer, B rows x 8 CTAs)", bound="hbm", achieved=a_gbs,
+    attn_roof = dict(kernel="decode_attn_kernel (Reuse layer, B rows x 8 CTAs)", bound="hbm", achieved=a_gbs,
                      peak=hbm, unit="GB/s", frac=a_gbs / hbm if hbm else None, traffic=ATTN_TRAFFIC.get((B, L)),
                      bytes_per_launch=a_bytes, ms_per_launch=a_ms, peak_source=peak_src)
     idx_roof = dict(kernel="block_score_kernel + block_select_kernel" + (" over entries (flat indexer)" if flat else ""),

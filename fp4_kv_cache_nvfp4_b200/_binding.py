@@ -73,6 +73,12 @@ def lib() -> ctypes.CDLL:
             L.csa2_abi_version.restype = _I32
             L.csa2_device_accessible.argtypes = [_P]
             L.csa2_device_accessible.restype = _I32
+            L.csa2_indexer_score_ids.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_Cache), _I32, _P, _P,
+                                                 _P, _P, _I32, _I32, _P, _P, _I32, _I64, _P, _P]
+            L.csa2_topk_merge.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _I32, _P]
+            L.csa2_attn_lse_merge.argtypes = [_I32, _P, _P, _P, _P, _I32, _P]
+            for n in ("csa2_indexer_score_ids", "csa2_topk_merge", "csa2_attn_lse_merge"):
+                getattr(L, n).restype = _I32
             L.csa2_test_empty_chain.argtypes = [_I32, _I32, _I32, _P, _P]
             L.csa2_test_empty_chain.restype = _I32
             L.csa2_test_set_wait_limit.argtypes = [ctypes.c_uint32]
@@ -109,6 +115,27 @@ def abi_version() -> int:
 def device_accessible(t) -> int:
     """1 if kernels can read the tensor (or raw address) in place, 0 if not, -1 on a CUDA error."""
     return int(lib().csa2_device_accessible(_ptr(t)))
+
+
+def indexer_score_ids(desc: LayerDesc, cache: KVCache, level: int, q_idx, w, seq_lens, ids, id_offset: int,
+                      scores, ids_out, n: int, max_len: int, err=None, stream=None) -> None:
+    """Scores of the given ids (exact chains) and the ids plus id_offset."""
+    _check(lib().csa2_indexer_score_ids(ctypes.byref(desc), ctypes.byref(cache.struct()), level, _ptr(q_idx),
+                                        _ptr(w), _ptr(seq_lens), _ptr(ids), ids.shape[-1], id_offset, _ptr(scores),
+                                        _ptr(ids_out), n, max_len, _ptr(err), _stream(stream)), "indexer_score_ids")
+
+
+def topk_merge(scores, ids, k: int, out, out_local=None, lo: int = 0, hi: int = 0, stream=None) -> None:
+    """Top-k of gathered (score, id) pairs [parts, n, part_len]; ids ascending in pair order."""
+    parts, n, plen = scores.shape
+    _check(lib().csa2_topk_merge(_ptr(scores), _ptr(ids), parts, plen, k, lo, hi, _ptr(out), _ptr(out_local), n,
+                                 _stream(stream)), "topk_merge")
+
+
+def attn_lse_merge(out_parts, lse_parts, out, lse, stream=None) -> None:
+    """Log-sum-exp merge of partial attention outputs [G, rows, 16, 128] / [G, rows, 16]."""
+    _check(lib().csa2_attn_lse_merge(out_parts.shape[0], _ptr(out_parts), _ptr(lse_parts), _ptr(out), _ptr(lse),
+                                     out_parts.shape[1], _stream(stream)), "attn_lse_merge")
 
 
 def test_set_wait_limit(polls: int) -> int:
@@ -167,6 +194,19 @@ class KVCache:
 
     def struct(self) -> _Cache:
         return self._s
+
+    def shard(self, page_lo: int, n_pages: int) -> "KVCache":
+        """A view of pages [page_lo, page_lo + n_pages) of every sequence: the
+        same cache arrays with that slice of the page table, so entry e of the
+        view is entry page_lo * page_size + e of the sequence (a context-parallel
+        shard)."""
+        v = KVCache.__new__(KVCache)
+        v.page_size, v.n_phys_pages = self.page_size, self.n_phys_pages
+        v.codes, v.scales, v.idx_k, v.pooled = self.codes, self.scales, self.idx_k, self.pooled
+        v.page_table = self.page_table[:, page_lo:page_lo + n_pages].contiguous()
+        v._s = _Cache(self._s.codes, self._s.scales, self._s.idx_k, self._s.idx_k_pooled, v.page_table.data_ptr(),
+                      self.page_size, v.page_table.shape[1], self.n_phys_pages)
+        return v
 
 
 def kv_quant_append(cache: KVCache, kv_src: torch.Tensor, idx_k_src, slot_mapping: torch.Tensor, ratio: int = 1,

@@ -38,24 +38,24 @@ constexpr int SWA_ROW = 528;   // staged bf16 token: 512 B + 16 B pad (bank spre
 constexpr int VT_ROW = 272;    // fp16 V tile row: 256 B + 16 B pad
 constexpr int OACC_ROW = 132;  // fp32 merged O row (floats)
 
-constexpr size_t ATT_OFF_FP4 = 0;
-constexpr size_t ATT_OFF_SWA = ATT_OFF_FP4 + 4 * KPW * FP4_ROW;
-constexpr size_t ATT_OFF_VT = ATT_OFF_SWA + KPW * SWA_ROW;
-constexpr size_t ATT_END_STAGE = ATT_OFF_VT + ATT_WARPS * KPW * VT_ROW;
-// per-warp rescaled O partials reuse the staging area once every warp is past P.V
-constexpr size_t ATT_OFF_OPART = 0;
-constexpr size_t ATT_END_OPART = ATT_OFF_OPART + (size_t)ATT_WARPS * kH * OACC_ROW * 4;
-constexpr size_t ATT_OFF_OACC = ATT_END_STAGE > ATT_END_OPART ? ATT_END_STAGE : ATT_END_OPART;
-constexpr size_t ATT_OFF_MS = ATT_OFF_OACC + kH * OACC_ROW * 4;
-constexpr size_t ATT_OFF_L = ATT_OFF_MS + ATT_WARPS * kH * 4;  // receive (max, sum): 2 x 16 floats
-constexpr size_t ATT_OFF_MC = ATT_OFF_L + 2 * 2 * ATT_SPLIT * 4;
-constexpr size_t ATT_OFF_LPART = ATT_OFF_MC + kH * 4;
-constexpr size_t ATT_OFF_VALID = ATT_OFF_LPART + ATT_WARPS * kH * 4;
-constexpr size_t ATT_OFF_FCT = ATT_OFF_VALID + ATT_WARPS * KPW * 4;  // merge factors [2][ATT_SPLIT] + sums [2]
-constexpr size_t ATT_SMEM = ATT_OFF_FCT + (2 * ATT_SPLIT + 2) * 4;
-static_assert(ATT_OFF_SWA % 16 == 0 && ATT_OFF_VT % 16 == 0 && ATT_OFF_OACC % 16 == 0 && ATT_OFF_MS % 16 == 0 &&
-                  ATT_OFF_VALID % 16 == 0,
-              "attention shared-memory layout");
+// Shared-memory layout of the decode kernel (byte offsets, all 16-aligned).
+constexpr int DA_KEYS = 4 * KPW + KPW;   // 64 selected + 16 window keys per CTA
+constexpr int DA_PROW = DA_KEYS * 2 + 16;  // fp16 P row [80 keys] + 16 B pad (ldmatrix without bank conflicts)
+constexpr int DA_RROW = kD + 4;          // received partial of one head: O[128], m, l, 2 pad (floats)
+constexpr uint32_t DA_RECV_BYTES = (uint32_t)ATT_SPLIT * 2 * (kD + 2) * 4;  // bytes each CTA receives
+constexpr size_t DA_OFF_FP4 = 0;                                         // [4 warps][16][144] staged rows
+constexpr size_t DA_OFF_SWA = DA_OFF_FP4 + 4 * KPW * FP4_ROW;            // [16][528] staged window rows
+constexpr size_t DA_OFF_VT = DA_OFF_SWA + KPW * SWA_ROW;                 // [80 keys][272 B] fp16 V tile
+constexpr size_t DA_OFF_P = DA_OFF_VT + (size_t)DA_KEYS * VT_ROW;        // [16 heads][DA_PROW] fp16 P
+constexpr size_t DA_OFF_RECV = DA_OFF_P + (size_t)kH * DA_PROW;          // [8 src][2 heads][DA_RROW] fp32
+constexpr size_t DA_OFF_WM = DA_OFF_RECV + (size_t)ATT_SPLIT * 2 * DA_RROW * 4;  // [5 warps][16] max
+constexpr size_t DA_OFF_WS = DA_OFF_WM + ATT_WARPS * kH * 4;             // [5 warps][16] sums
+constexpr size_t DA_OFF_VALID = DA_OFF_WS + ATT_WARPS * kH * 4;          // [80] key valid flags
+constexpr size_t DA_OFF_BAR = DA_OFF_VALID + DA_KEYS * 4;                // receive mbarrier
+constexpr size_t DA_SMEM = DA_OFF_BAR + 16;
+static_assert(DA_OFF_SWA % 16 == 0 && DA_OFF_VT % 16 == 0 && DA_OFF_P % 16 == 0 && DA_OFF_RECV % 16 == 0 &&
+                  DA_OFF_WM % 16 == 0 && DA_OFF_BAR % 16 == 0 && DA_PROW % 16 == 0,
+              "decode attention shared-memory layout");
 
 __device__ __forceinline__ uint32_t e2m1_low_byte_to_h2(uint32_t x) {
     uint32_t out;
@@ -85,33 +85,77 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                  : "r"(addr));
 }
 
-__global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
+// One 8-byte asynchronous store into a peer CTA's shared memory that counts
+// its bytes on that CTA's mbarrier (both addresses in the cluster window).
+__device__ __forceinline__ void st_async_f32x2(uint32_t addr, float a, float b, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "f"(a), "f"(b), "r"(mbar)
+                 : "memory");
+}
+// Wait for a phase of this CTA's mbarrier whose bytes come from peer CTAs
+// (acquire at cluster scope); gives up after `limit` polls.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+constexpr uint32_t kAttnWaitLimit = 1u << 22;
+
+// Decode attention.  A cluster of 8 CTAs per sequence; CTA s takes selected
+// keys [64s, 64s + 64) (warps 0-3, 16 each) and window keys [16s, 16s + 16)
+// (warp 4).
+//   before the wait (what exists before the previous layer ends): gather the
+//     keys' rows, dequantise K into the mma B fragments and V into a shared
+//     fp16 tile [80 keys][128], initialise the receive mbarrier and pass a
+//     cluster barrier (every peer's mbarrier is then ready);
+//   after the wait: each warp computes S = Q K^T for its 16 keys; the CTA
+//     takes one softmax over its 80 keys (per-warp maxima and fp16 P in shared
+//     memory, two CTA barriers); warp w (0-3) computes O = P V for dims
+//     [32w, 32w + 32); every CTA then sends its (O, max, sum) of heads 2c and
+//     2c + 1 to CTA c with st.async, counted in bytes on CTA c's mbarrier, and
+//     CTA c merges the 8 partials of its two heads by log-sum-exp and writes
+//     them.  No cluster barrier after the wait: a CTA only waits for the bytes
+//     it receives.
+__global__ void __launch_bounds__(ATT_THREADS) decode_attn_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int split = blockIdx.x % ATT_SPLIT;  // rank in the cluster (cluster = 8 consecutive CTAs)
     const int row = blockIdx.x / ATT_SPLIT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
-    const bool prefill = a.q_pos != nullptr;
-    float* oacc = reinterpret_cast<float*>(smem + ATT_OFF_OACC);
-    float* ms = reinterpret_cast<float*>(smem + ATT_OFF_MS);
-    float* lacc = reinterpret_cast<float*>(smem + ATT_OFF_L);
-    float* mc = reinterpret_cast<float*>(smem + ATT_OFF_MC);
-    float* opart = reinterpret_cast<float*>(smem + ATT_OFF_OPART);
-    float* lpart = reinterpret_cast<float*>(smem + ATT_OFF_LPART);
-    int* valid = reinterpret_cast<int*>(smem + ATT_OFF_VALID) + warp * KPW;
-    uint8_t* vt = smem + ATT_OFF_VT + warp * KPW * VT_ROW;
+    float* recv = reinterpret_cast<float*>(smem + DA_OFF_RECV);
+    float* wmax = reinterpret_cast<float*>(smem + DA_OFF_WM);
+    float* wsum = reinterpret_cast<float*>(smem + DA_OFF_WS);
+    int* valid = reinterpret_cast<int*>(smem + DA_OFF_VALID);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + DA_OFF_BAR);
+    uint8_t* vt = smem + DA_OFF_VT;  // key k (0..79) at row k
+    uint8_t* ps = smem + DA_OFF_P;
 
-    // Data that exists before the preceding layer finishes (a.pre: an earlier
-    // layer's index set, the cache, the SWA history) is gathered before waiting
-    // on the preceding kernel, so its latency overlaps that kernel's tail; q and
-    // the newest SWA row are read after the wait.  Every buffer offset below
-    // assumes a 16-byte-aligned dynamic shared base; the check is uniform over
-    // the grid, so no CTA waits on one that left.
+    // Every buffer offset assumes a 16-byte-aligned dynamic shared base; the
+    // check is uniform over the grid, so no CTA waits on one that left.
     if (smem_u32(smem) & 15u) {
         pdl_wait();
         if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
+    // The receive mbarrier expects one local arrival and DA_RECV_BYTES from the
+    // 8 CTAs of the cluster; the cluster barrier below makes its
+    // initialisation visible to them before any of them sends.  Neither reads
+    // global memory, so both run before the wait on the preceding kernel.
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, DA_RECV_BYTES);
+    }
+    cluster_arrive();
+
     const bool pre_idx = (a.pre & kPreIdx) != 0, pre_hist = (a.pre & kPreHist) != 0;
     bool waited = false;
     auto wait_once = [&]() {
@@ -122,41 +166,16 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     };
     if (!pre_idx && !pre_hist) wait_once();
 
-    // Q (A operand rows: heads g and g + 8, bf16 pairs) of this row
-    uint32_t qraw[8][4];
-    auto load_q = [&]() {
-        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
-        const uint32_t* qg8 = qg + 8 * kD / 2;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            qraw[c][0] = __ldg(qg + 8 * c + t);
-            qraw[c][1] = __ldg(qg8 + 8 * c + t);
-            qraw[c][2] = __ldg(qg + 8 * c + 4 + t);
-            qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
-        }
-    };
-
     // ---- sequence, window --------------------------------------------------
-    const int seq = prefill ? 0 : row;
-    const int32_t L = prefill ? a.seq_len_prefill : a.seq_lens[row];
-    const uint16_t* swa_base;
-    int n_swa, newest = -1;
-    if (prefill) {
-        const int p = a.q_pos[row];
-        const int lo = max(0, p - a.window + 1);
-        swa_base = a.swa + (int64_t)(lo - a.swa_start) * kCh;
-        n_swa = (lo >= a.swa_start) ? p - lo + 1 : 0;
-        if (lo < a.swa_start && tid == 0 && split == 0) dev_error(a.err, CSA2_DEV_INDEX);
-    } else {
-        swa_base = a.swa + (int64_t)row * a.window * kCh;
-        n_swa = a.swa_lens ? a.swa_lens[row] : (L < a.window ? L : a.window);
-        n_swa = max(0, min(n_swa, a.window));
-        if ((pre_idx || pre_hist) && L > 0) newest = (L - 1) % a.window;  // the newest row waits
-    }
+    const int32_t L = a.seq_lens[row];
+    const uint16_t* swa_base = a.swa + (int64_t)row * a.window * kCh;
+    int n_swa = a.swa_lens ? a.swa_lens[row] : (L < a.window ? L : a.window);
+    n_swa = max(0, min(n_swa, a.window));
+    const int newest = ((pre_idx || pre_hist) && L > 0) ? (L - 1) % a.window : -1;  // read after the wait
 
     // ---- gather this warp's 16 keys into shared memory ---------------------
-    uint8_t* st_fp4 = smem + ATT_OFF_FP4 + (warp < 4 ? warp : 0) * KPW * FP4_ROW;
-    uint8_t* st_swa = smem + ATT_OFF_SWA;
+    uint8_t* st_fp4 = smem + DA_OFF_FP4 + (warp < 4 ? warp : 0) * KPW * FP4_ROW;
+    uint8_t* st_swa = smem + DA_OFF_SWA;
     const int k0 = warp < 4 ? split * 64 + warp * KPW : split * KPW;
     if (warp < 4) {
         if (!pre_idx) wait_once();  // the index set comes from the preceding kernel
@@ -166,11 +185,11 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             if (kidx < a.topk) {
                 const int32_t pos = a.idx[(int64_t)row * a.topk + kidx];
                 if (pos >= 0) {
-                    if (pos < L) slot = entry_slot(a.cache, a.page_shift, seq, pos, a.err);
+                    if (pos < L) slot = entry_slot(a.cache, a.page_shift, row, pos, a.err);
                     else dev_error(a.err, CSA2_DEV_INDEX);
                 }
             }
-            valid[lane] = slot >= 0;
+            valid[warp * KPW + lane] = slot >= 0;
         }
         // 16 rows x 9 chunks of 16 B; every lane runs all 5 trips (the shuffle
         // needs the full warp), trips past the 144 chunks copy nothing
@@ -190,7 +209,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
             }
         }
     } else {
-        if (lane < KPW) valid[lane] = (k0 + lane) < n_swa;
+        if (lane < KPW) valid[4 * KPW + lane] = (k0 + lane) < n_swa;
         for (int c = lane; c < KPW * 32; c += 32) {
             const int r = c >> 5, ch = c & 31;
             uint8_t* dst = st_swa + r * SWA_ROW + ch * 16;
@@ -203,12 +222,13 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     }
     cp_async_commit();
 
-    // B fragments of S = Q K^T (fp16) for the warp's two n8 tiles of keys, and
-    // the fp16 V tile [key][dim] in shared memory.
+    // K of the warp's keys as the B fragments of S = Q K^T (two n8 tiles),
+    // V into rows [16 w, 16 w + 16) of the shared fp16 V tile; `only` >= 0
+    // rebuilds just that row (the newest window row, staged after the wait).
     uint32_t bk[2][8][2];
-    auto build_kv = [&]() {
+    auto build_kv = [&](int only) {
         const int key = lane >> 1, half = lane & 1;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(vt + (warp * KPW + key) * VT_ROW + half * 128);
         if (warp < 4) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -235,6 +255,7 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
         } else {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
+                if (only >= 0 && 8 * j + g != only) continue;
                 const uint32_t* r = reinterpret_cast<const uint32_t*>(st_swa + (8 * j + g) * SWA_ROW);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -242,46 +263,66 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
                     bk[j][c][1] = bf2_to_h2(r[8 * c + 4 + t]);
                 }
             }
-            const uint32_t* r = reinterpret_cast<const uint32_t*>(st_swa + key * SWA_ROW) + 64 + 32 * half;
+            if (only < 0 || key == only) {
+                const uint32_t* r = reinterpret_cast<const uint32_t*>(st_swa + key * SWA_ROW) + 64 + 32 * half;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]),
-                                                                    bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(
+                        bf2_to_h2(r[4 * i]), bf2_to_h2(r[4 * i + 1]), bf2_to_h2(r[4 * i + 2]), bf2_to_h2(r[4 * i + 3]));
+            }
         }
     };
-    if (warp == 4 && newest >= 0) {  // the newest window row is read after the wait
-        wait_once();
-        if (newest >= k0 && newest < k0 + KPW && newest < n_swa)
-            cp_async16(st_swa + (newest - k0) * SWA_ROW + lane * 16, swa_base + (int64_t)newest * kCh + lane * 8);
-        cp_async_commit();
-    }
     cp_async_wait<0>();
     __syncwarp();
-    build_kv();
+    build_kv(-1);
+    // the newest window row (computed from the previous layer's output) is read
+    // after the wait and patched into the fragments and the V tile
+    const int new_r = newest - k0;
+    const bool own_newest = warp == 4 && newest >= 0 && new_r >= 0 && new_r < KPW && newest < n_swa;
     wait_once();  // every thread has waited before anything is written
     pdl_trigger();
-    load_q();
+    if (own_newest) {
+        cp_async16(st_swa + new_r * SWA_ROW + lane * 16, swa_base + (int64_t)newest * kCh + lane * 8);
+        cp_async_commit();
+    }
+    // Q (A operand rows: heads g and g + 8, bf16 pairs) of this row
+    uint32_t qraw[8][4];
+    {
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q + (int64_t)row * kH * kD + g * kD);
+        const uint32_t* qg8 = qg + 8 * kD / 2;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            qraw[c][0] = __ldg(qg + 8 * c + t);
+            qraw[c][1] = __ldg(qg8 + 8 * c + t);
+            qraw[c][2] = __ldg(qg + 8 * c + 4 + t);
+            qraw[c][3] = __ldg(qg8 + 8 * c + 4 + t);
+        }
+    }
+    if (own_newest) {
+        cp_async_wait<0>();
+        __syncwarp();
+        build_kv(new_r);
+    }
 
     // ---- S = Q K^T (A operand: 16 heads x 128 dims, fp16) -------------------
     float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t qa[4] = {bf2_to_h2(qraw[c][0]), bf2_to_h2(qraw[c][1]), bf2_to_h2(qraw[c][2]),
-                                    bf2_to_h2(qraw[c][3])};
-            mma16816(S[0], qa, bk[0][c][0], bk[0][c][1]);
-            mma16816(S[1], qa, bk[1][c][0], bk[1][c][1]);
-        }
+    for (int c = 0; c < 8; ++c) {
+        const uint32_t qa[4] = {bf2_to_h2(qraw[c][0]), bf2_to_h2(qraw[c][1]), bf2_to_h2(qraw[c][2]),
+                                bf2_to_h2(qraw[c][3])};
+        mma16816(S[0], qa, bk[0][c][0], bk[0][c][1]);
+        mma16816(S[1], qa, bk[1][c][0], bk[1][c][1]);
     }
 
-    // ---- softmax over the warp's keys (log2 domain) ------------------------
+    // ---- one softmax over the CTA's 80 keys (log2 domain) ---------------------
     const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    const int kb = warp * KPW;  // this warp's first key in the CTA
     float mg = -INFINITY, mg8 = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const bool ok = valid[8 * j + 2 * t + e] != 0;
+            const bool ok = valid[kb + 8 * j + 2 * t + e] != 0;
             S[j][e] = ok ? S[j][e] * kScaleLog2 : -INFINITY;
             S[j][2 + e] = ok ? S[j][2 + e] * kScaleLog2 : -INFINITY;
             mg = fmaxf(mg, S[j][e]);
@@ -293,140 +334,116 @@ __global__ void __launch_bounds__(ATT_THREADS) sparse_attn_kernel(AttnArgs a) {
     mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 1));
     mg8 = fmaxf(mg8, __shfl_xor_sync(0xffffffffu, mg8, 2));
     if (t == 0) {
-        ms[warp * kH + g] = mg;
-        ms[warp * kH + g + 8] = mg8;
+        wmax[warp * kH + g] = mg;
+        wmax[warp * kH + g + 8] = mg8;
+    }
+    __syncthreads();  // every warp's maxima (and, with them, every V tile row)
+    float M = -INFINITY, M8 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < ATT_WARPS; ++w) {
+        M = fmaxf(M, wmax[w * kH + g]);
+        M8 = fmaxf(M8, wmax[w * kH + g + 8]);
     }
     float lg = 0.f, lg8 = 0.f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            S[j][e] = mg == -INFINITY ? 0.f : exp2f(S[j][e] - mg);
-            S[j][2 + e] = mg8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - mg8);
+            S[j][e] = M == -INFINITY ? 0.f : exp2f(S[j][e] - M);
+            S[j][2 + e] = M8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - M8);
             lg += S[j][e];
             lg8 += S[j][2 + e];
         }
+        // P (fp16) rows g and g + 8, keys kb + 8 j + 2 t, + 1
+        *reinterpret_cast<uint32_t*>(ps + g * DA_PROW + (kb + 8 * j + 2 * t) * 2) = f2_to_h2(S[j][0], S[j][1]);
+        *reinterpret_cast<uint32_t*>(ps + (g + 8) * DA_PROW + (kb + 8 * j + 2 * t) * 2) = f2_to_h2(S[j][2], S[j][3]);
     }
     lg += __shfl_xor_sync(0xffffffffu, lg, 1);
     lg += __shfl_xor_sync(0xffffffffu, lg, 2);
     lg8 += __shfl_xor_sync(0xffffffffu, lg8, 1);
     lg8 += __shfl_xor_sync(0xffffffffu, lg8, 2);
+    if (t == 0) {
+        wsum[warp * kH + g] = lg;
+        wsum[warp * kH + g + 8] = lg8;
+    }
+    cluster_wait();   // every peer's receive mbarrier is initialised (arrived long before)
+    __syncthreads();  // P and the sums are complete
 
-    // ---- O = P V --------------------------------------------------------------
-    const uint32_t pa[4] = {f2_to_h2(S[0][0], S[0][1]), f2_to_h2(S[0][2], S[0][3]), f2_to_h2(S[1][0], S[1][1]),
-                            f2_to_h2(S[1][2], S[1][3])};
-    __syncwarp();
-    float O[16][4];
+    const uint32_t my_bar = smem_u32(bar);
+    if (warp < 4) {
+        // ---- O[16 heads][32 w .. 32 w + 31] = P[16][80] V[80][dims] ------------
+        float O[4][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-    {
+        for (int j = 0; j < 4; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+        const uint32_t pa_base = smem_u32(ps) + (((lane >> 3) & 1) * 8 + (lane & 7)) * DA_PROW + (lane >> 4) * 16;
         const int m = lane >> 3, r = lane & 7;
-        const uint32_t base = (uint32_t)__cvta_generic_to_shared(vt) + ((m & 1) * 8 + r) * VT_ROW + (m >> 1) * 16;
+        const uint32_t vb_base = smem_u32(vt) + ((m & 1) * 8 + r) * VT_ROW + (m >> 1) * 16 + warp * 64;
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(base + j * 16, b0, b1, b2, b3);
-            mma16816(O[j], pa, b0, b1);
-            mma16816(O[j + 1], pa, b2, b3);
-        }
-    }
-
-    // ---- merge: the 5 warps of this CTA in shared memory, then each CTA sends
-    // its (max, sum, O) of heads 2c, 2c+1 to CTA c of the cluster ------------
-    __syncthreads();  // ms complete
-    float Mg = -INFINITY, Mg8 = -INFINITY;
+        for (int ks = 0; ks < DA_KEYS / 16; ++ks) {
+            uint32_t pa[4];
+            ldsm_x4(pa_base + ks * 32, pa[0], pa[1], pa[2], pa[3]);
 #pragma unroll
-    for (int w = 0; w < ATT_WARPS; ++w) {
-        Mg = fmaxf(Mg, ms[w * kH + g]);
-        Mg8 = fmaxf(Mg8, ms[w * kH + g + 8]);
-    }
-    const float fg = mg == -INFINITY ? 0.f : exp2f(mg - Mg);
-    const float fg8 = mg8 == -INFINITY ? 0.f : exp2f(mg8 - Mg8);
-    {
-        float* part = opart + warp * kH * OACC_ROW;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            *reinterpret_cast<float2*>(part + g * OACC_ROW + 8 * j + 2 * t) = make_float2(O[j][0] * fg, O[j][1] * fg);
-            *reinterpret_cast<float2*>(part + (g + 8) * OACC_ROW + 8 * j + 2 * t) =
-                make_float2(O[j][2] * fg8, O[j][3] * fg8);
-        }
-        if (t == 0) {
-            lpart[warp * kH + g] = lg * fg;
-            lpart[warp * kH + g + 8] = lg8 * fg8;
-            if (warp == 0) {
-                mc[g] = Mg;
-                mc[g + 8] = Mg8;
+            for (int j = 0; j < 4; j += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_trans(vb_base + ks * 16 * VT_ROW + j * 16, b0, b1, b2, b3);
+                mma16816(O[j], pa, b0, b1);
+                mma16816(O[j + 1], pa, b2, b3);
             }
         }
-    }
-    __syncthreads();
-    // receive buffers (in this CTA): from CTA c, heads 2*split + hh
-    float* recv_o = oacc;                       // [ATT_SPLIT][2][kD]
-    float* recv_m = lacc;                       // [ATT_SPLIT][2]  (lacc/mc regions hold 16 floats each)
-    float* recv_l = recv_m + 2 * ATT_SPLIT;     // [ATT_SPLIT][2]
-    for (int i = tid; i < kH * kD / 4; i += ATT_THREADS) {
-        const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
-        float4 acc = *reinterpret_cast<const float4*>(opart + h * OACC_ROW + d4);
+        // ---- send: heads g, g + 8 to their owner CTAs, dims 32 w + 8 j + 2 t ----
+        const int hs[2] = {g, g + 8};
 #pragma unroll
-        for (int w = 1; w < ATT_WARPS; ++w) {
-            const float4 v = *reinterpret_cast<const float4*>(opart + w * kH * OACC_ROW + h * OACC_ROW + d4);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+        for (int hi = 0; hi < 2; ++hi) {
+            const int h = hs[hi];
+            const uint32_t owner = (uint32_t)(h >> 1);
+            const uint32_t rb = mapa_shared(my_bar, owner);
+            const uint32_t ro = mapa_shared(smem_u32(recv + (split * 2 + (h & 1)) * DA_RROW), owner);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                st_async_f32x2(ro + (uint32_t)(32 * warp + 8 * j + 2 * t) * 4u, O[j][2 * hi], O[j][2 * hi + 1], rb);
         }
-        const uint32_t dst = smem_u32(recv_o + (split * 2 + (h & 1)) * kD + d4);
-        st_cluster_f32x4(mapa_shared(dst, (uint32_t)(h >> 1)), acc);
-    }
-    if (tid < kH) {
-        float l = 0.f;
+    } else if (lane < kH) {
+        // ---- send the CTA's (max, sum) of head `lane` to its owner --------------
+        const int h = lane;
+        float mx = -INFINITY, sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < ATT_WARPS; ++w) l += lpart[w * kH + tid];
-        const uint32_t rank = (uint32_t)(tid >> 1), slot = (uint32_t)(split * 2 + (tid & 1));
-        st_cluster_u32(mapa_shared(smem_u32(recv_m + slot), rank), __float_as_uint(mc[tid]));
-        st_cluster_u32(mapa_shared(smem_u32(recv_l + slot), rank), __float_as_uint(l));
+        for (int w = 0; w < ATT_WARPS; ++w) mx = fmaxf(mx, wmax[w * kH + h]);
+#pragma unroll
+        for (int w = 0; w < ATT_WARPS; ++w) sum += wsum[w * kH + h];
+        const uint32_t owner = (uint32_t)(h >> 1);
+        st_async_f32x2(mapa_shared(smem_u32(recv + (split * 2 + (h & 1)) * DA_RROW + kD), owner), mx, sum,
+                       mapa_shared(my_bar, owner));
     }
-    cluster_sync_all();  // the only exchange: afterwards every CTA reads its own memory
 
-    float (*fct)[ATT_SPLIT] = reinterpret_cast<float (*)[ATT_SPLIT]>(smem + ATT_OFF_FCT);
-    float* sden = reinterpret_cast<float*>(smem + ATT_OFF_FCT) + 2 * ATT_SPLIT;
-    if (warp == 0) {
-        const int hh = (lane >> 3) & 1, c = lane & 7;
-        const float mcv = lane < 2 * ATT_SPLIT ? recv_m[c * 2 + hh] : -INFINITY;
-        const float lv = lane < 2 * ATT_SPLIT ? recv_l[c * 2 + hh] : 0.f;
-        float M = mcv;
-#pragma unroll
-        for (int o = 1; o < ATT_SPLIT; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float f = (lane < 2 * ATT_SPLIT && mcv != -INFINITY) ? exp2f(mcv - M) : 0.f;
-        float den = lv * f;
-#pragma unroll
-        for (int o = 1; o < ATT_SPLIT; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        if (lane < 2 * ATT_SPLIT) {
-            fct[hh][c] = f;
-            if (c == 0) {
-                sden[hh] = den;
-                a.lse[(int64_t)row * kH + 2 * split + hh] =
-                    den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
-            }
-        }
+    // ---- receive the 8 partials of heads 2 split, 2 split + 1 and merge -------
+    if (!mbar_wait_cluster(bar, 0u, kAttnWaitLimit)) {
+        if (tid == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+        return;  // nothing was received in time: leave out and lse unwritten
     }
-    __syncthreads();
-    for (int i = tid; i < 2 * kD / 4; i += ATT_THREADS) {
-        const int hh = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
+    if (tid < 2 * kD / 4) {
+        const int hh = tid / (kD / 4), d4 = (tid % (kD / 4)) * 4;
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < ATT_SPLIT; ++c) Mx = fmaxf(Mx, recv[(c * 2 + hh) * DA_RROW + kD]);
         float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        float den = 0.f;
 #pragma unroll
         for (int c = 0; c < ATT_SPLIT; ++c) {
-            const float4 v = *reinterpret_cast<const float4*>(recv_o + (c * 2 + hh) * kD + d4);
-            const float f = fct[hh][c];
+            const float* p = recv + (c * 2 + hh) * DA_RROW;
+            const float mc = p[kD];
+            const float f = mc == -INFINITY ? 0.f : exp2f(mc - Mx);
+            const float4 v = *reinterpret_cast<const float4*>(p + d4);
             num.x += v.x * f;
             num.y += v.y * f;
             num.z += v.z * f;
             num.w += v.w * f;
+            den += p[kD + 1] * f;
         }
-        const float den = sden[hh];
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        *reinterpret_cast<float4*>(a.out + ((int64_t)row * kH + 2 * split + hh) * kD + d4) =
+        const int h = 2 * split + hh;
+        *reinterpret_cast<float4*>(a.out + ((int64_t)row * kH + h) * kD + d4) =
             make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+        if (d4 == 0) a.lse[(int64_t)row * kH + h] = den > 0.f ? (Mx + log2f(den)) * 0.6931471805599453f : -INFINITY;
     }
 }
 
@@ -917,8 +934,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!init[dev]) {
-        e = cudaFuncSetAttribute((const void*)sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ATT_SMEM);
+        e = cudaFuncSetAttribute((const void*)decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)DA_SMEM);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute((const void*)prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)PA_SMEM);
@@ -940,8 +957,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
         LaunchCfg c(dim3((unsigned)a.rows), dim3(PA_THREADS), PA_SMEM, stream);
         return cudaLaunchKernelEx(&c.cfg, prefill_attn_kernel, a);
     }
-    LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), ATT_SMEM, stream, ATT_SPLIT);
-    return cudaLaunchKernelEx(&c.cfg, sparse_attn_kernel, a);
+    LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), DA_SMEM, stream, ATT_SPLIT);
+    return cudaLaunchKernelEx(&c.cfg, decode_attn_kernel, a);
 }
 
 }  // namespace csa2

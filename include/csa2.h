@@ -264,6 +264,45 @@ CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc*
                                void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Context-parallel decode of one long sequence over G shards (one per GPU).
+ * Pages: native context window of one million tokens (conexaotc.com.br,
+ * opening paragraphs); Top-512 and the hierarchical indexer of up to 2048
+ * blocks of 8 (CSA2 paragraph).  Shard g holds the entries [g*S, g*S + S) of
+ * the sequence (S a multiple of the page size) in a cache whose page table is
+ * that slice of the sequence's; it runs csa2_indexer_topk and
+ * csa2_sparse_attn_decode on its own entries (positions local to the shard).
+ * Since every member of the global Top-K lies in its own shard's local Top-K,
+ * merging the shards' local lists gives exactly the single-GPU selection:
+ *   1. csa2_indexer_score_ids: the scores of a shard's selected ids (block ids
+ *      at level BLOCK, entry positions at level TOKEN), computed with the
+ *      sequential FMA chains of the selection (bit-equal scores), and the ids
+ *      made global by adding id_offset (-1 stays -1, score -inf);
+ *   2. the (score, global id) lists of all shards are gathered rank by rank
+ *      (an all-gather into [G][n][k]: the ids of a row are then ascending in
+ *      pair order, shard by shard);
+ *   3. csa2_topk_merge: the Top-k of the gathered pairs by (score desc, id asc)
+ *      -- the global set, ascending, -1 padded -- and, if out_local is given,
+ *      its members in [lo, hi) minus lo: the shard's local share;
+ *   4. attention per shard over its local share (the window on one shard),
+ *      then csa2_attn_lse_merge of the gathered partial (out, lse).
+ *   ids [n][k], scores and ids_out [n][k] (ids_out nullable); id_offset >= 0.
+ *   scores, ids [n_parts][n][part_len], n_parts * part_len <= 16384 (8 shards x
+ *   2048), k <= 2048; out, out_local [n][k].
+ *   out_parts [n_parts][rows][16][128], lse_parts [n_parts][rows][16] (natural
+ *   log, -inf for an empty partial); out [rows][16][128], lse [rows][16];
+ *   out = sum_g e^(lse_g - M) out_g / sum_g e^(lse_g - M), lse = M + log(sum). */
+CSA2_API csa2_status csa2_indexer_score_ids(const csa2_layer_desc* desc, const csa2_kv_cache* cache, int32_t level,
+                                            const uint16_t* q_idx, const float* w, const int32_t* seq_lens,
+                                            const int32_t* ids, int32_t k, int32_t id_offset, float* scores,
+                                            int32_t* ids_out, int32_t n, int64_t max_len, int32_t* err_word,
+                                            void* stream);
+CSA2_API csa2_status csa2_topk_merge(const float* scores, const int32_t* ids, int32_t n_parts, int32_t part_len,
+                                     int32_t k, int32_t lo, int32_t hi, int32_t* out, int32_t* out_local, int32_t n,
+                                     void* stream);
+CSA2_API csa2_status csa2_attn_lse_merge(int32_t n_parts, const float* out_parts, const float* lse_parts, float* out,
+                                         float* lse, int32_t rows, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Allocation-free decode indexer.  The pages have no counterpart to this call:
  * it is an integration convenience for callers that cannot allocate device
  * memory where they run the indexer -- plug-ins whose host framework owns all
