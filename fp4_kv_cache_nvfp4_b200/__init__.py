@@ -14,6 +14,6 @@ import os
 from ._binding import (  # noqa: F401
     BLOCK, BF16, CSA2Error, F32, FULL, KVCache, LayerDesc, REINDEX, REUSE, TOKEN, abi_version, attn_lse_merge,
     decode_layers, default_desc, device_accessible, indexer_score_ids, indexer_topk, indexer_topk_noalloc,
-    kv_quant_append, lib, lib_path, schedule, sparse_attn_decode, sparse_attn_prefill, test_empty_chain,
+    kv_quant_append, lib, lib_path, schedule, sparse_attn_decode, sparse_attn_prefill, swa_replay, test_empty_chain,
     test_set_wait_limit, topk_merge, workspace_bytes,
 )

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
             L.csa2_attn_lse_merge.argtypes = [_I32, _P, _P, _P, _P, _I32, _P]
             for n in ("csa2_indexer_score_ids", "csa2_topk_merge", "csa2_attn_lse_merge"):
                 getattr(L, n).restype = _I32
+            L.csa2_swa_replay.argtypes = [_P, _P, _P, _P, _I32, _I32, _I32, _P, _P]
+            L.csa2_swa_replay.restype = _I32
             L.csa2_test_empty_chain.argtypes = [_I32, _I32, _I32, _P, _P]
             L.csa2_test_empty_chain.restype = _I32
             L.csa2_test_set_wait_limit.argtypes = [ctypes.c_uint32]
@@ -136,6 +138,13 @@ def attn_lse_merge(out_parts, lse_parts, out, lse, stream=None) -> None:
     """Log-sum-exp merge of partial attention outputs [G, rows, 16, 128] / [G, rows, 16]."""
     _check(lib().csa2_attn_lse_merge(out_parts.shape[0], _ptr(out_parts), _ptr(lse_parts), _ptr(out), _ptr(lse),
                                      out_parts.shape[1], _stream(stream)), "attn_lse_merge")
+
+
+def swa_replay(h, w_kv, seq_lens, swa_kv, B: int, window: int = 128, err=None, stream=None) -> None:
+    """Recompute the window K|V rows of B sequences from their hidden states
+    h [B, window, d_model] and the projection w_kv [256, d_model] (bf16 bits)."""
+    _check(lib().csa2_swa_replay(_ptr(h), _ptr(w_kv), _ptr(seq_lens), _ptr(swa_kv), B, h.shape[-1], window,
+                                 _ptr(err), _stream(stream)), "swa_replay")
 
 
 def test_set_wait_limit(polls: int) -> int:

@@ -46,6 +46,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
+#include "tc.cuh"
 
 namespace csa2 {
 
@@ -1314,37 +1315,6 @@ constexpr int PT_SPLIT = 2048;    // entries per CTA (grid.y splits the entry ra
 constexpr int PT_CAND = 768;      // approximate candidates per query
 constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit threshold) -> exact fallback
 
-// ---- tcgen05 helpers (5th-generation tensor cores, accumulators in TMEM) ----
-// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand tile
-// (rows of 128 B, 8-row groups 1024 B apart, chunk c of row r at c ^ (r & 7);
-// the tile starts on a 1024-byte boundary).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// D[128 x n] (+)= A[128 x 16] . B[n x 16]^T, bf16 inputs, fp32 accumulators in TMEM
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
-        "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(addr));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
 // K5a on tcgen05: a CTA scores 128 queries (MMA M, one TMEM lane each) against
 // its range of entries, 64 at a time (MMA N), all four heads (4 accumulators
 // of 64 columns, double-buffered: 512 TMEM columns).
@@ -1830,21 +1800,6 @@ static cudaError_t ensure_smem(const void* fn, size_t bytes, bool* done) {
         done[dev] = true;
     }
     return cudaSuccess;
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        else
-            (void)cudaGetLastError();
-    }
-    return fn;
 }
 
 // The indexer-K rows as a 2-D tensor [n_slots][64] bf16 read in 64-row boxes,

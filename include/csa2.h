@@ -264,6 +264,26 @@ CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc*
                                void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* SWA Bounded Replay, attention part.  Pages: "FP4 KV, repeticion limitada y
+ * otras extensiones" (7minutos.es) -- on a miss only 128 tokens are
+ * recomputed -- and "Como funciona" (e-cogni.com.br) -- the replay avoids
+ * persisting the SWA cache at the cost of a small recompute in prefill.
+ * Recomputes one layer's window K|V rows from the hidden states of the window's
+ * tokens:
+ *   swa_kv[b][p % window][c] = bf16_RNE( sum_k h[b][t][k] * w_kv[c][k] )
+ * for the last n_b = min(window, seq_lens[b]) tokens, t = 0..n_b-1 oldest
+ * first, p = seq_lens[b] - n_b + t; c = 0..255 (K channels 0..127, V
+ * 128..255); fp32 accumulation on the tensor cores.  Rows of swa_kv outside
+ * the window and rows t >= n_b of h are not touched / not used.
+ *   h      [B][window][d_model] bf16, 16-byte aligned
+ *   w_kv   [256][d_model] bf16 (row c = output channel c), 16-byte aligned
+ *   swa_kv [B][window][256] bf16 (the ring csa2_sparse_attn_decode reads)
+ * d_model a multiple of 64 (<= 65536; UNSUPPORTED otherwise); window <= 128. */
+CSA2_API csa2_status csa2_swa_replay(const uint16_t* h, const uint16_t* w_kv, const int32_t* seq_lens,
+                                     uint16_t* swa_kv, int32_t B, int32_t d_model, int32_t window, int32_t* err_word,
+                                     void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Context-parallel decode of one long sequence over G shards (one per GPU).
  * Pages: native context window of one million tokens (conexaotc.com.br,
  * opening paragraphs); Top-512 and the hierarchical indexer of up to 2048

@@ -95,6 +95,7 @@ def _declare(L: ctypes.CDLL) -> None:
     L.orc_visible_entries.argtypes = [_I64, _I32, _I64]
     L.orc_prefill_indexer.argtypes = [_I64, _P, _I32, _I64, _P, _P, _P, _I64, _P]
     L.orc_prefill_attn.argtypes = [_I64, _P, _P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _P]
+    L.orc_swa_replay.argtypes = [_P, _P, _I64, _I64, _P]
     L.orc_cache_bytes_per_token.restype = ctypes.c_double
     L.orc_cache_bytes_per_token.argtypes = [_I32, _P, ctypes.c_double, ctypes.c_double]
 
@@ -315,6 +316,16 @@ def prefill_attn(q_pos, q, idx, codes, scales, swa, swa_start: int, window: int 
     lib().orc_prefill_attn(T, _p(q_pos), _p(q), _p(idx), idx.shape[1], _p(codes), _p(scales), _p(swa), swa_start,
                            window, _p(out), _p(lse))
     return out, lse
+
+
+def swa_replay(h, w_kv) -> np.ndarray:
+    """Replayed window rows: bf16 bits [n, 256] = bf16(h [n, d] . w_kv [256, d]^T)."""
+    h, w_kv = _c(h, np.uint16), _c(w_kv, np.uint16)
+    n, d = h.shape
+    assert w_kv.shape == (CH, d)
+    out = np.empty((n, CH), np.uint16)
+    lib().orc_swa_replay(_p(h), _p(w_kv), n, d, _p(out))
+    return out
 
 
 def cache_bytes_per_token(full_ratios, main_entry_bytes: float, idx_entry_bytes: float) -> float:

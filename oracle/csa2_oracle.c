@@ -49,6 +49,9 @@
  *   R10 decode window = last min(128, L) tokens including the current one;
  *       prefill window of the query at p = tokens [max(0, p-127), p]; entry j
  *       is visible to query p iff (j+1)*ratio - 1 <= p.
+ *   R12 SWA Bounded Replay: a layer's window K|V row of a token is bf16(h . W)
+ *       with h the token's hidden state and W the layer's K|V projection
+ *       (synthetic here: the pages' weights are not available).
  *   R11 the pages place the hierarchical indexer in the decoder only; the
  *       encoder's Full layers (ratio 2) select their Top-512 over every entry
  *       of the context ("flat"), as its prefill does.  A decode step with
@@ -528,6 +531,27 @@ void orc_prefill_attn(int64_t T, const int32_t* q_pos, const uint16_t* q, const 
         orc_attend(q + t * ORC_H * ORC_D, idx + t * topk, topk, codes, scales, swa + (lo - swa_start) * ORC_CH,
                    p - lo + 1, out + t * ORC_H * ORC_D, lse + t * ORC_H);
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* SWA Bounded Replay, attention part ([P5] "FP4 KV, repeticion        */
+/* limitada...": on a miss only 128 tokens are recomputed; [P4] "Como   */
+/* funciona": the replay avoids persisting the SWA cache)              */
+/* ------------------------------------------------------------------ */
+
+/* R12 (reading): a layer's SWA K|V row of a token is its hidden state h
+ * (bf16, d_model values) times the layer's K|V projection w (bf16, 256 output
+ * channels x d_model), rounded to bf16: out[t][c] = bf16_RNE(sum_k h[t][k] *
+ * w[c][k]).  The sum is taken in fp64 (it decides no integer), rounded to fp32
+ * and then to bf16.  h [n][d], w [256][d], out [n][256]. */
+void orc_swa_replay(const uint16_t* h, const uint16_t* w, int64_t n, int64_t d, uint16_t* out) {
+    for (int64_t t = 0; t < n; ++t)
+        for (int c = 0; c < ORC_CH; ++c) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < d; ++k)
+                acc += (double)orc_bf16_to_f32(h[t * d + k]) * (double)orc_bf16_to_f32(w[(int64_t)c * d + k]);
+            out[t * ORC_CH + c] = orc_f32_to_bf16((float)acc);
+        }
 }
 
 /* ------------------------------------------------------------------ */

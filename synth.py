@@ -26,7 +26,8 @@ import math
 import numpy as np
 
 ROLES = {"gain": 1, "kv": 2, "idx_k": 3, "q": 4, "q_idx": 5, "w": 6, "swa": 7, "lens": 8, "pages": 9, "burst": 10,
-         "tok": 11}
+         "tok": 11, "hidden": 12, "w_kv": 13}
+D_MODEL = 4096  # hidden size of the synthetic SWA replay (the pages give none)
 CHUNK = 4096  # rows per independently seeded chunk
 CH, IDD, H, D, IH = 256, 64, 16, 128, 4
 
@@ -107,6 +108,19 @@ def swa_rows(seed: int, layer: int, seq: int, n: int, g: np.ndarray | None = Non
     """SWA K|V rows [n, 256] bf16 bits of one layer."""
     g = gain(seed) if g is None else g
     return to_bf16_bits(_normal(rng(seed, "swa", layer, seq), (n, CH)) * g[None, :])
+
+
+def hidden_rows(seed: int, layer: int, seq: int, n: int, d: int = D_MODEL) -> np.ndarray:
+    """Synthetic hidden states [n, d] bf16 bits N(0,1) of a layer's window tokens
+    (the input of the SWA Bounded Replay)."""
+    return to_bf16_bits(_normal(rng(seed, "hidden", layer, seq), (n, d)))
+
+
+def kv_projection(seed: int, layer: int, d: int = D_MODEL) -> np.ndarray:
+    """Synthetic K|V projection [256, d] bf16 bits: N(0, 1/d) times the per-channel
+    gain, so the replayed rows have the SWA rows' distribution."""
+    g = gain(seed)
+    return to_bf16_bits(_normal(rng(seed, "w_kv", layer), (CH, d)) * (g[:, None] / np.float32(math.sqrt(d))))
 
 
 def ragged_lens(seed: int, B: int, lo: int, hi: int) -> np.ndarray:
