@@ -1,5 +1,6 @@
-// K6/K7: sparse attention over gathered FP4 main-KV entries plus the layer's
-// bf16 SWA window, merged by log-sum-exp.
+// K6: decode attention over gathered FP4 main-KV entries plus the layer's
+// bf16 SWA window, merged by log-sum-exp (prefill attention, K7, is in
+// prefill_attn.cu).
 //
 // Pages: "Como funciona" (e-cogni.com.br): a Reuse layer runs sparse attention
 // directly on the re-used Top-K indices; every layer keeps its own global Q and
@@ -7,22 +8,21 @@
 // (conexaotc.com.br, Causal Encoder-Decoder paragraph).  Merge of the two
 // branches by log-sum-exp: workload statement.
 //
-// Design (one "row" = one decode sequence or one prefill query, 16 heads that
-// share one K and one V):
+// Design (one row = one decode sequence, 16 heads that share one K and one V):
 //   * a cluster of 8 CTAs per row; CTA s takes selected keys [64s, 64s+64)
 //     (four warps of 16) and window keys [16s, 16s+16) (a fifth warp);
 //   * each warp gathers its 16 rows (144 B per FP4 entry: codes + scales, or
 //     512 B per bf16 window token) with cp.async, dequantises E2M1 x E4M3 to
 //     fp16 in registers (exact: <= 6 significant bits, magnitudes 2^-10..2688)
 //     straight into the mma.sync B fragments of S = Q K^T (m16n8k16, the 16
-//     heads are the M dimension), takes an exp2-domain softmax over its keys,
-//     and multiplies P (fp16) by V (fp16 tile in shared memory, ldmatrix.trans);
-//   * warps merge their (max, sum, O) in shared memory, CTAs of the cluster
-//     through distributed shared memory: CTA s writes heads 2s and 2s+1.
+//     heads are the M dimension), and writes V as an fp16 tile;
+//   * one softmax over the CTA's 80 keys (per-warp maxima and fp16 P in shared
+//     memory), then P V split by output dims over four warps;
+//   * the CTAs' partials go to the CTA that owns each head pair by st.async,
+//     counted on its mbarrier (details at decode_attn_kernel).
 // The work per row is ~5 MFLOP against 136 KiB of gathered bytes, so the kernel
 // is bound by gather latency and HBM/L2 bandwidth; mma.sync keeps the math off
 // the critical path.
-#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -36,7 +36,6 @@ constexpr int KPW = 16;        // keys per warp
 constexpr int FP4_ROW = 144;   // staged FP4 entry: 128 code bytes + 16 scale bytes
 constexpr int SWA_ROW = 528;   // staged bf16 token: 512 B + 16 B pad (bank spread)
 constexpr int VT_ROW = 272;    // fp16 V tile row: 256 B + 16 B pad
-constexpr int OACC_ROW = 132;  // fp32 merged O row (floats)
 
 // Shared-memory layout of the decode kernel (byte offsets, all 16-aligned).
 constexpr int DA_KEYS = 4 * KPW + KPW;   // 64 selected + 16 window keys per CTA
@@ -85,28 +84,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                  : "r"(addr));
 }
 
-// One 8-byte asynchronous store into a peer CTA's shared memory that counts
-// its bytes on that CTA's mbarrier (both addresses in the cluster window).
-__device__ __forceinline__ void st_async_f32x2(uint32_t addr, float a, float b, uint32_t mbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
-                 "f"(a), "f"(b), "r"(mbar)
-                 : "memory");
-}
-// Wait for a phase of this CTA's mbarrier whose bytes come from peer CTAs
-// (acquire at cluster scope); gives up after `limit` polls.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t it = 0; it < limit; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
 constexpr uint32_t kAttnWaitLimit = 1u << 22;
 
 // Decode attention.  A cluster of 8 CTAs per sequence; CTA s takes selected
@@ -447,488 +424,9 @@ __global__ void __launch_bounds__(ATT_THREADS) decode_attn_kernel(AttnArgs a) {
     }
 }
 
-// ============================================================================
-// Prefill attention, selected entries: one CTA per query, no cluster.  Four
-// warps each take 16 of the query's selected entries per chunk over 8 chunks
-// (512 entries).  Each warp runs its own double-buffered cp.async pipeline
-// (gather chunk c + 2 while computing chunk c), reads the query's Q as an fp16
-// tile through ldmatrix, and carries an online softmax (running max, sum and
-// O) across its chunks.  The merge folds in the window partial that
-// prefill_swa_kernel left in out / lse: the window branch is computed once per
-// 16 consecutive queries there, not per query here.
-// ============================================================================
-constexpr int PA_CHUNKS = 8;
-constexpr int PA_WARPS = 4;                 // entry warps; merge slot 4 holds the window partial
-constexpr int PA_THREADS = PA_WARPS * 32;
-constexpr size_t PA_STAGE = (size_t)PA_WARPS * KPW * FP4_ROW;
-constexpr size_t PA_OFF_VT = 2 * PA_STAGE;
-constexpr size_t PA_END_LOOP = PA_OFF_VT + (size_t)PA_WARPS * KPW * VT_ROW;
-constexpr size_t PA_END_OPART = (size_t)ATT_WARPS * kH * OACC_ROW * 4;  // merge partials reuse the ring
-constexpr int PA_QROW = 272;  // fp16 Q tile row: 256 B + 16 B pad (ldmatrix without bank conflicts)
-constexpr size_t PA_OFF_MS = align16(PA_END_LOOP > PA_END_OPART ? PA_END_LOOP : PA_END_OPART);
-constexpr size_t PA_OFF_LP = PA_OFF_MS + ATT_WARPS * kH * 4;
-constexpr size_t PA_OFF_Q = align16(PA_OFF_LP + ATT_WARPS * kH * 4);          // [16][136] fp16
-constexpr size_t PA_OFF_SLOT = align16(PA_OFF_Q + (size_t)kH * PA_QROW);       // [4 warps][8 chunks][16] int32
-constexpr size_t PA_SMEM = align16(PA_OFF_SLOT + 4 * PA_CHUNKS * KPW * 4);
-static_assert(PA_STAGE % 16 == 0 && PA_OFF_VT % 16 == 0, "prefill attention shared-memory layout");
-
-__global__ void __launch_bounds__(PA_THREADS, 3) prefill_attn_kernel(AttnArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int row = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    float* opart = reinterpret_cast<float*>(smem);
-    float* ms = reinterpret_cast<float*>(smem + PA_OFF_MS);
-    float* lpart = reinterpret_cast<float*>(smem + PA_OFF_LP);
-    uint8_t* qs = smem + PA_OFF_Q;
-    int32_t* s_slot = reinterpret_cast<int32_t*>(smem + PA_OFF_SLOT) + warp * PA_CHUNKS * KPW;
-    uint8_t* vt = smem + PA_OFF_VT + warp * KPW * VT_ROW;
-
-    pdl_wait();
-    pdl_trigger();
-    if (smem_u32(smem) & 15u) {  // uniform over the grid
-        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
-        return;
-    }
-    const int32_t L = a.seq_len_prefill;
-
-    // physical slots of the entry warps' keys, chunk c key r at s_slot[16 c + r]
-    if (lane < KPW) {
-        int32_t pos[PA_CHUNKS];
-#pragma unroll
-        for (int c = 0; c < PA_CHUNKS; ++c) {
-            const int kidx = c * 64 + warp * KPW + lane;
-            pos[c] = kidx < a.topk ? a.idx[(int64_t)row * a.topk + kidx] : -1;
-        }
-#pragma unroll
-        for (int c = 0; c < PA_CHUNKS; ++c) {
-            int32_t sl = -1;
-            if (pos[c] >= 0) {
-                if (pos[c] < L) sl = (int32_t)entry_slot(a.cache, a.page_shift, 0, pos[c], a.err);
-                else dev_error(a.err, CSA2_DEV_INDEX);
-            }
-            s_slot[c * KPW + lane] = sl;
-        }
-    }
-    __syncwarp();
-    auto stage_of = [&](int c) { return smem + (size_t)(c & 1) * PA_STAGE; };
-    auto gather = [&](int c) {  // chunk c of this warp into ring slot c & 1 (commits a group)
-        if (c < PA_CHUNKS) {
-            uint8_t* st = stage_of(c) + warp * KPW * FP4_ROW;
-#pragma unroll
-            for (int it = 0; it < (KPW * 9 + 31) / 32; ++it) {
-                const int q = lane + 32 * it;
-                const int r = min(q / 9, KPW - 1), ch = q % 9;
-                const int32_t sl = s_slot[c * KPW + r];
-                if (q < KPW * 9) {
-                    uint8_t* dst = st + r * FP4_ROW + ch * 16;
-                    if (sl >= 0) {
-                        if (ch < 8) cp_async16(dst, a.cache.codes + (int64_t)sl * kCodeBytes + ch * 16);
-                        else cp_async16(dst, a.cache.scales + (int64_t)sl * kScales);
-                    } else {
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-                    }
-                }
-            }
-        }
-        cp_async_commit();
-    };
-    gather(0);
-    gather(1);
-
-    // Q [16 heads][128] as an fp16 tile in shared memory (A operand via ldmatrix)
-    for (int i = tid; i < kH * kD / 8; i += PA_THREADS) {
-        const int h = i >> 4, c8 = i & 15;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)row * kH + h) * kD) + c8);
-        *reinterpret_cast<uint4*>(qs + h * PA_QROW + c8 * 16) =
-            make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
-    }
-    __syncthreads();
-    // lane address of the A fragment of k-step cc: matrix m = lane / 8 holds
-    // heads (m & 1) * 8 + (lane & 7), dims 16 cc + (m >> 1) * 8
-    const uint32_t qa_base = smem_u32(qs) + (((lane >> 3) & 1) * 8 + (lane & 7)) * PA_QROW + (lane >> 4) * 16;
-
-    const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    float m_run = -INFINITY, m_run8 = -INFINITY, l_run = 0.f, l_run8 = 0.f;
-    float O[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-
-    for (int c = 0; c < PA_CHUNKS; ++c) {
-        cp_async_wait<1>();
-        __syncwarp();
-        const uint8_t* st = stage_of(c) + warp * KPW * FP4_ROW;
-        // validity of the 16 keys of this chunk (same rule as the gather)
-        const uint32_t vmask = __ballot_sync(0xffffffffu, lane < KPW && s_slot[c * KPW + (lane & (KPW - 1))] >= 0);
-        // S = Q K^T one n8 tile (8 keys) at a time, B fragments dequantised
-        // straight from the staged rows; then the fp16 V tile [key][dim]
-        float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            uint32_t bk[8][2];
-            {
-                // the row's K codes (64 B) and K scales (8 B) in five vector loads
-                const uint8_t* r = st + (8 * j + g) * FP4_ROW;
-                uint32_t w[16];
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 x = *reinterpret_cast<const uint4*>(r + 16 * v);
-                    w[4 * v] = x.x;
-                    w[4 * v + 1] = x.y;
-                    w[4 * v + 2] = x.z;
-                    w[4 * v + 3] = x.w;
-                }
-                const uint2 scs = *reinterpret_cast<const uint2*>(r + 128);
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t sc = e4m3_to_h2((uint8_t)(((cc < 4 ? scs.x : scs.y) >> (8 * (cc & 3))) & 0xffu));
-                    bk[cc][0] = hmul2(e2m1_low_byte_to_h2(w[2 * cc] >> (8 * t)), sc);
-                    bk[cc][1] = hmul2(e2m1_low_byte_to_h2(w[2 * cc + 1] >> (8 * t)), sc);
-                }
-            }
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint32_t qa[4];
-                ldsm_x4(qa_base + cc * 32, qa[0], qa[1], qa[2], qa[3]);
-                mma16816(S[j], qa, bk[cc][0], bk[cc][1]);
-            }
-        }
-        {
-            const int key = lane >> 1, half = lane & 1;
-            uint32_t* dst = reinterpret_cast<uint32_t*>(vt + key * VT_ROW + half * 128);
-            {
-                // half a row of V: 32 code bytes and 4 scale bytes in three vector loads
-                const uint8_t* r = st + key * FP4_ROW;
-                const uint4 v0 = *reinterpret_cast<const uint4*>(r + 64 + 32 * half);
-                const uint4 v1 = *reinterpret_cast<const uint4*>(r + 64 + 32 * half + 16);
-                const uint32_t scw = *reinterpret_cast<const uint32_t*>(r + 128 + 8 + 4 * half);
-                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t sc = e4m3_to_h2((uint8_t)((scw >> (8 * (i >> 1))) & 0xffu));
-                    uint32_t h0, h1, h2, h3;
-                    e2m1x8_to_h2x4(w[i], h0, h1, h2, h3);
-                    *reinterpret_cast<uint4*>(dst + 4 * i) =
-                        make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
-                }
-            }
-        }
-        __syncwarp();      // the staged rows are no longer read; the V tile is written
-        gather(c + 2);     // refill this ring slot while the chunk is finished
-
-        // online softmax (log2 domain) over this chunk's keys
-        float cm = -INFINITY, cm8 = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const bool ok = (vmask >> (8 * j + 2 * t + e)) & 1u;
-                S[j][e] = ok ? S[j][e] * kScaleLog2 : -INFINITY;
-                S[j][2 + e] = ok ? S[j][2 + e] * kScaleLog2 : -INFINITY;
-                cm = fmaxf(cm, S[j][e]);
-                cm8 = fmaxf(cm8, S[j][2 + e]);
-            }
-        }
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
-        cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 1));
-        cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 2));
-        const float mn = fmaxf(m_run, cm), mn8 = fmaxf(m_run8, cm8);
-        const float f = m_run == -INFINITY ? 0.f : exp2f(m_run - mn);
-        const float f8 = m_run8 == -INFINITY ? 0.f : exp2f(m_run8 - mn8);
-        m_run = mn;
-        m_run8 = mn8;
-        float lg = 0.f, lg8 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                S[j][e] = mn == -INFINITY ? 0.f : exp2f(S[j][e] - mn);
-                S[j][2 + e] = mn8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - mn8);
-                lg += S[j][e];
-                lg8 += S[j][2 + e];
-            }
-        }
-        lg += __shfl_xor_sync(0xffffffffu, lg, 1);
-        lg += __shfl_xor_sync(0xffffffffu, lg, 2);
-        lg8 += __shfl_xor_sync(0xffffffffu, lg8, 1);
-        lg8 += __shfl_xor_sync(0xffffffffu, lg8, 2);
-        l_run = l_run * f + lg;
-        l_run8 = l_run8 * f8 + lg8;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            O[j][0] *= f;
-            O[j][1] *= f;
-            O[j][2] *= f8;
-            O[j][3] *= f8;
-        }
-        const uint32_t pa[4] = {f2_to_h2(S[0][0], S[0][1]), f2_to_h2(S[0][2], S[0][3]), f2_to_h2(S[1][0], S[1][1]),
-                                f2_to_h2(S[1][2], S[1][3])};
-        {
-            const int m = lane >> 3, r = lane & 7;
-            const uint32_t base = smem_u32(vt) + ((m & 1) * 8 + r) * VT_ROW + (m >> 1) * 16;
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(base + j * 16, b0, b1, b2, b3);
-                mma16816(O[j], pa, b0, b1);
-                mma16816(O[j + 1], pa, b2, b3);
-            }
-        }
-        __syncwarp();  // the V tile is read before the next chunk rewrites it
-    }
-    cp_async_wait<0>();
-
-    // ---- merge: the four warps and the window partial (slot 4) ---------------
-    if (t == 0) {
-        ms[warp * kH + g] = m_run;
-        ms[warp * kH + g + 8] = m_run8;
-    }
-    if (tid < kH) {  // window partial: out is normalised (sum 1 at max lse), log2 domain
-        const float l = a.lse[(int64_t)row * kH + tid];
-        ms[PA_WARPS * kH + tid] = l == -INFINITY ? -INFINITY : l * 1.4426950408889634f;
-    }
-    __syncthreads();  // every warp is past its loop: the ring may hold the partials
-    float Mg = -INFINITY, Mg8 = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < ATT_WARPS; ++w) {
-        Mg = fmaxf(Mg, ms[w * kH + g]);
-        Mg8 = fmaxf(Mg8, ms[w * kH + g + 8]);
-    }
-    const float fg = m_run == -INFINITY ? 0.f : exp2f(m_run - Mg);
-    const float fg8 = m_run8 == -INFINITY ? 0.f : exp2f(m_run8 - Mg8);
-    {
-        float* part = opart + warp * kH * OACC_ROW;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            *reinterpret_cast<float2*>(part + g * OACC_ROW + 8 * j + 2 * t) = make_float2(O[j][0] * fg, O[j][1] * fg);
-            *reinterpret_cast<float2*>(part + (g + 8) * OACC_ROW + 8 * j + 2 * t) =
-                make_float2(O[j][2] * fg8, O[j][3] * fg8);
-        }
-        if (t == 0) {
-            lpart[warp * kH + g] = l_run * fg;
-            lpart[warp * kH + g + 8] = l_run8 * fg8;
-        }
-    }
-    for (int i = tid; i < kH * kD / 4; i += PA_THREADS) {  // the window partial, rescaled the same way
-        const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < ATT_WARPS; ++w) M = fmaxf(M, ms[w * kH + h]);
-        const float m5 = ms[PA_WARPS * kH + h];
-        const float f5 = m5 == -INFINITY ? 0.f : exp2f(m5 - M);
-        const float4 v = *reinterpret_cast<const float4*>(a.out + ((int64_t)row * kH + h) * kD + d4);
-        *reinterpret_cast<float4*>(opart + PA_WARPS * kH * OACC_ROW + h * OACC_ROW + d4) =
-            make_float4(v.x * f5, v.y * f5, v.z * f5, v.w * f5);
-        if (d4 == 0) lpart[PA_WARPS * kH + h] = f5;
-    }
-    __syncthreads();
-    for (int i = tid; i < kH * kD / 4; i += PA_THREADS) {
-        const int h = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
-        float4 acc = *reinterpret_cast<const float4*>(opart + h * OACC_ROW + d4);
-        float den = lpart[h];
-#pragma unroll
-        for (int w = 1; w < ATT_WARPS; ++w) {
-            const float4 v = *reinterpret_cast<const float4*>(opart + w * kH * OACC_ROW + h * OACC_ROW + d4);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
-            den += lpart[w * kH + h];
-        }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        *reinterpret_cast<float4*>(a.out + ((int64_t)row * kH + h) * kD + d4) =
-            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        if (d4 == 0) {
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < ATT_WARPS; ++w) M = fmaxf(M, ms[w * kH + h]);
-            a.lse[(int64_t)row * kH + h] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
-        }
-    }
-}
-
-// ============================================================================
-// Prefill attention, window branch: a CTA takes 16 consecutive queries (one
-// warp each) and walks the union of their windows once, 16 tokens at a time,
-// so each bf16 window row is staged and converted once for all 16 queries
-// instead of once per query.  Every warp keeps its query's online softmax over
-// the window and writes the normalised partial (out) and its natural-log lse;
-// prefill_attn_kernel then merges the selected entries into them.
-// ============================================================================
-constexpr int PW_Q = 16;                  // queries per CTA, one warp each
-constexpr int PW_THREADS = PW_Q * 32;
-constexpr size_t PW_OFF_Q = 0;                                        // [16 q][16 h] rows of PA_QROW bytes (fp16)
-constexpr size_t PW_OFF_ST = PW_OFF_Q + (size_t)PW_Q * kH * PA_QROW;  // 2 x [16 rows][SWA_ROW]
-constexpr size_t PW_OFF_INFO = PW_OFF_ST + 2 * (size_t)KPW * SWA_ROW;  // lo[16], p[16]
-constexpr size_t PW_SMEM = PW_OFF_INFO + 2 * PW_Q * 4;
-static_assert(PW_OFF_ST % 16 == 0 && PW_OFF_INFO % 16 == 0, "window kernel shared-memory layout");
-
-__global__ void __launch_bounds__(PW_THREADS, 1) prefill_swa_kernel(AttnArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    int* s_lo = reinterpret_cast<int*>(smem + PW_OFF_INFO);
-    int* s_p = s_lo + PW_Q;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int t0 = blockIdx.x * PW_Q, row = t0 + warp;
-    pdl_wait();
-    pdl_trigger();
-    if (smem_u32(smem) & 15u) {  // uniform over the grid
-        if (tid == 0) dev_error(a.err, CSA2_DEV_ALIGN);
-        return;
-    }
-    // window [lo, p] of each query (empty: lo > p)
-    if (tid < PW_Q) {
-        int lo = 1, p = 0;
-        if (t0 + tid < a.rows) {
-            p = a.q_pos[t0 + tid];
-            lo = max(0, p - a.window + 1);
-            if (lo < a.swa_start) {  // the window's rows are not all in swa_kv
-                dev_error(a.err, CSA2_DEV_INDEX);
-                lo = p + 1;
-            }
-        }
-        s_lo[tid] = lo;
-        s_p[tid] = p;
-    }
-    // Q of the 16 queries, fp16, row (q, h)
-    for (int i = tid; i < PW_Q * kH * (kD / 8); i += PW_THREADS) {
-        const int r = i >> 4, c8 = i & 15, q = r / kH;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t0 + q < a.rows) v = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)t0 * kH + r) * kD) + c8);
-        *reinterpret_cast<uint4*>(smem + PW_OFF_Q + r * PA_QROW + c8 * 16) =
-            make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
-    }
-    __syncthreads();
-    int u0 = INT_MAX, u1 = -1;  // union of the non-empty windows
-    for (int q = 0; q < PW_Q; ++q)
-        if (s_lo[q] <= s_p[q]) {
-            u0 = min(u0, s_lo[q]);
-            u1 = max(u1, s_p[q]);
-        }
-    const int my_lo = s_lo[warp], my_p = s_p[warp];
-    const int nchunk = u1 >= u0 ? (u1 - u0 + KPW) / KPW : 0;
-    auto stage = [&](int c) { return smem + PW_OFF_ST + (size_t)(c & 1) * KPW * SWA_ROW; };
-    auto issue = [&](int c) {  // one 16-byte chunk per thread: 16 rows x 32 chunks
-        if (c < nchunk) {
-            const int r = tid >> 5, ch = tid & 31, k = u0 + c * KPW + r;
-            uint8_t* dst = stage(c) + r * SWA_ROW + ch * 16;
-            if (k <= u1) cp_async16(dst, a.swa + (int64_t)(k - a.swa_start) * kCh + ch * 8);
-            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
-        cp_async_commit();
-    };
-    issue(0);
-    issue(1);
-    const uint32_t qa_base = smem_u32(smem + PW_OFF_Q) +
-                             (warp * kH + ((lane >> 3) & 1) * 8 + (lane & 7)) * PA_QROW + (lane >> 4) * 16;
-    const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    float m_run = -INFINITY, m_run8 = -INFINITY, l_run = 0.f, l_run8 = 0.f;
-    float O[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-    for (int c = 0; c < nchunk; ++c) {
-        cp_async_wait<1>();
-        __syncthreads();  // chunk c is staged (bf16)
-        {
-            uint4* pv = reinterpret_cast<uint4*>(stage(c) + (tid >> 5) * SWA_ROW + (tid & 31) * 16);
-            const uint4 v = *pv;
-            *pv = make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
-        }
-        __syncthreads();  // chunk c is fp16
-        const int k0 = u0 + c * KPW;
-        if (k0 <= my_p && k0 + KPW - 1 >= my_lo) {  // the chunk meets this query's window
-            const uint8_t* st = stage(c);
-            float S[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t* r = reinterpret_cast<const uint32_t*>(st + (8 * j + g) * SWA_ROW);
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint32_t qa[4];
-                    ldsm_x4(qa_base + cc * 32, qa[0], qa[1], qa[2], qa[3]);
-                    mma16816(S[j], qa, r[8 * cc + t], r[8 * cc + 4 + t]);
-                }
-            }
-            float cm = -INFINITY, cm8 = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int k = k0 + 8 * j + 2 * t + e;
-                    const bool ok = k >= my_lo && k <= my_p;
-                    S[j][e] = ok ? S[j][e] * kScaleLog2 : -INFINITY;
-                    S[j][2 + e] = ok ? S[j][2 + e] * kScaleLog2 : -INFINITY;
-                    cm = fmaxf(cm, S[j][e]);
-                    cm8 = fmaxf(cm8, S[j][2 + e]);
-                }
-            }
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
-            cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 1));
-            cm8 = fmaxf(cm8, __shfl_xor_sync(0xffffffffu, cm8, 2));
-            const float mn = fmaxf(m_run, cm), mn8 = fmaxf(m_run8, cm8);
-            const float f = m_run == -INFINITY ? 0.f : exp2f(m_run - mn);
-            const float f8 = m_run8 == -INFINITY ? 0.f : exp2f(m_run8 - mn8);
-            m_run = mn;
-            m_run8 = mn8;
-            float lg = 0.f, lg8 = 0.f;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    S[j][e] = mn == -INFINITY ? 0.f : exp2f(S[j][e] - mn);
-                    S[j][2 + e] = mn8 == -INFINITY ? 0.f : exp2f(S[j][2 + e] - mn8);
-                    lg += S[j][e];
-                    lg8 += S[j][2 + e];
-                }
-            }
-            lg += __shfl_xor_sync(0xffffffffu, lg, 1);
-            lg += __shfl_xor_sync(0xffffffffu, lg, 2);
-            lg8 += __shfl_xor_sync(0xffffffffu, lg8, 1);
-            lg8 += __shfl_xor_sync(0xffffffffu, lg8, 2);
-            l_run = l_run * f + lg;
-            l_run8 = l_run8 * f8 + lg8;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                O[j][0] *= f;
-                O[j][1] *= f;
-                O[j][2] *= f8;
-                O[j][3] *= f8;
-            }
-            const uint32_t pa[4] = {f2_to_h2(S[0][0], S[0][1]), f2_to_h2(S[0][2], S[0][3]),
-                                    f2_to_h2(S[1][0], S[1][1]), f2_to_h2(S[1][2], S[1][3])};
-            const int m = lane >> 3, r = lane & 7;
-            const uint32_t base = smem_u32(st) + ((m & 1) * 8 + r) * SWA_ROW + 256 + (m >> 1) * 16;
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(base + j * 16, b0, b1, b2, b3);
-                mma16816(O[j], pa, b0, b1);
-                mma16816(O[j + 1], pa, b2, b3);
-            }
-        }
-        __syncthreads();  // every warp has read stage c & 1
-        issue(c + 2);
-    }
-    cp_async_wait<0>();
-    if (row >= a.rows) return;
-    // the window partial of heads g and g + 8: normalised O and natural-log lse
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f, inv8 = l_run8 > 0.f ? 1.f / l_run8 : 0.f;
-    float* o = a.out + (int64_t)row * kH * kD;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        *reinterpret_cast<float2*>(o + g * kD + 8 * j + 2 * t) = make_float2(O[j][0] * inv, O[j][1] * inv);
-        *reinterpret_cast<float2*>(o + (g + 8) * kD + 8 * j + 2 * t) = make_float2(O[j][2] * inv8, O[j][3] * inv8);
-    }
-    if (t == 0) {
-        a.lse[(int64_t)row * kH + g] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
-        a.lse[(int64_t)row * kH + g + 8] = l_run8 > 0.f ? (m_run8 + log2f(l_run8)) * 0.6931471805599453f : -INFINITY;
-    }
-}
-
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
     static bool init[64];
+    static int n_sm[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -937,26 +435,12 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
         e = cudaFuncSetAttribute((const void*)decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)DA_SMEM);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute((const void*)prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)PA_SMEM);
-        if (e != cudaSuccess) return e;
-        // several query CTAs per SM: ask for the largest shared-memory carveout
-        e = cudaFuncSetAttribute((const void*)prefill_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute((const void*)prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)PW_SMEM);
+        e = cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         init[dev] = true;
     }
     if (a.rows <= 0) return cudaSuccess;
-    if (a.q_pos) {  // prefill: the window branch per 16 queries, then the selected entries per query
-        LaunchCfg cw(dim3((unsigned)((a.rows + PW_Q - 1) / PW_Q)), dim3(PW_THREADS), PW_SMEM, stream);
-        e = cudaLaunchKernelEx(&cw.cfg, prefill_swa_kernel, a);
-        if (e != cudaSuccess) return e;
-        LaunchCfg c(dim3((unsigned)a.rows), dim3(PA_THREADS), PA_SMEM, stream);
-        return cudaLaunchKernelEx(&c.cfg, prefill_attn_kernel, a);
-    }
+    if (a.q_pos) return launch_prefill_attn_tc(a, n_sm[dev], stream);  // one persistent CTA per SM
     LaunchCfg c(dim3((unsigned)a.rows * ATT_SPLIT), dim3(ATT_THREADS), DA_SMEM, stream, ATT_SPLIT);
     return cudaLaunchKernelEx(&c.cfg, decode_attn_kernel, a);
 }

@@ -494,6 +494,14 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     uint32_t* bitmap = a.bitmap + (int64_t)b * (a.nblk_pad >> 5);
     uint64_t* bnd = a.bnd + (int64_t)b * a.nblk_pad;
     constexpr int U = kFlat ? 8 : 4;  // loads in flight per thread
+    // Block rows: each warp lists its boundary rows in shared memory (the
+    // finalize's bitmaps, unused until then) and the CTA reserves its range of
+    // the sequence's boundary list with one atomic, instead of one atomic per
+    // ballot on the sequence's counter.
+    constexpr int WCAP = K3_CHUNK / (K3_THREADS / 32);  // rows per warp and chunk
+    uint64_t* wlist = reinterpret_cast<uint64_t*>(smem) + wid * WCAP;
+    uint32_t wn = 0;
+    const unsigned lt = (1u << lane) - 1u;
     for (int32_t base = c0 + wid * 32; base < c1; base += U * K3_THREADS) {
         float v[U];
 #pragma unroll
@@ -519,15 +527,27 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
                 const uint32_t at = pos + __popc(mgt & ((1u << lane) - 1u));
                 if (((mgt >> lane) & 1u) && at < (uint32_t)kMaxTopk) a.abv[(int64_t)b * kMaxTopk + at] = j;
             }
-            if (meq) {
+            if (!kFlat) {
+                if ((meq >> lane) & 1u) wlist[wn + __popc(meq & lt)] = ((uint64_t)key << 32) | (uint64_t)j;
+                wn += __popc(meq);
+            } else if (meq) {
                 const int leader = __ffs(meq) - 1;
                 uint32_t pos = 0;
                 if (lane == leader) pos = atomicAdd(&a.bnd_cnt[b], (uint32_t)__popc(meq));
                 pos = __shfl_sync(0xffffffffu, pos, leader);
-                if ((meq >> lane) & 1u)
-                    bnd[pos + __popc(meq & ((1u << lane) - 1u))] = ((uint64_t)key << 32) | (uint64_t)j;
+                if ((meq >> lane) & 1u) bnd[pos + __popc(meq & lt)] = ((uint64_t)key << 32) | (uint64_t)j;
             }
         }
+    }
+    if (!kFlat) {  // one reservation per CTA, then each warp copies its list
+        uint32_t* ftmp = reinterpret_cast<uint32_t*>(smem) + 2 * K3_WORDS + 1024;
+        uint32_t n_cta;
+        const uint32_t woff = __shfl_sync(
+            0xffffffffu, block_excl_scan(lane == 0 ? wn : 0u, ftmp, &n_cta), 0);
+        if (threadIdx.x == 0) ftmp[63] = n_cta ? atomicAdd(&a.bnd_cnt[b], n_cta) : 0u;
+        __syncthreads();
+        const uint32_t at = ftmp[63] + woff;
+        for (uint32_t i = lane; i < wn; i += 32) bnd[at + i] = wlist[i];
     }
     __threadfence();
     __syncthreads();
@@ -553,12 +573,13 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     uint32_t* tie = gm ? a.tie + (int64_t)b * (a.nblk_pad >> 5) : sm_bm + K3_WORDS;
     const uint32_t n_bnd = __ldcg(&a.bnd_cnt[b]);
     const uint64_t* B = bnd;
-    if (n_bnd <= (uint32_t)K3_BND_CAP) {  // stage the boundary list (the common case)
-        load_words(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd), 2 * (int)n_bnd);
-        B = sbnd;
-    }
+    // stage the boundary list (the common case) and the row bitmap, every
+    // load of both in flight at once
+    const bool stage_bnd = n_bnd <= (uint32_t)K3_BND_CAP;
+    load_words2(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd),
+                stage_bnd ? 2 * (int)n_bnd : 0, bm, bitmap, gm ? 0 : nwords);
+    if (stage_bnd) B = sbnd;
     if (!gm) {
-        load_words(bm, bitmap, nwords);
         for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
     } else {  // 16-byte groups: a sequence's bitmaps are 1 KiB aligned, padded to 256 words
         for (int i = threadIdx.x; i < (nwords + 3) / 4; i += K3_THREADS)

@@ -108,6 +108,8 @@ struct AttnArgs {
 constexpr int kPreIdx = 1;
 constexpr int kPreHist = 2;
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+// Prefill attention on tcgen05 (prefill_attn.cu): a persistent kernel over at most n_ctas CTAs.
+cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int n_ctas, cudaStream_t stream);
 
 // Copies the FP4 rows of a decode index set into the staged cache (stage.cu).
 struct StageArgs {

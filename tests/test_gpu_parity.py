@@ -359,6 +359,43 @@ def test_prefill_scattered_queries(csa2, orc):
     assert ps.errors() == 0
 
 
+def test_prefill_early_queries(csa2, orc):
+    # queries from the first token on: windows shorter than 128 tokens, fewer
+    # than 512 visible entries (sets padded with -1), and more queries than
+    # the persistent attention kernel has CTAs, so every CTA reuses both of
+    # its query buffers several times
+    seed = 1003
+    tokens = 2400
+    n_ent = tokens // 2
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 1, 0, tokens)
+    idx_k = synth.idx_k_rows(seed, 1, 0, n_ent)
+    ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=777)
+    kvb = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+    codes, scales = orc.quant_rows(kvb, ratio=2)
+    q_pos = np.arange(0, tokens, 2, dtype=np.int32)
+    T = len(q_pos)
+    q_idx = synth.q_idx(seed, 1, 0, T)
+    w = synth.w_idx(seed, 1, 0, T)
+    d = csa2.default_desc(csa2.FULL, 2)
+    ws = _ws(csa2, T, n_ent, prefill=True)
+    out_idx = torch.empty((T, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q_idx), dev(w), dev(np.array([n_ent], np.int32)), out_idx, T,
+                      n_ent, ws, q_pos=dev(q_pos), err=ps.err)
+    want = orc.prefill_indexer(q_pos, 2, n_ent, idx_k, q_idx, w)
+    check_sets(out_idx.cpu().numpy(), want, "prefill indexer, early queries")
+    assert (want[0] == -1).all() and (want[-1] >= 0).all()
+    swa = synth.swa_rows(seed, 1, 0, tokens)
+    q = synth.q_heads(seed, 1, 0, T)
+    out = torch.empty((T, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_prefill(d, ps.cache, bits16(q), out_idx, dev(q_pos), bits16(swa), 0, n_ent, out, lse, T,
+                             err=ps.err)
+    ro, rl = orc.prefill_attn(q_pos, q, want, codes, scales, swa, 0)
+    check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, "prefill attention, early queries")
+    assert ps.errors() == 0
+
+
 def test_prefill_indexer_exact_fallback_on_ties(csa2, orc):
     # Entries 0..4999 share one indexer-K row, so their scores tie exactly.  A
     # query that sees more than 2048 of them has too many candidates at the

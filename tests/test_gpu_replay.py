@@ -1,8 +1,10 @@
 """SWA Bounded Replay on the GPU (tcgen05 projection) against the oracle: the
-replayed window rows within one bf16 ulp of the fp64 definition (the tensor
-core accumulates in fp32, in its own order), ring slots outside the window
-untouched, and the decode attention over the replayed window within max-abs
-2e-3 / rel-L2 1e-3 of the oracle's attention over its own replayed rows."""
+replayed window rows within the bound of their two bf16 roundings plus fp32
+accumulation over d_model products of the fp64 definition (the tensor core
+accumulates in fp32, in its own order; almost every row element is equal),
+ring slots outside the window untouched, and the decode attention over the
+replayed window within max-abs 2e-3 / rel-L2 1e-3 of the oracle's attention
+over the same rows."""
 import numpy as np
 import pytest
 import torch
@@ -46,15 +48,22 @@ def test_replay_rows_and_window_attention(csa2, orc, d_model):
         torch.cuda.synchronize()
     assert int(err.item()) == 0
     got = swa.cpu().numpy().view(np.uint16)
-    ref_rows = []
     for b, L in enumerate(lens):
         n = min(W, L)
         want = orc.swa_replay(h[b, :n], w_kv)
-        ref_rows.append(want)
         slots = (L - n + np.arange(n)) % W
+        # bound: the two roundings to bf16 (half an ulp each; an ulp is at most
+        # 2^-7 of the value, at the bottom of a binade) plus fp32 accumulation
+        # over d_model products, |err| <= d 2^-24 sum|h w|
+        hf = orc.bf16_to_f32(h[b, :n]).astype(np.float64)
+        wf = orc.bf16_to_f32(w_kv).astype(np.float64)
+        gf = orc.bf16_to_f32(got[b, slots]).astype(np.float64)
+        rf = orc.bf16_to_f32(want).astype(np.float64)
+        bound = 2.0 ** -7 * np.abs(rf) + 2.0 * d_model * 2.0 ** -24 * (np.abs(hf) @ np.abs(wf).T)
+        excess = np.abs(gf - rf) - bound
+        assert excess.max() <= 0, f"seq {b}: beyond the bound by {excess.max()}"
         u = _ulps(got[b, slots], want)
-        assert u.max() <= 1, f"seq {b}: {u.max()} ulps"
-        assert (u == 0).mean() > 0.97
+        assert (u == 0).mean() > 0.97 and (u <= 1).mean() > 0.999, f"seq {b}: {(u == 0).mean()}"
         untouched = np.setdiff1d(np.arange(W), slots)
         assert (got[b, untouched] == sentinel).all()
 
@@ -75,6 +84,9 @@ def test_replay_rows_and_window_attention(csa2, orc, d_model):
     assert ps.errors() == 0
     out, lse = out.cpu().numpy(), lse.cpu().numpy()
     for b, L in enumerate(lens):
+        # the oracle's attention over the very rows the kernel replayed (the
+        # rows themselves were checked against the oracle's replay above)
+        n = min(W, L)
         codes, scales = orc.quant_rows(synth.kv_rows(SEED, b, 0, L))
-        ro, rl = orc.attend(q[b], idx[b], codes, scales, ref_rows[b])
+        ro, rl = orc.attend(q[b], idx[b], codes, scales, got[b, (L - n + np.arange(n)) % W])
         check_attn(out[b], lse[b], ro, rl, f"replayed window, seq {b}")
