@@ -40,12 +40,14 @@ csa2_status check_cache(const csa2_kv_cache* c, bool need_idx, bool need_pooled)
 
 // Where p lives: 0 device (or managed) memory, 1 host memory mapped into the
 // device address space at p, -1 host memory the device cannot read in place.
-// The answer for the last pointer asked is kept, so repeated calls (and calls
-// under stream capture) do not query the driver again.
+// The answers for the last two pointers asked are kept, so repeated calls (and
+// calls under stream capture) do not query the driver again.
 int memory_kind(const void* p) {
-    static thread_local const void* last = nullptr;
-    static thread_local int last_kind = 0;
-    if (p == last) return last_kind;
+    static thread_local const void* last[2] = {nullptr, nullptr};
+    static thread_local int last_kind[2] = {0, 0};
+    static thread_local int next = 0;
+    for (int i = 0; i < 2; ++i)
+        if (p == last[i]) return last_kind[i];
     cudaPointerAttributes at{};
     int kind = 0;
     if (cudaPointerGetAttributes(&at, p) == cudaSuccess) {
@@ -54,8 +56,9 @@ int memory_kind(const void* p) {
     } else {
         (void)cudaGetLastError();
     }
-    last = p;
-    last_kind = kind;
+    last[next] = p;
+    last_kind[next] = kind;
+    next ^= 1;
     return kind;
 }
 
@@ -238,6 +241,7 @@ csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_
         !aligned(lse, 4))
         return CSA2_ERR_INVALID_ARG;
     if (err_word && !aligned(err_word, 4)) return CSA2_ERR_INVALID_ARG;
+    if ((cache->n_phys_pages << page_shift_of(*cache)) > INT32_MAX) return CSA2_ERR_UNSUPPORTED;  // int32 slots
     AttnArgs a{};
     a.cache = *cache;
     a.q = q;

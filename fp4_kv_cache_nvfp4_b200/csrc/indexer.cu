@@ -573,13 +573,12 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     uint32_t* tie = gm ? a.tie + (int64_t)b * (a.nblk_pad >> 5) : sm_bm + K3_WORDS;
     const uint32_t n_bnd = __ldcg(&a.bnd_cnt[b]);
     const uint64_t* B = bnd;
-    // stage the boundary list (the common case) and the row bitmap, every
-    // load of both in flight at once
-    const bool stage_bnd = n_bnd <= (uint32_t)K3_BND_CAP;
-    load_words2(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd),
-                stage_bnd ? 2 * (int)n_bnd : 0, bm, bitmap, gm ? 0 : nwords);
-    if (stage_bnd) B = sbnd;
+    if (n_bnd <= (uint32_t)K3_BND_CAP) {  // stage the boundary list (the common case)
+        load_words(reinterpret_cast<uint32_t*>(sbnd), reinterpret_cast<const uint32_t*>(bnd), 2 * (int)n_bnd);
+        B = sbnd;
+    }
     if (!gm) {
+        load_words(bm, bitmap, nwords);
         for (int i = threadIdx.x; i < nwords; i += K3_THREADS) tie[i] = 0;
     } else {  // 16-byte groups: a sequence's bitmaps are 1 KiB aligned, padded to 256 words
         for (int i = threadIdx.x; i < (nwords + 3) / 4; i += K3_THREADS)

@@ -26,19 +26,23 @@
 // 128): the next query of a prefill chunk adds one token, so one row is
 // converted instead of 128.  The softmax masks a window row whose token, the
 // one in [p - 127, p] congruent to the row, is before the window's start.
-//   warps 0-3   softmax and epilogue: thread = TMEM lane = key of a tile
-//               (S) and dim (O); per-head max and sum across the 4 warps
-//   warp 4      per query: the selected entries' physical slots, the window
-//               range, Q converted to fp16 in its swizzled tile
-//   warp 5      TMEM owner and MMA issue (one lane); order S(0), then S(j+1)
+//   warps 0-3   softmax: thread = TMEM lane = key of a tile (S) and dim (O);
+//               per-head max and sum across the 4 warps; the epilogue of
+//               query j - 1 runs after P of query j is out
+//   warp 4      TMEM owner and MMA issue (one lane); order S(0), then S(j+1)
 //               before O(j), so the softmax of query j overlaps the products
 //               of query j+1
-//   warps 6-13  operand producers: the window rows a query adds, then 8 FP4
-//               tiles per query (K of its 4 selected tiles, one query ahead,
-//               then V) into a 3-slot ring; each thread one half row per
-//               tile, the raw bytes of the next 4 tiles in flight in registers
-// Slots and windows rotate over three query buffers, Q, P and the 2 x 128
-// TMEM columns over two.
+//   warps 5-6   per query (alternating): the selected entries' physical
+//               slots, the window range, Q and the window rows the query
+//               adds, converted to fp16 in their swizzled tiles
+//   warps 7-14  converters: thread = one 16-byte quarter (32 channels) of two
+//               entries of a tile, read by plain loads (the four quarters of an
+//               entry's 64 K or V code bytes by four neighbouring lanes) one
+//               block of four tiles ahead of the block it converts, so 8 rows
+//               per thread are in flight; FP4 -> fp16 tile into a 3-slot ring.
+//               The 8 FP4 tiles of query j: its K, one query ahead, then its V.
+// TMEM holds four query buffers of 128 columns (S of 5 tiles at 0, O at 96),
+// Q and P^T two buffers each.
 #include <algorithm>
 #include <climits>
 
@@ -50,31 +54,33 @@ namespace csa2 {
 
 constexpr int PT_TILES = 5;                              // 4 selected tiles + the window
 constexpr int PT_NSLOT = 3;                              // operand ring slots
-constexpr int PT_NQB = 3;                                // slot-list / window buffers
-constexpr int PT_PREF = 4;                               // FP4 tiles whose raw bytes are in flight
+constexpr int PT_NQB = 4;                                // slot-list buffers
+constexpr int PT_NTB = 4;                                // TMEM query buffers
 constexpr uint32_t PT_HALF = 128 * 128;                  // one 64-dim half of a tile: 16 KiB
 constexpr uint32_t PT_TILE = 2 * PT_HALF;                // 32 KiB
 constexpr uint32_t PT_PTILE = 2 * 16 * 128;              // P^T of one tile: two 64-key halves x 16 heads x 128 B
-constexpr int PT_THREADS = 14 * 32;
-constexpr int PT_DQ0 = 6 * 32;                           // first producer thread
+constexpr int PT_W_MMA = 4, PT_W_SETUP = 5, PT_NSETUP = 3, PT_W_CONV = 8, PT_WARPS = 16;
+constexpr int PT_PTAB = 1024;                            // page-table entries kept in shared memory
+constexpr int PT_THREADS = PT_WARPS * 32;
 constexpr size_t PT_OFF_RING = 0;
 constexpr size_t PT_OFF_KW = PT_OFF_RING + (size_t)PT_NSLOT * PT_TILE;      // window K tile
 constexpr size_t PT_OFF_VW = PT_OFF_KW + PT_TILE;                           // window V tile
 constexpr size_t PT_OFF_P = PT_OFF_VW + PT_TILE;                            // [2][5][4 KiB]
 constexpr size_t PT_OFF_Q = PT_OFF_P + 2 * (size_t)PT_TILES * PT_PTILE;     // [2][2 halves][16][128 B]
 constexpr size_t PT_OFF_SLOT = PT_OFF_Q + 2 * 4096;                         // [3][512] int32
-constexpr size_t PT_OFF_WIN = PT_OFF_SLOT + (size_t)PT_NQB * 512 * 4;       // [3] (window start, query position)
-constexpr size_t PT_OFF_TAG = PT_OFF_WIN + 32;                              // [2][128] token of each window row
-constexpr size_t PT_OFF_RED = PT_OFF_TAG + 2 * 128 * 4;                     // [2][4 warps][16] floats
+constexpr size_t PT_OFF_PTAB = PT_OFF_SLOT + (size_t)PT_NQB * 512 * 4;      // [1024] the sequence's first pages
+constexpr size_t PT_OFF_WIN = PT_OFF_PTAB + (size_t)PT_PTAB * 4;            // [4] (window start, query position)
+constexpr size_t PT_OFF_RED = PT_OFF_WIN + 32;                              // [2][4 warps][16] floats
 constexpr size_t PT_OFF_BAR = PT_OFF_RED + 2 * 4 * 16 * 4;
-constexpr int PT_NBAR = 2 * PT_NSLOT + 2 * PT_NQB + 2 * 6 + 4;
+constexpr int PT_NBAR = 2 * PT_NSLOT + 2 * PT_NQB + 2 * 2 + 3 * PT_NTB + 2 + 2;
 constexpr size_t PT_OFF_MISC = PT_OFF_BAR + (size_t)PT_NBAR * 8;            // tmem base, timeout flag
 constexpr size_t PT_SMEM = PT_OFF_MISC + 16 + 1024;                         // + slack for the 1 KiB alignment
-static_assert(PT_OFF_KW % 1024 == 0 && PT_OFF_P % 1024 == 0 && PT_OFF_Q % 1024 == 0 && PT_OFF_BAR % 8 == 0,
+static_assert(PT_OFF_KW % 1024 == 0 && PT_OFF_P % 1024 == 0 && PT_OFF_Q % 1024 == 0 && PT_OFF_SLOT % 16 == 0 &&
+                  PT_OFF_BAR % 8 == 0,
               "K7 layout");
 static_assert(PT_SMEM <= 227 * 1024, "K7 shared memory");
 constexpr uint32_t kPtWaitLimit = 1u << 22;
-constexpr uint32_t PT_TMEM_COLS = 256;  // per query buffer: S of 5 tiles (80 columns) at 0, O (16) at 96
+constexpr uint32_t PT_TMEM_COLS = 128 * PT_NTB;
 
 // Shared-memory descriptor of an MN-major, 128-byte-swizzled operand: rows of
 // 128 B (64 M-elements of one K index), 8-row groups SBO = 1024 B apart along
@@ -93,36 +99,41 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t 
         : "memory");
 }
 
-// Raw bytes of one producer thread's half row of one FP4 tile.
-struct PtRaw {
-    uint4 c0, c1;  // 32 code bytes = 64 channels
-    uint32_t sc;   // their 4 scales
-    uint32_t ok;   // 0: the entry is absent (a zero row)
-};
+// 2^x (the hardware approximation; P is rounded to fp16 afterwards)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 8 dims (one 16-byte chunk ch of the 16 of a K or V row) of a bf16 window row
+// into row `row` of a window tile, as fp16
+__device__ __forceinline__ void win_store(uint8_t* tile, int row, int ch, uint4 x) {
+    *reinterpret_cast<uint4*>(tile + (size_t)(ch >> 3) * PT_HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
+        make_uint4(bf2_to_h2(x.x), bf2_to_h2(x.y), bf2_to_h2(x.z), bf2_to_h2(x.w));
+}
 
 __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PT_OFF_BAR);
-    uint64_t* full = bars;                       // [3] ring slot filled (8 producer warps)
+    uint64_t* full = bars;                       // [3] ring slot converted (8 converter warps)
     uint64_t* empty = full + PT_NSLOT;           // [3] ring slot read by the tensor core
-    uint64_t* slot_ready = empty + PT_NSLOT;     // [3] slots and window range of a query (warp 4)
-    uint64_t* slot_free = slot_ready + PT_NQB;   // [3] (8 producer warps + 4 softmax warps)
-    uint64_t* q_ready = slot_free + PT_NQB;      // [2] Q tile written (warp 4)
+    uint64_t* slot_ready = empty + PT_NSLOT;     // [4] slots and window range of a query (setup warp)
+    uint64_t* slot_free = slot_ready + PT_NQB;   // [4] (8 converter warps + 4 softmax warps)
+    uint64_t* q_ready = slot_free + PT_NQB;      // [2] Q tile and the query's window K rows written
     uint64_t* q_free = q_ready + 2;              // [2] Q tile read (MMA commit)
-    uint64_t* s_full = q_free + 2;               // [2] S complete (MMA commit)
-    uint64_t* p_ready = s_full + 2;              // [2] P^T written (4 softmax warps)
-    uint64_t* o_full = p_ready + 2;              // [2] O complete (MMA commit)
-    uint64_t* tmem_free = o_full + 2;            // [2] S and O read (4 softmax warps)
-    uint64_t* kw_ready = tmem_free + 2;          // window K rows of the next query written (8 warps)
-    uint64_t* kw_done = kw_ready + 1;            // window K tile read (MMA commit)
-    uint64_t* vw_ready = kw_done + 1;
-    uint64_t* vw_done = vw_ready + 1;
+    uint64_t* s_full = q_free + 2;               // [4] S complete (MMA commit)
+    uint64_t* o_full = s_full + PT_NTB;          // [4] O complete (MMA commit)
+    uint64_t* tmem_free = o_full + PT_NTB;       // [4] S and O read (4 softmax warps)
+    uint64_t* p_ready = tmem_free + PT_NTB;      // [2] P^T written (4 softmax warps)
+    uint64_t* vw_ready = p_ready + 2;            // window V rows of a query written (setup warp)
+    uint64_t* mma_done = vw_ready + 1;           // every product complete
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + PT_OFF_MISC);
-    int* s_timeout = reinterpret_cast<int*>(smem + PT_OFF_MISC + 4);
+    volatile int* s_timeout = reinterpret_cast<volatile int*>(smem + PT_OFF_MISC + 4);
     int32_t* s_slot = reinterpret_cast<int32_t*>(smem + PT_OFF_SLOT);
     int2* s_win = reinterpret_cast<int2*>(smem + PT_OFF_WIN);
-    int32_t* s_tag = reinterpret_cast<int32_t*>(smem + PT_OFF_TAG);  // [0..127] K rows, [128..255] V rows
+    int32_t* s_ptab = reinterpret_cast<int32_t*>(smem + PT_OFF_PTAB);
     float* s_red = reinterpret_cast<float*>(smem + PT_OFF_RED);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     // this CTA's contiguous range of queries
@@ -141,25 +152,24 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
         for (int b = 0; b < 2; ++b) {
             mbar_init(&q_ready[b], 1);
             mbar_init(&q_free[b], 1);
+        }
+        for (int b = 0; b < PT_NTB; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_ready[b], 4);
             mbar_init(&o_full[b], 1);
             mbar_init(&tmem_free[b], 4);
         }
-        mbar_init(kw_ready, 8);
-        mbar_init(kw_done, 1);
-        mbar_init(vw_ready, 8);
-        mbar_init(vw_done, 1);
+        mbar_init(&p_ready[0], 4);
+        mbar_init(&p_ready[1], 4);
+        mbar_init(vw_ready, 1);
+        mbar_init(mma_done, 1);
         *s_timeout = 0;
         fence_mbar_init();
     }
     // window tiles start as zeros (a masked row still meets P = 0 in P V, so it
-    // must hold a finite value) with no token in any row
+    // must hold a finite value)
     for (int i = tid; i < 2 * (int)PT_TILE / 16; i += PT_THREADS)
         reinterpret_cast<uint4*>(smem + PT_OFF_KW)[i] = make_uint4(0, 0, 0, 0);
-    for (int i = tid; i < 256; i += PT_THREADS) s_tag[i] = INT32_MIN;
-    fence_proxy_async_smem();
-    if (wid == 5) {
+    if (wid == PT_W_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                      "r"(PT_TMEM_COLS)
                      : "memory");
@@ -172,75 +182,52 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
     pdl_wait();
     pdl_trigger();
     const int32_t L = a.seq_len_prefill;
-    auto timeout = [&]() { *s_timeout = 1; };
-
-    if (wid == 4) {
-        // ============ slots, window range and Q of each query ============
-        for (int j = 0; j < nq; ++j) {
-            const int q = q0 + j, sb = j % PT_NQB, qb = j & 1;
-            if (j >= PT_NQB && !mbar_wait(&slot_free[sb], (uint32_t)((j - PT_NQB) / PT_NQB) & 1u, kPtWaitLimit))
-                timeout();
-            if (j >= 2 && !mbar_wait(&q_free[qb], (uint32_t)((j - 2) >> 1) & 1u, kPtWaitLimit)) timeout();
-            int32_t* sl = s_slot + sb * 512;
-            for (int k = lane; k < 512; k += 32) {
-                int32_t slot = -1;
-                const int32_t pos = k < a.topk ? a.idx[(int64_t)q * a.topk + k] : -1;
-                if (pos >= 0) {
-                    if (pos < L) slot = (int32_t)entry_slot(a.cache, a.page_shift, 0, pos, a.err);
-                    else dev_error(a.err, CSA2_DEV_INDEX);
-                }
-                sl[k] = slot;
-            }
-            if (lane == 0) {
-                const int p = a.q_pos[q];
-                int lo = max(0, p - a.window + 1);
-                if (lo < a.swa_start) {  // the window's rows are not all in swa_kv: no window
-                    dev_error(a.err, CSA2_DEV_INDEX);
-                    lo = p + 1;
-                }
-                s_win[sb] = make_int2(lo, p);
-            }
-            // Q: 16 heads x 128 dims, fp16, half h of the dims at +2 KiB, head rows of 128 B
-            uint8_t* qt = smem + PT_OFF_Q + (size_t)qb * 4096;
-            for (int i = lane; i < 16 * 16; i += 32) {
-                const int h = i >> 4, c8 = i & 15, half = c8 >> 3, c = c8 & 7;
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)q * kH + h) * kD) + c8);
-                *reinterpret_cast<uint4*>(qt + half * 2048 + h * 128 + ((c ^ (h & 7)) << 4)) =
-                    make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
-            }
-            fence_proxy_async_smem();  // Q is read by the tensor core
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&slot_ready[sb]);
-                mbar_arrive(&q_ready[qb]);
-            }
+    // window of a query: tokens [lo, p] (lo = p + 1: none, when its rows are not all in swa_kv)
+    auto window_of = [&](int q) -> int2 {
+        const int p = __ldg(a.q_pos + q);
+        const int lo = max(0, p - a.window + 1);
+        return make_int2(lo < a.swa_start ? p + 1 : lo, p);
+    };
+    // the sequence's first pages (its whole table, when it fits)
+    const int n_ptab = min(a.cache.max_pages_per_seq, PT_PTAB);
+    for (int i = tid; i < n_ptab; i += PT_THREADS) s_ptab[i] = __ldg(a.cache.page_table + i);
+    // every row of the first query's window (later queries add their new tokens)
+    if (nq > 0) {
+        const int2 w0 = window_of(q0);
+        for (int c = tid; c < (w0.y - w0.x + 1) * 32; c += PT_THREADS) {
+            const int tok = w0.x + (c >> 5), ch = c & 31;
+            const uint4 x = __ldg(reinterpret_cast<const uint4*>(a.swa + (int64_t)(tok - a.swa_start) * kCh) + ch);
+            win_store(smem + (ch < 16 ? PT_OFF_KW : PT_OFF_VW), tok & 127, ch & 15, x);
         }
-    } else if (wid == 5) {
+    }
+    fence_proxy_async_smem();  // the rows are read by the tensor core
+    __syncthreads();
+    auto wait = [&](uint64_t* bar, uint32_t parity) {  // bounded; after one timeout every wait returns at once
+        if (*s_timeout) return;
+        if (!mbar_wait(bar, parity, kPtWaitLimit)) *s_timeout = 1;
+    };
+
+    if (wid == PT_W_MMA) {
         // ================= MMA issue: S(0), then S(j + 1) before O(j) =================
-        if (lane == 0) {
+        if (lane == 0 && nq > 0) {
             uint32_t pos = 0;  // ring position
-            auto ring_wait = [&](int& s) {
-                s = (int)(pos % PT_NSLOT);
-                if (!mbar_wait(&full[s], (pos / PT_NSLOT) & 1u, kPtWaitLimit)) timeout();
-                tc_fence_after();
-            };
             auto mma_s = [&](int j) {  // S^T(j) = K^ Q^T over the 4 selected tiles and the window tile
-                const int qb = j & 1;
-                const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-                if (!mbar_wait(&q_ready[qb], ph, kPtWaitLimit)) timeout();
-                if (j >= 2 && !mbar_wait(&tmem_free[qb], ph ^ 1u, kPtWaitLimit)) timeout();
-                const uint32_t tS = tmem + (uint32_t)qb * 128u;
+                const int qb = j & 1, tb = j & (PT_NTB - 1);
+                wait(&q_ready[qb], (uint32_t)(j >> 1) & 1u);
+                if (j >= PT_NTB) wait(&tmem_free[tb], (uint32_t)((j / PT_NTB) - 1) & 1u);
+                tc_fence_after();
+                const uint32_t tS = tmem + (uint32_t)tb * 128u;
                 const uint32_t qaddr = smem_u32(smem + PT_OFF_Q + (size_t)qb * 4096);
                 for (int t = 0; t < PT_TILES; ++t) {
                     uint32_t ka;
                     int s = -1;
                     if (t < 4) {
-                        ring_wait(s);
+                        s = (int)(pos % PT_NSLOT);
+                        wait(&full[s], (pos / PT_NSLOT) & 1u);
+                        tc_fence_after();
                         ka = smem_u32(smem + PT_OFF_RING + (size_t)s * PT_TILE);
                     } else {
-                        if (!mbar_wait(kw_ready, (uint32_t)j & 1u, kPtWaitLimit)) timeout();
-                        tc_fence_after();
-                        ka = smem_u32(smem + PT_OFF_KW);
+                        ka = smem_u32(smem + PT_OFF_KW);  // written with Q (q_ready)
                     }
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {  // 16 dims per step; dims 64.. in the second half
@@ -254,27 +241,26 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                     }
                 }
                 umma_commit(&q_free[qb]);
-                umma_commit(kw_done);
-                umma_commit(&s_full[qb]);
+                umma_commit(&s_full[tb]);
             };
-            auto mma_o = [&](int j) {  // O^T(j) += V^T P^T over the 4 selected tiles and the window tile
-                const int qb = j & 1;
-                const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-                if (!mbar_wait(&p_ready[qb], ph, kPtWaitLimit)) timeout();
+            auto mma_o = [&](int j) {  // O^T(j) = V^T P^T over the 4 selected tiles and the window tile
+                const int tb = j & (PT_NTB - 1);
+                wait(&p_ready[j & 1], (uint32_t)(j >> 1) & 1u);
+                wait(vw_ready, (uint32_t)j & 1u);
                 tc_fence_after();
-                const uint32_t tO = tmem + (uint32_t)qb * 128u + 96u;
+                const uint32_t tO = tmem + (uint32_t)tb * 128u + 96u;
                 for (int t = 0; t < PT_TILES; ++t) {
                     uint32_t va;
                     int s = -1;
                     if (t < 4) {
-                        ring_wait(s);
+                        s = (int)(pos % PT_NSLOT);
+                        wait(&full[s], (pos / PT_NSLOT) & 1u);
+                        tc_fence_after();
                         va = smem_u32(smem + PT_OFF_RING + (size_t)s * PT_TILE);
                     } else {
-                        if (!mbar_wait(vw_ready, (uint32_t)j & 1u, kPtWaitLimit)) timeout();
-                        tc_fence_after();
                         va = smem_u32(smem + PT_OFF_VW);
                     }
-                    const uint32_t pa = smem_u32(smem + PT_OFF_P + ((size_t)qb * PT_TILES + t) * PT_PTILE);
+                    const uint32_t pa = smem_u32(smem + PT_OFF_P + ((size_t)(j & 1) * PT_TILES + t) * PT_PTILE);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step: two 8-key groups of 1024 B
                         const uint64_t da = umma_desc_sw128_mn(va + (uint32_t)ks * 2048u, PT_HALF);
@@ -286,142 +272,242 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                         ++pos;
                     }
                 }
-                umma_commit(vw_done);
-                umma_commit(&o_full[qb]);
+                umma_commit(&o_full[tb]);
             };
-            if (nq > 0) mma_s(0);
+            mma_s(0);
             for (int j = 0; j < nq; ++j) {
                 if (j + 1 < nq) mma_s(j + 1);
                 mma_o(j);
             }
+            umma_commit(mma_done);
+            wait(mma_done, 0u);
         }
         __syncwarp();
-    } else if (wid >= 6) {
-        // ============ operand producers ============
-        // Tile jobs in ring order: K of query 0, then per query j the K of
-        // query j + 1 and the V of query j; job n < 4: K(0) tile n; job
-        // 4 + 8 j + r: K(j + 1) tile r (r < 4, absent for the last query) or
-        // V(j) tile r - 4.
-        const int dt = tid - PT_DQ0, key = dt >> 1, h = dt & 1;
-        const int nend = 8 * nq + 4;
-        auto job_of = [&](int n, int& j, int& v, int& t) -> bool {
-            if (n < 4) {
-                j = 0, v = 0, t = n;
-                return nq > 0;
+    } else if (wid >= PT_W_SETUP && wid < PT_W_SETUP + PT_NSETUP) {
+        // ======= per query (three warps in turn): slots, window range, Q, new window rows =======
+        // physical slot of an entry (pos >= 0), the page from the cached table when it is there
+        auto slot_of = [&](int32_t pos) -> int32_t {
+            const int32_t pg = pos >> a.page_shift;
+            if (pg >= n_ptab) return (int32_t)entry_slot(a.cache, a.page_shift, 0, pos, a.err);
+            const int32_t phys = s_ptab[pg];
+            if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                dev_error(a.err, CSA2_DEV_PAGE);
+                return -1;
             }
-            const int m = n - 4, jj = m >> 3, r = m & 7;
-            if (r < 4) {
-                j = jj + 1, v = 0, t = r;
-                return jj + 1 < nq;
-            }
-            j = jj, v = 1, t = r - 4;
-            return jj < nq;
+            return (phys << a.page_shift) | (pos & ((1 << a.page_shift) - 1));
         };
-        int seen = -1;  // last query whose slot list the prefetch waited for
-        auto fetch = [&](int n, PtRaw& r) {  // raw bytes of job n (any n; absent jobs give a zero row)
-            int j, v, t;
-            r.ok = 0u;
-            if (n >= nend || !job_of(n, j, v, t)) return;
+        for (int j = wid - PT_W_SETUP; j < nq; j += PT_NSETUP) {
+            const int q = q0 + j, b = j % PT_NQB, qb = j & 1;
+            const int2 win = window_of(q);
+            // the tokens of this window that the previous query's window lacks:
+            // [win.x, min(win.y, prev.x - 1)] and [max(win.x, prev.y + 1), win.y]
+            // (an empty window is [p + 1, p]; the first query's was written whole)
+            const int2 prev = j == 0 ? win : window_of(q - 1);
+            const int a0 = win.x, a1 = min(win.y, prev.x - 1), b0 = max(win.x, prev.y + 1), b1 = win.y;
+            const int n1 = max(0, a1 - a0 + 1), n_new = n1 + max(0, b1 - b0 + 1);
+            auto new_tok = [&](int k) { return k < n1 ? a0 + k : b0 + (k - n1); };
+            // every global load of the query in flight at once
+            int32_t pos[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int k = lane + 32 * i;
+                pos[i] = k < a.topk ? __ldg(a.idx + (int64_t)q * a.topk + k) : -1;
+            }
+            uint4 qv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qv[i] = __ldg(reinterpret_cast<const uint4*>(a.q + (int64_t)q * kH * kD) + lane + 32 * i);
+            uint4 wx = make_uint4(0, 0, 0, 0);  // chunk `lane` of the first new token's row (K: lanes < 16)
+            if (n_new > 0)
+                wx = __ldg(reinterpret_cast<const uint4*>(a.swa + (int64_t)(new_tok(0) - a.swa_start) * kCh) + lane);
+            if (j >= PT_NQB) wait(&slot_free[b], (uint32_t)((j / PT_NQB) - 1) & 1u);
+            int32_t* sl = s_slot + b * 512;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                int32_t slot = -1;
+                if (pos[i] >= 0) {
+                    if (pos[i] < L) slot = slot_of(pos[i]);
+                    else dev_error(a.err, CSA2_DEV_INDEX);
+                }
+                sl[lane + 32 * i] = slot;
+            }
+            if (lane == 0) {
+                if (win.x > win.y) dev_error(a.err, CSA2_DEV_INDEX);  // the window's rows are not all in swa_kv
+                s_win[b] = win;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&slot_ready[b]);
+            // Q: 16 heads x 128 dims, fp16, half h of the dims at +2 KiB, head rows of 128 B
+            if (j >= 2) wait(&q_free[qb], (uint32_t)((j >> 1) - 1) & 1u);
+            uint8_t* qt = smem + PT_OFF_Q + (size_t)qb * 4096;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane + 32 * i, h = e >> 4, c8 = e & 15, half = c8 >> 3, c = c8 & 7;
+                *reinterpret_cast<uint4*>(qt + half * 2048 + h * 128 + ((c ^ (h & 7)) << 4)) =
+                    make_uint4(bf2_to_h2(qv[i].x), bf2_to_h2(qv[i].y), bf2_to_h2(qv[i].z), bf2_to_h2(qv[i].w));
+            }
+            // the new K rows, once the previous query's S has read the window tile.
+            // The per-query barriers of the TMEM buffers say so without aliasing:
+            // the two setup warps take turns, so a barrier completed once per
+            // query may be two phases behind this warp's last wait on it.
+            if (j >= 1) wait(&s_full[(j - 1) & (PT_NTB - 1)], (uint32_t)((j - 1) / PT_NTB) & 1u);
+            for (int k = 0; k < n_new; ++k) {
+                const int tok = new_tok(k);
+                const uint4 x = k == 0 ? wx
+                                       : __ldg(reinterpret_cast<const uint4*>(a.swa + (int64_t)(tok - a.swa_start) * kCh) +
+                                               lane);
+                if (lane < 16) win_store(smem + PT_OFF_KW, tok & 127, lane, x);  // V chunks: below
+            }
+            fence_proxy_async_smem();  // Q and the rows are read by the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_ready[qb]);
+            // the new V rows, once the previous query's O has read the window tile
+            if (j >= 1) wait(&o_full[(j - 1) & (PT_NTB - 1)], (uint32_t)((j - 1) / PT_NTB) & 1u);
+            for (int k = 0; k < n_new; ++k) {
+                const int tok = new_tok(k);
+                const uint4 x = k == 0 ? wx
+                                       : __ldg(reinterpret_cast<const uint4*>(a.swa + (int64_t)(tok - a.swa_start) * kCh) +
+                                               lane);
+                if (lane >= 16) win_store(smem + PT_OFF_VW, tok & 127, lane - 16, x);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(vw_ready);
+        }
+    } else if (wid >= PT_W_CONV) {
+        // ============ converters: FP4 rows -> fp16 operand tiles ============
+        // Thread ct owns quarter qt (channels 32 qt .. 32 qt + 31 of K or V) of
+        // entries e0 = ct / 4 and e0 + 64 of every tile.  The tiles come in blocks
+        // of four (one query's K or V): K(0), then K(j + 1), V(j) for each j.
+        // Block b + 1's rows are loaded while block b is converted.
+        const int ct = tid - PT_W_CONV * 32, qt = ct & 3, hq = qt >> 1, cq = (qt & 1) * 4, e0 = ct >> 2;
+        const int nb = 2 * nq;
+        auto block_of = [&](int b, int& j, int& v) {
+            if (b == 0) {
+                j = 0, v = 0;
+                return;
+            }
+            const int i = b - 1, p = i >> 1;
+            if (p == nq - 1) j = nq - 1, v = 1;
+            else if (i & 1) j = p, v = 1;
+            else j = p + 1, v = 0;
+        };
+        struct Rows {
+            uint4 c[2];     // 16 code bytes of each of the two entries (zeros: absent)
+            uint32_t s[2];  // word qt of each entry's 16 scale bytes (K's 8, then V's)
+        };
+        // The scale words of a query's K block serve its V block too: lanes 2, 3
+        // of an entry's four hold V's scales.  Kept per query parity (V(j) follows K(j + 1)).
+        uint32_t sv0[8], sv1[8];
+        int seen = -1;  // last query whose slot list was waited for
+        auto fetch_block = [&](int b, Rows (&R)[4]) {
+            int j, v;
+            block_of(b, j, v);
             if (j > seen) {
-                if (!mbar_wait(&slot_ready[j % PT_NQB], (uint32_t)(j / PT_NQB) & 1u, kPtWaitLimit)) timeout();
+                wait(&slot_ready[j % PT_NQB], (uint32_t)(j / PT_NQB) & 1u);
                 seen = j;
             }
-            const int32_t slot = s_slot[(j % PT_NQB) * 512 + t * 128 + key];
-            if (slot < 0) return;
-            const uint4* cp = reinterpret_cast<const uint4*>(a.cache.codes + (int64_t)slot * kCodeBytes + (v ? 64 : 0) +
-                                                              32 * h);
-            r.c0 = __ldg(cp);
-            r.c1 = __ldg(cp + 1);
-            r.sc = __ldg(reinterpret_cast<const uint32_t*>(a.cache.scales + (int64_t)slot * kScales + (v ? 8 : 0) +
-                                                           4 * h));
-            r.ok = 1u;
-        };
-        // the window rows query j adds to tile K (v = 0) or V (v = 1): rows of
-        // tokens in [lo, p] whose tag differs; 16 threads per row, 8 dims each
-        const GroupBar pb{2, 256};
-        auto window_rows = [&](int j, int v) {
-            const int2 win = s_win[j % PT_NQB];
-            int32_t* tag = s_tag + v * 128;
-            uint8_t* tile = smem + (v ? PT_OFF_VW : PT_OFF_KW);
-            const int n = win.y - win.x + 1;  // tokens in the window (<= 128; 0: none)
-            for (int c = dt; c < n * 16; c += 256) {
-                const int tok = win.x + (c >> 4), ch = c & 15, row = tok & 127;
-                if (tag[row] == tok) continue;
-                const uint4 x = __ldg(reinterpret_cast<const uint4*>(a.swa + (int64_t)(tok - a.swa_start) * kCh +
-                                                                      (v ? 128 : 0)) + ch);
-                *reinterpret_cast<uint4*>(tile + (size_t)(ch >> 3) * PT_HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
-                    make_uint4(bf2_to_h2(x.x), bf2_to_h2(x.y), bf2_to_h2(x.z), bf2_to_h2(x.w));
-            }
-            pb.sync();  // every thread has read the tags
-            for (int c = dt; c < n; c += 256) tag[(win.x + c) & 127] = win.x + c;
-            fence_proxy_async_smem();  // the rows are read by the tensor core
-            pb.sync();
-            if (lane == 0) mbar_arrive(v ? vw_ready : kw_ready);
-        };
-        PtRaw r0, r1, r2, r3;  // raw bytes of jobs n .. n + 3
-        int n = 0;
-        while (n < nend) {  // skip absent jobs at the front
-            int j, v, t;
-            if (job_of(n, j, v, t)) break;
-            ++n;
-        }
-        fetch(n, r0);
-        fetch(n + 1, r1);
-        fetch(n + 2, r2);
-        fetch(n + 3, r3);
-        uint32_t pos = 0;  // ring position
-        for (; n < nend; ++n) {
-            int j, v, t;
-            if (!job_of(n, j, v, t)) {  // an absent job: its prefetched bytes move down
-                r0 = r1, r1 = r2, r2 = r3;
-                fetch(n + 4, r3);
-                continue;
-            }
-            if (t == 0) {  // the window rows of this query, before its first tile of the kind
-                if (j >= 1 && !mbar_wait(v ? vw_done : kw_done, (uint32_t)(j - 1) & 1u, kPtWaitLimit)) timeout();
-                window_rows(j, v);
-            }
-            const int s = (int)(pos % PT_NSLOT);
-            if (pos >= PT_NSLOT && !mbar_wait(&empty[s], ((pos / PT_NSLOT) - 1) & 1u, kPtWaitLimit)) timeout();
-            uint8_t* dst = smem + PT_OFF_RING + (size_t)s * PT_TILE + (size_t)h * PT_HALF + key * 128;
-            const uint32_t words[8] = {r0.c0.x, r0.c0.y, r0.c0.z, r0.c0.w, r0.c1.x, r0.c1.y, r0.c1.z, r0.c1.w};
+            const int32_t* sl = s_slot + (j % PT_NQB) * 512 + e0;
+            int32_t slot[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {  // 8 channels per chunk, scale (c / 2) of the four
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (r0.ok) {
-                    const uint32_t sc = e4m3_to_h2((uint8_t)((r0.sc >> (8 * (c >> 1))) & 0xffu));
-                    uint32_t h0, h1, h2, h3;
-                    e2m1x8_to_h2x4(words[c], h0, h1, h2, h3);
-                    o = make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
+            for (int i = 0; i < 8; ++i) slot[i] = sl[(i >> 1) * 128 + (i & 1) * 64];
+            if (v == 1) {  // query j's slot list is read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&slot_free[j % PT_NQB]);
+            }
+            const uint8_t* cbase = a.cache.codes + v * 64 + qt * 16;
+            const uint8_t* sbase = a.cache.scales + qt * 4;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint4 c = make_uint4(0u, 0u, 0u, 0u);
+                if (slot[i] >= 0) c = __ldg(reinterpret_cast<const uint4*>(cbase + (int64_t)slot[i] * kCodeBytes));
+                R[i >> 1].c[i & 1] = c;
+                if (v == 0) {
+                    uint32_t w = 0u;
+                    if (slot[i] >= 0) w = __ldg(reinterpret_cast<const uint32_t*>(sbase + (int64_t)slot[i] * kScales));
+                    R[i >> 1].s[i & 1] = w;
+                    if (j & 1) sv1[i] = w;
+                    else sv0[i] = w;
+                } else {
+                    R[i >> 1].s[i & 1] = (j & 1) ? sv1[i] : sv0[i];
                 }
-                *reinterpret_cast<uint4*>(dst + ((c ^ (key & 7)) << 4)) = o;
+            }
+        };
+        auto convert_tile = [&](int m, int v, const Rows& R) {
+            const int s = m % PT_NSLOT;
+            if (m >= PT_NSLOT) wait(&empty[s], (uint32_t)((m / PT_NSLOT) - 1) & 1u);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int key = e0 + 64 * e;
+                uint8_t* dst = smem + PT_OFF_RING + (size_t)s * PT_TILE + (size_t)hq * PT_HALF + key * 128;
+                // this quarter's two scale bytes: word 2 v + qt / 2 of the entry, from its lane
+                const uint32_t wsc = __shfl_sync(0xffffffffu, R.s[e], (lane & ~3) | (2 * v + (qt >> 1)));
+                const uint32_t b2 = (wsc >> (16 * (qt & 1))) & 0xffffu;
+                // both scales of the quarter in one conversion, each then in both halves
+                const __half2_raw sh = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+                const uint32_t s2 = (uint32_t)sh.x | ((uint32_t)sh.y << 16);
+                const uint32_t sc_lo = __byte_perm(s2, 0u, 0x1010), sc_hi = __byte_perm(s2, 0u, 0x3232);
+                const uint32_t w[4] = {R.c[e].x, R.c[e].y, R.c[e].z, R.c[e].w};
+                const bool rot = qt >> 1;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    // the two quarters of one half store in rotated order (word
+                    // i + 2), so their chunks sit in other banks
+                    const int wi = rot ? (i + 2) & 3 : i;
+                    const uint32_t sc = (rot ? ((i + 2) & 3) >> 1 : i >> 1) ? sc_hi : sc_lo;
+                    uint32_t h0, h1, h2, h3;
+                    e2m1x8_to_h2x4(rot ? w[(i + 2) & 3] : w[i], h0, h1, h2, h3);
+                    *reinterpret_cast<uint4*>(dst + (((cq + wi) ^ (key & 7)) << 4)) =
+                        make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
+                }
             }
             fence_proxy_async_smem();  // the tile is read by the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
-            ++pos;
-            if (v == 1 && t == 3 && lane == 0) mbar_arrive(&slot_free[j % PT_NQB]);  // done with query j's slots
-            r0 = r1, r1 = r2, r2 = r3;
-            fetch(n + 4, r3);
+        };
+        Rows RA[4], RB[4];
+        if (nb > 0) fetch_block(0, RA);
+        for (int b = 0; b < nb; b += 2) {
+            if (b + 1 < nb) fetch_block(b + 1, RB);
+            int jj, va, vb;
+            block_of(b, jj, va);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) convert_tile(4 * b + t, va, RA[t]);
+            if (b + 1 >= nb) break;
+            if (b + 2 < nb) fetch_block(b + 2, RA);
+            block_of(b + 1, jj, vb);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) convert_tile(4 * (b + 1) + t, vb, RB[t]);
         }
     } else {
         // ============ softmax and epilogue: warps 0-3, thread = TMEM lane ============
         const GroupBar sb{1, 128};
         const uint32_t lane_base = tmem + ((uint32_t)(32 * wid) << 16);
         const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+        float inv[16];  // 1 / sum of the query whose epilogue is pending
+        auto epilogue = [&](int jj) {  // O(jj) (thread = dim) / sum -> out; its TMEM buffer is free after
+            const uint32_t tb = (uint32_t)jj & (PT_NTB - 1);
+            uint32_t ov[16];
+            tmem_ld16(lane_base + tb * 128u + 96u, ov);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_free[tb]);
+            float* out = a.out + (int64_t)(q0 + jj) * kH * kD;
+#pragma unroll
+            for (int hh = 0; hh < 16; ++hh) out[hh * kD + tid] = __uint_as_float(ov[hh]) * inv[hh];
+        };
         for (int j = 0; j < nq; ++j) {
-            const int q = q0 + j, qb = j & 1, wb = j % PT_NQB;
-            const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-            // the slots and the window of this query (written by warp 4), then its scores
-            if (!mbar_wait(&slot_ready[wb], (uint32_t)(j / PT_NQB) & 1u, kPtWaitLimit)) timeout();
-            if (!mbar_wait(&s_full[qb], ph, kPtWaitLimit)) timeout();
+            const int q = q0 + j, tb = j & (PT_NTB - 1), wb = j % PT_NQB;
+            // the slots and the window of this query (setup warp), then its scores
+            wait(&slot_ready[wb], (uint32_t)(j / PT_NQB) & 1u);
+            wait(&s_full[tb], (uint32_t)(j / PT_NTB) & 1u);
             tc_fence_after();
             const int32_t* sl = s_slot + wb * 512;
             const int2 win = s_win[wb];
             // window row `tid` holds the token of [p - 127, p] congruent to it
             const int wtok = win.y - ((win.y - tid) & 127);
             const bool wok = wtok >= win.x;
-            const uint32_t tS = lane_base + (uint32_t)qb * 128u;
+            const uint32_t tS = lane_base + (uint32_t)tb * 128u;
             // pass 1: the per-head maximum over the 640 keys (log2 domain)
             float m[16];
 #pragma unroll
@@ -448,11 +534,12 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
 #pragma unroll
             for (int hh = 0; hh < 16; ++hh)
                 m[hh] = fmaxf(fmaxf(red[hh], red[16 + hh]), fmaxf(red[32 + hh], red[48 + hh]));
+            // P^T buffer j & 1 was read by O(j - 2), waited for before the epilogue of j - 2
             // pass 2: P = exp2(S - max) as fp16 into P^T, and the per-head sums
             float l[16];
 #pragma unroll
             for (int hh = 0; hh < 16; ++hh) l[hh] = 0.f;
-            uint8_t* pt = smem + PT_OFF_P + (size_t)qb * PT_TILES * PT_PTILE;
+            uint8_t* pt = smem + PT_OFF_P + (size_t)(j & 1) * PT_TILES * PT_PTILE;
             const int k = tid;  // key within the tile
             const int ke = k & ~1, odd = k & 1;
 #pragma unroll 1
@@ -464,7 +551,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                 float p[16];
 #pragma unroll
                 for (int hh = 0; hh < 16; ++hh) {
-                    p[hh] = (ok && m[hh] != -INFINITY) ? exp2f(__uint_as_float(v[hh]) * kScaleLog2 - m[hh]) : 0.f;
+                    p[hh] = (ok && m[hh] != -INFINITY) ? ex2(__uint_as_float(v[hh]) * kScaleLog2 - m[hh]) : 0.f;
                     l[hh] += p[hh];
                 }
                 // P^T tile t: [key half][16 heads][128 B], key k of head h at chunk ((k & 63) >> 3) ^ (h & 7);
@@ -483,7 +570,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             fence_proxy_async_smem();  // P^T is read by the tensor core
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&p_ready[qb]);
+                mbar_arrive(&p_ready[j & 1]);
                 mbar_arrive(&slot_free[wb]);
             }
 #pragma unroll
@@ -497,21 +584,6 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             sb.sync();
 #pragma unroll
             for (int hh = 0; hh < 16; ++hh) l[hh] = (red[hh] + red[16 + hh]) + (red[32 + hh] + red[48 + hh]);
-            // ---- O^T (thread = dim) once every P V product is done ----
-            if (!mbar_wait(&o_full[qb], ph, kPtWaitLimit)) timeout();
-            tc_fence_after();
-            uint32_t ov[16];
-            tmem_ld16(lane_base + (uint32_t)qb * 128u + 96u, ov);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_free[qb]);
-            float* out = a.out + (int64_t)q * kH * kD;
-#pragma unroll
-            for (int hh = 0; hh < 16; ++hh) {
-                const float inv = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
-                out[hh * kD + tid] = __uint_as_float(ov[hh]) * inv;
-            }
             if (tid < 16) {
                 float lt = 0.f, mt = 0.f;
 #pragma unroll
@@ -522,11 +594,23 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                     }
                 a.lse[(int64_t)q * kH + tid] = lt > 0.f ? (mt + log2f(lt)) * 0.6931471805599453f : -INFINITY;
             }
+            if (j >= 1) {
+                wait(&o_full[(j - 1) & (PT_NTB - 1)], (uint32_t)((j - 1) / PT_NTB) & 1u);
+                tc_fence_after();
+                epilogue(j - 1);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 16; ++hh) inv[hh] = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
+        }
+        if (nq > 0) {
+            wait(&o_full[(nq - 1) & (PT_NTB - 1)], (uint32_t)((nq - 1) / PT_NTB) & 1u);
+            tc_fence_after();
+            epilogue(nq - 1);
         }
     }
     tc_fence_before();
     __syncthreads();  // every accumulator has been read
-    if (wid == 5) {
+    if (wid == PT_W_MMA) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(PT_TMEM_COLS)
                      : "memory");
@@ -547,6 +631,8 @@ cudaError_t launch_prefill_attn_tc(const AttnArgs& a, int n_ctas, cudaStream_t s
         init[dev] = true;
     }
     if (a.rows <= 0) return cudaSuccess;
+    // slots are kept as int32
+    if ((a.cache.n_phys_pages << a.page_shift) > INT32_MAX) return cudaErrorInvalidValue;
     LaunchCfg c(dim3((unsigned)std::min(a.rows, n_ctas)), dim3(PT_THREADS), PT_SMEM, stream);
     return cudaLaunchKernelEx(&c.cfg, prefill_attn_tc_kernel, a);
 }

@@ -100,31 +100,6 @@ __device__ __forceinline__ void load_words(uint32_t* dst, const uint32_t* src, i
     for (int j = 4 * n4 + threadIdx.x; j < n32; j += nt) dst[j] = __ldcg(src + j);
 }
 
-// Copy two word arrays global -> shared with up to 16 16-byte loads per thread
-// in flight at once (both sources and destinations 16-byte aligned).
-__device__ __forceinline__ void load_words2(uint32_t* d1, const uint32_t* s1, int n1, uint32_t* d2,
-                                            const uint32_t* s2, int n2) {
-    const int nt = blockDim.x, q1 = n1 >> 2, q2 = n2 >> 2, tot = q1 + q2;
-    const uint4* a4 = reinterpret_cast<const uint4*>(s1);
-    const uint4* b4 = reinterpret_cast<const uint4*>(s2);
-    for (int base = 0; base < tot; base += 16 * nt) {
-        uint4 v[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int i = base + threadIdx.x + k * nt;
-            v[k] = i < q1 ? __ldcg(a4 + i) : i < tot ? __ldcg(b4 + (i - q1)) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int i = base + threadIdx.x + k * nt;
-            if (i < q1) reinterpret_cast<uint4*>(d1)[i] = v[k];
-            else if (i < tot) reinterpret_cast<uint4*>(d2)[i - q1] = v[k];
-        }
-    }
-    for (int j = 4 * q1 + threadIdx.x; j < n1; j += nt) d1[j] = __ldcg(s1 + j);
-    for (int j = 4 * q2 + threadIdx.x; j < n2; j += nt) d2[j] = __ldcg(s2 + j);
-}
-
 // ----------------------------------------------------------------------------
 // Threshold refinement: the first digit b1 (key bits 31..20) holds the kk-th
 // largest key and `need` of its members are still to be taken.  Two 10-bit

@@ -223,7 +223,8 @@ CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_layer_desc* desc, const 
  * bf16 K|V rows of tokens swa_start, swa_start+1, ... and the window of the
  * query at p is tokens [max(0, p - window + 1), p] (requires swa_start <= that
  * start); seq_len = entries in the cache; out [T][16][128], lse [T][16].
- * q, swa_kv and out must be 16-byte aligned (INVALID_ARG otherwise). */
+ * q, swa_kv and out must be 16-byte aligned (INVALID_ARG otherwise); the
+ * cache must hold fewer than 2^31 slots (UNSUPPORTED otherwise). */
 CSA2_API csa2_status csa2_sparse_attn_prefill(const csa2_layer_desc* desc, const csa2_kv_cache* cache, const uint16_t* q,
                                      const int32_t* topk_idx, const int32_t* q_pos, const uint16_t* swa_kv,
                                      int32_t swa_start, int32_t seq_len, float* out, float* lse, int32_t T,
