@@ -50,12 +50,12 @@ __global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (e >= a.n) return;
+    // Every load that does not need this entry's slot is issued with it: the
+    // source rows, the next entry's slot, and (for the block's pooled row) the
+    // slots and indexer-K source rows of the 7 entries before this one.  The
+    // cache rows of a block's earlier entries follow once the slot is known:
+    // two round trips in all.
     const int64_t slot = a.slot_mapping[e];
-    if (slot < 0 || slot >= a.n_slots) {
-        if (lane == 0) dev_error(a.err, CSA2_DEV_SLOT);
-        return;
-    }
-
     float x[8];
     if (a.ratio == 2) {
         float y[8];
@@ -65,6 +65,22 @@ __global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
         for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(__fadd_rn(x[i], y[i]), 0.5f);
     } else {
         load8<kBf16>(a.src, e, lane, x);
+    }
+    const bool has_idx = a.idx_src != nullptr, pooled = has_idx && a.cache.idx_k_pooled != nullptr;
+    uint32_t ws[8];       // indexer-K source row of entry e - d, lane's word
+    int64_t pm[8];        // slot of entry e - d (d >= 1)
+#pragma unroll
+    for (int d = 0; d < 8; ++d) {
+        const int64_t ed = e - d;
+        ws[d] = (has_idx && (d == 0 || pooled) && ed >= 0)
+                    ? __ldg(reinterpret_cast<const uint32_t*>(a.idx_src + ed * kID) + lane)
+                    : 0u;
+        pm[d] = (d > 0 && pooled && ed >= 0) ? __ldg(a.slot_mapping + ed) : -1;
+    }
+    const int64_t next = (pooled && e + 1 < a.n) ? __ldg(a.slot_mapping + e + 1) : -1;
+    if (slot < 0 || slot >= a.n_slots) {
+        if (lane == 0) dev_error(a.err, CSA2_DEV_SLOT);
+        return;
     }
 
     // block amax over the lane pair, scale = E4M3(amax / 6)
@@ -83,34 +99,33 @@ __global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
     reinterpret_cast<uint32_t*>(a.cache.codes + slot * kCodeBytes)[lane] = packed;
     if ((lane & 1) == 0) a.cache.scales[slot * kScales + (lane >> 1)] = (uint8_t)sb;
 
-    if (a.idx_src == nullptr) return;
-    const uint32_t kw = __ldg(reinterpret_cast<const uint32_t*>(a.idx_src + e * kID) + lane);
-    reinterpret_cast<uint32_t*>(a.cache.idx_k + slot * kID)[lane] = kw;
+    if (!has_idx) return;
+    reinterpret_cast<uint32_t*>(a.cache.idx_k + slot * kID)[lane] = ws[0];
 
-    if (a.cache.idx_k_pooled == nullptr) return;
+    if (!pooled) return;
     // The last appended entry of a block of 8 recomputes that block's pooled row
     // over the entries present (slot % 8 + 1 of them).  Entries appended by this
     // call are read from the source rows (other warps are still storing them),
     // earlier ones from the cache.
-    const bool last_in_block = (e == a.n - 1) || ((a.slot_mapping[e + 1] >> 3) != (slot >> 3));
+    const bool last_in_block = (e == a.n - 1) || ((next >> 3) != (slot >> 3));
     if (!last_in_block) return;
     const int64_t s0 = slot & ~int64_t(7);
     const int cnt = int(slot - s0) + 1;
-    // all slot-mapping probes, then all row loads, issued together (two round trips)
-    int64_t probe[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t er = e - (slot - (s0 + r));
-        probe[r] = (r < cnt && er >= 0) ? __ldg(a.slot_mapping + er) : -1;
-    }
     uint32_t wr[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t sr = s0 + r, er = e - (slot - sr);
+    for (int r = 0; r < 8; ++r) {  // slot s0 + r is entry e - d of this call when the slot mapping says so
+        const int d = int(slot - (s0 + r));
         wr[r] = 0u;
         if (r < cnt) {
-            if (probe[r] == sr) wr[r] = __ldg(reinterpret_cast<const uint32_t*>(a.idx_src + er * kID) + lane);
-            else wr[r] = reinterpret_cast<const uint32_t*>(a.cache.idx_k + sr * kID)[lane];
+            bool src = d == 0;
+#pragma unroll
+            for (int dd = 1; dd < 8; ++dd)
+                if (dd == d) src = pm[dd] == s0 + r;
+            uint32_t v = 0u;
+#pragma unroll
+            for (int dd = 0; dd < 8; ++dd)
+                if (dd == d) v = ws[dd];
+            wr[r] = src ? v : reinterpret_cast<const uint32_t*>(a.cache.idx_k + (s0 + r) * kID)[lane];
         }
     }
     float acc0 = 0.f, acc1 = 0.f;
