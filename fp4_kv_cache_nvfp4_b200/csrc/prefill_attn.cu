@@ -26,21 +26,25 @@
 // 128): the next query of a prefill chunk adds one token, so one row is
 // converted instead of 128.  The softmax masks a window row whose token, the
 // one in [p - 127, p] congruent to the row, is before the window's start.
-//   warps 0-3   softmax: thread = TMEM lane = key of a tile (S) and dim (O);
-//               per-head max and sum across the 4 warps; the epilogue of
-//               query j - 1 runs after P of query j is out
-//   warp 4      TMEM owner and MMA issue (one lane); order S(0), then S(j+1)
+//   warps 0-7   softmax: warp w reads TMEM lane quarter w % 4 (thread = key
+//               of a tile for S, dim for O) for heads 8 (w / 4) .. + 7; per-head
+//               max and sum across the 4 warps of a head group; the epilogue
+//               of query j - 1 runs after P of query j is out
+//   warp 8      TMEM owner and MMA issue (one lane); order S(0), then S(j+1)
 //               before O(j), so the softmax of query j overlaps the products
 //               of query j+1
-//   warps 5-6   per query (alternating): the selected entries' physical
-//               slots, the window range, Q and the window rows the query
-//               adds, converted to fp16 in their swizzled tiles
-//   warps 7-14  converters: thread = one 16-byte quarter (32 channels) of two
-//               entries of a tile, read by plain loads (the four quarters of an
+//   warps 9-11  per query (in turn): the selected entries' physical slots
+//               (the sequence's page table cached in shared memory), the
+//               window range, Q and the window rows the query adds, converted
+//               to fp16 in their swizzled tiles
+//   warps 12-27 converters: thread = one 16-byte quarter (32 channels) of one
+//               entry of a tile, read by plain loads (the four quarters of an
 //               entry's 64 K or V code bytes by four neighbouring lanes) one
-//               block of four tiles ahead of the block it converts, so 8 rows
-//               per thread are in flight; FP4 -> fp16 tile into a 3-slot ring.
-//               The 8 FP4 tiles of query j: its K, one query ahead, then its V.
+//               block of four tiles ahead of the block it converts; FP4 ->
+//               fp16 tile into a 3-slot ring.  The 8 FP4 tiles of query j: its
+//               K, one query ahead, then its V.  The proxy fence that hands a
+//               tile to the tensor core does not wait for the loads in flight
+//               (measured).
 // TMEM holds four query buffers of 128 columns (S of 5 tiles at 0, O at 96),
 // Q and P^T two buffers each.
 #include <algorithm>
@@ -59,7 +63,7 @@ constexpr int PT_NTB = 4;                                // TMEM query buffers
 constexpr uint32_t PT_HALF = 128 * 128;                  // one 64-dim half of a tile: 16 KiB
 constexpr uint32_t PT_TILE = 2 * PT_HALF;                // 32 KiB
 constexpr uint32_t PT_PTILE = 2 * 16 * 128;              // P^T of one tile: two 64-key halves x 16 heads x 128 B
-constexpr int PT_W_MMA = 4, PT_W_SETUP = 5, PT_NSETUP = 3, PT_W_CONV = 8, PT_WARPS = 16;
+constexpr int PT_NSOFT = 8, PT_W_MMA = 8, PT_W_SETUP = 9, PT_NSETUP = 3, PT_W_CONV = 12, PT_NCONV = 16, PT_WARPS = 28;
 constexpr int PT_PTAB = 1024;                            // page-table entries kept in shared memory
 constexpr int PT_THREADS = PT_WARPS * 32;
 constexpr size_t PT_OFF_RING = 0;
@@ -70,8 +74,9 @@ constexpr size_t PT_OFF_Q = PT_OFF_P + 2 * (size_t)PT_TILES * PT_PTILE;     // [
 constexpr size_t PT_OFF_SLOT = PT_OFF_Q + 2 * 4096;                         // [3][512] int32
 constexpr size_t PT_OFF_PTAB = PT_OFF_SLOT + (size_t)PT_NQB * 512 * 4;      // [1024] the sequence's first pages
 constexpr size_t PT_OFF_WIN = PT_OFF_PTAB + (size_t)PT_PTAB * 4;            // [4] (window start, query position)
-constexpr size_t PT_OFF_RED = PT_OFF_WIN + 32;                              // [2][4 warps][16] floats
-constexpr size_t PT_OFF_BAR = PT_OFF_RED + 2 * 4 * 16 * 4;
+constexpr size_t PT_OFF_RED = PT_OFF_WIN + 32;                              // [2][2 head groups][4 quarters][8] floats
+constexpr size_t PT_OFF_INV = PT_OFF_RED + 2 * 2 * 4 * 8 * 4;              // [2][16] 1 / sum per head
+constexpr size_t PT_OFF_BAR = PT_OFF_INV + 2 * 16 * 4;
 constexpr int PT_NBAR = 2 * PT_NSLOT + 2 * PT_NQB + 2 * 2 + 3 * PT_NTB + 2 + 2;
 constexpr size_t PT_OFF_MISC = PT_OFF_BAR + (size_t)PT_NBAR * 8;            // tmem base, timeout flag
 constexpr size_t PT_SMEM = PT_OFF_MISC + 16 + 1024;                         // + slack for the 1 KiB alignment
@@ -99,6 +104,13 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t 
         : "memory");
 }
 
+// 8 consecutive TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(addr));
+}
+
 // 2^x (the hardware approximation; P is rounded to fp16 afterwards)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -117,16 +129,16 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PT_OFF_BAR);
-    uint64_t* full = bars;                       // [3] ring slot converted (8 converter warps)
+    uint64_t* full = bars;                       // [3] ring slot converted (16 converter warps)
     uint64_t* empty = full + PT_NSLOT;           // [3] ring slot read by the tensor core
     uint64_t* slot_ready = empty + PT_NSLOT;     // [4] slots and window range of a query (setup warp)
-    uint64_t* slot_free = slot_ready + PT_NQB;   // [4] (8 converter warps + 4 softmax warps)
+    uint64_t* slot_free = slot_ready + PT_NQB;   // [4] (16 converter warps + 8 softmax warps)
     uint64_t* q_ready = slot_free + PT_NQB;      // [2] Q tile and the query's window K rows written
     uint64_t* q_free = q_ready + 2;              // [2] Q tile read (MMA commit)
     uint64_t* s_full = q_free + 2;               // [4] S complete (MMA commit)
     uint64_t* o_full = s_full + PT_NTB;          // [4] O complete (MMA commit)
-    uint64_t* tmem_free = o_full + PT_NTB;       // [4] S and O read (4 softmax warps)
-    uint64_t* p_ready = tmem_free + PT_NTB;      // [2] P^T written (4 softmax warps)
+    uint64_t* tmem_free = o_full + PT_NTB;       // [4] S and O read (8 softmax warps)
+    uint64_t* p_ready = tmem_free + PT_NTB;      // [2] P^T written (8 softmax warps)
     uint64_t* vw_ready = p_ready + 2;            // window V rows of a query written (setup warp)
     uint64_t* mma_done = vw_ready + 1;           // every product complete
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + PT_OFF_MISC);
@@ -135,6 +147,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
     int2* s_win = reinterpret_cast<int2*>(smem + PT_OFF_WIN);
     int32_t* s_ptab = reinterpret_cast<int32_t*>(smem + PT_OFF_PTAB);
     float* s_red = reinterpret_cast<float*>(smem + PT_OFF_RED);
+    float* s_inv = reinterpret_cast<float*>(smem + PT_OFF_INV);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     // this CTA's contiguous range of queries
     const int per = (a.rows + (int)gridDim.x - 1) / (int)gridDim.x;
@@ -142,12 +155,12 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
 
     if (tid == 0) {
         for (int s = 0; s < PT_NSLOT; ++s) {
-            mbar_init(&full[s], 8);
+            mbar_init(&full[s], PT_NCONV);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < PT_NQB; ++b) {
             mbar_init(&slot_ready[b], 1);
-            mbar_init(&slot_free[b], 12);
+            mbar_init(&slot_free[b], PT_NCONV + PT_NSOFT);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&q_ready[b], 1);
@@ -156,10 +169,10 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
         for (int b = 0; b < PT_NTB; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&o_full[b], 1);
-            mbar_init(&tmem_free[b], 4);
+            mbar_init(&tmem_free[b], PT_NSOFT);
         }
-        mbar_init(&p_ready[0], 4);
-        mbar_init(&p_ready[1], 4);
+        mbar_init(&p_ready[0], PT_NSOFT);
+        mbar_init(&p_ready[1], PT_NSOFT);
         mbar_init(vw_ready, 1);
         mbar_init(mma_done, 1);
         *s_timeout = 0;
@@ -376,9 +389,9 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
     } else if (wid >= PT_W_CONV) {
         // ============ converters: FP4 rows -> fp16 operand tiles ============
         // Thread ct owns quarter qt (channels 32 qt .. 32 qt + 31 of K or V) of
-        // entries e0 = ct / 4 and e0 + 64 of every tile.  The tiles come in blocks
-        // of four (one query's K or V): K(0), then K(j + 1), V(j) for each j.
-        // Block b + 1's rows are loaded while block b is converted.
+        // entry e0 = ct / 4 of every tile.  The tiles come in blocks of four (one
+        // query's K or V): K(0), then K(j + 1), V(j) for each j.  Block b + 1's
+        // rows are loaded while block b is converted.
         const int ct = tid - PT_W_CONV * 32, qt = ct & 3, hq = qt >> 1, cq = (qt & 1) * 4, e0 = ct >> 2;
         const int nb = 2 * nq;
         auto block_of = [&](int b, int& j, int& v) {
@@ -391,15 +404,15 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             else if (i & 1) j = p, v = 1;
             else j = p + 1, v = 0;
         };
-        struct Rows {
-            uint4 c[2];     // 16 code bytes of each of the two entries (zeros: absent)
-            uint32_t s[2];  // word qt of each entry's 16 scale bytes (K's 8, then V's)
+        struct Row {
+            uint4 c;     // 16 code bytes of the entry (zeros: absent)
+            uint32_t s;  // word qt of the entry's 16 scale bytes (K's 8, then V's)
         };
         // The scale words of a query's K block serve its V block too: lanes 2, 3
         // of an entry's four hold V's scales.  Kept per query parity (V(j) follows K(j + 1)).
-        uint32_t sv0[8], sv1[8];
+        uint32_t sv0[4], sv1[4];
         int seen = -1;  // last query whose slot list was waited for
-        auto fetch_block = [&](int b, Rows (&R)[4]) {
+        auto fetch_block = [&](int b, Row (&R)[4]) {
             int j, v;
             block_of(b, j, v);
             if (j > seen) {
@@ -407,9 +420,9 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                 seen = j;
             }
             const int32_t* sl = s_slot + (j % PT_NQB) * 512 + e0;
-            int32_t slot[8];
+            int32_t slot[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) slot[i] = sl[(i >> 1) * 128 + (i & 1) * 64];
+            for (int t = 0; t < 4; ++t) slot[t] = sl[t * 128];
             if (v == 1) {  // query j's slot list is read
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&slot_free[j % PT_NQB]);
@@ -417,54 +430,50 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             const uint8_t* cbase = a.cache.codes + v * 64 + qt * 16;
             const uint8_t* sbase = a.cache.scales + qt * 4;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int t = 0; t < 4; ++t) {
                 uint4 c = make_uint4(0u, 0u, 0u, 0u);
-                if (slot[i] >= 0) c = __ldg(reinterpret_cast<const uint4*>(cbase + (int64_t)slot[i] * kCodeBytes));
-                R[i >> 1].c[i & 1] = c;
+                if (slot[t] >= 0) c = __ldg(reinterpret_cast<const uint4*>(cbase + (int64_t)slot[t] * kCodeBytes));
+                R[t].c = c;
                 if (v == 0) {
                     uint32_t w = 0u;
-                    if (slot[i] >= 0) w = __ldg(reinterpret_cast<const uint32_t*>(sbase + (int64_t)slot[i] * kScales));
-                    R[i >> 1].s[i & 1] = w;
-                    if (j & 1) sv1[i] = w;
-                    else sv0[i] = w;
+                    if (slot[t] >= 0) w = __ldg(reinterpret_cast<const uint32_t*>(sbase + (int64_t)slot[t] * kScales));
+                    R[t].s = w;
+                    if (j & 1) sv1[t] = w;
+                    else sv0[t] = w;
                 } else {
-                    R[i >> 1].s[i & 1] = (j & 1) ? sv1[i] : sv0[i];
+                    R[t].s = (j & 1) ? sv1[t] : sv0[t];
                 }
             }
         };
-        auto convert_tile = [&](int m, int v, const Rows& R) {
+        auto convert_tile = [&](int m, int v, const Row& R) {
             const int s = m % PT_NSLOT;
             if (m >= PT_NSLOT) wait(&empty[s], (uint32_t)((m / PT_NSLOT) - 1) & 1u);
+            uint8_t* dst = smem + PT_OFF_RING + (size_t)s * PT_TILE + (size_t)hq * PT_HALF + e0 * 128;
+            // this quarter's two scale bytes: word 2 v + qt / 2 of the entry, from its lane
+            const uint32_t wsc = __shfl_sync(0xffffffffu, R.s, (lane & ~3) | (2 * v + (qt >> 1)));
+            const uint32_t b2 = (wsc >> (16 * (qt & 1))) & 0xffffu;
+            // both scales of the quarter in one conversion, each then in both halves
+            const __half2_raw sh = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+            const uint32_t s2 = (uint32_t)sh.x | ((uint32_t)sh.y << 16);
+            const uint32_t sc_lo = __byte_perm(s2, 0u, 0x1010), sc_hi = __byte_perm(s2, 0u, 0x3232);
+            const uint32_t w[4] = {R.c.x, R.c.y, R.c.z, R.c.w};
+            const bool rot = qt >> 1;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int key = e0 + 64 * e;
-                uint8_t* dst = smem + PT_OFF_RING + (size_t)s * PT_TILE + (size_t)hq * PT_HALF + key * 128;
-                // this quarter's two scale bytes: word 2 v + qt / 2 of the entry, from its lane
-                const uint32_t wsc = __shfl_sync(0xffffffffu, R.s[e], (lane & ~3) | (2 * v + (qt >> 1)));
-                const uint32_t b2 = (wsc >> (16 * (qt & 1))) & 0xffffu;
-                // both scales of the quarter in one conversion, each then in both halves
-                const __half2_raw sh = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
-                const uint32_t s2 = (uint32_t)sh.x | ((uint32_t)sh.y << 16);
-                const uint32_t sc_lo = __byte_perm(s2, 0u, 0x1010), sc_hi = __byte_perm(s2, 0u, 0x3232);
-                const uint32_t w[4] = {R.c[e].x, R.c[e].y, R.c[e].z, R.c[e].w};
-                const bool rot = qt >> 1;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    // the two quarters of one half store in rotated order (word
-                    // i + 2), so their chunks sit in other banks
-                    const int wi = rot ? (i + 2) & 3 : i;
-                    const uint32_t sc = (rot ? ((i + 2) & 3) >> 1 : i >> 1) ? sc_hi : sc_lo;
-                    uint32_t h0, h1, h2, h3;
-                    e2m1x8_to_h2x4(rot ? w[(i + 2) & 3] : w[i], h0, h1, h2, h3);
-                    *reinterpret_cast<uint4*>(dst + (((cq + wi) ^ (key & 7)) << 4)) =
-                        make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
-                }
+            for (int i = 0; i < 4; ++i) {
+                // the two quarters of one half store in rotated order (word
+                // i + 2), so their chunks sit in other banks
+                const int wi = rot ? (i + 2) & 3 : i;
+                const uint32_t sc = (rot ? ((i + 2) & 3) >> 1 : i >> 1) ? sc_hi : sc_lo;
+                uint32_t h0, h1, h2, h3;
+                e2m1x8_to_h2x4(rot ? w[(i + 2) & 3] : w[i], h0, h1, h2, h3);
+                *reinterpret_cast<uint4*>(dst + (((cq + wi) ^ (e0 & 7)) << 4)) =
+                    make_uint4(hmul2(h0, sc), hmul2(h1, sc), hmul2(h2, sc), hmul2(h3, sc));
             }
             fence_proxy_async_smem();  // the tile is read by the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         };
-        Rows RA[4], RB[4];
+        Row RA[4], RB[4];
         if (nb > 0) fetch_block(0, RA);
         for (int b = 0; b < nb; b += 2) {
             if (b + 1 < nb) fetch_block(b + 1, RB);
@@ -479,22 +488,26 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             for (int t = 0; t < 4; ++t) convert_tile(4 * (b + 1) + t, vb, RB[t]);
         }
     } else {
-        // ============ softmax and epilogue: warps 0-3, thread = TMEM lane ============
-        const GroupBar sb{1, 128};
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * wid) << 16);
+        // ============ softmax and epilogue: warps 0-7 ============
+        // warp w: TMEM lane quarter w & 3 (thread = key r of a tile for S, dim r
+        // for O) and heads 8 hg .. 8 hg + 7, hg = w >> 2; per-head max and sum
+        // across the 4 warps of a head group
+        const int wq = wid & 3, hg = wid >> 2, r = 32 * wq + lane;
+        const GroupBar sb{1, 32 * PT_NSOFT};
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16) + 8u * (uint32_t)hg;
         const float kScaleLog2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-        float inv[16];  // 1 / sum of the query whose epilogue is pending
         auto epilogue = [&](int jj) {  // O(jj) (thread = dim) / sum -> out; its TMEM buffer is free after
             const uint32_t tb = (uint32_t)jj & (PT_NTB - 1);
-            uint32_t ov[16];
-            tmem_ld16(lane_base + tb * 128u + 96u, ov);
+            uint32_t ov[8];
+            tmem_ld8(lane_base + tb * 128u + 96u, ov);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_free[tb]);
-            float* out = a.out + (int64_t)(q0 + jj) * kH * kD;
+            float* out = a.out + ((int64_t)(q0 + jj) * kH + 8 * hg) * kD;
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh) out[hh * kD + tid] = __uint_as_float(ov[hh]) * inv[hh];
+            for (int hh = 0; hh < 8; ++hh)
+                out[hh * kD + r] = __uint_as_float(ov[hh]) * s_inv[(jj & 1) * 16 + 8 * hg + hh];
         };
         for (int j = 0; j < nq; ++j) {
             const int q = q0 + j, tb = j & (PT_NTB - 1), wb = j % PT_NQB;
@@ -504,63 +517,61 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
             tc_fence_after();
             const int32_t* sl = s_slot + wb * 512;
             const int2 win = s_win[wb];
-            // window row `tid` holds the token of [p - 127, p] congruent to it
-            const int wtok = win.y - ((win.y - tid) & 127);
+            // window row r holds the token of [p - 127, p] congruent to it
+            const int wtok = win.y - ((win.y - r) & 127);
             const bool wok = wtok >= win.x;
             const uint32_t tS = lane_base + (uint32_t)tb * 128u;
             // pass 1: the per-head maximum over the 640 keys (log2 domain)
-            float m[16];
+            float m[8];
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh) m[hh] = -INFINITY;
+            for (int hh = 0; hh < 8; ++hh) m[hh] = -INFINITY;
 #pragma unroll 1
             for (int t = 0; t < PT_TILES; ++t) {
-                const bool ok = t < 4 ? sl[t * 128 + tid] >= 0 : wok;
-                uint32_t v[16];
-                tmem_ld16(tS + 16u * t, v);
+                const bool ok = t < 4 ? sl[t * 128 + r] >= 0 : wok;
+                uint32_t v[8];
+                tmem_ld8(tS + 16u * t, v);
                 tmem_wait_ld();
                 if (ok)
 #pragma unroll
-                    for (int hh = 0; hh < 16; ++hh) m[hh] = fmaxf(m[hh], __uint_as_float(v[hh]) * kScaleLog2);
+                    for (int hh = 0; hh < 8; ++hh) m[hh] = fmaxf(m[hh], __uint_as_float(v[hh]) * kScaleLog2);
             }
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh)
+            for (int hh = 0; hh < 8; ++hh)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m[hh] = fmaxf(m[hh], __shfl_xor_sync(0xffffffffu, m[hh], o));
-            float* red = s_red + (j & 1) * 64;  // alternate buffers: a fast warp's next query never overwrites this one
+            // alternate buffers: a fast warp's next query never overwrites this one
+            float* red = s_red + (j & 1) * 64 + hg * 32;
             if (lane == 0)
 #pragma unroll
-                for (int hh = 0; hh < 16; ++hh) red[wid * 16 + hh] = m[hh];
+                for (int hh = 0; hh < 8; ++hh) red[wq * 8 + hh] = m[hh];
             sb.sync();
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh)
-                m[hh] = fmaxf(fmaxf(red[hh], red[16 + hh]), fmaxf(red[32 + hh], red[48 + hh]));
+            for (int hh = 0; hh < 8; ++hh) m[hh] = fmaxf(fmaxf(red[hh], red[8 + hh]), fmaxf(red[16 + hh], red[24 + hh]));
             // P^T buffer j & 1 was read by O(j - 2), waited for before the epilogue of j - 2
             // pass 2: P = exp2(S - max) as fp16 into P^T, and the per-head sums
-            float l[16];
+            float l[8];
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh) l[hh] = 0.f;
+            for (int hh = 0; hh < 8; ++hh) l[hh] = 0.f;
             uint8_t* pt = smem + PT_OFF_P + (size_t)(j & 1) * PT_TILES * PT_PTILE;
-            const int k = tid;  // key within the tile
-            const int ke = k & ~1, odd = k & 1;
+            const int ke = r & ~1, odd = r & 1;
 #pragma unroll 1
             for (int t = 0; t < PT_TILES; ++t) {
-                const bool ok = t < 4 ? sl[t * 128 + tid] >= 0 : wok;
-                uint32_t v[16];
-                tmem_ld16(tS + 16u * t, v);
+                const bool ok = t < 4 ? sl[t * 128 + r] >= 0 : wok;
+                uint32_t v[8];
+                tmem_ld8(tS + 16u * t, v);
                 tmem_wait_ld();
-                float p[16];
-#pragma unroll
-                for (int hh = 0; hh < 16; ++hh) {
-                    p[hh] = (ok && m[hh] != -INFINITY) ? ex2(__uint_as_float(v[hh]) * kScaleLog2 - m[hh]) : 0.f;
-                    l[hh] += p[hh];
-                }
                 // P^T tile t: [key half][16 heads][128 B], key k of head h at chunk ((k & 63) >> 3) ^ (h & 7);
-                // lanes k and k ^ 1 pair up: the even lane stores heads 0..7, the odd one heads 8..15
-                uint8_t* ptt = pt + (size_t)t * PT_PTILE + (size_t)(k >> 6) * 2048;
+                // lanes r and r ^ 1 pair up: the even lane stores heads 8 hg + 0..3, the odd one 8 hg + 4..7
+                uint8_t* ptt = pt + (size_t)t * PT_PTILE + (size_t)(r >> 6) * 2048;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int hs = odd ? 8 + i : i;   // head this lane stores
-                    const float mine = odd ? p[8 + i] : p[i], give = odd ? p[i] : p[8 + i];
+                for (int i = 0; i < 4; ++i) {  // heads 8 hg + i and 8 hg + 4 + i
+                    const float p0 = (ok && m[i] != -INFINITY) ? ex2(__uint_as_float(v[i]) * kScaleLog2 - m[i]) : 0.f;
+                    const float p1 =
+                        (ok && m[4 + i] != -INFINITY) ? ex2(__uint_as_float(v[4 + i]) * kScaleLog2 - m[4 + i]) : 0.f;
+                    l[i] += p0;
+                    l[4 + i] += p1;
+                    const int hs = 8 * hg + (odd ? 4 + i : i);  // head this lane stores
+                    const float mine = odd ? p1 : p0, give = odd ? p0 : p1;
                     const float got = __shfl_xor_sync(0xffffffffu, give, 1);
                     const float lo = odd ? got : mine, hi = odd ? mine : got;  // keys ke, ke + 1
                     *reinterpret_cast<uint32_t*>(ptt + hs * 128 + ((((ke & 63) >> 3) ^ (hs & 7)) << 4) + (ke & 7) * 2) =
@@ -574,33 +585,38 @@ __global__ void __launch_bounds__(PT_THREADS, 1) prefill_attn_tc_kernel(AttnArgs
                 mbar_arrive(&slot_free[wb]);
             }
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh)
+            for (int hh = 0; hh < 8; ++hh)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) l[hh] += __shfl_xor_sync(0xffffffffu, l[hh], o);
             sb.sync();  // every warp has read the maxima: the buffer takes the sums
             if (lane == 0)
 #pragma unroll
-                for (int hh = 0; hh < 16; ++hh) red[wid * 16 + hh] = l[hh];
+                for (int hh = 0; hh < 8; ++hh) red[wq * 8 + hh] = l[hh];
             sb.sync();
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh) l[hh] = (red[hh] + red[16 + hh]) + (red[32 + hh] + red[48 + hh]);
-            if (tid < 16) {
+            for (int hh = 0; hh < 8; ++hh) l[hh] = (red[hh] + red[8 + hh]) + (red[16 + hh] + red[24 + hh]);
+            if (wq == 0 && lane < 8) {  // lse of head 8 hg + lane
                 float lt = 0.f, mt = 0.f;
 #pragma unroll
-                for (int hh = 0; hh < 16; ++hh)
-                    if (hh == tid) {
+                for (int hh = 0; hh < 8; ++hh)
+                    if (hh == lane) {
                         lt = l[hh];
                         mt = m[hh];
                     }
-                a.lse[(int64_t)q * kH + tid] = lt > 0.f ? (mt + log2f(lt)) * 0.6931471805599453f : -INFINITY;
+                a.lse[(int64_t)q * kH + 8 * hg + lane] = lt > 0.f ? (mt + log2f(lt)) * 0.6931471805599453f : -INFINITY;
             }
             if (j >= 1) {
                 wait(&o_full[(j - 1) & (PT_NTB - 1)], (uint32_t)((j - 1) / PT_NTB) & 1u);
                 tc_fence_after();
                 epilogue(j - 1);
             }
+            if (wq == 0 && lane < 8) {  // 1 / sum of this query, read by its epilogue (after two more barriers)
+                float lt = 0.f;
 #pragma unroll
-            for (int hh = 0; hh < 16; ++hh) inv[hh] = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
+                for (int hh = 0; hh < 8; ++hh)
+                    if (hh == lane) lt = l[hh];
+                s_inv[(j & 1) * 16 + 8 * hg + lane] = lt > 0.f ? 1.f / lt : 0.f;
+            }
         }
         if (nq > 0) {
             wait(&o_full[(nq - 1) & (PT_NTB - 1)], (uint32_t)((nq - 1) / PT_NTB) & 1u);

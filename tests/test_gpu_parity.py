@@ -396,6 +396,43 @@ def test_prefill_early_queries(csa2, orc):
     assert ps.errors() == 0
 
 
+@pytest.mark.parametrize("T", [1, 37, 150, 300])
+def test_prefill_attention_few_queries_per_cta(csa2, orc, T):
+    # fewer queries than the persistent attention kernel has CTAs (T = 1, 37:
+    # CTAs of one query or none), two per CTA (150, 300 over 148 CTAs): the
+    # pipeline's first and last query paths and the deferred epilogue at a
+    # CTA's end.  Index sets are given directly: sorted visible entries with
+    # -1 padding and -1 holes.
+    seed = 1005
+    tokens = 2048 + 320
+    n_ent = tokens // 2
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 2, 0, tokens)
+    ps.append(0, 0, synth.to_bf16_bits(kv), synth.idx_k_rows(seed, 2, 0, n_ent), ratio=2, chunk=999)
+    kvb = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+    codes, scales = orc.quant_rows(kvb, ratio=2)
+    q_pos = np.arange(tokens - T, tokens, dtype=np.int32)
+    rng = np.random.default_rng(T)
+    sets = np.full((T, 512), -1, np.int32)
+    for i, p in enumerate(q_pos):
+        vis = int(p) // 2 + 1
+        k = int(rng.integers(300, 513))
+        sel = np.sort(rng.choice(vis, min(k, vis), replace=False)).astype(np.int32)
+        sel[rng.random(sel.size) < 0.05] = -1  # holes
+        sets[i, :sel.size] = sel
+    swa_start = int(q_pos[0]) - 127
+    swa = synth.swa_rows(seed, 2, 0, tokens - swa_start)
+    q = synth.q_heads(seed, 2, 0, T)
+    d = csa2.default_desc(csa2.REUSE, 2)
+    out = torch.empty((T, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_prefill(d, ps.cache, bits16(q), dev(sets), dev(q_pos), bits16(swa), swa_start, n_ent, out, lse,
+                             T, err=ps.err)
+    ro, rl = orc.prefill_attn(q_pos, q, sets, codes, scales, swa, swa_start)
+    check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, f"prefill attention, T = {T}")
+    assert ps.errors() == 0
+
+
 def test_prefill_indexer_exact_fallback_on_ties(csa2, orc):
     # Entries 0..4999 share one indexer-K row, so their scores tie exactly.  A
     # query that sees more than 2048 of them has too many candidates at the
