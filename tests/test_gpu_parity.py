@@ -433,6 +433,40 @@ def test_prefill_attention_few_queries_per_cta(csa2, orc, T):
     assert ps.errors() == 0
 
 
+@pytest.mark.parametrize("window,topk", [(64, 256), (100, 512), (128, 384)])
+def test_prefill_attention_window_and_topk(csa2, orc, window, topk):
+    # a window shorter than 128 tokens (rows of the 128-row window tile whose
+    # token is older than the window stay masked) and index sets narrower than
+    # 512 (slots past topk are absent), over 400 consecutive queries
+    seed = 1006
+    tokens = 3000
+    n_ent = tokens // 2
+    T = 400
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 3, 0, tokens)
+    ps.append(0, 0, synth.to_bf16_bits(kv), synth.idx_k_rows(seed, 3, 0, n_ent), ratio=2, chunk=999)
+    kvb = orc.bf16_to_f32(synth.to_bf16_bits(kv)).reshape(kv.shape)
+    codes, scales = orc.quant_rows(kvb, ratio=2)
+    q_pos = np.arange(tokens - T, tokens, dtype=np.int32)
+    rng = np.random.default_rng(window + topk)
+    sets = np.full((T, topk), -1, np.int32)
+    for i, p in enumerate(q_pos):
+        vis = int(p) // 2 + 1
+        sel = np.sort(rng.choice(vis, min(topk, vis), replace=False)).astype(np.int32)
+        sets[i, :sel.size] = sel
+    swa_start = int(q_pos[0]) - window + 1
+    swa = synth.swa_rows(seed, 3, 0, tokens - swa_start)
+    q = synth.q_heads(seed, 3, 0, T)
+    d = csa2.default_desc(csa2.REUSE, 2, window=window, topk=topk)
+    out = torch.empty((T, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T, 16), dtype=torch.float32, device="cuda")
+    csa2.sparse_attn_prefill(d, ps.cache, bits16(q), dev(sets), dev(q_pos), bits16(swa), swa_start, n_ent, out, lse,
+                             T, err=ps.err)
+    ro, rl = orc.prefill_attn(q_pos, q, sets, codes, scales, swa, swa_start, window=window)
+    check_attn(out.cpu().numpy(), lse.cpu().numpy(), ro, rl, f"prefill attention, window {window}, topk {topk}")
+    assert ps.errors() == 0
+
+
 def test_prefill_indexer_exact_fallback_on_ties(csa2, orc):
     # Entries 0..4999 share one indexer-K row, so their scores tie exactly.  A
     # query that sees more than 2048 of them has too many candidates at the
