@@ -103,6 +103,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int32_t 
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
+// 1-D bulk copy, global -> this CTA's shared memory, completion counted in
+// bytes on `bar`: both addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -288,9 +296,14 @@ __device__ __forceinline__ void group_find_kth_bin(const uint32_t* hist, int nbi
     // each thread owns a contiguous run of bins counted from the top
     int per = (nbins + g.n - 1) / g.n;
     int hi = nbins - 1 - (int)threadIdx.x * per;  // first (highest) bin of this thread
+    // the run is summed from a per-thread starting point, so that the lanes of
+    // a warp read distinct banks (runs of `per` words apart would collide)
+    const int rot = (int)(((uint32_t)threadIdx.x * (uint32_t)per / 32u) % (uint32_t)per);
     uint32_t mine = 0;
     for (int i = 0; i < per; ++i) {
-        int b = hi - i;
+        int r = i + rot;
+        if (r >= per) r -= per;
+        int b = hi - r;
         if (b >= 0) mine += hist[b];
     }
     uint32_t total;

@@ -57,19 +57,6 @@ namespace csa2 {
 // fused multiply-add, rounded to nearest, in each 32-bit half, so the low half
 // follows row k's scalar FMA chain and the high half row m's, bit for bit.
 // qp[2 d + j] holds ((q_2j, q_2j), (q_2j+1, q_2j+1)) of dimension d, j = 0, 1.
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
 __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32_t (&m)[32],
                                            const ulonglong2* __restrict__ qp, float4 w, float& s_k, float& s_m) {
     uint64_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;  // (row k, row m) dot of head h; zero bits are (+0, +0)
@@ -1569,39 +1556,96 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     if (tid == 0 && *s_timeout) dev_error(a.err, CSA2_DEV_TIMEOUT);
 }
 
+constexpr int PC_THREADS = 320;                       // 3 rounds of exact rescoring cover 960 candidates
+constexpr int PC_CTAS = 4;                            // resident CTAs per SM the layout is sized for
+constexpr int PC_CH = (kMaxCand / 8 + PC_THREADS - 1) / PC_THREADS;  // 16-byte chunks of 8 keys per thread (at most)
+constexpr int PC_SB = 512;                            // sample histogram: 1/64 binade per bin, 8 binades
+constexpr int PC_SAMPLE_CAND = 800;                   // candidates the sample's threshold aims at
+constexpr int PC_CAND_LO = 600;                       // fewer -> the threshold from every key instead
+// Region A: the visible entries' 16-bit keys while the candidates are chosen;
+// afterwards the candidates' exact keys, the select's histogram and lists.
+constexpr size_t PC_OFF_K16 = 0;                                   // [16384] u16
+constexpr size_t PC_OFF_CK = 0;                                    // [2048] u32
+constexpr size_t PC_OFF_HIST = PC_OFF_CK + PT_CAND_MAX * 4;        // [4096] u32
+constexpr size_t PC_OFF_L0 = PC_OFF_HIST + kHistBins * 4;          // [2048] u16
+constexpr size_t PC_OFF_L1 = PC_OFF_L0 + PT_CAND_MAX * 2;          // [2048] u16
+// Region B: the sample histogram, then the sequence's page table.
+constexpr size_t PC_OFF_HS = (size_t)kMaxCand * 2;                 // [512] u32, one key per chunk
+constexpr size_t PC_OFF_PTAB = PC_OFF_HS;                          // [1536] i32 physical page per page index
+constexpr int PC_PTAB = 1536;
+// Region C: the histogram of every key, then the candidate list.
+constexpr size_t PC_OFF_HE = PC_OFF_PTAB + PC_PTAB * 4;            // [1024] u32
+constexpr size_t PC_OFF_CAND = PC_OFF_HE;                          // [2048] u16 candidate entries
+constexpr size_t PC_OFF_QD = PC_OFF_CAND + PT_CAND_MAX * 2;        // [64] float4
+constexpr size_t PC_OFF_TMP = PC_OFF_QD + kID * 16;                // [64] u32
+constexpr size_t PC_OFF_MISC = PC_OFF_TMP + 64 * 4;                // w (float4), l1[4], kmax bits, largest exact key, mbarrier
+constexpr size_t PC_SMEM = PC_OFF_MISC + 48;
+static_assert(PC_OFF_L1 + PT_CAND_MAX * 2 <= PC_OFF_HS, "K5b region A");
+static_assert(PC_SB <= PC_PTAB && 1024 * 4 == PT_CAND_MAX * 2, "K5b regions B and C");
+static_assert(54 + PC_THREADS / 32 <= 64, "K5b scratch words");
+static_assert(PC_CH * 8 * PC_THREADS >= kMaxCand && PC_CH <= 8 && PC_THREADS % 32 == 0, "K5b key chunks");
+static_assert(PC_OFF_QD % 16 == 0 && PC_OFF_MISC % 16 == 0 && PC_OFF_HIST % 16 == 0, "K5b shared-memory layout");
+static_assert(PC_CTAS * (PC_SMEM + 1024) <= 228 * 1024, "K5b residency");
+
+// Key j (0..7) of a chunk of eight 16-bit keys.
+__device__ __forceinline__ uint32_t chunk_key(const uint4& v, int j) {
+    const uint32_t w = j < 2 ? v.x : j < 4 ? v.y : j < 6 ? v.z : v.w;
+    return (j & 1) ? w >> 16 : w & 0xffffu;
+}
+// Largest key of a chunk whose first nv entries are visible.
+__device__ __forceinline__ uint32_t chunk_max(const uint4& v, int nv) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < nv) m = max(m, chunk_key(v, j));
+    return m;
+}
+// Bit j set when key j is >= thr and entry j is visible.  The high key of a
+// word is >= thr exactly when the word is >= thr << 16.
+__device__ __forceinline__ uint32_t chunk_sel(const uint4& v, uint32_t thr, int nv) {
+    const uint32_t th = thr << 16;
+    const uint32_t m = (uint32_t)((v.x << 16) >= th) | ((uint32_t)(v.x >= th) << 1) |
+                       ((uint32_t)((v.y << 16) >= th) << 2) | ((uint32_t)(v.y >= th) << 3) |
+                       ((uint32_t)((v.z << 16) >= th) << 4) | ((uint32_t)(v.z >= th) << 5) |
+                       ((uint32_t)((v.w << 16) >= th) << 6) | ((uint32_t)(v.w >= th) << 7);
+    return nv >= 8 ? m : m & ((1u << max(nv, 0)) - 1u);
+}
+// Histogram (top bin = mx) of the visible keys lying dlo..dhi values below mx.
+__device__ __forceinline__ void chunk_hist_range(const uint4* k16v, int n_ch, int n_vis, uint32_t mx, uint32_t dlo,
+                                                 uint32_t dhi, uint32_t* h) {
+    for (int i = threadIdx.x; i < n_ch; i += PC_THREADS) {
+        const uint4 v = k16v[i];
+        const int nv = n_vis - 8 * i;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t dist = mx - chunk_key(v, j);
+            hist_add(h, 1023u - dist, j < nv && dist - dlo <= dhi - dlo);
+        }
+    }
+}
+
 // float value of an order-preserving key (inverse of score_key)
 __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-constexpr int PC_THREADS = 256;
-constexpr size_t PC_OFF_K16 = 0;                                      // [16384] u16
-constexpr size_t PC_OFF_CK = PC_OFF_K16 + (size_t)kMaxCand * 2;        // [2048] u32 exact keys
-constexpr size_t PC_OFF_CAND = PC_OFF_CK + PT_CAND_MAX * 4;            // [2048] u16 entries
-constexpr size_t PC_OFF_HIST = PC_OFF_CAND + PT_CAND_MAX * 2;          // [4096]
-constexpr size_t PC_OFF_L0 = PC_OFF_HIST + kHistBins * 4;              // [2048] u16
-constexpr size_t PC_OFF_L1 = PC_OFF_L0 + PT_CAND_MAX * 2;              // [2048] u16
-constexpr size_t PC_OFF_QD = PC_OFF_L1 + PT_CAND_MAX * 2;              // [64] float4
-constexpr size_t PC_OFF_TMP = PC_OFF_QD + kID * 16;                    // [64] u32
-constexpr size_t PC_OFF_MISC = PC_OFF_TMP + 64 * 4;                    // w (float4), l1[4], kmax, thr, count
-constexpr size_t PC_SMEM = PC_OFF_MISC + 64;
-static_assert(PC_OFF_QD % 16 == 0 && PC_OFF_MISC % 16 == 0 && PC_OFF_HIST % 16 == 0, "K5b shared-memory layout");
-// the visible entries' page ids (pages hold >= 8 entries) fit in the l0/l1 lists' space
-static_assert((kMaxCand / 8) * 4 <= PC_OFF_QD - PC_OFF_L0, "K5b page-id staging");
-
-__global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(PC_THREADS, PC_CTAS) prefill_candidates_kernel(PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint16_t* k16 = reinterpret_cast<uint16_t*>(smem + PC_OFF_K16);
+    uint4* k16v = reinterpret_cast<uint4*>(smem + PC_OFF_K16);
     uint32_t* ck = reinterpret_cast<uint32_t*>(smem + PC_OFF_CK);
-    uint16_t* cand = reinterpret_cast<uint16_t*>(smem + PC_OFF_CAND);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + PC_OFF_HIST);
     uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + PC_OFF_L0);
     uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + PC_OFF_L1);
+    uint32_t* hs = reinterpret_cast<uint32_t*>(smem + PC_OFF_HS);
+    uint32_t* he = reinterpret_cast<uint32_t*>(smem + PC_OFF_HE);
+    int32_t* ptab = reinterpret_cast<int32_t*>(smem + PC_OFF_PTAB);
+    uint16_t* cand = reinterpret_cast<uint16_t*>(smem + PC_OFF_CAND);
     float4* qd = reinterpret_cast<float4*>(smem + PC_OFF_QD);
     uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + PC_OFF_TMP);
     float4& s_w = *reinterpret_cast<float4*>(smem + PC_OFF_MISC);
     float* s_l1 = reinterpret_cast<float*>(smem + PC_OFF_MISC + 16);       // [4]
-    uint32_t* s_u = reinterpret_cast<uint32_t*>(smem + PC_OFF_MISC + 32);  // kmax bits, count
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(smem + PC_OFF_MISC + 32);  // kmax bits, largest exact key
+    uint64_t* kbar = reinterpret_cast<uint64_t*>(smem + PC_OFF_MISC + 40);  // the keys' bulk copy
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int t = blockIdx.x;
     pdl_wait();
@@ -1631,83 +1675,177 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
     }
     if (tid == 0) {
         s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)t * kIH);
-        s_u[1] = 0;
+        s_u[1] = 0u;
     }
-    {  // the visible entries' 16-bit keys, 16 B at a time (rows are 128 B aligned)
-        const uint4* src = reinterpret_cast<const uint4*>(a.keys16 + (int64_t)t * a.stride);
-        for (int i = tid; i < (n_vis + 7) / 8; i += PC_THREADS) reinterpret_cast<uint4*>(k16)[i] = __ldcg(src + i);
+    // the visible entries' 16-bit keys, 8 to a 16-byte chunk: one bulk copy
+    // (rows are 128 B aligned)
+    const int n_ch = (n_vis + 7) >> 3;
+    if (tid == 0) {
+        mbar_init(kbar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(kbar, (uint32_t)n_ch * 16u);
+        bulk_load(k16v, a.keys16 + (int64_t)t * a.stride, (uint32_t)n_ch * 16u, kbar);
     }
-    for (int i = tid; i < 1024; i += PC_THREADS) hist[i] = 0;
-    __syncthreads();
-
-    // ---- candidates: entries whose 16-bit key is >= that of the PT_CAND-th
-    // largest.  The histogram counts each key's distance below the row's
-    // largest key (one bin per key value, 1024 values = 8 binades); distances
-    // beyond are not counted, and a row whose PT_CAND-th key lies beyond takes
-    // the exact fallback.
     const bool limited = n_vis > PT_CAND;
+    __syncthreads();  // the barrier is initialised; query and weights are staged
+    if (!mbar_wait(kbar, 0u, kWaitLimit)) {
+        if (tid == 0) {
+            dev_error(a.err, CSA2_DEV_TIMEOUT);
+            a.flags[t] = 1;
+        }
+        mbar_wait(kbar, 0u, kWaitLimit);  // the copy may still land: bounded second wait
+        return;
+    }
+
+    // ---- candidates: entries whose 16-bit key is >= thr16.  A histogram of
+    // one key per chunk (entry 8i), counted from the sample's largest key,
+    // puts thr16 at the lower edge of the bin that holds the sample's key of
+    // the rank about PC_SAMPLE_CAND keys clear.  When the count falls outside
+    // [PC_CAND_LO, PT_CAND_MAX], or the sample has too few keys within 8
+    // binades of its largest, thr16 is the PT_CAND-th largest key instead, from
+    // a histogram of every key within 8 binades of the row's largest (a row
+    // whose PT_CAND-th key lies lower takes the exact fallback).  Any threshold
+    // is sound: the candidates' Top-K is verified below against the best score
+    // a non-candidate can reach.
     uint32_t thr16 = 0u;
+    bool sampled = false, need_exact = false;
     if (limited) {
+        for (int i = tid; i < PC_SB; i += PC_THREADS) hs[i] = 0;
+        uint32_t smp[PC_CH];
+        uint32_t smx = 0;
+#pragma unroll
+        for (int c = 0; c < PC_CH; ++c) {
+            const int i = tid + c * PC_THREADS;
+            smp[c] = i < n_ch ? (reinterpret_cast<const uint32_t*>(k16v)[4 * i] & 0xffffu) : 0u;  // entry 8i
+            smx = max(smx, smp[c]);
+        }
+        smx = __reduce_max_sync(0xffffffffu, smx);
+        if (lane == 0) tmp[wid] = smx;
+        __syncthreads();
+        smx = 0;
+        for (int v = 0; v < PC_THREADS / 32; ++v) smx = max(smx, tmp[v]);
+#pragma unroll
+        for (int c = 0; c < PC_CH; ++c) {
+            const uint32_t dist = smx - smp[c];
+            hist_add(hs, (PC_SB - 1) - (dist >> 1), tid + c * PC_THREADS < n_ch && dist < 1024u);
+        }
+        __syncthreads();
+        const uint32_t ks = (uint32_t)(((int64_t)PC_SAMPLE_CAND * n_ch + n_vis - 1) / n_vis);
+        int b;
+        uint32_t above, counted;
+        group_find_kth_bin(hs, PC_SB, ks, tmp, &b, &above, GroupBar{0, PC_THREADS}, &counted);
+        if (counted >= ks) {
+            thr16 = smx - (2u * (uint32_t)(PC_SB - 1 - b) + 1u);
+            sampled = true;
+        } else {
+            need_exact = true;
+        }
+    }
+    // the sample histogram is read: region B takes the page table (loads in
+    // flight through the compaction)
+    const int n_pg = min(((n_vis - 1) >> a.page_shift) + 1, PC_PTAB);
+    for (int j = tid; j < n_pg; j += PC_THREADS)
+        ptab[j] = j < a.cache.max_pages_per_seq ? __ldg(a.cache.page_table + j) : -1;
+    // thr16 = the PT_CAND-th largest key within 8 binades of the maximum;
+    // false (and the row flagged) when fewer keys lie there
+    auto exact_threshold = [&]() -> bool {
         uint32_t mx = 0;
-        for (int i = tid; i < n_vis; i += PC_THREADS) mx = max(mx, (uint32_t)k16[i]);
-        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) tmp[wid] = mx;
+        for (int i = tid; i < n_ch; i += PC_THREADS) mx = max(mx, chunk_max(k16v[i], n_vis - 8 * i));
+        for (int i = tid; i < 1024; i += PC_THREADS) he[i] = 0;
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) tmp[54 + wid] = mx;
         __syncthreads();
         mx = 0;
-        for (int v = 0; v < PC_THREADS / 32; ++v) mx = max(mx, tmp[v]);
-        __syncthreads();
-        for (int i = tid; i < n_vis; i += PC_THREADS) {
-            const uint32_t dist = mx - (uint32_t)k16[i];
-            hist_add(hist, 1023u - dist, dist < 1024u);
-        }
+        for (int v = 0; v < PC_THREADS / 32; ++v) mx = max(mx, tmp[54 + v]);
+        chunk_hist_range(k16v, n_ch, n_vis, mx, 0u, 1023u, he);
         __syncthreads();
         int b;
         uint32_t above, counted;
-        group_find_kth_bin(hist, 1024, PT_CAND, tmp, &b, &above, GroupBar{0, PC_THREADS}, &counted);
-        if (counted < (uint32_t)PT_CAND) {  // the threshold lies more than 8 binades below the maximum
+        group_find_kth_bin(he, 1024, PT_CAND, tmp, &b, &above, GroupBar{0, PC_THREADS}, &counted);
+        if (counted < (uint32_t)PT_CAND) {
             if (tid == 0) a.flags[t] = 1;
-            return;
+            return false;
         }
         thr16 = mx - (1023u - (uint32_t)b);
+        return true;
+    };
+    if (need_exact && !exact_threshold()) return;
+
+    // ---- compaction in entry order (the output must come out ascending):
+    // lane l of warp v owns a contiguous run of cpl chunks (16-byte reads
+    // 16 * cpl bytes apart, distinct banks within each 8-lane phase); the
+    // counting pass keeps each chunk's 8-bit selection mask for the writing
+    // pass, which needs one prefix over the lanes and warps
+    const int cpw = ((n_ch + PC_THREADS / 32 - 1) / (PC_THREADS / 32) + 31) & ~31;
+    const int cpl = cpw >> 5;
+    const int c0 = wid * cpw + lane * cpl;
+    uint32_t mlo = 0, mhi = 0, off = 0;
+    int m = 0;
+    auto count_pass = [&]() {
+        uint32_t mine = 0;
+        mlo = 0;
+        mhi = 0;
+#pragma unroll
+        for (int s = 0; s < PC_CH; ++s) {
+            const int i = c0 + s;
+            uint32_t mk = 0;
+            if (s < cpl && i < n_ch) mk = chunk_sel(k16v[i], thr16, n_vis - 8 * i);
+            mine += __popc(mk);
+            if (s < 4) mlo |= mk << (8 * s);
+            else mhi |= mk << (8 * (s - 4));
+        }
+        const uint32_t inc = warp_incl_scan(mine);
+        if (lane == 31) tmp[wid] = inc;
+        __syncthreads();
+        uint32_t tot = 0;
+        off = inc - mine;
+        for (int v = 0; v < PC_THREADS / 32; ++v) {
+            if (v < wid) off += tmp[v];
+            tot += tmp[v];
+        }
+        m = (int)tot;
+    };
+    count_pass();
+    if (sampled && (m < PC_CAND_LO || m > PT_CAND_MAX)) {
+        if (!exact_threshold()) return;
+        count_pass();
     }
-    // compact in entry order (the output must come out ascending): warp v
-    // walks a contiguous segment, counts, then writes at its prefix offset
-    const int seg = ((n_vis + PC_THREADS / 32 - 1) / (PC_THREADS / 32) + 31) & ~31;
-    const int lo = wid * seg, hi = min(n_vis, lo + seg);
-    uint32_t mine = 0;
-    for (int b = lo; b < hi; b += 32) {
-        const int i = b + lane;
-        mine += __popc(__ballot_sync(0xffffffffu, i < hi && (!limited || (uint32_t)k16[i] >= thr16)));
-    }
-    __syncthreads();
-    if (lane == 0) tmp[wid] = mine;
-    __syncthreads();
-    uint32_t off = 0, m_total = 0;
-    for (int v = 0; v < PC_THREADS / 32; ++v) {
-        if (v < wid) off += tmp[v];
-        m_total += tmp[v];
-    }
-    const int m = (int)m_total;
     if (m > PT_CAND_MAX) {  // too many ties at the 16-bit threshold: exact fallback
         if (tid == 0) a.flags[t] = 1;
         return;
     }
-    for (int b = lo; b < hi; b += 32) {
-        const int i = b + lane;
-        const bool in = i < hi && (!limited || (uint32_t)k16[i] >= thr16);
-        const unsigned bm = __ballot_sync(0xffffffffu, in);
-        if (in) cand[off + __popc(bm & ((1u << lane) - 1u))] = (uint16_t)i;
-        off += __popc(bm);
+#pragma unroll
+    for (int s = 0; s < PC_CH; ++s) {
+        uint32_t mk = (s < 4 ? mlo >> (8 * s) : mhi >> (8 * (s - 4))) & 0xffu;
+        while (mk) {
+            cand[off++] = (uint16_t)(8 * (c0 + s) + __ffs(mk) - 1);
+            mk &= mk - 1u;
+        }
     }
     __syncthreads();
 
     // ---- exact scores of the candidates (the oracle's sequential FMA chains)
+    // and the largest of them
     const float4 w = s_w;
+    const int64_t pmask = (int64_t(1) << a.page_shift) - 1;
+    uint32_t cmx = 0u;
     for (int i = tid; i < m; i += PC_THREADS) {
         const int e = cand[i];
-        const int64_t slot = entry_slot(a.cache, a.page_shift, 0, e, a.err);
-        uint32_t kr[32];
+        int64_t slot;
+        if ((e >> a.page_shift) < n_pg) {
+            const int32_t phys = ptab[e >> a.page_shift];
+            if (phys < 0 || phys >= a.cache.n_phys_pages) {
+                dev_error(a.err, CSA2_DEV_PAGE);
+                slot = -1;
+            } else {
+                slot = ((int64_t)phys << a.page_shift) | ((int64_t)e & pmask);
+            }
+        } else {
+            slot = entry_slot(a.cache, a.page_shift, 0, e, a.err);
+        }
+        uint32_t key = 0u;
         if (slot >= 0) {
+            uint32_t kr[32];
             const uint4* src = reinterpret_cast<const uint4*>(a.cache.idx_k + slot * kID);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -1717,32 +1855,100 @@ __global__ void __launch_bounds__(PC_THREADS) prefill_candidates_kernel(PrefillA
                 kr[4 * c + 2] = v.z;
                 kr[4 * c + 3] = v.w;
             }
-            ck[i] = score_key(idx_score1(kr, qd, w));
-        } else {
-            ck[i] = 0u;
+            key = score_key(idx_score1(kr, qd, w));
         }
+        ck[i] = key;
+        cmx = max(cmx, key);
     }
-    for (int i = tid; i < kHistBins; i += PC_THREADS) hist[i] = 0;
+    for (int i = tid; i < 1024; i += PC_THREADS) hist[i] = 0;
+    cmx = __reduce_max_sync(0xffffffffu, cmx);
+    if (lane == 0) atomicMax(&s_u[1], cmx);
     __syncthreads();
 
-    // ---- exact Top-K among the candidates
-    uint32_t nv = 0;
+    // ---- exact Top-K among the candidates.  First digit: key >> 16 counted
+    // from 1022 values below the largest key's (lower keys share bin 0).  The
+    // K-th key's bin, taken whole or holding at most 32 keys, is resolved by
+    // one warp; otherwise (or when the K-th key lies in the shared bin 0) the
+    // three-digit radix select over the whole key finds it.
+    const uint32_t top16 = s_u[1] >> 16;
+    const uint32_t base = top16 > 1022u ? top16 - 1022u : 0u;
     for (int i = tid; i < m; i += PC_THREADS) {
-        nv += ck[i] != 0u;
-        hist_add(hist, ck[i] >> 20, ck[i] != 0u);
+        const uint32_t k = ck[i];
+        hist_add(hist, (k >> 16) >= base ? (k >> 16) - base : 0u, k != 0u);
     }
-    uint32_t n_valid;
-    block_excl_scan(nv, tmp, &n_valid);
-    const uint32_t kk = min((uint32_t)a.topk, n_valid);
-    if (kk == 0) {
+    __syncthreads();
+    int b1;
+    uint32_t above, n_valid;
+    group_find_kth_bin(hist, 1024, (uint32_t)a.topk, tmp, &b1, &above, GroupBar{0, PC_THREADS}, &n_valid);
+    if (n_valid == 0u) {
         for (int i = tid; i < a.topk; i += PC_THREADS) out[i] = -1;
         if (tid == 0) a.flags[t] = 0;
         return;
     }
-    int b1;
-    uint32_t above, T, need;
-    find_kth_bin(hist, kHistBins, kk, tmp, &b1, &above);
-    refine_threshold(ck, m, (uint32_t)b1, kk - above, hist, l0, l1, tmp, &T, &need);
+    uint32_t kk, T = 0u, need = 0u;
+    if (n_valid <= (uint32_t)a.topk) {
+        kk = n_valid;  // every valid candidate: the keys above 0
+        if (limited) {  // a non-candidate may belong to the Top-K
+            if (tid == 0) a.flags[t] = 1;
+            return;
+        }
+    } else {
+        kk = (uint32_t)a.topk;
+        need = kk - above;
+        const uint32_t nb = hist[b1];
+        const uint32_t hb = base + (uint32_t)b1;  // key >> 16 of the bin's keys (unless the shared bin 0)
+        const bool shared0 = b1 == 0 && base > 0u;
+        if (!shared0 && hb > 0u && nb == need) {  // the bin is taken whole: T just below it, no ties
+            T = (hb << 16) - 1u;
+            need = 0u;
+        } else if (!shared0 && nb <= 32u) {
+            uint32_t* bk = reinterpret_cast<uint32_t*>(l0);  // the bin's keys
+            if (tid == 0) tmp[50] = 0u;
+            __syncthreads();
+            for (int i0 = wid * 32; i0 < m; i0 += PC_THREADS) {
+                const int i = i0 + lane;
+                const uint32_t k = i < m ? ck[i] : 0u;
+                const bool in = k != 0u && (k >> 16) == hb;
+                const unsigned bm = __ballot_sync(0xffffffffu, in);
+                if (bm) {
+                    const int leader = __ffs(bm) - 1;
+                    uint32_t pos = 0;
+                    if (lane == leader) pos = atomicAdd(&tmp[50], (uint32_t)__popc(bm));
+                    pos = __shfl_sync(0xffffffffu, pos, leader);
+                    if (in) bk[pos + __popc(bm & ((1u << lane) - 1u))] = k;
+                }
+            }
+            __syncthreads();
+            if (wid == 0) {  // T = the need-th largest key of the bin
+                const bool mine = (uint32_t)lane < nb;
+                const uint32_t kl = mine ? bk[lane] : 0u;
+                uint32_t ge = 0;
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t kj = __shfl_sync(0xffffffffu, kl, j);
+                    ge += ((uint32_t)j < nb && kj >= kl) ? 1u : 0u;
+                }
+                const uint32_t Tw = __reduce_max_sync(0xffffffffu, mine && ge >= need ? kl : 0u);
+                const uint32_t gt = __popc(__ballot_sync(0xffffffffu, mine && kl > Tw));
+                if (lane == 0) {
+                    tmp[51] = Tw;
+                    tmp[52] = need - gt;
+                }
+            }
+            __syncthreads();
+            T = tmp[51];
+            need = tmp[52];
+        } else {
+            __syncthreads();  // every thread has read hist[b1]
+            for (int i = tid; i < kHistBins; i += PC_THREADS) hist[i] = 0;
+            __syncthreads();
+            for (int i = tid; i < m; i += PC_THREADS) hist_add(hist, ck[i] >> 20, ck[i] != 0u);
+            __syncthreads();
+            int g1;
+            uint32_t ab;
+            find_kth_bin(hist, kHistBins, kk, tmp, &g1, &ab);
+            refine_threshold(ck, m, (uint32_t)g1, kk - ab, hist, l0, l1, tmp, &T, &need);
+        }
+    }
     // ---- no entry outside the candidates can reach the K-th exact score
     if (limited) {
         const double bound = (double)key_value(thr16 << 16);  // non-candidates score below this (approximately)

@@ -8,6 +8,22 @@
 
 namespace csa2 {
 
+// Two fp32 lanes in one 64-bit register; fma.rn.f32x2 rounds each lane as
+// fma.rn.f32 does (the two-row score chains of the block-level scorer).
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
 // Score of one indexer-K row held as 32 bf16x2 words, qd[d] = (q_0..q_3)[d] in
 // fp32: each head's dot product is a sequential FMA chain over d = 0..63 and
 // the head sum a sequential FMA chain over h = 0..3 of w_h * max(dot_h, 0).

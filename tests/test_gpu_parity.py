@@ -495,6 +495,35 @@ def test_prefill_indexer_exact_fallback_on_ties(csa2, orc):
     assert ps.errors() == 0
 
 
+def test_prefill_indexer_sampled_entries_lead(csa2, orc):
+    # Every eighth entry's indexer-K row is scaled by 4, so those entries hold
+    # the largest scores.  A threshold estimated from one key per 8 entries then
+    # sits far too high and the candidates kernel must count the remaining keys
+    # too; the sets must still equal the oracle's.
+    seed = 1003
+    n_ent = 8000
+    tokens = 2 * n_ent
+    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    kv = synth.kv_rows(seed, 2, 0, tokens)
+    kf = orc.bf16_to_f32(synth.idx_k_rows(seed, 2, 0, n_ent)).reshape(n_ent, 64)
+    kf[::8] *= 4.0
+    idx_k = synth.to_bf16_bits(kf)
+    ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=999)
+    q_pos = np.concatenate([np.arange(3000, 3100), np.arange(tokens - 300, tokens)]).astype(np.int32)
+    T = len(q_pos)
+    q_idx = synth.q_idx(seed, 2, 0, T)
+    w = synth.w_idx(seed, 2, 0, T)
+    d = csa2.default_desc(csa2.FULL, 2)
+    ws = _ws(csa2, T, n_ent, prefill=True)
+    out_idx = torch.empty((T, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q_idx), dev(w), dev(np.array([n_ent], np.int32)), out_idx, T,
+                      n_ent, ws, q_pos=dev(q_pos), err=ps.err)
+    want = orc.prefill_indexer(q_pos, 2, n_ent, idx_k, q_idx, w)
+    assert (want[-1] % 8 == 0).mean() > 0.5  # the scaled entries dominate the sets
+    check_sets(out_idx.cpu().numpy(), want, "prefill indexer, sampled entries lead")
+    assert ps.errors() == 0
+
+
 # ---------------------------------------------------------------------------
 # device-side error reporting (bounds checks turn bad input into flags)
 # ---------------------------------------------------------------------------
