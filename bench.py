@@ -276,10 +276,10 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    if flat:  # Full: block_score + block_select over entries (token kernel at <= 16,384), then attention
-        launches_per_step = 1 + sum((3 if L > 16384 else 2) if m != csa2.REUSE else 1 for m in modes)
+    if flat:  # Full: block_score + block_select over entries (token score + select at <= 16,384), then attention
+        launches_per_step = 1 + sum(3 if m != csa2.REUSE else 1 for m in modes)
     else:
-        launches_per_step = 1 + sum({csa2.FULL: 4, csa2.REINDEX: 2, csa2.REUSE: 1}[m] for m in modes)
+        launches_per_step = 1 + sum({csa2.FULL: 5, csa2.REINDEX: 3, csa2.REUSE: 1}[m] for m in modes)
     if args.kv_host:  # each new index set's rows are staged on the device once
         launches_per_step += n_idx
 

@@ -28,9 +28,11 @@
 //                              collect the bin's members; the last CTA refines
 //                              the boundary and emits the kept rows in order
 //                              (a flat selection lists and sorts them).
-//   token_topk_kernel   (K4)  one 8-CTA cluster per sequence scores the
-//                              <= 16,384 candidates (1 KiB runs of 8 indexer-K
-//                              rows) and selects the Top-K across the cluster.
+//   token_score_kernel  (K4a) 16 CTAs per sequence score the <= 16,384
+//                              candidates (1 KiB runs of 8 indexer-K rows) into
+//                              the workspace;
+//   token_select_kernel (K4b) one 8-CTA cluster per sequence selects the
+//                              Top-K across the cluster.
 //   prefill_tc_score_kernel / prefill_candidates_kernel: prefill, approximate
 //                              scores on tcgen05, exact rescoring of the
 //                              candidates and a verified exact Top-K per query;
@@ -799,40 +801,46 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
 }
 
 // ============================================================================
-// K4: token scores over the candidates + Top-K, one 8-CTA cluster per sequence
+// K4: token scores over the candidates + Top-K, in two kernels.
 //
-// CTA r of a sequence's cluster scores candidate slots [2048 r, 2048 r + 2048):
-// each warp copies the indexer-K rows of its candidate blocks (a block's 8 rows
-// are one 1 KiB run) with 16-byte cp.async into its own slice of a 2-stage
-// ring, and every thread scores one row per round.  The radix select then runs
-// across the cluster: each CTA adds its digit histogram into every CTA's
-// receive buffer (red.shared::cluster), one cluster barrier follows, every CTA
-// locates the bin holding the K-th key, and the next digit repeats this on the
-// survivors only; a bin whose keys are all taken ends the search.  The ordered
-// emission exchanges per-CTA counts the same way, so every CTA writes its
-// selected positions at its own offset, ascending.
+// K4a token_score_kernel: 16 CTAs per sequence; CTA p scores candidate slots
+// [1024 p, 1024 p + 1024).  Warp w copies the indexer-K rows of its 8
+// candidate blocks (a block's 8 rows are one 1 KiB run) into its own 8 KiB of
+// shared memory, as 8-row tensor boxes (128-byte swizzled, counted on the
+// warp's barrier) or with 16-byte cp.async into the same layout; lane l then
+// scores the warp's rows l and l + 32 with the two-row packed chains.  The
+// exact keys go to the workspace, 0 for slots without a candidate.
+//
+// K4b token_select_kernel: one CTA per sequence; thread t holds keys
+// [16 t, 16 t + 16) in registers.  First digit: key >> 16 counted from 1022
+// values below the largest key's (lower keys share bin 0), a histogram whose
+// atomics spread over hundreds of bins.  The K-th key's bin, taken whole or
+// holding at most 32 keys, is resolved by one warp; otherwise (or when the
+// K-th key lies in the shared bin 0) a 12-bit digit and two 10-bit digits
+// over the shrinking survivor lists find it.  The emission takes two block
+// scans (ties at the threshold, then selected counts) and writes each
+// thread's positions in slot order.
 // ============================================================================
-constexpr int TK_CL = 8;
-constexpr int TK_THREADS = 512;
-constexpr int TK_SLOTS = kMaxCand / TK_CL;  // 2048 candidate slots per CTA
-constexpr int TK_ROUND = TK_THREADS;        // rows per round
-constexpr int TK_BLKS = TK_SLOTS / kBlk;    // 256 candidate blocks per CTA
-constexpr size_t TK_STAGE_BYTES = (size_t)TK_ROUND * 128;
-constexpr size_t TK_OFF_KEYS = 2 * TK_STAGE_BYTES;
-constexpr size_t TK_OFF_HIST = align16(TK_OFF_KEYS + TK_SLOTS * 4);
-constexpr size_t TK_OFF_G1 = align16(TK_OFF_HIST + kHistBins * 4);
-constexpr size_t TK_OFF_G2 = align16(TK_OFF_G1 + kHistBins * 4);
-constexpr size_t TK_OFF_G3 = align16(TK_OFF_G2 + 1024 * 4);
-constexpr size_t TK_OFF_GCNT = align16(TK_OFF_G3 + 1024 * 4);
-constexpr size_t TK_OFF_L0 = align16(TK_OFF_GCNT + 2 * TK_CL * 4);
-constexpr size_t TK_OFF_L1 = align16(TK_OFF_L0 + TK_SLOTS * 2);
-constexpr size_t TK_OFF_BSLOT = align16(TK_OFF_L1 + TK_SLOTS * 2);
-constexpr size_t TK_OFF_BPOS = align16(TK_OFF_BSLOT + TK_BLKS * 8);
-constexpr size_t TK_OFF_QD = align16(TK_OFF_BPOS + TK_BLKS * 4);
-constexpr size_t TK_OFF_TMP = align16(TK_OFF_QD + kID * 16);
-constexpr size_t TK_OFF_MISC = align16(TK_OFF_TMP + 64 * 4);  // w (float4), two counters
-constexpr size_t TK_SMEM = align16(TK_OFF_MISC + 32);
-static_assert(TK_OFF_BSLOT % 8 == 0 && TK_OFF_QD % 16 == 0 && TK_OFF_MISC % 16 == 0, "K4 shared-memory layout");
+constexpr int TS_PARTS = 16;
+constexpr int TS_SLOTS = kMaxCand / TS_PARTS;  // 1024 candidate slots per CTA
+constexpr int TS_THREADS = 512;               // two rows per thread
+constexpr int TS_BLKS = TS_SLOTS / kBlk;       // 128 candidate blocks per CTA, 8 per warp
+constexpr size_t TS_OFF_QP = (size_t)TS_SLOTS * 128;                // rows | q pairs [128] float4
+constexpr size_t TS_OFF_MISC = TS_OFF_QP + 2 * kID * 16;             // w (float4)
+constexpr size_t TS_OFF_BAR = TS_OFF_MISC + 16;                      // [16] per-warp copy barriers
+constexpr size_t TS_SMEM = TS_OFF_BAR + (TS_THREADS / 32) * 8;
+static_assert(TS_BLKS == 8 * (TS_THREADS / 32), "K4a: 8 candidate blocks per warp");
+
+constexpr int TK_THREADS = 1024;
+constexpr int TK_PER = kMaxCand / TK_THREADS;                        // 16 keys per thread
+constexpr size_t TK_OFF_KEYS = 0;                                   // [16384] u32
+constexpr size_t TK_OFF_HIST = TK_OFF_KEYS + (size_t)kMaxCand * 4;   // [4096] u32
+constexpr size_t TK_OFF_L0 = TK_OFF_HIST + kHistBins * 4;            // [16384] u16
+constexpr size_t TK_OFF_L1 = TK_OFF_L0 + (size_t)kMaxCand * 2;       // [16384] u16
+constexpr size_t TK_OFF_TMP = TK_OFF_L1 + (size_t)kMaxCand * 2;      // [64] u32
+constexpr size_t TK_OFF_BK = TK_OFF_TMP + 64 * 4;                    // [32] u32 keys of the K-th bin
+constexpr size_t TK_SMEM = TK_OFF_BK + 32 * 4;
+static_assert(kMaxCand == kMaxKeep * kBlk && TK_PER % 4 == 0, "K4b shared-memory layout");
 
 // The earlier (non-cluster) layout constants are still used by the prefill select.
 constexpr size_t K4_OFF_HIST = (size_t)kMaxCand * 4;
@@ -847,262 +855,254 @@ struct TokenArgs {
     const int32_t* seq_lens;
     const int32_t* cand;  // [n][keep] or null (flat)
     int32_t* out;         // [n][topk]
+    uint32_t* keys;       // [n][16384] exact keys, K4a -> K4b
     int32_t* err;
     int64_t max_len;
     int keep, topk, page_shift;
     int pre;  // 1: the lengths, cand and the cache may be read before the preceding kernel completes
+    int tma;  // 1: candidate blocks arrive as 8-row tensor boxes (else 16-byte cp.async)
 };
 
-// Push this CTA's histogram (nonzero bins only) into the receive histogram of
-// every CTA of the cluster.  Whole CTA.
-__device__ __forceinline__ void push_hist(const uint32_t* lhist, int nbins, uint32_t* recv) {
-    const uint32_t base = smem_u32(recv);
-    for (int i = threadIdx.x; i < nbins; i += blockDim.x) {
-        const uint32_t v = lhist[i];
-        if (v) {
-#pragma unroll
-            for (int c = 0; c < TK_CL; ++c) red_add_cluster(mapa_shared(base + 4u * i, c), v);
-        }
+// Candidate slot range [s0, s1) of a CTA holding `span` slots from s0, and the
+// first position of candidate block k of the sequence (-1: none).
+struct TokenSlots {
+    int32_t L;
+    int s0, s1;
+    __device__ TokenSlots(const TokenArgs& a, int b, int part, int span, bool report) {
+        L = seq_len_checked(a.seq_lens, b, a.max_len, report ? a.err : nullptr);
+        const int32_t cap = a.keep * kBlk;
+        const int nslots = a.cand ? cap : min(L, cap);
+        if (!a.cand && L > cap && report && threadIdx.x == 0) dev_error(a.err, CSA2_DEV_LEN);
+        s0 = part * span;
+        s1 = max(s0, min(s0 + span, nslots));
     }
-}
+    __device__ int32_t block_pos(const TokenArgs& a, int b, int i) const {  // i: first slot of the block
+        if (i >= s1) return -1;
+        const int32_t blk = a.cand ? __ldg(a.cand + (int64_t)b * a.keep + (i >> 3)) : (i >> 3);
+        return (blk >= 0 && blk * kBlk < L) ? blk * kBlk : -1;
+    }
+};
 
-__global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS)
-    token_topk_kernel(TokenArgs a) {
+__global__ void __launch_bounds__(TS_THREADS, 1)
+    token_score_kernel(const __grid_constant__ CUtensorMap tmap, TokenArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + TK_OFF_KEYS);
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);    // local histogram
-    uint32_t* g1 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G1);        // received, digit 1 (4096)
-    uint32_t* g2 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G2);        // received, digit 2 (1024)
-    uint32_t* g3 = reinterpret_cast<uint32_t*>(smem + TK_OFF_G3);        // received, digit 3 (1024)
-    uint32_t* gcnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_GCNT);    // received per-CTA counts [8][2]
-    uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L0);
-    uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L1);
-    int64_t* bslot = reinterpret_cast<int64_t*>(smem + TK_OFF_BSLOT);
-    int32_t* bpos = reinterpret_cast<int32_t*>(smem + TK_OFF_BPOS);
-    float4* qd = reinterpret_cast<float4*>(smem + TK_OFF_QD);
-    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
-    float4& s_w = *reinterpret_cast<float4*>(smem + TK_OFF_MISC);
-    uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + TK_OFF_MISC + 16);
-    const int r = blockIdx.x % TK_CL;
-    const int b = blockIdx.x / TK_CL;
+    float4* qp = reinterpret_cast<float4*>(smem + TS_OFF_QP);
+    float4& s_w = *reinterpret_cast<float4*>(smem + TS_OFF_MISC);
+    const int part = blockIdx.x % TS_PARTS;
+    const int b = blockIdx.x / TS_PARTS;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
     // With a.pre (a Reindex layer inside the decode driver: its candidates come
     // from the Full layer, launches back) the candidates' slots are resolved
-    // and their first rows copied before waiting on the preceding kernel; q_idx
-    // and w, which a model computes from the previous layer's output, are read
+    // and their rows copied before waiting on the preceding kernel; q_idx and
+    // w, which a model computes from the previous layer's output, are read
     // after the wait.
     const bool pre = a.pre != 0;
     if (!pre) {
         pdl_wait();
         pdl_trigger();
     }
-    // 16-byte copies and vector reads need an aligned base; the check is
-    // uniform over the grid, so no CTA waits at a cluster barrier for one that left
-    if (smem_u32(smem) & 15u) {
+    // 16-byte copies need a 16-byte aligned base, 128-byte-swizzled tensor
+    // boxes a 1 KiB aligned one (uniform over the grid)
+    if (smem_u32(smem) & (a.tma ? 1023u : 15u)) {
         if (pre) pdl_wait();
-        if (tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_ALIGN);
+        if (tid == 0 && part == 0) dev_error(a.err, CSA2_DEV_ALIGN);
         return;
     }
-    const int32_t L = seq_len_checked(a.seq_lens, b, a.max_len, a.err);
-    const int32_t cap = a.keep * kBlk;
-    const int nslots = a.cand ? cap : min(L, cap);
-    if (!a.cand && L > cap && tid == 0 && r == 0) dev_error(a.err, CSA2_DEV_LEN);
-    const int s0 = r * TK_SLOTS, s1 = max(s0, min(s0 + TK_SLOTS, nslots));
-
-    // candidate blocks of this CTA: first position and first slot
-    for (int k = tid; k < TK_BLKS; k += TK_THREADS) {
-        const int i = s0 + k * kBlk;
-        int32_t p = -1;
-        int64_t sl = -1;
-        if (i < s1) {
-            const int32_t blk = a.cand ? __ldg(a.cand + (int64_t)b * a.keep + (i >> 3)) : (i >> 3);
-            if (blk >= 0 && blk * kBlk < L) {
-                p = blk * kBlk;
-                sl = entry_slot(a.cache, a.page_shift, b, p, a.err);
-            }
+    const TokenSlots ts(a, b, part, TS_SLOTS, part == 0);
+    // warp w: candidate blocks 8 w + j (lane j < 8 resolves one), rows 64 w ..
+    uint8_t* wrows = smem + (size_t)wid * 64 * 128;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + TS_OFF_BAR) + wid;
+    int32_t mypos = -1;
+    int64_t myslot = -1;
+    if (lane < 8) {
+        const int32_t p = ts.block_pos(a, b, ts.s0 + (8 * wid + lane) * kBlk);
+        if (p >= 0) {
+            myslot = entry_slot(a.cache, a.page_shift, b, p, a.err);
+            mypos = myslot >= 0 ? p : -1;
         }
-        bpos[k] = sl >= 0 ? p : -1;
-        bslot[k] = sl;
     }
-    for (int i = tid; i < kHistBins; i += TK_THREADS) {
-        hist[i] = 0;
-        g1[i] = 0;
-    }
-    for (int i = tid; i < 1024; i += TK_THREADS) {
-        g2[i] = 0;
-        g3[i] = 0;
-    }
-    if (tid < 2 * TK_CL) gcnt[tid] = 0;
-    __syncthreads();
-    cluster_arrive();  // receive buffers are zero; peers wait for this before pushing
-
-    // Rows of round k: slot s0 + 512 k + 32 w + l belongs to lane l of warp w,
-    // which scores it.  The warp copies its 32 rows (4 candidate blocks of 8
-    // contiguous indexer-K rows) into its own slice of a 2-stage ring with
-    // 16-byte cp.async, lane l moving chunk l & 7 of row 4 j + l / 8, and
-    // waits only for its own copies.
-    const int nrounds = (s1 - s0 + TK_ROUND - 1) / TK_ROUND;
-    const uint8_t* idx_k = reinterpret_cast<const uint8_t*>(a.cache.idx_k);
-    auto row_src = [&](int k) {  // physical entry of this lane's row in round k, -1 if none
-        const int my = k * TK_ROUND + tid;
-        const int blk = my >> 3, e = my & 7;
-        return (s0 + my < s1 && bpos[blk] >= 0 && bpos[blk] + e < L) ? (int32_t)(bslot[blk] + e) : -1;
-    };
-    auto issue = [&](int k) {
-        const int32_t src = k < nrounds ? row_src(k) : -1;
-        uint8_t* slice = smem + (size_t)(k & 1) * TK_STAGE_BYTES + (size_t)wid * (32 * 128);
+    if (a.tma) {
+        if (lane == 0) {
+            mbar_init(bar, 1);  // lane 0's expect-tx arrival
+            fence_mbar_init();
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, myslot >= 0);
+        if (lane == 0) mbar_arrive_expect_tx(bar, 1024u * (uint32_t)__popc(m));
+        __syncwarp();
+        if (myslot >= 0) tma_load_2d(wrows + lane * 1024, &tmap, 0, (int32_t)myslot, bar);
+    } else {
+        // lane l moves chunk l & 7 of row 4 j + l / 8 into the swizzled layout
+        const uint8_t* idx_k = reinterpret_cast<const uint8_t*>(a.cache.idx_k);
         const int c = lane & 7;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
             const int rr = 4 * j + (lane >> 3);
-            const int32_t ps = __shfl_sync(0xffffffffu, src, rr);
-            if (ps >= 0) cp_async16(slice + rr * 128 + ((c ^ (rr & 7)) << 4), idx_k + (int64_t)ps * 128 + c * 16);
+            const int64_t sl = __shfl_sync(0xffffffffu, myslot, rr >> 3);
+            if (sl >= 0) cp_async16(wrows + rr * 128 + ((c ^ (rr & 7)) << 4), idx_k + (sl + (rr & 7)) * 128 + c * 16);
         }
-        cp_async_commit();  // possibly empty: the wait below always leaves the newest group
-    };
-    issue(0);
-    issue(1);
+        cp_async_commit();
+    }
     if (pre) {
         pdl_wait();
         pdl_trigger();
     }
-    load_q_idx(a.q_idx + (int64_t)b * kIH * kID, qd);
+    load_q_pairs(a.q_idx + (int64_t)b * kIH * kID, qp, tid, TS_THREADS);
     if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
-    __syncthreads();  // qd and s_w
-    for (int k = 0; k < nrounds; ++k) {
-        cp_async_wait<1>();
-        __syncwarp();  // the other lanes' copies of this warp's rows are visible
-        uint32_t key = 0u;
-        if (row_src(k) >= 0) {
-            uint32_t kr[32];
-            read_row(smem + (size_t)(k & 1) * TK_STAGE_BYTES + (size_t)wid * (32 * 128), lane, kr);
-            key = score_key(idx_score1(kr, qd, s_w));
-        }
-        keys[k * TK_ROUND + tid] = key;
-        hist_add(hist, key >> 20, key != 0u);
-        __syncwarp();  // every lane has read the slice before it is refilled
-        issue(k + 2);
+    __syncthreads();  // q pairs and w
+    if (a.tma) {
+        if (!mbar_wait(bar, 0u, kWaitLimit) && lane == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
+    } else {
+        cp_async_wait<0>();
     }
-    for (int i = nrounds * TK_ROUND + tid; i < TK_SLOTS; i += TK_THREADS) keys[i] = 0u;
-    __syncthreads();  // the local histogram is complete
+    __syncwarp();  // the warp's rows are visible to all its lanes
+    const int32_t pA = __shfl_sync(0xffffffffu, mypos, lane >> 3);
+    const int32_t pB = __shfl_sync(0xffffffffu, mypos, 4 + (lane >> 3));
+    uint32_t kA[32], kB[32];
+    read_row(wrows, lane, kA);
+    read_row(wrows, lane + 32, kB);
+    float sA, sB;
+    idx_score2(kA, kB, reinterpret_cast<const ulonglong2*>(qp), s_w, sA, sB);
+    uint32_t* keys = a.keys + (int64_t)b * kMaxCand + ts.s0 + 64 * wid;
+    keys[lane] = (pA >= 0 && pA + (lane & 7) < ts.L) ? score_key(sA) : 0u;
+    keys[lane + 32] = (pB >= 0 && pB + (lane & 7) < ts.L) ? score_key(sB) : 0u;
+}
 
-    // ---- cluster radix select: every CTA receives every CTA's histogram -----
-    cluster_wait();  // peers' receive buffers are zero
-    push_hist(hist, kHistBins, g1);
-    cluster_sync_all();
-    uint32_t nv = 0;
-    for (int i = tid; i < kHistBins; i += TK_THREADS) nv += g1[i];
-    uint32_t n_valid;
-    block_excl_scan(nv, tmp, &n_valid);
-    const uint32_t kk = min((uint32_t)a.topk, n_valid);
+__global__ void __launch_bounds__(TK_THREADS, 1) token_select_kernel(TokenArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + TK_OFF_KEYS);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + TK_OFF_HIST);
+    uint16_t* l0 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L0);
+    uint16_t* l1 = reinterpret_cast<uint16_t*>(smem + TK_OFF_L1);
+    uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + TK_OFF_TMP);
+    uint32_t* bk = reinterpret_cast<uint32_t*>(smem + TK_OFF_BK);
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
+    if (tid == 0) tmp[50] = 0u;  // the K-th bin's key count
+    pdl_wait();
+    pdl_trigger();
+    if (smem_u32(smem) & 15u) {  // vector reads need an aligned base (uniform)
+        if (tid == 0 && b == 0) dev_error(a.err, CSA2_DEV_ALIGN);
+        return;
+    }
+    // every load at once: the length, the two candidate blocks of this
+    // thread's 16 slots (blocks 2t, 2t + 1) and its keys (0: no candidate)
+    static_assert(TK_PER == 2 * kBlk, "K4b: two candidate blocks per thread");
+    const int32_t Lraw = __ldg(a.seq_lens + b);
+    int32_t c0 = 2 * tid, c1 = 2 * tid + 1;
+    if (a.cand) {
+        c0 = c0 < a.keep ? __ldg(a.cand + (int64_t)b * a.keep + c0) : -1;
+        c1 = c1 < a.keep ? __ldg(a.cand + (int64_t)b * a.keep + c1) : -1;
+    }
+    uint32_t kr[TK_PER];
+    uint32_t mx = 0u;
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(a.keys + (int64_t)b * kMaxCand) + tid * (TK_PER / 4);
+#pragma unroll
+        for (int j = 0; j < TK_PER / 4; ++j) {
+            const uint4 v = __ldcg(src + j);
+            kr[4 * j] = v.x;
+            kr[4 * j + 1] = v.y;
+            kr[4 * j + 2] = v.z;
+            kr[4 * j + 3] = v.w;
+            reinterpret_cast<uint4*>(keys)[tid * (TK_PER / 4) + j] = v;
+        }
+#pragma unroll
+        for (int j = 0; j < TK_PER; ++j) mx = max(mx, kr[j]);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) tmp[wid] = mx;
+    __syncthreads();
+    mx = 0u;
+    for (int v = 0; v < TK_THREADS / 32; ++v) mx = max(mx, tmp[v]);
+    const uint32_t top16 = mx >> 16;
+    const uint32_t base = top16 > 1022u ? top16 - 1022u : 0u;
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        const uint32_t k = kr[j];
+        hist_add(hist, (k >> 16) >= base ? (k >> 16) - base : 0u, k != 0u);
+    }
+    __syncthreads();  // every thread has read tmp; the histogram is complete
+    int b1;
+    uint32_t above, n_valid;
+    group_find_kth_bin(hist, 1024, (uint32_t)a.topk, tmp, &b1, &above, GroupBar{0, TK_THREADS}, &n_valid);
     int32_t* out = a.out + (int64_t)b * a.topk;
-    uint32_t T = 0xffffffffu, need = 0;
-    if (kk > 0) {  // uniform across the cluster
-        int b1, d2, d3;
-        uint32_t above;
-        find_kth_bin(g1, kHistBins, kk, tmp, &b1, &above);
+    uint32_t kk, T = 0u, need = 0u;  // selected: keys > T and the first `need` keys == T
+    if (n_valid <= (uint32_t)a.topk) {
+        kk = n_valid;  // every valid candidate: the keys above 0
+    } else {
+        kk = (uint32_t)a.topk;
         need = kk - above;
-        // A bin whose keys are all taken ends the search: T just below it, no
-        // ties (the histograms are the cluster's, so every CTA decides alike).
-        if (b1 > 0 && g1[b1] == need) {
-            T = ((uint32_t)b1 << 20) - 1u;
-            need = 0;
-        } else {
-            // digit 2 (bits 19..10) over this CTA's survivors of digit 1
-            if (tid == 0) {
-                s_cnt[0] = 0;
-                s_cnt[1] = 0;
-            }
-            for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
-            __syncthreads();
-            for (int base = wid * 32; base < TK_SLOTS; base += TK_THREADS) {
-                const int i = base + lane;
-                const uint32_t k = keys[i];
-                const bool in = k != 0u && (int)(k >> 20) == b1;
-                list_append(l0, &s_cnt[0], (uint32_t)i, in);
-                hist_add(hist, (k >> 10) & 1023u, in);
+        const uint32_t nb = hist[b1];
+        const uint32_t hb = base + (uint32_t)b1;  // key >> 16 of the bin's keys (unless the shared bin 0)
+        const bool shared0 = b1 == 0 && base > 0u;
+        if (!shared0 && hb > 0u && nb == need) {  // the bin is taken whole: T just below it, no ties
+            T = (hb << 16) - 1u;
+            need = 0u;
+        } else if (!shared0 && nb <= 32u) {
+#pragma unroll
+            for (int j = 0; j < TK_PER; ++j) {
+                const uint32_t k = kr[j];
+                if (k != 0u && (k >> 16) == hb) bk[atomicAdd(&tmp[50], 1u)] = k;
             }
             __syncthreads();
-            push_hist(hist, 1024, g2);
-            cluster_sync_all();
-            find_kth_bin(g2, 1024, need, tmp, &d2, &above);
-            need -= above;
-            if (g2[d2] == need) {
-                T = (((uint32_t)b1 << 20) | ((uint32_t)d2 << 10)) - 1u;
-                need = 0;
-            } else {
-                const int n0 = (int)s_cnt[0];
-                for (int i = tid; i < 1024; i += TK_THREADS) hist[i] = 0;
-                __syncthreads();
-                for (int base = wid * 32; base < n0; base += TK_THREADS) {
-                    const int i = base + lane;
-                    const int slot = i < n0 ? (int)l0[i] : 0;
-                    const uint32_t k = i < n0 ? keys[slot] : 0u;
-                    const bool in = i < n0 && (int)((k >> 10) & 1023u) == d2;
-                    list_append(l1, &s_cnt[1], (uint32_t)slot, in);
-                    hist_add(hist, k & 1023u, in);
+            if (wid == 0) {  // T = the need-th largest key of the bin
+                const bool mine = (uint32_t)lane < nb;
+                const uint32_t kl = mine ? bk[lane] : 0u;
+                uint32_t ge = 0;
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t kj = __shfl_sync(0xffffffffu, kl, j);
+                    ge += ((uint32_t)j < nb && kj >= kl) ? 1u : 0u;
                 }
-                __syncthreads();
-                push_hist(hist, 1024, g3);
-                cluster_sync_all();
-                find_kth_bin(g3, 1024, need, tmp, &d3, &above);
-                need -= above;
-                T = ((uint32_t)b1 << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+                const uint32_t Tw = __reduce_max_sync(0xffffffffu, mine && ge >= need ? kl : 0u);
+                const uint32_t gt = __popc(__ballot_sync(0xffffffffu, mine && kl > Tw));
+                if (lane == 0) {
+                    tmp[51] = Tw;
+                    tmp[52] = need - gt;
+                }
             }
+            __syncthreads();
+            T = tmp[51];
+            need = tmp[52];
+        } else {  // three digits over the whole key
+            __syncthreads();  // every thread has read hist[b1]
+            for (int i = tid; i < kHistBins; i += TK_THREADS) hist[i] = 0;
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < TK_PER; ++j) hist_add(hist, kr[j] >> 20, kr[j] != 0u);
+            __syncthreads();
+            int g1;
+            uint32_t ab;
+            find_kth_bin(hist, kHistBins, kk, tmp, &g1, &ab);
+            refine_threshold(keys, kMaxCand, (uint32_t)g1, kk - ab, hist, l0, l1, tmp, &T, &need);
         }
     }
-
-    // ---- ordered emission: per-CTA counts to every CTA, then own offsets -----
-    const unsigned lt = (1u << lane) - 1u;
-    constexpr int SEG = TK_SLOTS / (TK_THREADS / 32);  // 128 slots per warp
-    uint32_t n_gt = 0, n_eq = 0;
-    for (int base = wid * SEG; base < wid * SEG + SEG; base += 32) {
-        const uint32_t k = keys[base + lane];
-        n_gt += __popc(__ballot_sync(0xffffffffu, k > T && T != 0xffffffffu));
-        n_eq += __popc(__ballot_sync(0xffffffffu, k == T));
+    // ---- emission in slot order: one scan of (ties at T, keys above T); the
+    // ties taken before this thread are min(its tie prefix, need)
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        gt += kr[j] > T ? 1u : 0u;
+        eq += (kr[j] == T && kr[j] != 0u) ? 1u : 0u;
     }
-    __syncthreads();
-    if (lane == 0) {
-        tmp[wid] = n_eq;
-        tmp[32 + wid] = n_gt;
+    uint32_t tot;
+    __syncthreads();  // tmp is free
+    const uint32_t pre = block_excl_scan((eq << 16) | gt, tmp, &tot);  // both counts < 2^15
+    const uint32_t tie_base = pre >> 16;
+    const uint32_t take = tie_base >= need ? 0u : min(eq, need - tie_base);
+    uint32_t pos = (pre & 0xffffu) + min(tie_base, need), ties = 0;
+    const int32_t L = (Lraw >= 1 && Lraw <= a.max_len) ? Lraw : 0;
+    const int32_t p0 = (c0 >= 0 && c0 * kBlk < L) ? c0 * kBlk : -1;
+    const int32_t p1 = (c1 >= 0 && c1 * kBlk < L) ? c1 * kBlk : -1;
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        const uint32_t k = kr[j];
+        const bool tie = k == T && k != 0u;
+        if (k > T || (tie && ties < take)) out[pos++] = (j < kBlk ? p0 : p1) + (j & 7);
+        ties += tie ? 1u : 0u;
     }
-    __syncthreads();
-    if (tid < TK_CL) {  // lane c sends this CTA's totals to CTA c
-        uint32_t e = 0, g = 0;
-        for (int v = 0; v < TK_THREADS / 32; ++v) {
-            e += tmp[v];
-            g += tmp[32 + v];
-        }
-        st_cluster_u32(mapa_shared(smem_u32(gcnt + 2 * r), tid), e);
-        st_cluster_u32(mapa_shared(smem_u32(gcnt + 2 * r + 1), tid), g);
-    }
-    cluster_sync_all();  // last exchange: no CTA touches another's memory after this
-    uint32_t tie_base = 0, sel_base = 0;
-    for (int c = 0; c < r; ++c) {
-        const uint32_t e = gcnt[2 * c], g = gcnt[2 * c + 1];
-        const uint32_t take = tie_base >= need ? 0u : min(e, need - tie_base);
-        sel_base += g + take;
-        tie_base += e;
-    }
-    for (int v = 0; v < wid; ++v) {
-        const uint32_t take = tie_base >= need ? 0u : min(tmp[v], need - tie_base);
-        sel_base += tmp[32 + v] + take;
-        tie_base += tmp[v];
-    }
-    for (int base = wid * SEG; base < wid * SEG + SEG; base += 32) {
-        const int i = base + lane;
-        const uint32_t k = keys[i];
-        const unsigned meq = __ballot_sync(0xffffffffu, k == T);
-        const uint32_t rank = tie_base + __popc(meq & lt);
-        const bool sel = (k > T && T != 0xffffffffu) || (k == T && rank < need);
-        const unsigned msel = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[sel_base + __popc(msel & lt)] = bpos[i >> 3] + (i & 7);
-        sel_base += __popc(msel);
-        tie_base += __popc(meq);
-    }
-    if (r == 0)
-        for (int i = (int)kk + tid; i < a.topk; i += TK_THREADS) out[i] = -1;
+    for (int i = (int)kk + tid; i < a.topk; i += TK_THREADS) out[i] = -1;
 }
 
 // ============================================================================
@@ -2030,12 +2030,12 @@ static cudaError_t ensure_smem(const void* fn, size_t bytes, bool* done) {
 
 // The indexer-K rows as a 2-D tensor [n_slots][64] bf16 read in 64-row boxes,
 // 128-byte swizzled.  Returns false when the map cannot be made.
-static bool entry_row_map(const csa2_kv_cache& cache, CUtensorMap* map) {
+static bool entry_row_map(const csa2_kv_cache& cache, CUtensorMap* map, uint32_t box_rows = 64u) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)kID, (cuuint64_t)(cache.n_phys_pages * cache.page_size)};
     const cuuint64_t strides[1] = {(cuuint64_t)kID * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kID, 64u};
+    const cuuint32_t box[2] = {(cuuint32_t)kID, box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void*)cache.idx_k, dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -2119,10 +2119,10 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
                               const int32_t* seq_lens, const int32_t* cand_blocks, int keep, int topk, int32_t* out,
                               int n, int64_t max_len, char* ws, int32_t* err, cudaStream_t stream,
                               int pre) {
-    static bool d4[64];
-    cudaError_t e = ensure_smem((const void*)token_topk_kernel, TK_SMEM, d4);
+    static bool d4[64], d5[64];
+    cudaError_t e = ensure_smem((const void*)token_score_kernel, TS_SMEM, d4);
+    if (e == cudaSuccess) e = ensure_smem((const void*)token_select_kernel, TK_SMEM, d5);
     if (e != cudaSuccess) return e;
-    (void)ws;
     TokenArgs a{};
     a.cache = cache;
     a.q_idx = q_idx;
@@ -2130,14 +2130,23 @@ cudaError_t launch_token_topk(const csa2_kv_cache& cache, const uint16_t* q_idx,
     a.seq_lens = seq_lens;
     a.cand = cand_blocks;
     a.out = out;
+    a.keys = reinterpret_cast<uint32_t*>(ws + decode_ws_layout(n, max_len, false).tok_keys);
     a.err = err;
     a.max_len = max_len;
     a.keep = keep;
     a.topk = topk;
     a.page_shift = page_shift_of(cache);
     a.pre = pre;
-    LaunchCfg c(dim3((unsigned)n * TK_CL), dim3(TK_THREADS), TK_SMEM, stream);
-    return cudaLaunchKernelEx(&c.cfg, token_topk_kernel, a);
+    // candidate blocks as 8-row tensor boxes when every slot is an int32
+    // coordinate (a block's 8 rows lie in one page: pages hold >= 8 entries)
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    a.tma = (cache.n_phys_pages << a.page_shift) <= INT32_MAX && entry_row_map(cache, &map, kBlk) ? 1 : 0;
+    LaunchCfg c1(dim3((unsigned)n * TS_PARTS), dim3(TS_THREADS), TS_SMEM, stream);
+    e = cudaLaunchKernelEx(&c1.cfg, token_score_kernel, map, a);
+    if (e != cudaSuccess) return e;
+    LaunchCfg c2(dim3((unsigned)n), dim3(TK_THREADS), TK_SMEM, stream);
+    return cudaLaunchKernelEx(&c2.cfg, token_select_kernel, a);
 }
 
 cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_idx, const float* w,
