@@ -833,7 +833,7 @@ def run_launch_floor(args, local_rank: int) -> dict:
     sink = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     out = {}
-    for n, ctas in ((28, 64), (28, 148), (28, 296), (20, 148), (1, 148)):
+    for n, ctas in ((33, 148), (28, 64), (28, 148), (28, 296), (20, 148), (1, 148)):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             csa2.test_empty_chain(n, ctas, 160, sink, stream=stream)
