@@ -586,17 +586,53 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
     __syncthreads();
     find_kth_bin(hist, 1024, need, tmp, &d2, &above);
     need -= above;
-    for (int i = threadIdx.x; i < 1024; i += K3_THREADS) hist[i] = 0;
-    __syncthreads();
-    for (int base = wid * 32; base < (int)n_bnd; base += K3_THREADS) {
-        const int i = base + lane;
-        const uint32_t key = i < (int)n_bnd ? (uint32_t)(B[i] >> 32) : 0u;
-        hist_add(hist, key & 1023u, i < (int)n_bnd && (int)((key >> 10) & 1023u) == d2);
+    const uint32_t nb2 = hist[d2];  // boundary rows in the second digit's bin
+    const uint32_t hi22 = (bstar << 20) | ((uint32_t)d2 << 10);
+    uint32_t T;
+    if (hi22 > 0u && nb2 == need) {  // the bin is taken whole: T just below it, no ties
+        T = hi22 - 1u;
+        need = 0u;
+    } else if (nb2 <= 32u) {  // one warp ranks the bin's keys
+        uint32_t* bk = hist;  // [32] keys (the histogram is read), counter at tmp[55]
+        if (threadIdx.x == 0) tmp[55] = 0u;
+        __syncthreads();  // every thread has read hist[d2]
+        for (uint32_t i = threadIdx.x; i < n_bnd; i += K3_THREADS) {
+            const uint32_t key = (uint32_t)(B[i] >> 32);
+            if ((key >> 10) == (hi22 >> 10)) bk[atomicAdd(&tmp[55], 1u)] = key;
+        }
+        __syncthreads();
+        if (wid == 0) {  // T = the need-th largest key of the bin
+            const bool mine = (uint32_t)lane < nb2;
+            const uint32_t kl = mine ? bk[lane] : 0u;
+            uint32_t ge = 0;
+            for (int j = 0; j < 32; ++j) {
+                const uint32_t kj = __shfl_sync(0xffffffffu, kl, j);
+                ge += ((uint32_t)j < nb2 && kj >= kl) ? 1u : 0u;
+            }
+            const uint32_t Tw = __reduce_max_sync(0xffffffffu, mine && ge >= need ? kl : 0u);
+            const uint32_t gt = __popc(__ballot_sync(0xffffffffu, mine && kl > Tw));
+            if (lane == 0) {
+                tmp[53] = Tw;
+                tmp[54] = need - gt;
+            }
+        }
+        __syncthreads();
+        T = tmp[53];
+        need = tmp[54];
+    } else {  // the third digit over the bin's rows
+        __syncthreads();  // every thread has read hist[d2]
+        for (int i = threadIdx.x; i < 1024; i += K3_THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int base = wid * 32; base < (int)n_bnd; base += K3_THREADS) {
+            const int i = base + lane;
+            const uint32_t key = i < (int)n_bnd ? (uint32_t)(B[i] >> 32) : 0u;
+            hist_add(hist, key & 1023u, i < (int)n_bnd && (int)((key >> 10) & 1023u) == d2);
+        }
+        __syncthreads();
+        find_kth_bin(hist, 1024, need, tmp, &d3, &above);
+        need -= above;
+        T = hi22 | (uint32_t)d3;
     }
-    __syncthreads();
-    find_kth_bin(hist, 1024, need, tmp, &d3, &above);
-    need -= above;
-    const uint32_t T = (bstar << 20) | ((uint32_t)d2 << 10) | (uint32_t)d3;
     if (kFlat) {
         // A flat selection takes keep (<= 512) of up to 2^21 rows: list them
         // (the rows above the K-th's bin, the boundary rows above T and the
@@ -757,8 +793,56 @@ __global__ void __launch_bounds__(K3_THREADS) block_select_kernel(BlockArgs a) {
                 }
                 base += __shfl_sync(0xffffffffu, incl, 31);
             }
-        } else {  // the block level's short chunk
-            // thread t owns words [t*per, (t+1)*per) of the chunk
+        } else if (cn <= 8 * K3_THREADS) {  // a short chunk (contexts up to 1M): thread t owns words [8t, 8t + 8)
+            const int w0 = 8 * threadIdx.x;
+            uint32_t wb[8], wt[8];
+            if (w0 + 8 <= cn) {  // 16-byte reads (the chunk starts 16-byte aligned)
+                const uint4 b0 = reinterpret_cast<const uint4*>(cbm + w0)[0], b1 = reinterpret_cast<const uint4*>(cbm + w0)[1];
+                const uint4 t0 = reinterpret_cast<const uint4*>(ctie + w0)[0], t1 = reinterpret_cast<const uint4*>(ctie + w0)[1];
+                wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w; wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
+                wt[0] = t0.x; wt[1] = t0.y; wt[2] = t0.z; wt[3] = t0.w; wt[4] = t1.x; wt[5] = t1.y; wt[6] = t1.z; wt[7] = t1.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    wb[k] = w0 + k < cn ? cbm[w0 + k] : 0u;
+                    wt[k] = w0 + k < cn ? ctie[w0 + k] : 0u;
+                }
+            }
+            // one scan of (ties, rows above T): fewer than keep <= 2048 rows lie above T
+            // (12 bits), at most 2^20 rows tie (20 bits); the ties taken before this
+            // thread are min(its tie prefix, need), lowest index first
+            uint32_t my_ties = 0, my_above = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                my_ties += __popc(wt[k]);
+                my_above += __popc(wb[k]);
+            }
+            uint32_t tot;
+            const uint32_t pre = block_excl_scan((my_ties << 12) | my_above, tmp, &tot);
+            const uint32_t tie_base = rank0 + (pre >> 12);
+            const uint32_t taken0 = min(rank0, need);  // ties the earlier chunks took
+            const uint32_t take = tie_base >= need ? 0u : min(my_ties, need - tie_base);
+            uint32_t pos = base0 + (pre & 0xfffu) + min(tie_base, need) - taken0, taken = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                uint32_t t = wt[k], kept = 0;
+                while (t && taken < take) {  // the lowest-index ties
+                    const uint32_t lb = t & (0u - t);
+                    kept |= lb;
+                    t ^= lb;
+                    ++taken;
+                }
+                uint32_t m = wb[k] | kept;
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (pos < (uint32_t)a.keep) out[pos] = (c0w + w0 + k) * 32 + bit;
+                    ++pos;
+                }
+            }
+            n_ties = tot >> 12;
+            n_sel = (tot & 0xfffu) + min(rank0 + n_ties, need) - taken0;
+        } else {  // a longer chunk: thread t owns words [t*per, (t+1)*per)
             const int per = (cn + K3_THREADS - 1) / K3_THREADS;
             const int w0 = threadIdx.x * per, w1 = min(cn, w0 + per);
             uint32_t my_ties = 0;
