@@ -162,6 +162,44 @@ def test_token_topk_bitexact(csa2, orc, lens):
     assert ps.errors() == 0
 
 
+def test_token_select_ties_and_wide_range(csa2, orc):
+    # Two cases the token select's one-warp bin resolution does not cover.
+    # Sequence 0: q = 0, so every score is 0 and all 16,384 candidates tie;
+    # the lowest 512 positions win.  Sequence 1: one indexer-K row is +-2^100
+    # with the signs of head 0's query, so its score lies ~100 binades above
+    # the others and the K-th key falls more than 8 binades below the largest;
+    # that entry is selected, the rest must match the oracle.  Both take the
+    # three-digit select.
+    lens = [20000, 20000]
+    B, max_len = len(lens), max(lens)
+    ps = PagedSeqs(csa2, lens)
+    q, w = _indexer_inputs(B)
+    q[0] = 0
+    idx0 = synth.idx_k_rows(SEED, 0, 0, lens[0])
+    kf = orc.bf16_to_f32(synth.idx_k_rows(SEED, 1, 0, lens[1])).reshape(lens[1], 64)
+    qf = orc.bf16_to_f32(q[1]).reshape(4, 64)
+    kf[12345] = np.where(qf[0] >= 0, 1.0, -1.0) * 2.0 ** 100
+    idx1 = synth.to_bf16_bits(kf)
+    for b, (L, idx) in enumerate(zip(lens, (idx0, idx1))):
+        ps.append(b, 0, synth.kv_rows(SEED, b, 0, L), idx)
+    ws = _ws(csa2, B, max_len)
+    sl = dev(np.array(lens, np.int32))
+    d = csa2.default_desc(csa2.FULL, 1)
+    blocks = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.BLOCK, bits16(q), dev(w), sl, blocks, B, max_len, ws, err=ps.err)
+    out = torch.empty((B, 512), dtype=torch.int32, device="cuda")
+    csa2.indexer_topk(d, ps.cache, csa2.TOKEN, bits16(q), dev(w), sl, out, B, max_len, ws, cand_blocks=blocks,
+                      err=ps.err)
+    got = out.cpu().numpy()
+    assert got[0].tolist() == list(range(512))
+    for b, idx in ((0, idx0), (1, idx1)):
+        ob = orc.select_blocks(orc.pool_blocks(idx), lens[b], q[b], w[b])
+        want = orc.select_tokens(idx, lens[b], ob, q[b], w[b])
+        check_sets(got[b], want, f"seq {b}")
+    assert 12345 in got[1].tolist()
+    assert ps.errors() == 0
+
+
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------
