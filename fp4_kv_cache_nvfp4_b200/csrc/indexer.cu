@@ -1208,6 +1208,7 @@ struct PrefillArgs {
     int32_t* err;
     int64_t stride;
     int T, ratio, topk, n_entries, page_shift, kmax_parts;
+    int tma_k;         // 1: K5a's entry tiles arrive as 64-row tensor boxes (pages of >= 64 entries)
 };
 
 __device__ __forceinline__ int visible(int p, int ratio, int n) { return min((p + 1) / ratio, n); }
@@ -1409,31 +1410,34 @@ constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit thresho
 // K5a on tcgen05: a CTA scores 128 queries (MMA M, one TMEM lane each) against
 // its range of entries, 64 at a time (MMA N), all four heads (4 accumulators
 // of 64 columns, double-buffered: 512 TMEM columns).
-//   warps 0-7  epilogue: warps w and w + 4 read lane quarter w of the four
-//              accumulators (one query per thread, half of the 64 entries
-//              each) with tcgen05.ld, compute sum_h w_h relu(.), write keys
-//   warp 8     producer: K tiles by cp.async into a 4-stage ring (chunk
-//              swizzle of the canonical 128-byte layout); it waits for its
-//              own copies two tiles behind, fences them for the tensor core
-//              (generic -> async proxy) and marks the stage full
+//   warps 0-7  epilogue: warp w reads lane quarter w & 3 of the four
+//              accumulators (one query per thread, entries 32 (w >> 2) ..
+//              + 31 of the 64) with tcgen05.ld, computes sum_h w_h relu(.)
+//              and writes the keys
+//   warp 8     producer: each K tile as one 64-row tensor box (pages of >= 64
+//              entries) or by cp.async (the canonical 128-byte swizzle either
+//              way) into a 6-stage ring; the cp.async path waits for its own
+//              copies two tiles behind and fences them for the tensor core
 //   warp 9     MMA: one thread issues 16 tcgen05.mma per tile and commits to
 //              the tile's "done" and the stage's "empty" barriers
 //   warp 10    max |k| of every staged tile (the verification bound)
 constexpr int TC_Q = 128;
 constexpr int TC_E = 64;
-constexpr int TC_STAGES = 4;
-constexpr int TC_THREADS = 11 * 32;
-constexpr int TC_EPI_WARPS = 8;
+constexpr int TC_STAGES = 6;
+constexpr int TC_EPI_WARPS = 8;                      // 2 per TMEM lane quarter, 32 entries of a tile each
+constexpr int TC_W_PROD = TC_EPI_WARPS, TC_W_MMA = TC_EPI_WARPS + 1, TC_W_KMAX = TC_EPI_WARPS + 2;
+constexpr int TC_THREADS = (TC_EPI_WARPS + 3) * 32;
 constexpr size_t TC_OFF_Q = 0;                                          // 4 heads x [128][128 B]
-constexpr size_t TC_OFF_K = TC_OFF_Q + (size_t)kIH * TC_Q * 128;        // 4 stages x [64][128 B]
-constexpr size_t TC_OFF_BAR = TC_OFF_K + (size_t)TC_STAGES * TC_E * 128;  // full[4] empty[4] done[2] free[2]
-constexpr size_t TC_OFF_MISC = TC_OFF_BAR + 12 * 8;                     // tmem base, timeout
+constexpr size_t TC_OFF_K = TC_OFF_Q + (size_t)kIH * TC_Q * 128;        // stages x [64][128 B]
+constexpr size_t TC_OFF_BAR = TC_OFF_K + (size_t)TC_STAGES * TC_E * 128;  // full[S] empty[S] done[2] free[2]
+constexpr size_t TC_OFF_MISC = TC_OFF_BAR + (2 * TC_STAGES + 4) * 8;    // tmem base, timeout
 constexpr size_t TC_OFF_PG = TC_OFF_MISC + 16;                          // physical pages of the entry range
 constexpr int TC_MAX_PG = PT_SPLIT / kBlk;                              // pages are >= 8 entries
 constexpr size_t TC_SMEM = 120 * 1024;                                  // one CTA per SM: it owns all of TMEM
 static_assert(TC_OFF_PG + TC_MAX_PG * 4 <= TC_SMEM && TC_OFF_K % 1024 == 0, "K5a (tcgen05) shared-memory layout");
 
-__global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    prefill_tc_score_kernel(const __grid_constant__ CUtensorMap tmap, PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
     uint64_t* empty = full + TC_STAGES;
@@ -1494,7 +1498,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     fence_proxy_async_smem();  // the Q tiles are read by the tensor core
-    if (wid == 9) {
+    if (wid == TC_W_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                      "r"(512)
                      : "memory");
@@ -1505,7 +1509,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (wid == 8) {
+    if (wid == TC_W_PROD && a.tma_k) {
+        // ============ producer, tensor boxes: a tile's 64 entries lie in one page ============
+        if (lane == 0) {
+            const int32_t emask = (1 << sh) - 1;
+            for (int i = 0; i < ntile; ++i) {
+                const int s = i % TC_STAGES, e0 = e_beg + i * TC_E;
+                if (i >= TC_STAGES && !mbar_wait(&empty[s], (uint32_t)((i / TC_STAGES) - 1) & 1u, kWaitLimit))
+                    *s_timeout = 1;
+                int32_t phys = s_pg[(e0 >> sh) - pg0];
+                if (phys < 0) phys = 0;  // flagged above; the copy stays in bounds
+                mbar_arrive_expect_tx(&full[s], (uint32_t)TC_E * 128u);
+                tma_load_2d(smem + TC_OFF_K + (size_t)s * TC_E * 128, &tmap, 0, (phys << sh) | (e0 & emask), &full[s]);
+            }
+        }
+        __syncwarp();
+    } else if (wid == TC_W_PROD) {
         // ================= producer =================
         const int32_t emask = (1 << sh) - 1;
         auto issue = [&](int i) {
@@ -1541,7 +1560,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
                 publish(i - 2);
             }
         }
-    } else if (wid == 9) {
+    } else if (wid == TC_W_MMA) {
         // ================= MMA issue =================
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_E >> 3) << 17) |
@@ -1565,7 +1584,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
             }
         }
         __syncwarp();
-    } else if (wid == 10) {
+    } else if (wid == TC_W_KMAX) {
         // ================= max |k| of the staged tiles =================
         uint32_t kmax_bits = 0;
         for (int i = 0; i < ntile; ++i) {
@@ -1633,7 +1652,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) prefill_tc_score_kernel(Prefill
     }
     tc_fence_before();
     __syncthreads();  // every accumulator has been read
-    if (wid == 9) {
+    if (wid == TC_W_MMA) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
@@ -2265,9 +2284,17 @@ cudaError_t launch_prefill_topk(const csa2_kv_cache& cache, const uint16_t* q_id
     // tensor-core scores -> candidates, exact rescoring and verification; then
     // the exact CUDA-core path for the queries that failed the check (it exits
     // at once for the others)
+    // entry tiles as 64-row tensor boxes when a tile lies in one page and every
+    // slot is an int32 coordinate
+    CUtensorMap kmap;
+    memset(&kmap, 0, sizeof(kmap));
+    a.tma_k = cache.page_size >= TC_E && (cache.n_phys_pages << a.page_shift) <= INT32_MAX &&
+                      entry_row_map(cache, &kmap)
+                  ? 1
+                  : 0;
     LaunchCfg c0(dim3((unsigned)((T + TC_Q - 1) / TC_Q), (unsigned)((max_len + PT_SPLIT - 1) / PT_SPLIT)),
                  dim3(TC_THREADS), TC_SMEM, stream);
-    e = cudaLaunchKernelEx(&c0.cfg, prefill_tc_score_kernel, a);
+    e = cudaLaunchKernelEx(&c0.cfg, prefill_tc_score_kernel, kmap, a);
     if (e != cudaSuccess) return e;
     LaunchCfg cc(dim3((unsigned)T), dim3(PC_THREADS), PC_SMEM, stream);
     e = cudaLaunchKernelEx(&cc.cfg, prefill_candidates_kernel, a);
