@@ -360,14 +360,16 @@ def test_prefill_parity(csa2, orc):
     assert ps.errors() == 0
 
 
-def test_prefill_scattered_queries(csa2, orc):
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_prefill_scattered_queries(csa2, orc, page_size):
     # queries at non-consecutive positions, in no particular order: the window
     # branch walks the union of 16 queries' windows, the indexer's query tiles
-    # and the per-query kernels see unrelated neighbours
+    # and the per-query kernels see unrelated neighbours.  Pages of 16 entries
+    # take the scorer's cp.async producer, pages of 64 its tensor boxes.
     seed = 1003
     tokens = 4096 + 62
     n_ent = tokens // 2
-    ps = PagedSeqs(csa2, [n_ent], pooled=False)
+    ps = PagedSeqs(csa2, [n_ent], pooled=False, page_size=page_size)
     kv = synth.kv_rows(seed, 0, 0, tokens)
     idx_k = synth.idx_k_rows(seed, 0, 0, n_ent)
     ps.append(0, 0, synth.to_bf16_bits(kv), idx_k, ratio=2, chunk=999)
