@@ -70,9 +70,9 @@ extern "C" CSA2_API csa2_status csa2_indexer_topk_noalloc(const csa2_layer_desc*
     // The block-level and flat-row kernels expect their counters and
     // histograms at zero.  The previous call may have used another (n, max_len)
     // and so another layout: clear the zero-state head of this call's layout
-    // first (a memset, no allocation).  The token-level kernel (a hierarchical
+    // first (a memset, no allocation).  The token-level kernels (a hierarchical
     // Reindex/Full token call, or a flat call over at most 16,384 entries)
-    // keeps all its state on chip and reads no scratch, so it needs no clear.
+    // write every key they read back, so they need no clear.
     const bool flat = desc->keep_blocks == 0;
     const bool uses_scratch = level == CSA2_LEVEL_BLOCK || (flat && max_len > kMaxCand);
     if (uses_scratch) {

@@ -26,7 +26,8 @@
  *     descriptor/cache structs and the per-layer pointer tables of
  *     csa2_decode_layers, which are HOST memory read during the call;
  *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *     default stream) and may be captured in a CUDA graph;
+ *     default stream) and may be captured in a CUDA graph (stated for every
+ *     call except csa2_indexer_topk_noalloc);
  *   - kernels are launched with programmatic dependent launch: each waits for
  *     the preceding kernel in the stream before touching memory (inside
  *     csa2_decode_layers, see there);
@@ -344,11 +345,11 @@ CSA2_API csa2_status csa2_attn_lse_merge(int32_t n_parts, const float* out_parts
  *     1.3 * 2^20 entries (one sequence of 2^20 needs about 12.4 MiB, two need
  *     about 24.8 MiB);
  *   - the first call on a device looks up the array's device address, and the
- *     first call of each level and mode runs the kernels' one-time set-up
- *     (shared-memory attributes, and for flat rows the tensor-map entry
- *     point); make those first calls before any stream capture;
+ *     first call of each level and mode runs the kernels' one-time host set-up
+ *     (shared-memory attributes and the tensor-map entry point);
  *   - block-level and flat-row calls clear the counters they need (a memset on
- *     `stream`); token-level calls read no scratch.  Otherwise the array keeps
+ *     `stream`); token-level calls need no clear (they write every key they
+ *     read back).  Otherwise the array keeps
  *     what the previous call left; all calls share one array per device, so
  *     calls that overlap on the GPU (other streams, other threads) race and
  *     must be serialised by the caller. */
