@@ -31,8 +31,8 @@
 //   token_score_kernel  (K4a) 16 CTAs per sequence score the <= 16,384
 //                              candidates (1 KiB runs of 8 indexer-K rows) into
 //                              the workspace;
-//   token_select_kernel (K4b) one 8-CTA cluster per sequence selects the
-//                              Top-K across the cluster.
+//   token_select_kernel (K4b) one CTA per sequence selects the Top-K of
+//                              the sequence's keys.
 //   prefill_tc_score_kernel / prefill_candidates_kernel: prefill, approximate
 //                              scores on tcgen05, exact rescoring of the
 //                              candidates and a verified exact Top-K per query;
@@ -1391,11 +1391,13 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
 // ============================================================================
 // Prefill indexer on tensor cores, exact by verification
 //
-// K5a scores every (query, visible entry) pair with mma.sync bf16 x bf16 ->
-// fp32 (exact products, fp32 sums in the tensor core's order) and writes the
-// top 16 bits of each score's order-preserving key.  K5b, one CTA per query,
-// takes the approximate Top-1024 as candidates, rescores them with the exact
-// sequential-FMA chain and selects the exact Top-K among them; it then checks
+// K5a scores every (query, visible entry) pair on the tensor cores, bf16 x bf16
+// -> fp32 (exact products, fp32 sums in the tensor core's order), and writes
+// the top 16 bits of each score's order-preserving key.  K5b, one CTA per
+// query, takes the entries at or above a 16-bit threshold B as candidates
+// (about 800: B from a sample of the keys, or the 768th largest key), rescores
+// them with the exact sequential-FMA chain and selects the exact Top-K among
+// them; it then checks
 // that no other entry can reach that Top-K: every non-candidate's approximate
 // score lies below the candidates' 16-bit threshold B, and
 // |approximate - exact| <= delta = 2^-12 sum_h |w_h| ||q_h||_1 max|k|, a bound
@@ -1404,7 +1406,7 @@ __global__ void __launch_bounds__(PSEL_THREADS) prefill_select_kernel(PrefillArg
 // CUDA-core kernels recompute it.  The output is therefore the exact Top-K.
 // ============================================================================
 constexpr int PT_SPLIT = 2048;    // entries per CTA (grid.y splits the entry range)
-constexpr int PT_CAND = 768;      // approximate candidates per query
+constexpr int PT_CAND = 768;      // candidates per query when the threshold comes from every key
 constexpr int PT_CAND_MAX = 2048; // more candidates (ties at the 16-bit threshold) -> exact fallback
 
 // K5a on tcgen05: a CTA scores 128 queries (MMA M, one TMEM lane each) against
