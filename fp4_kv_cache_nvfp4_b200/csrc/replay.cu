@@ -9,22 +9,28 @@
 //   swa[b][(p) % window][c] = bf16( sum_k h[b][t][k] * w_kv[c][k] ),
 // p = L_b - n_b + t the position of row t of the last n_b = min(window, L_b)
 // tokens, c = 0..255 (K channels 0..127, V channels 128..255), fp32
-// accumulation on the tensor cores, round to nearest even.
+// accumulation, round to nearest even.
 //
-// One CTA per (sequence, slice of 32 of the 256 channels), so a layer's
-// replay of B sequences spreads over 8 B SMs: D[128 tokens x 32 ch] =
-// H[128 x d_model] . W_slice[32 x d_model]^T as tcgen05.mma kind::f16 (bf16 x
-// bf16 -> fp32, M 128, N 32, K 16), the fp32 accumulator in 32 TMEM columns.
-// The slices of one sequence read the same hidden states (from L2 after the
-// first).
+// A cluster of 4 CTAs per (sequence, slice of 64 of the 256 channels), the
+// cluster's CTAs splitting d_model four ways, so a layer's replay of B
+// sequences spreads over 16 B SMs and every CTA reads a quarter of the
+// hidden states it needs: D_r[128 tokens x 64 ch] = H[128 x d_r] .
+// W_slice[64 x d_r]^T over its quarter d_r, tcgen05.mma kind::f16 (bf16 x bf16
+// -> fp32, M 128, N 64, K 16), the fp32 partial in 64 TMEM columns.  The four
+// partials meet through distributed shared memory: CTA r owns channels
+// 16 r .. 16 r + 15 of the slice and receives the other three CTAs' partials
+// of them (8 KiB each), then sums the four in rank order (fixed, so the result
+// does not depend on timing) and rounds once to bf16.
 //   warp 0   producer: one lane loads 64-dim slices of H and W_slice as
-//            128-byte-swizzled TMA tensor boxes (no multicast) into a 4-stage
+//            128-byte-swizzled TMA tensor boxes (no multicast) into a 7-stage
 //            ring, completion counted in bytes on the stage's mbarrier;
 //   warp 1   MMA: allocates TMEM, one lane issues 4 MMAs per slice and commits
 //            to the stage's "empty" barrier, and to "done" after the last;
-//   warps 2-5  epilogue: warp w reads TMEM lane quarter w % 4 (one token per
-//            thread, 32 fp32 columns), rounds to bf16 and stores its part of
-//            the row.
+//   warps 2-5  epilogue: warp w owns TMEM lane quarter w % 4 (one token per
+//            thread): it stores the three foreign 16-channel parts of its rows
+//            into their owners' shared memory, and after the cluster barrier
+//            sums the four partials of its own part and stores the bf16 row
+//            part.
 #include <cstring>
 
 #include "common.cuh"
@@ -34,19 +40,24 @@
 namespace csa2 {
 
 constexpr int RP_M = 128;       // tokens per CTA (the window)
-constexpr int RP_N = 32;        // channels per CTA
-constexpr int RP_SLICES = kCh / RP_N;  // CTAs per sequence
+constexpr int RP_N = 64;        // channels per CTA
+constexpr int RP_SLICES = kCh / RP_N;  // channel slices per sequence
+constexpr int RP_KSPLIT = 4;    // CTAs of a cluster, splitting d_model
+constexpr int RP_OWN = RP_N / RP_KSPLIT;  // channels each CTA of the cluster sums and stores
 constexpr int RP_KS = 64;       // d_model slice per stage (128 B of bf16)
-constexpr int RP_STAGES = 4;
+constexpr int RP_STAGES = 7;
 constexpr int RP_THREADS = 6 * 32;
 constexpr uint32_t RP_TILE = RP_M * RP_KS * 2;           // 16 KiB: H slice [128 tokens][64 dims]
-constexpr uint32_t RP_TILE_B = RP_N * RP_KS * 2;         // 4 KiB: W slice [32 channels][64 dims]
+constexpr uint32_t RP_TILE_B = RP_N * RP_KS * 2;         // 8 KiB: W slice [64 channels][64 dims]
 constexpr size_t RP_OFF_A = 0;                           // [stages][128][128 B]
-constexpr size_t RP_OFF_B = RP_OFF_A + (size_t)RP_STAGES * RP_TILE;    // [stages][32][128 B]
-constexpr size_t RP_OFF_BAR = RP_OFF_B + (size_t)RP_STAGES * RP_TILE_B;  // full[4] empty[4] done
+constexpr size_t RP_OFF_B = RP_OFF_A + (size_t)RP_STAGES * RP_TILE;    // [stages][64][128 B]
+constexpr size_t RP_OFF_RED = RP_OFF_B + (size_t)RP_STAGES * RP_TILE_B;  // [source rank][4][128 rows][16 B]
+constexpr size_t RP_OFF_BAR = RP_OFF_RED + (size_t)RP_KSPLIT * RP_M * RP_OWN * 4;  // full[] empty[] done
 constexpr size_t RP_OFF_MISC = RP_OFF_BAR + (2 * RP_STAGES + 1) * 8;   // tmem base, timeout
 constexpr size_t RP_SMEM = RP_OFF_MISC + 16 + 1024;                    // + slack to align the base to 1 KiB
 constexpr uint32_t kReplayWaitLimit = 1u << 22;
+static_assert(RP_OWN == 16, "one 16-column TMEM load per owner part");
+static_assert(RP_SMEM <= 227 * 1024, "shared memory");
 
 struct ReplayArgs {
     const int32_t* seq_lens;
@@ -59,7 +70,8 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
                                                                     const __grid_constant__ CUtensorMap map_w,
                                                                     ReplayArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 128-byte-swizzled tiles need a 1 KiB-aligned base: round up inside the slack
+    // 128-byte-swizzled tiles need a 1 KiB-aligned base: round up inside the
+    // slack (the same offset in every CTA, so peer addresses line up)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + RP_OFF_BAR);
     uint64_t* empty = full + RP_STAGES;
@@ -67,8 +79,12 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + RP_OFF_MISC);
     int* s_timeout = reinterpret_cast<int*>(smem + RP_OFF_MISC + 4);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int b = blockIdx.x / RP_SLICES, n0 = (blockIdx.x % RP_SLICES) * RP_N;
+    // blockIdx.x = (b * RP_SLICES + slice) * RP_KSPLIT + rank; clusters are RP_KSPLIT consecutive CTAs
+    const int rank = (int)(blockIdx.x % RP_KSPLIT);
+    const int b = (int)(blockIdx.x / (RP_KSPLIT * RP_SLICES));
+    const int n0 = (int)((blockIdx.x / RP_KSPLIT) % RP_SLICES) * RP_N;
     const int nk = a.d_model / RP_KS;
+    const int k_begin = rank * nk / RP_KSPLIT, my_nk = (rank + 1) * nk / RP_KSPLIT - k_begin;
 
     if (tid == 0) {
         for (int s = 0; s < RP_STAGES; ++s) {
@@ -88,25 +104,31 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // every CTA of the cluster has started before any peer stores reach it:
+    // arrive now, wait just before the first remote store
+    cluster_arrive();
     const uint32_t tmem = *s_tmem;
     pdl_wait();  // the hidden states come from the preceding kernel
     pdl_trigger();
+    // the sequence length, read early by the epilogue warps (its latency hides behind the products)
+    const int32_t L = wid >= 2 ? a.seq_lens[b] : 0;
 
     if (wid == 0) {
         // ================= producer: TMA boxes of H and W =================
         if (lane == 0) {
-            for (int i = 0; i < nk; ++i) {
+            for (int i = 0; i < my_nk; ++i) {
                 const int s = i % RP_STAGES;
                 if (i >= RP_STAGES &&
                     !mbar_wait(&empty[s], (uint32_t)((i / RP_STAGES) - 1) & 1u, kReplayWaitLimit))
                     *s_timeout = 1;
                 mbar_arrive_expect_tx(&full[s], RP_TILE + RP_TILE_B);
                 // x = 64 i dims (128 B multiples), y = first row of the box
-                tma_load_2d(smem + RP_OFF_A + (size_t)s * RP_TILE, &map_h, i * RP_KS, b * a.window, &full[s]);
-                tma_load_2d(smem + RP_OFF_B + (size_t)s * RP_TILE_B, &map_w, i * RP_KS, n0, &full[s]);
+                const int x = (k_begin + i) * RP_KS;
+                tma_load_2d(smem + RP_OFF_A + (size_t)s * RP_TILE, &map_h, x, b * a.window, &full[s]);
+                tma_load_2d(smem + RP_OFF_B + (size_t)s * RP_TILE_B, &map_w, x, n0, &full[s]);
             }
             // the last stages' boxes have landed before this thread leaves (bounded)
-            for (int i = max(0, nk - RP_STAGES); i < nk; ++i)
+            for (int i = max(0, my_nk - RP_STAGES); i < my_nk; ++i)
                 if (!mbar_wait(&full[i % RP_STAGES], (uint32_t)(i / RP_STAGES) & 1u, kReplayWaitLimit))
                     *s_timeout = 1;
         }
@@ -115,8 +137,8 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
         // ================= MMA issue =================
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(RP_N >> 3) << 17) |
-                                   ((uint32_t)(RP_M >> 4) << 24);  // bf16 x bf16 -> f32, K-major, M 128, N 32
-            for (int i = 0; i < nk; ++i) {
+                                   ((uint32_t)(RP_M >> 4) << 24);  // bf16 x bf16 -> f32, K-major, M 128, N 64
+            for (int i = 0; i < my_nk; ++i) {
                 const int s = i % RP_STAGES;
                 if (!mbar_wait(&full[s], (uint32_t)(i / RP_STAGES) & 1u, kReplayWaitLimit)) *s_timeout = 1;
                 tc_fence_after();
@@ -127,36 +149,98 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
                     umma_bf16(tmem, da + 2u * kk, db + 2u * kk, idesc, (i | kk) > 0 ? 1u : 0u);
                 umma_commit(&empty[s]);
             }
-            umma_commit(done);
+            if (my_nk > 0)
+                umma_commit(done);
+            else
+                mbar_arrive(done);  // no products: the epilogue takes a zero partial
         }
         __syncwarp();
-    } else {
-        // ================= epilogue: thread = token = TMEM lane, 32 channels =================
-        const int quarter = wid & 3, t = 32 * quarter + lane;
-        const int32_t L = a.seq_lens[b];
-        const int n_b = L < 1 ? 0 : min(L, a.window);
-        if (L < 1 && lane == 0 && quarter == 0) dev_error(a.err, CSA2_DEV_LEN);
+    }
+
+    // ================= exchange: the partials of each owner's 16 channels =================
+    // Receive area [source rank][chunk c of 4 floats][128 rows][16 B]: one warp's store of a
+    // chunk is 512 contiguous bytes, and the owner's reads of a chunk by consecutive rows are
+    // free of bank conflicts.
+    const int quarter = wid & 3, t = 32 * quarter + lane;  // epilogue warps: TMEM lane quarter, token row
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+    auto red_off = [](int src, int row, int c) { return (uint32_t)(((src * 4 + c) * RP_M + row) * 16); };
+    uint32_t part[RP_KSPLIT][RP_OWN];  // this thread's row of the CTA's partial, by owner
+    if (wid >= 2) {
         if (!mbar_wait(done, 0u, kReplayWaitLimit)) *s_timeout = 1;
         tc_fence_after();
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
-        const int64_t p = (int64_t)L - n_b + t;  // position of this row's token
-        uint16_t* dst = a.swa + ((int64_t)b * a.window + (p % a.window + a.window) % a.window) * kCh + n0;
-#pragma unroll 1
-        for (int c = 0; c < RP_N; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(lane_base + (uint32_t)c, v);
-            tmem_wait_ld();
-            uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int r = 0; r < RP_KSPLIT; ++r) tmem_ld16(lane_base + (uint32_t)(r * RP_OWN), part[r]);
+        tmem_wait_ld();
+        if (my_nk == 0)  // d_model split four ways left this CTA nothing: its partial is zero
+#pragma unroll
+            for (int r = 0; r < RP_KSPLIT; ++r)
+#pragma unroll
+                for (int e = 0; e < RP_OWN; ++e) part[r][e] = 0u;
+    }
+    __syncwarp();
+    cluster_wait();  // the peers have started (their receive areas exist)
+    if (wid >= 2) {
+        const uint32_t red_local = smem_u32(smem + RP_OFF_RED);
+        // rounds j = 1, 2, 3 to owner rank + j: the four CTAs store to different peers at a
+        // time (the owner's part is picked by selects, so `part` stays in registers)
+#pragma unroll
+        for (int j = 1; j < RP_KSPLIT; ++j) {
+            const int r = (rank + j) % RP_KSPLIT;
+            float v[RP_OWN];
+#pragma unroll
+            for (int e = 0; e < RP_OWN; ++e) {
+                uint32_t x = part[0][e];
+#pragma unroll
+                for (int q = 1; q < RP_KSPLIT; ++q) x = r == q ? part[q][e] : x;
+                v[e] = __uint_as_float(x);
             }
-            if (t < n_b) {
-                uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-                d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            const uint32_t ra = mapa_shared(red_local, (uint32_t)r);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                st_cluster_f32x4(ra + red_off(rank, t, c), make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+        }
+    }
+    __syncwarp();
+    cluster_arrive();  // release: this CTA's stores into its peers
+    cluster_wait();    // acquire: the peers' stores into this CTA
+
+    if (wid >= 2) {
+        // ================= sum in rank order, round to bf16, store =================
+        const int n_b = L < 1 ? 0 : min(L, a.window);
+        if (L < 1 && lane == 0 && quarter == 0 && n0 == 0 && rank == 0) dev_error(a.err, CSA2_DEV_LEN);
+        float acc[RP_OWN];
+#pragma unroll
+        for (int e = 0; e < RP_OWN; ++e) acc[e] = 0.f;
+        const uint8_t* red = smem + RP_OFF_RED;
+#pragma unroll
+        for (int src = 0; src < RP_KSPLIT; ++src) {
+            if (src == rank) {
+#pragma unroll
+                for (int e = 0; e < RP_OWN; ++e) acc[e] += __uint_as_float(part[src][e]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 x = *reinterpret_cast<const float4*>(red + red_off(src, t, c));
+                    acc[4 * c] += x.x;
+                    acc[4 * c + 1] += x.y;
+                    acc[4 * c + 2] += x.z;
+                    acc[4 * c + 3] += x.w;
+                }
             }
+        }
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        if (t < n_b) {
+            const int64_t p = (int64_t)L - n_b + t;  // position of this row's token
+            uint16_t* dst = a.swa + ((int64_t)b * a.window + (p % a.window + a.window) % a.window) * kCh + n0 +
+                            rank * RP_OWN;
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
     }
     tc_fence_before();
@@ -216,7 +300,8 @@ extern "C" CSA2_API csa2_status csa2_swa_replay(const uint16_t* h, const uint16_
         !bf16_rows_map(w_kv, kCh, d_model, RP_N, &mw))
         return CSA2_ERR_CUDA;
     ReplayArgs a{seq_lens, swa_kv, err_word, B, d_model, window};
-    LaunchCfg c(dim3((unsigned)B * RP_SLICES), dim3(RP_THREADS), RP_SMEM, (cudaStream_t)stream);
+    LaunchCfg c(dim3((unsigned)B * RP_SLICES * RP_KSPLIT), dim3(RP_THREADS), RP_SMEM, (cudaStream_t)stream,
+                RP_KSPLIT);
     if (cudaLaunchKernelEx(&c.cfg, swa_replay_kernel, mh, mw, a) != cudaSuccess) {
         (void)cudaGetLastError();
         return CSA2_ERR_CUDA;

@@ -275,7 +275,9 @@ CSA2_API csa2_status csa2_decode_layers(int32_t n_layers, const csa2_layer_desc*
  *   swa_kv[b][p % window][c] = bf16_RNE( sum_k h[b][t][k] * w_kv[c][k] )
  * for the last n_b = min(window, seq_lens[b]) tokens, t = 0..n_b-1 oldest
  * first, p = seq_lens[b] - n_b + t; c = 0..255 (K channels 0..127, V
- * 128..255); fp32 accumulation on the tensor cores.  Rows of swa_kv outside
+ * 128..255); fp32 accumulation (tensor-core sums over four quarters of
+ * d_model, added in a fixed order, so the result does not vary from run to
+ * run).  Rows of swa_kv outside
  * the window and rows t >= n_b of h are not touched / not used.
  *   h      [B][window][d_model] bf16, 16-byte aligned
  *   w_kv   [256][d_model] bf16 (row c = output channel c), 16-byte aligned
