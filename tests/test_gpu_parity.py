@@ -101,10 +101,12 @@ def _indexer_inputs(B, layer=0, seed=SEED):
     return q, w
 
 
-def test_block_topk_bitexact(csa2, orc):
+@pytest.mark.parametrize("page_size", [64, 16])
+def test_block_topk_bitexact(csa2, orc, page_size):
+    # pooled rows in 1 KiB page runs (64 entries a page) or 256-byte ones (16)
     lens = [16392, 20001, 70000, 1000, 16384]
     B, max_len = len(lens), max(lens)
-    ps = PagedSeqs(csa2, lens)
+    ps = PagedSeqs(csa2, lens, page_size=page_size)
     idxs = [_fill(ps, b, L)[1] for b, L in enumerate(lens)]
     q, w = _indexer_inputs(B)
     ws = _ws(csa2, B, max_len)
