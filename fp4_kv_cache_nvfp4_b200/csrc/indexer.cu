@@ -56,31 +56,32 @@ namespace csa2 {
 // score of one indexer-K row held as 32 bf16x2 words; qd[d] = (q_0..q_3)[d]
 // ----------------------------------------------------------------------------
 // Two rows at once with packed fp32 arithmetic: fma.rn.f32x2 performs one
-// fused multiply-add, rounded to nearest, in each 32-bit half, so the low half
-// follows row k's scalar FMA chain and the high half row m's, bit for bit.
-// qp[2 d + j] holds ((q_2j, q_2j), (q_2j+1, q_2j+1)) of dimension d, j = 0, 1.
+// fused multiply-add, rounded to nearest, in each 32-bit half.  The halves hold
+// two heads of one row, so every (row, head) dot follows the scalar FMA chain
+// over the dimensions bit for bit.  qh[d] = (q_0, q_1, q_2, q_3)[d]: one 16-byte
+// load gives the head pairs (0, 1) and (2, 3) of dimension d for both rows.
 __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32_t (&m)[32],
-                                           const ulonglong2* __restrict__ qp, float4 w, float& s_k, float& s_m) {
-    uint64_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;  // (row k, row m) dot of head h; zero bits are (+0, +0)
+                                           const ulonglong2* __restrict__ qh, float4 w, float& s_k, float& s_m) {
+    uint64_t k01 = 0, k23 = 0, m01 = 0, m23 = 0;  // (head h, head h + 1) dots of rows k and m; zero bits are +0
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const uint64_t x0 = pack2(bf16_lo(k[i]), bf16_lo(m[i]));  // dimension 2i
-        const uint64_t x1 = pack2(bf16_hi(k[i]), bf16_hi(m[i]));  // dimension 2i + 1
-        const ulonglong2 q01a = qp[4 * i], q23a = qp[4 * i + 1], q01b = qp[4 * i + 2], q23b = qp[4 * i + 3];
-        c0 = ffma2(q01a.x, x0, c0);
-        c1 = ffma2(q01a.y, x0, c1);
-        c2 = ffma2(q23a.x, x0, c2);
-        c3 = ffma2(q23a.y, x0, c3);
-        c0 = ffma2(q01b.x, x1, c0);
-        c1 = ffma2(q01b.y, x1, c1);
-        c2 = ffma2(q23b.x, x1, c2);
-        c3 = ffma2(q23b.y, x1, c3);
+        const ulonglong2 qa = qh[2 * i], qb = qh[2 * i + 1];  // dimensions 2i and 2i + 1
+        const float xk0 = bf16_lo(k[i]), xk1 = bf16_hi(k[i]), xm0 = bf16_lo(m[i]), xm1 = bf16_hi(m[i]);
+        const uint64_t dk0 = pack2(xk0, xk0), dm0 = pack2(xm0, xm0), dk1 = pack2(xk1, xk1), dm1 = pack2(xm1, xm1);
+        k01 = ffma2(qa.x, dk0, k01);
+        k23 = ffma2(qa.y, dk0, k23);
+        m01 = ffma2(qa.x, dm0, m01);
+        m23 = ffma2(qa.y, dm0, m23);
+        k01 = ffma2(qb.x, dk1, k01);
+        k23 = ffma2(qb.y, dk1, k23);
+        m01 = ffma2(qb.x, dm1, m01);
+        m23 = ffma2(qb.y, dm1, m23);
     }
     float a0, a1, a2, a3, b0, b1, b2, b3;
-    unpack2(c0, a0, b0);
-    unpack2(c1, a1, b1);
-    unpack2(c2, a2, b2);
-    unpack2(c3, a3, b3);
+    unpack2(k01, a0, a1);
+    unpack2(k23, a2, a3);
+    unpack2(m01, b0, b1);
+    unpack2(m23, b2, b3);
     float s = 0.f, t = 0.f;
     s = __fmaf_rn(w.x, a0 > 0.f ? a0 : 0.f, s);
     t = __fmaf_rn(w.x, b0 > 0.f ? b0 : 0.f, t);
@@ -94,14 +95,12 @@ __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32
     s_m = t;
 }
 
-// Load q_idx [4][64] bf16 of one row into the duplicated layout idx_score2 reads.
-__device__ __forceinline__ void load_q_pairs(const uint16_t* q, float4* qp, int tid, int nt) {
-    for (int d = tid; d < kID; d += nt) {
-        const float q0 = bf16_bits_to_f32(q[d]), q1 = bf16_bits_to_f32(q[kID + d]);
-        const float q2 = bf16_bits_to_f32(q[2 * kID + d]), q3 = bf16_bits_to_f32(q[3 * kID + d]);
-        qp[2 * d] = make_float4(q0, q0, q1, q1);
-        qp[2 * d + 1] = make_float4(q2, q2, q3, q3);
-    }
+// Load q_idx [4][64] bf16 of one row into the layout idx_score2 reads:
+// qh[d] = (q_0, q_1, q_2, q_3)[d].
+__device__ __forceinline__ void load_q_heads(const uint16_t* q, float4* qh, int tid, int nt) {
+    for (int d = tid; d < kID; d += nt)
+        qh[d] = make_float4(bf16_bits_to_f32(q[d]), bf16_bits_to_f32(q[kID + d]), bf16_bits_to_f32(q[2 * kID + d]),
+                            bf16_bits_to_f32(q[3 * kID + d]));
 }
 
 
@@ -149,7 +148,7 @@ constexpr int K2_PROWS = K2_TILE / K2_PWARPS;   // 128 rows copied per producer 
 constexpr int K2_CROWS = K2_TILE / K2_CWARPS;   // 64 rows scored per consumer warp
 constexpr size_t K2_OFF_HIST = K2_STAGES * K2_STAGE_BYTES;
 constexpr size_t K2_OFF_QD = align16(K2_OFF_HIST + kHistBins * 4);
-constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 32);  // q in pairs: 64 x 32 B
+constexpr size_t K2_OFF_TMP = align16(K2_OFF_QD + kID * 16);  // q by dimension: 64 x 16 B
 constexpr size_t K2_OFF_TS = align16(K2_OFF_TMP + 64 * 4);
 constexpr size_t K2_OFF_NBLK = align16(K2_OFF_TS + (K2_MAX_SEQS + 1) * 4);
 constexpr size_t K2_OFF_BAR = align16(K2_OFF_NBLK + K2_MAX_SEQS * 4);  // full[3], empty[3]
@@ -413,7 +412,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid
         const int b = seq_of_tile(tile_start, a.n, t);
         if (b != cur_b) {
             if (cur_b >= 0) flush(cur_b, nloc);
-            load_q_pairs(a.q_idx + (int64_t)b * kIH * kID, qd, tid, K2_CTHREADS);
+            load_q_heads(a.q_idx + (int64_t)b * kIH * kID, qd, tid, K2_CTHREADS);
             if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
             cur_b = b;
             nloc = 0;
@@ -909,8 +908,8 @@ constexpr int TS_PARTS = 16;
 constexpr int TS_SLOTS = kMaxCand / TS_PARTS;  // 1024 candidate slots per CTA
 constexpr int TS_THREADS = 512;               // two rows per thread
 constexpr int TS_BLKS = TS_SLOTS / kBlk;       // 128 candidate blocks per CTA, 8 per warp
-constexpr size_t TS_OFF_QP = (size_t)TS_SLOTS * 128;                // rows | q pairs [128] float4
-constexpr size_t TS_OFF_MISC = TS_OFF_QP + 2 * kID * 16;             // w (float4)
+constexpr size_t TS_OFF_QP = (size_t)TS_SLOTS * 128;                // rows | q by dimension [64] float4
+constexpr size_t TS_OFF_MISC = TS_OFF_QP + kID * 16;                 // w (float4)
 constexpr size_t TS_OFF_BAR = TS_OFF_MISC + 16;                      // [16] per-warp copy barriers
 constexpr size_t TS_SMEM = TS_OFF_BAR + (TS_THREADS / 32) * 8;
 static_assert(TS_BLKS == 8 * (TS_THREADS / 32), "K4a: 8 candidate blocks per warp");
@@ -1031,9 +1030,9 @@ __global__ void __launch_bounds__(TS_THREADS, 1)
         pdl_wait();
         pdl_trigger();
     }
-    load_q_pairs(a.q_idx + (int64_t)b * kIH * kID, qp, tid, TS_THREADS);
+    load_q_heads(a.q_idx + (int64_t)b * kIH * kID, qp, tid, TS_THREADS);
     if (tid == 0) s_w = *reinterpret_cast<const float4*>(a.w + (int64_t)b * kIH);
-    __syncthreads();  // q pairs and w
+    __syncthreads();  // q and w
     if (a.tma) {
         if (!mbar_wait(bar, 0u, kWaitLimit) && lane == 0) dev_error(a.err, CSA2_DEV_TIMEOUT);
     } else {
