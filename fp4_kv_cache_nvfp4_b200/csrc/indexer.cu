@@ -1615,6 +1615,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             vis = visible(a.q_pos[t], a.ratio, a.n_entries);
         }
         const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+        // (w_h, w_h) pairs: fma.rn.f32x2 rounds each half as the scalar FMA chain over the heads does
+        const uint64_t wx2 = pack2(w.x, w.x), wy2 = pack2(w.y, w.y), wz2 = pack2(w.z, w.z), ww2 = pack2(w.w, w.w);
         for (int i = 0; i < ntile; ++i) {
             const int buf = i & 1, e0 = e_beg + i * TC_E;
             if (!mbar_wait(&done[buf], (uint32_t)(i >> 1) & 1u, kWaitLimit)) *s_timeout = 1;
@@ -1630,15 +1632,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 tmem_wait_ld();
                 uint32_t pk[8];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float s = 0.f;
-                    s = __fmaf_rn(w.x, fmaxf(__uint_as_float(v0[j]), 0.f), s);
-                    s = __fmaf_rn(w.y, fmaxf(__uint_as_float(v1[j]), 0.f), s);
-                    s = __fmaf_rn(w.z, fmaxf(__uint_as_float(v2[j]), 0.f), s);
-                    s = __fmaf_rn(w.w, fmaxf(__uint_as_float(v3[j]), 0.f), s);
-                    const uint32_t k16 = e0 + 16 * c + j < vis ? score_key(s) >> 16 : 0u;
-                    if (j & 1) pk[j >> 1] |= k16 << 16;
-                    else pk[j >> 1] = k16;
+                for (int j = 0; j < 16; j += 2) {  // entries j and j + 1 in the halves of packed FMAs
+                    const auto relu2 = [](uint32_t lo, uint32_t hi) {
+                        return pack2(fmaxf(__uint_as_float(lo), 0.f), fmaxf(__uint_as_float(hi), 0.f));
+                    };
+                    uint64_t s2 = ffma2(wx2, relu2(v0[j], v0[j + 1]), 0ull);
+                    s2 = ffma2(wy2, relu2(v1[j], v1[j + 1]), s2);
+                    s2 = ffma2(wz2, relu2(v2[j], v2[j + 1]), s2);
+                    s2 = ffma2(ww2, relu2(v3[j], v3[j + 1]), s2);
+                    float sa, sb;
+                    unpack2(s2, sa, sb);
+                    const uint32_t ka = e0 + 16 * c + j < vis ? score_key(sa) >> 16 : 0u;
+                    const uint32_t kb = e0 + 16 * c + j + 1 < vis ? score_key(sb) >> 16 : 0u;
+                    pk[j >> 1] = ka | (kb << 16);
                 }
                 if (t < a.T) {
                     uint4* dst = reinterpret_cast<uint4*>(a.keys16 + (int64_t)t * a.stride + e0 + 16 * c);

@@ -90,3 +90,37 @@ def test_replay_rows_and_window_attention(csa2, orc, d_model):
         codes, scales = orc.quant_rows(synth.kv_rows(SEED, b, 0, L))
         ro, rl = orc.attend(q[b], idx[b], codes, scales, got[b, (L - n + np.arange(n)) % W])
         check_attn(out[b], lse[b], ro, rl, f"replayed window, seq {b}")
+
+
+@pytest.mark.parametrize("d_model,W", [(64, 64), (192, 128), (320, 32)])
+def test_replay_small_d_model_and_short_window(csa2, orc, d_model, W):
+    """d_model split four ways leaves some CTAs of a cluster with no slice (64:
+    three of four; 192: one; 320: slices of 1, 1, 1, 2) and their partial is
+    zero; a window shorter than the 128-row tile reads the next sequence's rows
+    past n_b and discards them.  Rows within the bound of the oracle, other ring
+    slots untouched."""
+    lens = [W // 2, W, 3 * W + 5, 1]
+    B = len(lens)
+    layer = 5
+    h = np.stack([synth.hidden_rows(SEED, layer, b, W, d_model) for b in range(B)])
+    w_kv = synth.kv_projection(SEED, layer, d_model)
+    sentinel = np.uint16(0x7F7F)
+    swa = torch.full((B, W, 256), int(sentinel), dtype=torch.int16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa2.swa_replay(bits16(h), bits16(w_kv), dev(np.array(lens, np.int32)), swa, B, W, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = swa.cpu().numpy().view(np.uint16)
+    for b, L in enumerate(lens):
+        n = min(W, L)
+        want = orc.swa_replay(h[b, :n], w_kv)
+        slots = (L - n + np.arange(n)) % W
+        hf = orc.bf16_to_f32(h[b, :n]).astype(np.float64)
+        wf = orc.bf16_to_f32(w_kv).astype(np.float64)
+        gf = orc.bf16_to_f32(got[b, slots]).astype(np.float64)
+        rf = orc.bf16_to_f32(want).astype(np.float64)
+        bound = 2.0 ** -7 * np.abs(rf) + 2.0 * d_model * 2.0 ** -24 * (np.abs(hf) @ np.abs(wf).T)
+        assert (np.abs(gf - rf) - bound).max() <= 0, f"seq {b}"
+        assert (_ulps(got[b, slots], want) <= 1).mean() > 0.999
+        untouched = np.setdiff1d(np.arange(W), slots)
+        assert (got[b, untouched] == sentinel).all()
