@@ -166,6 +166,13 @@ __device__ __forceinline__ void st_async_f32x2(uint32_t addr, float a, float b, 
                  "f"(a), "f"(b), "r"(mbar)
                  : "memory");
 }
+// The same with 16 bytes.
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, float4 v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mbar)
+                 : "memory");
+}
 // Wait for a phase of this CTA's mbarrier whose bytes come from peer CTAs
 // (acquire at cluster scope); gives up after `limit` polls.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {

@@ -19,8 +19,10 @@
 // -> fp32, M 128, N 64, K 16), the fp32 partial in 64 TMEM columns.  The four
 // partials meet through distributed shared memory: CTA r owns channels
 // 16 r .. 16 r + 15 of the slice and receives the other three CTAs' partials
-// of them (8 KiB each), then sums the four in rank order (fixed, so the result
-// does not depend on timing) and rounds once to bf16.
+// of them (8 KiB each, asynchronous remote stores counted in bytes on its
+// mbarrier: no cluster barrier after the products), then sums the four in rank
+// order (fixed, so the result does not depend on timing) and rounds once to
+// bf16.
 //   warp 0   producer: one lane loads 64-dim slices of H and W_slice as
 //            128-byte-swizzled TMA tensor boxes (no multicast) into a 7-stage
 //            ring, completion counted in bytes on the stage's mbarrier;
@@ -28,9 +30,9 @@
 //            to the stage's "empty" barrier, and to "done" after the last;
 //   warps 2-5  epilogue: warp w owns TMEM lane quarter w % 4 (one token per
 //            thread): it stores the three foreign 16-channel parts of its rows
-//            into their owners' shared memory, and after the cluster barrier
-//            sums the four partials of its own part and stores the bf16 row
-//            part.
+//            into their owners' shared memory, and once its own mbarrier has
+//            counted the peers' 24 KiB sums the four partials of its own part
+//            and stores the bf16 row part.
 #include <cstring>
 
 #include "common.cuh"
@@ -52,8 +54,9 @@ constexpr uint32_t RP_TILE_B = RP_N * RP_KS * 2;         // 8 KiB: W slice [64 c
 constexpr size_t RP_OFF_A = 0;                           // [stages][128][128 B]
 constexpr size_t RP_OFF_B = RP_OFF_A + (size_t)RP_STAGES * RP_TILE;    // [stages][64][128 B]
 constexpr size_t RP_OFF_RED = RP_OFF_B + (size_t)RP_STAGES * RP_TILE_B;  // [source rank][4][128 rows][16 B]
-constexpr size_t RP_OFF_BAR = RP_OFF_RED + (size_t)RP_KSPLIT * RP_M * RP_OWN * 4;  // full[] empty[] done
-constexpr size_t RP_OFF_MISC = RP_OFF_BAR + (2 * RP_STAGES + 1) * 8;   // tmem base, timeout
+constexpr size_t RP_OFF_BAR = RP_OFF_RED + (size_t)RP_KSPLIT * RP_M * RP_OWN * 4;  // full[] empty[] done recv
+constexpr uint32_t RP_RECV_BYTES = (uint32_t)(RP_KSPLIT - 1) * RP_M * RP_OWN * 4;   // 24 KiB from the peers
+constexpr size_t RP_OFF_MISC = RP_OFF_BAR + (2 * RP_STAGES + 2) * 8;   // tmem base, timeout
 constexpr size_t RP_SMEM = RP_OFF_MISC + 16 + 1024;                    // + slack to align the base to 1 KiB
 constexpr uint32_t kReplayWaitLimit = 1u << 22;
 static_assert(RP_OWN == 16, "one 16-column TMEM load per owner part");
@@ -76,6 +79,7 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + RP_OFF_BAR);
     uint64_t* empty = full + RP_STAGES;
     uint64_t* done = empty + RP_STAGES;
+    uint64_t* recv = done + 1;  // the peers' partials of this CTA's channels, counted in bytes
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + RP_OFF_MISC);
     int* s_timeout = reinterpret_cast<int*>(smem + RP_OFF_MISC + 4);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -92,6 +96,8 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
+        mbar_init(recv, 1);
+        mbar_arrive_expect_tx(recv, RP_RECV_BYTES);
         *s_timeout = 0;
         fence_mbar_init();
     }
@@ -195,14 +201,16 @@ __global__ void __launch_bounds__(RP_THREADS, 1) swa_replay_kernel(const __grid_
                 v[e] = __uint_as_float(x);
             }
             const uint32_t ra = mapa_shared(red_local, (uint32_t)r);
+            const uint32_t rb = mapa_shared(smem_u32(recv), (uint32_t)r);
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                st_cluster_f32x4(ra + red_off(rank, t, c), make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+                st_async_f32x4(ra + red_off(rank, t, c), make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]),
+                               rb);
         }
     }
-    __syncwarp();
-    cluster_arrive();  // release: this CTA's stores into its peers
-    cluster_wait();    // acquire: the peers' stores into this CTA
+    // no barrier: an owner waits only for the bytes it receives (the senders' stores complete on its
+    // mbarrier; a CTA leaves only after its own partials arrived, so every store finds its target)
+    if (wid >= 2 && !mbar_wait_cluster(recv, 0u, kReplayWaitLimit)) *s_timeout = 1;
 
     if (wid >= 2) {
         // ================= sum in rank order, round to bf16, store =================
