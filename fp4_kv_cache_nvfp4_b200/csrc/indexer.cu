@@ -95,6 +95,53 @@ __device__ __forceinline__ void idx_score2(const uint32_t (&k)[32], const uint32
     s_m = t;
 }
 
+// The same two rows read from a 128-byte-swizzled tile in shared memory chunk by
+// chunk as the dimensions advance (rows ra and rb of the tile; chunk c of row r
+// at c ^ (r & 7)), so the rows never occupy 64 registers at once.
+__device__ __forceinline__ void idx_score2_tile(const uint8_t* tile, int ra, int rb, const ulonglong2* __restrict__ qh,
+                                                float4 w, float& s_k, float& s_m) {
+    uint64_t k01 = 0, k23 = 0, m01 = 0, m23 = 0;
+    const uint8_t* pa = tile + ra * 128;
+    const uint8_t* pb = tile + rb * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // 16-byte chunk c: dimensions 8c .. 8c + 7
+        const uint4 va = *reinterpret_cast<const uint4*>(pa + ((c ^ (ra & 7)) << 4));
+        const uint4 vb = *reinterpret_cast<const uint4*>(pb + ((c ^ (rb & 7)) << 4));
+        const uint32_t ka[4] = {va.x, va.y, va.z, va.w}, kb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = 4 * c + u;
+            const ulonglong2 qa = qh[2 * i], qb = qh[2 * i + 1];
+            const float xk0 = bf16_lo(ka[u]), xk1 = bf16_hi(ka[u]), xm0 = bf16_lo(kb[u]), xm1 = bf16_hi(kb[u]);
+            const uint64_t dk0 = pack2(xk0, xk0), dm0 = pack2(xm0, xm0), dk1 = pack2(xk1, xk1), dm1 = pack2(xm1, xm1);
+            k01 = ffma2(qa.x, dk0, k01);
+            k23 = ffma2(qa.y, dk0, k23);
+            m01 = ffma2(qa.x, dm0, m01);
+            m23 = ffma2(qa.y, dm0, m23);
+            k01 = ffma2(qb.x, dk1, k01);
+            k23 = ffma2(qb.y, dk1, k23);
+            m01 = ffma2(qb.x, dm1, m01);
+            m23 = ffma2(qb.y, dm1, m23);
+        }
+    }
+    float a0, a1, a2, a3, b0, b1, b2, b3;
+    unpack2(k01, a0, a1);
+    unpack2(k23, a2, a3);
+    unpack2(m01, b0, b1);
+    unpack2(m23, b2, b3);
+    float s = 0.f, t = 0.f;
+    s = __fmaf_rn(w.x, a0 > 0.f ? a0 : 0.f, s);
+    t = __fmaf_rn(w.x, b0 > 0.f ? b0 : 0.f, t);
+    s = __fmaf_rn(w.y, a1 > 0.f ? a1 : 0.f, s);
+    t = __fmaf_rn(w.y, b1 > 0.f ? b1 : 0.f, t);
+    s = __fmaf_rn(w.z, a2 > 0.f ? a2 : 0.f, s);
+    t = __fmaf_rn(w.z, b2 > 0.f ? b2 : 0.f, t);
+    s = __fmaf_rn(w.w, a3 > 0.f ? a3 : 0.f, s);
+    t = __fmaf_rn(w.w, b3 > 0.f ? b3 : 0.f, t);
+    s_k = s;
+    s_m = t;
+}
+
 // Load q_idx [4][64] bf16 of one row into the layout idx_score2 reads:
 // qh[d] = (q_0, q_1, q_2, q_3)[d].
 __device__ __forceinline__ void load_q_heads(const uint16_t* q, float4* qh, int tid, int nt) {
@@ -421,13 +468,10 @@ __global__ void __launch_bounds__(K2_THREADS, 1) block_score_kernel(const __grid
         if (!mbar_wait(&full[s], (uint32_t)(i / K2_STAGES) & 1u, a.wait_limit)) s_timeout = 1;
         const uint8_t* stage = smem + (size_t)s * K2_STAGE_BYTES;
         const int r0 = K2_CROWS * wid + lane;  // rows r0 and r0 + 32 of the tile
-        uint32_t k[32], m[32];
-        read_row(stage, r0, k);
-        read_row(stage, r0 + 32, m);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // the stage's rows of this warp are in registers
         float s0, s1;
-        idx_score2(k, m, reinterpret_cast<const ulonglong2*>(qd), s_w, s0, s1);
+        idx_score2_tile(stage, r0, r0 + 32, reinterpret_cast<const ulonglong2*>(qd), s_w, s0, s1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // the warp has read its rows of the stage
         const int32_t j = (t - tile_start[b]) * K2_TILE + r0;
         const int32_t nblk = s_nblk[b];
         float* sc = a.scores + (int64_t)b * a.nblk_pad;
