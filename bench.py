@@ -116,8 +116,8 @@ def attn_bytes_per_row(L: int) -> int:
 ATTN_TRAFFIC = {(8, 1 << 20): 4 * 518144}
 # dram__bytes_read.sum + dram__bytes_write.sum of one flat indexer launch
 # (block_score_kernel + block_select_kernel<1>) keyed by (B, entries), taken at
-# B = 2 (139,576,576 B) and scaled by the rows scored
-FLAT_TRAFFIC = {(8, 1 << 19): 558306304}
+# B = 2 (140,038,400 B) and scaled by the rows scored
+FLAT_TRAFFIC = {(8, 1 << 19): 4 * 140038400}
 
 
 class ClockSampler:
